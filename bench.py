@@ -1,0 +1,451 @@
+"""Benchmark of the 2:4 sparse FFN hot path on B200.
+
+One step = the whole path on one GPT-2 FFN (default: the 355M shape, fp16,
+8192 tokens):
+  mask step on W1 and W2 (transposable 2:4 search, flip count against the
+  previous mask, compression of both orientations), forward GEMMs
+  (X -> gelu(X W1m^T) -> H W2m^T), input-gradient GEMMs (dY -> dH with the
+  gelu' epilogue -> dX), masked decay on both gradients.
+The weights alternate between W and a N(0, 1e-4)-perturbed copy each step, so
+the flip count is live.  The metric is the dense-equivalent FLOPs of the four
+GEMMs divided by the step time (TFLOP/s); per-kernel times give the roofline.
+
+Multi-GPU: one process per GPU (torchrun), data-parallel replicas with their
+own token batch; masks are computed redundantly and bit-identically, so no
+collective runs on the data path (weak scaling).  Timing: W untimed warm-up
+steps, then exactly K steps between barrier + synchronize; L2 is flushed
+(256 MiB write) before every timed step outside the step's events; the step
+time is the sum of CUDA-event step times, max over ranks.
+
+--impl reference times the CPU oracle (the only other implementation this
+project has) on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic_inputs as si  # noqa: E402
+
+METRIC = "2:4 FFN GEMM TFLOP/s (% sparse TC peak); mask-search GB/s (% HBM) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_seeds(wl: si.FFNWorkload, rank: int) -> dict:
+    """Per-rank seeds: every replica holds the same weights and its own token batch."""
+    seeds = dict(wl.seeds)
+    seeds["X"] = wl.seeds["X"] + 1000 * rank
+    seeds["dY"] = wl.seeds["dY"] + 1000 * rank
+    return seeds
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/sp24_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ our arm
+
+class FFNStep:
+    """Device buffers and the launch sequence of one step (kernel launches only)."""
+
+    KERNELS = ("mask_step", "gemm_fwd", "gemm_dgrad", "masked_decay")
+
+    def __init__(self, wl: si.FFNWorkload, rank: int):
+        import torch
+        import structured_sparse_transformer_b200 as sp
+        self.sp, self.torch, self.wl = sp, torch, wl
+        tdt = si.DTYPES[wl.dtype]
+        T, d, ff = wl.tokens, wl.d, wl.ff
+        seeds = rank_seeds(wl, rank)
+        wl_r = si.FFNWorkload(wl.name, wl.d, wl.ff, wl.tokens, wl.dtype, wl.steps, wl.lam, seeds)
+        W1, W2 = wl_r.weights()
+        X, dY = wl_r.activations()
+        G1, G2 = wl_r.grads()
+        self.host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
+        dev = "cuda"
+        self.W = [[W1.to(dev), si.perturb(W1, wl.perturb_seed(0, 0)).to(dev)],
+                  [W2.to(dev), si.perturb(W2, wl.perturb_seed(0, 1)).to(dev)]]
+        self.X, self.dY = X.to(dev), dY.to(dev)
+        self.G = [G1.to(dev), G2.to(dev)]
+        self.idx = [[torch.zeros(ff // 4, d // 4, dtype=torch.uint8, device=dev) for _ in range(2)],
+                    [torch.zeros(d // 4, ff // 4, dtype=torch.uint8, device=dev) for _ in range(2)]]
+        self.flips = torch.zeros(2, dtype=torch.int64, device=dev)
+        self.c = [sp.alloc_compressed(ff, d, tdt), sp.alloc_compressed(d, ff, tdt)]
+        self.H = torch.empty(T, ff, dtype=tdt, device=dev)
+        self.Hpre = torch.empty(T, ff, dtype=tdt, device=dev)
+        self.dH = torch.empty(T, ff, dtype=tdt, device=dev)
+        self.Y = torch.empty(T, d, dtype=tdt, device=dev)
+        self.dX = torch.empty(T, d, dtype=tdt, device=dev)
+        self.step_no = 0
+        self.launches_per_step = 8
+
+    def run(self, events=None):
+        """Enqueue one step; if `events` is a dict, record (start, end) CUDA events per kernel."""
+        sp, torch, wl = self.sp, self.torch, self.wl
+        d, ff = wl.d, wl.ff
+        cur, prev = self.step_no % 2, (self.step_no + 1) % 2
+
+        def timed(name, fn):
+            if events is None:
+                fn()
+                return
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            events.setdefault(name, []).append((s, e))
+
+        for li in range(2):
+            c = self.c[li]
+            timed("mask_step", lambda li=li, c=c: sp.sp24_mask_step(
+                self.W[li][cur], self.idx[li][cur], self.idx[li][prev], self.flips[li:li + 1], *c))
+        c1, c2 = self.c
+        timed("gemm_fwd", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu", self.Hpre))
+        timed("gemm_fwd", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y))
+        timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre))
+        timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dH, c1[2], c1[3], d, self.dX))
+        for li in range(2):
+            timed("masked_decay", lambda li=li: sp.sp24_masked_decay(self.G[li], self.W[li][cur], self.idx[li][cur],
+                                                                      wl.lam))
+        self.step_no += 1
+
+    # algorithmic bytes / flops per launch of each kernel
+    def work(self):
+        wl = self.wl
+        n_el = wl.d * wl.ff
+        return {
+            # read W (2 B/el), idx_prev (1/16), write idx (1/16), values of both orientations (2 B/el),
+            # metadata of both orientations (2 x 1/8 B/el)
+            "mask_step": ("GB/s", n_el * (2 + 1 / 16 + 1 / 16 + 2 + 0.25)),
+            "gemm_fwd": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
+            "gemm_dgrad": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
+            # read g (4), W (2), idx (1/16), write g (4)
+            "masked_decay": ("GB/s", n_el * (10 + 1 / 16)),
+        }
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import structured_sparse_transformer_b200 as sp
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    step = FFNStep(wl, rank)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {sp.sp24_status_string(st)}")
+
+    events, step_ev = {}, []
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            step.run(events)
+            e.record()
+            step_ev.append((s, e))
+        barrier()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {sp.sp24_status_string(st)}")
+    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
+    total_ms = max_over_ranks(step_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    flops = wl.gemm_flops()
+    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    peaks, peak_kind = load_peaks()
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    kernels = {}
+    for name, (unit, amount) in step.work().items():
+        times = [s.elapsed_time(e) * 1e-3 for s, e in events.get(name, [])]
+        if not times:
+            continue
+        avg = sum(times) / len(times)
+        achieved = amount / avg / (1e12 if unit == "TFLOP/s" else 1e9)
+        peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
+        kernels[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
+                         "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
+    g = {k: kernels[k] for k in ("gemm_fwd", "gemm_dgrad")}
+    g_time = sum(v["avg_us"] * v["launches"] for v in g.values())
+    g_launches = sum(v["launches"] for v in g.values())
+    g_avg = g_time / g_launches * 1e-6
+    g_ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
+    roofline = {"bound": "tensor", "achieved": round(g_ach, 1), "peak": sparse_peak, "unit": "TFLOP/s",
+                "frac": round(g_ach / sparse_peak, 4), "traffic": args.gemm_traffic,
+                "kernel": "sp24_gemm_kernel (fwd + dgrad launches)",
+                "peak_source": f"2 x {peak_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s), "
+                               "the nominal 2:4 sparse ratio"}
+    mask = kernels["mask_step"]
+
+    e2e = run_e2e(args, step, wl, world, dev, barrier)
+    clocks = clk.summary()
+    flips = [int(x) for x in step.flips.cpu().tolist()]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
+        "config": {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff, "tokens_per_gpu": wl.tokens,
+                   "global_tokens": wl.tokens * world, "parallelism": f"dp{world} replicas, no collective",
+                   "l2": "flushed before every timed step (256 MiB write, outside the step events)"},
+        "roofline": roofline,
+        "mask_search_roofline": {"bound": "hbm", "achieved": mask["achieved"], "peak": peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": mask["frac"], "traffic": args.mask_traffic,
+                                 "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": clocks,
+        "last_flip_counts": flips,
+        "peaks": peak_kind,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_tokens)
+    return line
+
+
+def run_e2e(args, step, wl, world, dev, barrier):
+    """Same metric through the C ABI with host buffers: H2D of the step's inputs from pinned
+    memory and D2H of its results inside the timed region."""
+    import torch
+    h = {k: v.pin_memory() for k, v in step.host.items()}
+    out_y = torch.empty(step.Y.shape, dtype=step.Y.dtype).pin_memory()
+    out_dx = torch.empty(step.dX.shape, dtype=step.dX.dtype).pin_memory()
+    out_g = [torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in step.G]
+    out_f = torch.empty(2, dtype=torch.int64).pin_memory()
+
+    def one():
+        step.W[0][step.step_no % 2].copy_(h["W1"], non_blocking=True)
+        step.W[1][step.step_no % 2].copy_(h["W2"], non_blocking=True)
+        step.X.copy_(h["X"], non_blocking=True)
+        step.dY.copy_(h["dY"], non_blocking=True)
+        step.G[0].copy_(h["G1"], non_blocking=True)
+        step.G[1].copy_(h["G2"], non_blocking=True)
+        step.run()
+        out_y.copy_(step.Y, non_blocking=True)
+        out_dx.copy_(step.dX, non_blocking=True)
+        out_g[0].copy_(step.G[0], non_blocking=True)
+        out_g[1].copy_(step.G[1], non_blocking=True)
+        out_f.copy_(step.flips, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        one()
+    e.record()
+    barrier()
+    ms = max_over_ranks(s.elapsed_time(e), world, dev)
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = sum(t.numel() * t.element_size() for t in (out_y, out_dx, *out_g, out_f))
+    return {"value": round(wl.gemm_flops() * world * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / args.steps, 4)}
+
+
+# ---------------------------------------------------------- oracle (CPU) arm
+
+def oracle_step(wl, host, rows):
+    """One step of the CPU oracle on a token sample: both mask searches, both compressions,
+    the four GEMMs on `rows` token rows, GELU, masked decay on both gradients, flip counts.
+    Returns the GEMM FLOPs it processed."""
+    import numpy as np
+    import oracle
+    dt = wl.dtype
+    b1, b2 = si.bits16(host["W1"]), si.bits16(host["W2"])
+    i1, i2 = oracle.mask_search(b1, dt), oracle.mask_search(b2, dt)
+    oracle.compress_both(b1, i1)
+    oracle.compress_both(b2, i2)
+    k1, k2 = oracle.dense_mask(i1), oracle.dense_mask(i2)
+    w1, w2 = oracle.to_f64(b1, dt), oracle.to_f64(b2, dt)
+    x = oracle.to_f64(si.bits16(host["X"])[:rows], dt)
+    dy = oracle.to_f64(si.bits16(host["dY"])[:rows], dt)
+    pre = oracle.sparse_fwd(x, w1, k1)
+    h = oracle.gelu(pre)
+    oracle.sparse_fwd(h, w2, k2)
+    dh = oracle.sparse_dgrad(dy, w2, k2) * oracle.gelu_grad(pre)
+    oracle.sparse_dgrad(dh, w1, k1)
+    oracle.masked_decay(host["G1"].numpy(), b1, dt, i1, wl.lam)
+    oracle.masked_decay(host["G2"].numpy(), b2, dt, i2, wl.lam)
+    oracle.flip_count(i1, i1)
+    oracle.flip_count(i2, i2)
+    return 4 * 2.0 * rows * wl.d * wl.ff
+
+
+def cpu_baseline(wl, rows):
+    import oracle
+    oracle.build()
+    W1, W2 = wl.weights()
+    X, dY = wl.activations()
+    G1, G2 = wl.grads()
+    host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
+    t0 = time.perf_counter()
+    flops = oracle_step(wl, host, rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"one full oracle step of {wl.name} with the four GEMMs on the first {rows} of "
+                      f"{wl.tokens} token rows (mask search, compression, decay and flips in full)"}
+
+
+def run_reference(args, wl):
+    import oracle
+    oracle.build()
+    W1, W2 = wl.weights()
+    X, dY = wl.activations()
+    G1, G2 = wl.grads()
+    host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
+    rows = args.cpu_tokens
+    for _ in range(args.warmup):
+        oracle_step(wl, host, rows)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += oracle_step(wl, host, rows)
+    sec = time.perf_counter() - t0
+    value = flops / sec / 1e12
+    sample = (f"each step: the oracle's full {wl.name} step with the four GEMMs on the first {rows} of "
+              f"{wl.tokens} token rows")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff,
+                                            "tokens_per_gpu": wl.tokens, "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=si.GPT2_355M.name, choices=sorted(si.FFN_WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=256, help="token rows of the oracle's GEMM sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-traffic", type=float, default=None, help="ncu DRAM bytes per GEMM launch")
+    ap.add_argument("--mask-traffic", type=float, default=None, help="ncu DRAM bytes per mask-step launch")
+    args = ap.parse_args(argv)
+    wl = si.FFN_WORKLOADS[args.workload]
+    rank, world, local_rank = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, wl, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,209 @@
+/*
+ * sp24 -- 2:4 transposable-mask FFN kernels for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libsp24.so.  The operations come from "Accelerating Transformer
+ * Pre-training with 2:4 Sparsity" (Hu, Zhao, Huang, Chen, Zhu; ICML 2024):
+ *   - reproducibility table, Pseudocode row, Algorithm 1: transposable 2:4 mask
+ *     search by convolving |W| at stride 4 with the candidate 4x4 patterns and
+ *     taking the argmax per block;
+ *   - reproducibility table, Software Dependencies row: the pruning kernel and
+ *     the 2:4 sparse matrix multiplications, the masked decay kernel;
+ *   - abstract: masked decay on gradients, the flip rate that monitors mask
+ *     stability, and transposable masks so the backward product is 2:4 too.
+ *
+ * Conventions shared by every call
+ *   - Matrices are row-major.  W is [rows x cols] with leading dimension ldw
+ *     (elements).  A "block" is the 4x4 tile W[4i..4i+3][4j..4j+3].
+ *   - A mask is one uint8 pattern index per block, row-major
+ *     [rows/4][cols/4].  Index p in 0..89 names the p-th 4x4 0/1 pattern with
+ *     two ones in every row and column, in lexicographic order of the per-row
+ *     column pairs (each row's pair ranked (0,1)<(0,2)<(0,3)<(1,2)<(1,3)<(2,3),
+ *     row 0 most significant).  sp24_pattern_table() returns the patterns.
+ *   - Device pointers (marked "device") are caller-owned device memory; host
+ *     pointers (marked "host") are caller-owned host memory.  The library never
+ *     allocates, frees or keeps a pointer after a call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls that launch work are asynchronous and stream-ordered.
+ *   - Argument checks (shapes, dtypes, alignment, null pointers) run on the
+ *     host before anything is launched; a failed check launches nothing.
+ *   - Weights must be finite; results for NaN/Inf weights are unspecified
+ *     (never out-of-bounds accesses).
+ *   - A kernel that gives up waiting (bounded spin on an mbarrier) records it
+ *     in a per-device error word and exits; sp24_device_status() reports it.
+ */
+#ifndef SP24_H
+#define SP24_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SP24_API __attribute__((visibility("default")))
+#else
+#define SP24_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sp24_status {
+  SP24_OK = 0,
+  SP24_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum, ld < width */
+  SP24_ERR_UNSUPPORTED_SHAPE = 2, /* a size is not a multiple the call needs */
+  SP24_ERR_UNSUPPORTED_DTYPE = 3,
+  SP24_ERR_MISALIGNED = 4,        /* a pointer or row pitch is not 16-byte aligned */
+  SP24_ERR_CUDA = 5,              /* a CUDA runtime/driver call or launch failed */
+  SP24_ERR_TIMEOUT = 6,           /* a kernel gave up waiting (see sp24_device_status) */
+  SP24_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+} sp24_status;
+
+typedef enum sp24_dtype { SP24_F16 = 0, SP24_BF16 = 1 } sp24_dtype;
+
+typedef enum sp24_epilogue {
+  SP24_EPI_NONE = 0,
+  SP24_EPI_GELU = 1,  /* out = gelu(acc) (exact erf form); aux <- acc rounded to dtype */
+  SP24_EPI_DGELU = 2  /* out = acc * gelu'(aux); aux holds the pre-activation */
+} sp24_epilogue;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+SP24_API const char *sp24_status_string(sp24_status status);
+
+/* Copies the 90 candidate patterns (bit 4*i+j set <=> row i, column j kept)
+ * into out[0..89] (host).  Algorithm 1's filter set m. */
+SP24_API sp24_status sp24_pattern_table(uint16_t *out);
+
+/*
+ * Transposable 2:4 mask search (Algorithm 1).
+ * For every block, scores each of the 90 patterns by the exact sum of the |W|
+ * values it keeps and writes the index of the best one; ties go to the lowest
+ * index.  The result is bit-exact (scores are exact integer sums, never
+ * rounded).
+ *   W    device, dtype, [rows x ldw] row-major, 16-byte aligned, ldw % 8 == 0
+ *   idx  device, uint8 [rows/4][cols/4]
+ *   rows, cols multiples of 4 (>= 0; zero-sized calls return SP24_OK).
+ */
+SP24_API sp24_status sp24_mask_search(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,
+                             int64_t ldw, uint8_t *idx, void *stream);
+
+/*
+ * Sizes of one compressed orientation of an [rows x cols] matrix compressed
+ * along its rows (2 of every 4 values per row are kept):
+ *   vals_bytes = rows * cols/2 * 2       (values, row-major [rows][cols/2])
+ *   meta_bytes = ceil(rows/128) * ceil(cols/128) * 2048
+ * The forward operand of W [R x C] is sp24_compressed_size(R, C); the
+ * input-gradient operand (W^T compressed along its rows) is (C, R).
+ */
+SP24_API sp24_status sp24_compressed_size(int64_t rows, int64_t cols, sp24_dtype dtype, size_t *vals_bytes,
+                                 size_t *meta_bytes);
+
+/*
+ * Pruning and compression of W with a given mask (the pruning kernel of the
+ * Software Dependencies row), into the layout the sparse tensor cores read.
+ *   vals_row  device [rows][cols/2]   kept values of each row, in column order
+ *   meta_row  device, meta_bytes of (rows, cols): 2-bit positions, tiled in
+ *             128x128 chunks of 2048 bytes in tensor-memory lane order
+ *   vals_col  device [cols][rows/2]   kept values of each column of W (rows of W^T)
+ *   meta_col  device, meta_bytes of (cols, rows)
+ * Either orientation may be skipped by passing NULL for both of its pointers.
+ * rows % 16 == 0 and cols % 16 == 0.  Every byte of the metadata buffers is
+ * written (padding carries a valid code).  sp24_meta_to_canonical() maps the
+ * metadata to a canonical per-row form.
+ */
+SP24_API sp24_status sp24_prune_compress(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,
+                                int64_t ldw, const uint8_t *idx, void *vals_row, void *meta_row,
+                                void *vals_col, void *meta_col, void *stream);
+
+/*
+ * One mask update in a single pass over W: search (as sp24_mask_search),
+ * optionally the flip count against the previous mask (as sp24_flip_rate) and
+ * optionally the compression of both orientations (as sp24_prune_compress).
+ *   idx_prev, d_flip_count  both NULL or both set (device); *d_flip_count is
+ *                           overwritten with the number of changed mask entries
+ *   vals_row..meta_col      as sp24_prune_compress, or all NULL (search only)
+ * Compression requires rows % 16 == 0 and cols % 16 == 0.
+ */
+SP24_API sp24_status sp24_mask_step(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols, int64_t ldw,
+                           uint8_t *idx, const uint8_t *idx_prev,
+                           unsigned long long *d_flip_count, void *vals_row, void *meta_row,
+                           void *vals_col, void *meta_col, void *stream);
+
+/*
+ * 2:4 sparse FFN forward GEMM (Software Dependencies row): Y = X * (W*m)^T.
+ *   X         device [T x K] row-major, contiguous
+ *   vals_row, meta_row   device, W [N x K] compressed along K (sp24_prune_compress)
+ *   Y         device [T x N] row-major, contiguous
+ *   epi       SP24_EPI_NONE, or SP24_EPI_GELU: Y = gelu(acc) and aux[T x N] <- acc
+ *   aux       device [T x N] for SP24_EPI_GELU, else ignored (may be NULL)
+ * fp32 accumulation; outputs rounded to dtype.  K % 16 == 0, N % 16 == 0,
+ * T >= 0.  All pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const void *vals_row,
+                          const void *meta_row, int64_t N, sp24_dtype dtype, void *Y,
+                          sp24_epilogue epi, void *aux, void *stream);
+
+/*
+ * 2:4 sparse FFN input-gradient GEMM: dX = dY * (W*m).  Valid as a 2:4 product
+ * because the transposed mask is 2:4 as well (abstract: transposable masks).
+ *   dY        device [T x N] row-major, contiguous
+ *   vals_col, meta_col   device, W^T [K x N] compressed along N (sp24_prune_compress)
+ *   dX        device [T x K]
+ *   epi       SP24_EPI_NONE, or SP24_EPI_DGELU: dX = acc * gelu'(aux), aux [T x K]
+ * N % 16 == 0, K % 16 == 0.
+ */
+SP24_API sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *vals_col,
+                            const void *meta_col, int64_t K, sp24_dtype dtype, void *dX,
+                            sp24_epilogue epi, const void *aux, void *stream);
+
+/*
+ * Masked decay on gradients (abstract; masked decay kernel of the Software
+ * Dependencies row): grad <- grad + lambda * W where the mask is 0, unchanged
+ * where it is 1, as one fp32 fused multiply-add per pruned entry (in place).
+ *   grad  device fp32 [rows x cols] contiguous;  W device dtype [rows x cols]
+ *   idx   device uint8 [rows/4][cols/4];  rows % 4 == 0, cols % 4 == 0
+ */
+SP24_API sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows,
+                              int64_t cols, const uint8_t *idx, float lambda, void *stream);
+
+/*
+ * Flip count between two masks (abstract: the flip rate): *d_count is
+ * overwritten with the number of the 16*nblocks mask entries that differ.
+ * The flip rate is *d_count / (16 * nblocks).
+ *   idx_prev, idx_cur  device uint8 [nblocks];  d_count device
+ */
+SP24_API sp24_status sp24_flip_rate(const uint8_t *idx_prev, const uint8_t *idx_cur, int64_t nblocks,
+                           unsigned long long *d_count, void *stream);
+
+/*
+ * Maps the device metadata of an [rows x cols] matrix compressed along its
+ * rows (meta_bytes from sp24_compressed_size) to the canonical form: for row
+ * r, group g (columns 4g..4g+3) with kept offsets i0 < i1, the nibble
+ * i0 | i1 << 2 sits at bits 4*(g % 4) of canon[r * ceil(cols/16) + g / 4].
+ * Pure index permutation on host buffers; cols % 16 == 0.
+ */
+SP24_API sp24_status sp24_meta_to_canonical(const void *meta_dev_layout_host, int64_t rows, int64_t cols,
+                                   uint16_t *canon);
+
+/* Inverse of sp24_meta_to_canonical (host buffers); padding gets code 0x4. */
+SP24_API sp24_status sp24_meta_from_canonical(const uint16_t *canon, int64_t rows, int64_t cols,
+                                     void *meta_dev_layout_host);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's error
+ * word.  Returns SP24_ERR_TIMEOUT if a kernel gave up waiting since the last
+ * query, SP24_ERR_CUDA if synchronization failed, else SP24_OK.
+ */
+SP24_API sp24_status sp24_device_status(void *stream);
+
+/*
+ * Test hook: the spin budget, in SM clock cycles, of every bounded wait in
+ * the GEMM kernels on later launches (default 2^32, about 2 s).  A budget of
+ * 0 makes a wait give up unless its barrier has already completed.
+ */
+SP24_API sp24_status sp24_set_wait_budget(uint64_t cycles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP24_H */

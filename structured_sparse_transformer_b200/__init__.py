@@ -1,0 +1,221 @@
+"""Python binding of libsp24.so -- argument marshalling only.
+
+Each ``sp24_*`` function here has the name of the C entry point it calls
+(``include/sp24.h``), takes torch CUDA tensors (or raw pointers for the host
+helpers), passes their data pointers, sizes and the current CUDA stream, and
+raises ``Sp24Error`` on a non-OK status.  Every step of the computation runs in
+the library's kernels; there is no fallback of any kind.  Importing the package
+raises if ``libsp24.so`` is missing: build it with
+``python -m structured_sparse_transformer_b200.build``.
+
+Operations from "Accelerating Transformer Pre-training with 2:4 Sparsity":
+transposable 2:4 mask search (reproducibility table, Pseudocode row,
+Algorithm 1), pruning/compression and the 2:4 sparse FFN GEMMs (Software
+Dependencies row), masked decay and flip rate (abstract).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libsp24.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m structured_sparse_transformer_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P, I64, I32, U64, F32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_float
+_SIGNATURES = {
+    "sp24_pattern_table": [P],
+    "sp24_mask_search": [P, I32, I64, I64, I64, P, P],
+    "sp24_compressed_size": [I64, I64, I32, P, P],
+    "sp24_prune_compress": [P, I32, I64, I64, I64, P, P, P, P, P, P],
+    "sp24_mask_step": [P, I32, I64, I64, I64, P, P, P, P, P, P, P, P],
+    "sp24_gemm_fwd": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
+    "sp24_gemm_dgrad": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
+    "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
+    "sp24_flip_rate": [P, P, I64, P, P],
+    "sp24_meta_to_canonical": [P, I64, I64, P],
+    "sp24_meta_from_canonical": [P, I64, I64, P],
+    "sp24_device_status": [P],
+    "sp24_set_wait_budget": [U64],
+}
+for _name, _args in _SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = I32
+_lib.sp24_status_string.argtypes = [I32]
+_lib.sp24_status_string.restype = ctypes.c_char_p
+
+STATUS = {0: "SP24_OK", 1: "SP24_ERR_INVALID_ARG", 2: "SP24_ERR_UNSUPPORTED_SHAPE",
+          3: "SP24_ERR_UNSUPPORTED_DTYPE", 4: "SP24_ERR_MISALIGNED", 5: "SP24_ERR_CUDA",
+          6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE"}
+SP24_F16, SP24_BF16 = 0, 1
+SP24_EPI_NONE, SP24_EPI_GELU, SP24_EPI_DGELU = 0, 1, 2
+EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2}
+
+
+class Sp24Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {sp24_status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ctypes library, for callers that marshal raw pointers themselves."""
+    return _lib
+
+
+def sp24_status_string(status: int) -> str:
+    return _lib.sp24_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise Sp24Error(fn, status)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return SP24_F16
+    if t.dtype == torch.bfloat16:
+        return SP24_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("sp24 kernels take CUDA tensors only")
+
+
+# ------------------------------------------------------------ host helpers
+
+def sp24_pattern_table():
+    """The 90 candidate patterns as a list of uint16 bit sets (bit 4*i+j = row i, column j)."""
+    out = (ctypes.c_uint16 * 90)()
+    _check("sp24_pattern_table", _lib.sp24_pattern_table(out))
+    return list(out)
+
+
+def sp24_compressed_size(rows: int, cols: int, dtype: int = SP24_F16):
+    """(vals_bytes, meta_bytes) of one orientation of an [rows x cols] matrix compressed along rows."""
+    v, m = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("sp24_compressed_size", _lib.sp24_compressed_size(rows, cols, dtype, ctypes.byref(v), ctypes.byref(m)))
+    return v.value, m.value
+
+
+def sp24_meta_to_canonical(meta_bytes: bytes, rows: int, cols: int):
+    """Device-layout metadata (host bytes) -> canonical uint16 words [rows][cols/16] (numpy)."""
+    import numpy as np
+    src = np.frombuffer(bytes(meta_bytes), dtype=np.uint8).copy()
+    out = np.zeros((rows, cols // 16), dtype=np.uint16)
+    _check("sp24_meta_to_canonical", _lib.sp24_meta_to_canonical(src.ctypes.data, rows, cols, out.ctypes.data))
+    return out
+
+
+def sp24_meta_from_canonical(canon, rows: int, cols: int):
+    """Canonical uint16 words (numpy [rows][cols/16]) -> device-layout metadata bytes (numpy uint8)."""
+    import numpy as np
+    canon = np.ascontiguousarray(canon, dtype=np.uint16)
+    out = np.zeros(sp24_compressed_size(rows, cols)[1], dtype=np.uint8)
+    _check("sp24_meta_from_canonical",
+           _lib.sp24_meta_from_canonical(canon.ctypes.data, rows, cols, out.ctypes.data))
+    return out
+
+
+# ------------------------------------------------------------ device calls
+
+def sp24_mask_search(W, idx, stream=None):
+    """idx[R/4, C/4] (uint8, CUDA) <- Algorithm 1 on W [R, C] (fp16/bf16, CUDA, row-major)."""
+    _need_cuda(W, idx)
+    R, C = W.shape
+    _check("sp24_mask_search", _lib.sp24_mask_search(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx),
+                                                     _stream(stream)))
+
+
+def sp24_prune_compress(W, idx, vals_row, meta_row, vals_col, meta_col, stream=None):
+    _need_cuda(W, idx, vals_row, meta_row, vals_col, meta_col)
+    R, C = W.shape
+    _check("sp24_prune_compress",
+           _lib.sp24_prune_compress(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(vals_row),
+                                    _ptr(meta_row), _ptr(vals_col), _ptr(meta_col), _stream(stream)))
+
+
+def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_row=None, vals_col=None,
+                   meta_col=None, stream=None):
+    _need_cuda(W, idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col)
+    R, C = W.shape
+    _check("sp24_mask_step",
+           _lib.sp24_mask_step(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(idx_prev),
+                               _ptr(flip_count), _ptr(vals_row), _ptr(meta_row), _ptr(vals_col),
+                               _ptr(meta_col), _stream(stream)))
+
+
+def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=None):
+    """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None or 'gelu' (aux <- pre-activation)."""
+    _need_cuda(X, vals_row, meta_row, Y, aux)
+    T, K = X.shape
+    _check("sp24_gemm_fwd",
+           _lib.sp24_gemm_fwd(_ptr(X), T, K, _ptr(vals_row), _ptr(meta_row), N, _dtype_code(X), _ptr(Y),
+                              EPILOGUES[epi], _ptr(aux), _stream(stream)))
+
+
+def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stream=None):
+    """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None or 'dgelu' (uses aux [T, K])."""
+    _need_cuda(dY, vals_col, meta_col, dX, aux)
+    T, N = dY.shape
+    _check("sp24_gemm_dgrad",
+           _lib.sp24_gemm_dgrad(_ptr(dY), T, N, _ptr(vals_col), _ptr(meta_col), K, _dtype_code(dY), _ptr(dX),
+                                EPILOGUES[epi], _ptr(aux), _stream(stream)))
+
+
+def sp24_masked_decay(grad, W, idx, lam: float, stream=None):
+    """grad[R, C] (fp32, in place) <- grad + lam * W on pruned entries."""
+    _need_cuda(grad, W, idx)
+    R, C = W.shape
+    _check("sp24_masked_decay",
+           _lib.sp24_masked_decay(_ptr(grad), _ptr(W), _dtype_code(W), R, C, _ptr(idx), float(lam),
+                                  _stream(stream)))
+
+
+def sp24_flip_rate(idx_prev, idx_cur, count, stream=None):
+    """count[0] (int64 CUDA tensor, read as uint64) <- number of mask entries that differ."""
+    _need_cuda(idx_prev, idx_cur, count)
+    _check("sp24_flip_rate",
+           _lib.sp24_flip_rate(_ptr(idx_prev), _ptr(idx_cur), idx_cur.numel(), _ptr(count), _stream(stream)))
+
+
+def sp24_device_status(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the device error status code."""
+    return int(_lib.sp24_device_status(_stream(stream)))
+
+
+def sp24_set_wait_budget(cycles: int):
+    _check("sp24_set_wait_budget", _lib.sp24_set_wait_budget(int(cycles)))
+
+
+# ------------------------------------------------------------ conveniences
+
+def alloc_compressed(rows: int, cols: int, dtype, device="cuda"):
+    """Allocates (vals_row, meta_row, vals_col, meta_col) for W [rows x cols] with torch."""
+    import torch
+    vr, mr = sp24_compressed_size(rows, cols)
+    vc, mc = sp24_compressed_size(cols, rows)
+    return (torch.empty(rows, cols // 2, dtype=dtype, device=device),
+            torch.empty(mr, dtype=torch.uint8, device=device),
+            torch.empty(cols, rows // 2, dtype=dtype, device=device),
+            torch.empty(mc, dtype=torch.uint8, device=device))

@@ -1,0 +1,394 @@
+// libsp24: host side of the C ABI declared in include/sp24.h.
+//
+// Every entry point validates its arguments on the host first (nothing is
+// launched when a check fails), then enqueues its kernels on the caller's
+// stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "sp24.h"
+#include "gemm_sp.cuh"
+#include "mask_kernels.cuh"
+
+namespace {
+
+using namespace sp24;
+
+std::atomic<uint64_t> g_wait_budget{1ull << 32};
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_dtype(sp24_dtype d) { return d == SP24_F16 || d == SP24_BF16; }
+
+sp24_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return SP24_ERR_NO_DEVICE; }
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_NO_DEVICE;
+  }
+  return major == 10 ? SP24_OK : SP24_ERR_NO_DEVICE;
+}
+
+sp24_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// --------------------------------------------------------- tensor maps (TMA)
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [outer x inner] array of 16-bit elements.
+bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+
+template <bool BF16, int EPI>
+sp24_status launch_gemm_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                          void *out, void *aux, cudaStream_t stream) {
+  CUtensorMap ta, tb, tout, taux;
+  if (!make_map_2d(&ta, vals, (uint64_t)(Kd / 2), (uint64_t)M, (uint64_t)Kd, kGemmBKc, kGemmBM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tout, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, kGemmBM, kEpiTokens,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SP24_ERR_CUDA;
+  taux = tout;
+  if (EPI == kEpiGelu &&
+      !make_map_2d(&taux, aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, kGemmBM, kEpiTokens,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SP24_ERR_CUDA;
+  auto kernel = sp24_gemm_kernel<BF16, EPI>;
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
+      return SP24_ERR_CUDA;
+    configured = true;
+  }
+  const int num_kt = (int)((Kd + kGemmBK - 1) / kGemmBK);
+  dim3 grid((unsigned)((M + kGemmBM - 1) / kGemmBM), (unsigned)((T + kGemmBN - 1) / kGemmBN));
+  kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, tout, taux, static_cast<const uint8_t *>(meta),
+                                                         static_cast<const uint16_t *>(aux), (int)M, (int)T,
+                                                         num_kt, g_wait_budget.load());
+  return launch_status();
+}
+
+sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                        sp24_dtype dt, void *out, int epi, void *aux, cudaStream_t s) {
+  const bool bf = dt == SP24_BF16;
+  switch (epi) {
+    case kEpiNone: return bf ? launch_gemm_t<true, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_t<false, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiGelu: return bf ? launch_gemm_t<true, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_t<false, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s);
+    default: return bf ? launch_gemm_t<true, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s)
+                       : launch_gemm_t<false, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s);
+  }
+}
+
+sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                          sp24_dtype dt, const void *out, int epi, const void *aux, int allowed_epi) {
+  if (!B && T > 0) return SP24_ERR_INVALID_ARG;
+  if (!vals || !meta || (!out && T > 0)) return SP24_ERR_INVALID_ARG;
+  if (T < 0 || Kd <= 0 || M <= 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dt)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (epi != SP24_EPI_NONE && epi != allowed_epi) return SP24_ERR_INVALID_ARG;
+  if (epi != SP24_EPI_NONE && !aux) return SP24_ERR_INVALID_ARG;
+  if (Kd % 16 || M % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || M > INT32_MAX || Kd > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(B) || !aligned16(vals) || !aligned16(meta) || !aligned16(out) ||
+      (epi != SP24_EPI_NONE && !aligned16(aux)))
+    return SP24_ERR_MISALIGNED;
+  return SP24_OK;
+}
+
+// ------------------------------------------------------------ mask launches
+
+template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
+sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint8_t *idx, const uint8_t *prev,
+                          unsigned long long *flip, void *vr, void *mr, void *vc, void *mc, cudaStream_t s) {
+  dim3 grid((unsigned)((C + kTile - 1) / kTile), (unsigned)((R + kTile - 1) / kTile));
+  mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP><<<grid, kMaskThreads, 0, s>>>(
+      static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
+      static_cast<uint8_t *>(mr), static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc));
+  return launch_status();
+}
+
+template <bool SEARCH, bool COMPRESS, bool FLIP>
+sp24_status launch_mask_d(bool bf, const void *W, int64_t R, int64_t C, int64_t ldw, uint8_t *idx,
+                          const uint8_t *prev, unsigned long long *flip, void *vr, void *mr, void *vc, void *mc,
+                          cudaStream_t s) {
+  return bf ? launch_mask_t<true, SEARCH, COMPRESS, FLIP>(W, R, C, ldw, idx, prev, flip, vr, mr, vc, mc, s)
+            : launch_mask_t<false, SEARCH, COMPRESS, FLIP>(W, R, C, ldw, idx, prev, flip, vr, mr, vc, mc, s);
+}
+
+sp24_status validate_w(const void *W, sp24_dtype dt, int64_t rows, int64_t cols, int64_t ldw) {
+  if (rows < 0 || cols < 0 || ldw < cols) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dt)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (rows % 4 || cols % 4) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (rows > 0 && cols > 0) {
+    if (!W) return SP24_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8) return SP24_ERR_MISALIGNED;
+  }
+  return SP24_OK;
+}
+
+size_t meta_bytes_of(int64_t rows, int64_t cols) {
+  return (size_t)((rows + 127) / 128) * (size_t)((cols + 127) / 128) * 2048u;
+}
+
+// Byte offset, inside the device metadata of a [rows x cols] matrix, of the
+// nibble for row r, group g (columns 4g..4g+3), and the nibble's bit shift.
+inline size_t meta_nibble_pos(int64_t r, int64_t g, int64_t cols, int *shift) {
+  const int64_t kt_count = (cols + 127) / 128;
+  const int64_t mt = r / 128, m = r % 128;
+  const int64_t kt = g / 32, gk = g % 32;           // 32 groups per 128-column chunk
+  const int64_t kk = gk / 8, gg = gk % 8;           // 8 groups per 32-column K step
+  const int64_t lane = (m % 8) + 8 * (gg / 4) + 16 * (m / 16);
+  const int bit = 4 * (int)(gg % 4) + 16 * (int)((m / 8) % 2);
+  *shift = bit % 8;
+  return (size_t)(mt * kt_count + kt) * 2048 + (size_t)lane * 16 + (size_t)kk * 4 + (size_t)(bit / 8);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sp24_status_string(sp24_status st) {
+  switch (st) {
+    case SP24_OK: return "SP24_OK";
+    case SP24_ERR_INVALID_ARG: return "SP24_ERR_INVALID_ARG";
+    case SP24_ERR_UNSUPPORTED_SHAPE: return "SP24_ERR_UNSUPPORTED_SHAPE";
+    case SP24_ERR_UNSUPPORTED_DTYPE: return "SP24_ERR_UNSUPPORTED_DTYPE";
+    case SP24_ERR_MISALIGNED: return "SP24_ERR_MISALIGNED";
+    case SP24_ERR_CUDA: return "SP24_ERR_CUDA";
+    case SP24_ERR_TIMEOUT: return "SP24_ERR_TIMEOUT";
+    case SP24_ERR_NO_DEVICE: return "SP24_ERR_NO_DEVICE";
+  }
+  return "SP24_UNKNOWN_STATUS";
+}
+
+sp24_status sp24_pattern_table(uint16_t *out) {
+  if (!out) return SP24_ERR_INVALID_ARG;
+  constexpr PatternTables t = make_pattern_tables();
+  for (int p = 0; p < kNumPatterns; ++p) out[p] = t.bits[p];
+  return SP24_OK;
+}
+
+sp24_status sp24_compressed_size(int64_t rows, int64_t cols, sp24_dtype dtype, size_t *vals_bytes,
+                                 size_t *meta_bytes) {
+  if (!vals_bytes || !meta_bytes || rows < 0 || cols < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (rows % 4 || cols % 4) return SP24_ERR_UNSUPPORTED_SHAPE;
+  *vals_bytes = (size_t)rows * (size_t)(cols / 2) * 2u;
+  *meta_bytes = meta_bytes_of(rows, cols);
+  return SP24_OK;
+}
+
+sp24_status sp24_mask_step(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols, int64_t ldw, uint8_t *idx,
+                           const uint8_t *idx_prev, unsigned long long *d_flip_count, void *vals_row,
+                           void *meta_row, void *vals_col, void *meta_col, void *stream) {
+  sp24_status st = validate_w(W, dtype, rows, cols, ldw);
+  if (st != SP24_OK) return st;
+  const bool flip = idx_prev != nullptr;
+  if ((idx_prev == nullptr) != (d_flip_count == nullptr)) return SP24_ERR_INVALID_ARG;
+  const bool any_c = vals_row || meta_row || vals_col || meta_col;
+  const bool all_c = vals_row && meta_row && vals_col && meta_col;
+  if (any_c && !all_c) return SP24_ERR_INVALID_ARG;
+  if (!idx && rows > 0 && cols > 0) return SP24_ERR_INVALID_ARG;
+  if (all_c) {
+    if (rows % 16 || cols % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(vals_row) || !aligned16(meta_row) || !aligned16(vals_col) || !aligned16(meta_col))
+      return SP24_ERR_MISALIGNED;
+  }
+  if ((st = check_device()) != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (flip && cudaMemsetAsync(d_flip_count, 0, sizeof(unsigned long long), s) != cudaSuccess)
+    return SP24_ERR_CUDA;
+  if (rows == 0 || cols == 0) return SP24_OK;
+  const bool bf = dtype == SP24_BF16;
+  if (all_c && flip)
+    return launch_mask_d<true, true, true>(bf, W, rows, cols, ldw, idx, idx_prev, d_flip_count, vals_row, meta_row,
+                                           vals_col, meta_col, s);
+  if (all_c)
+    return launch_mask_d<true, true, false>(bf, W, rows, cols, ldw, idx, nullptr, nullptr, vals_row, meta_row,
+                                            vals_col, meta_col, s);
+  if (flip)
+    return launch_mask_d<true, false, true>(bf, W, rows, cols, ldw, idx, idx_prev, d_flip_count, nullptr, nullptr,
+                                            nullptr, nullptr, s);
+  return launch_mask_d<true, false, false>(bf, W, rows, cols, ldw, idx, nullptr, nullptr, nullptr, nullptr,
+                                           nullptr, nullptr, s);
+}
+
+sp24_status sp24_mask_search(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols, int64_t ldw, uint8_t *idx,
+                             void *stream) {
+  return sp24_mask_step(W, dtype, rows, cols, ldw, idx, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        stream);
+}
+
+sp24_status sp24_prune_compress(const void *W, sp24_dtype dtype, int64_t rows, int64_t cols, int64_t ldw,
+                                const uint8_t *idx, void *vals_row, void *meta_row, void *vals_col, void *meta_col,
+                                void *stream) {
+  sp24_status st = validate_w(W, dtype, rows, cols, ldw);
+  if (st != SP24_OK) return st;
+  if ((vals_row == nullptr) != (meta_row == nullptr) || (vals_col == nullptr) != (meta_col == nullptr))
+    return SP24_ERR_INVALID_ARG;
+  if (rows % 16 || cols % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (rows > 0 && cols > 0 && !idx) return SP24_ERR_INVALID_ARG;
+  if ((vals_row && (!aligned16(vals_row) || !aligned16(meta_row))) ||
+      (vals_col && (!aligned16(vals_col) || !aligned16(meta_col))))
+    return SP24_ERR_MISALIGNED;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (rows == 0 || cols == 0 || (!vals_row && !vals_col)) return SP24_OK;
+  return launch_mask_d<false, true, false>(dtype == SP24_BF16, W, rows, cols, ldw, const_cast<uint8_t *>(idx),
+                                           nullptr, nullptr, vals_row, meta_row, vals_col, meta_col,
+                                           as_stream(stream));
+}
+
+sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const void *vals_row, const void *meta_row, int64_t N,
+                          sp24_dtype dtype, void *Y, sp24_epilogue epi, void *aux, void *stream) {
+  sp24_status st = validate_gemm(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, SP24_EPI_GELU);
+  if (st != SP24_OK) return st;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (T == 0) return SP24_OK;
+  return launch_gemm(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, as_stream(stream));
+}
+
+sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *vals_col, const void *meta_col,
+                            int64_t K, sp24_dtype dtype, void *dX, sp24_epilogue epi, const void *aux,
+                            void *stream) {
+  sp24_status st = validate_gemm(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, aux, SP24_EPI_DGELU);
+  if (st != SP24_OK) return st;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (T == 0) return SP24_OK;
+  return launch_gemm(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, const_cast<void *>(aux), as_stream(stream));
+}
+
+sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,
+                              const uint8_t *idx, float lambda, void *stream) {
+  sp24_status st = validate_w(W, dtype, rows, cols, cols);
+  if (st != SP24_OK) return st;
+  if (rows > 0 && cols > 0 && (!grad || !idx)) return SP24_ERR_INVALID_ARG;
+  if (rows > 0 && cols > 0 && !aligned16(grad)) return SP24_ERR_MISALIGNED;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (rows == 0 || cols == 0) return SP24_OK;
+  const int64_t nblocks = (rows / 4) * (cols / 4);
+  const int64_t want = (nblocks + 255) / 256;
+  const int grid = (int)(want < (int64_t)sm_count() * 16 ? want : (int64_t)sm_count() * 16);
+  cudaStream_t s = as_stream(stream);
+  if (dtype == SP24_BF16)
+    masked_decay_kernel<true><<<grid, 256, 0, s>>>(grad, static_cast<const uint16_t *>(W), idx, rows, cols, lambda);
+  else
+    masked_decay_kernel<false><<<grid, 256, 0, s>>>(grad, static_cast<const uint16_t *>(W), idx, rows, cols, lambda);
+  return launch_status();
+}
+
+sp24_status sp24_flip_rate(const uint8_t *idx_prev, const uint8_t *idx_cur, int64_t nblocks,
+                           unsigned long long *d_count, void *stream) {
+  if (nblocks < 0 || !d_count || (nblocks > 0 && (!idx_prev || !idx_cur))) return SP24_ERR_INVALID_ARG;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (cudaMemsetAsync(d_count, 0, sizeof(unsigned long long), s) != cudaSuccess) return SP24_ERR_CUDA;
+  if (nblocks == 0) return SP24_OK;
+  const int64_t want = (nblocks / 16 + 255) / 256 + 1;
+  const int grid = (int)(want < (int64_t)sm_count() * 8 ? want : (int64_t)sm_count() * 8);
+  flip_count_kernel<<<grid, 256, 0, s>>>(idx_prev, idx_cur, nblocks, d_count);
+  return launch_status();
+}
+
+sp24_status sp24_meta_to_canonical(const void *meta_dev_layout_host, int64_t rows, int64_t cols, uint16_t *canon) {
+  if (!meta_dev_layout_host || !canon || rows < 0 || cols < 0) return SP24_ERR_INVALID_ARG;
+  if (rows % 4 || cols % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
+  const uint8_t *dev = static_cast<const uint8_t *>(meta_dev_layout_host);
+  const int64_t words = cols / 16;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t w = 0; w < words; ++w) {
+      uint16_t v = 0;
+      for (int e = 0; e < 4; ++e) {
+        int shift = 0;
+        const size_t pos = meta_nibble_pos(r, 4 * w + e, cols, &shift);
+        v |= (uint16_t)(((dev[pos] >> shift) & 0xF) << (4 * e));
+      }
+      canon[r * words + w] = v;
+    }
+  return SP24_OK;
+}
+
+sp24_status sp24_meta_from_canonical(const uint16_t *canon, int64_t rows, int64_t cols, void *meta_dev_layout_host) {
+  if (!meta_dev_layout_host || !canon || rows < 0 || cols < 0) return SP24_ERR_INVALID_ARG;
+  if (rows % 4 || cols % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
+  uint8_t *dev = static_cast<uint8_t *>(meta_dev_layout_host);
+  memset(dev, 0x44, meta_bytes_of(rows, cols));
+  const int64_t words = cols / 16;
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t w = 0; w < words; ++w)
+      for (int e = 0; e < 4; ++e) {
+        int shift = 0;
+        const size_t pos = meta_nibble_pos(r, 4 * w + e, cols, &shift);
+        const uint8_t nib = (uint8_t)((canon[r * words + w] >> (4 * e)) & 0xF);
+        dev[pos] = (uint8_t)((dev[pos] & ~(0xF << shift)) | (nib << shift));
+      }
+  return SP24_OK;
+}
+
+sp24_status sp24_device_status(void *stream) {
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SP24_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess) return SP24_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SP24_ERR_CUDA;
+  return (word & kDevErrTimeout) ? SP24_ERR_TIMEOUT : SP24_OK;
+}
+
+sp24_status sp24_set_wait_budget(uint64_t cycles) {
+  g_wait_budget.store(cycles);
+  return SP24_OK;
+}
+
+}  // extern "C"

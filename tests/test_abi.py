@@ -1,0 +1,131 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every entry
+point that include/sp24.h declares, rejects bad arguments on the host before any
+CUDA call, and its host-side metadata maps agree with the oracle's canonical
+layout.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic_inputs as si
+import structured_sparse_transformer_b200 as sp
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sp24.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SP24_API[^;(]*?\b(sp24_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 14
+    lib = sp.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    expected = {"sp24_mask_search", "sp24_prune_compress", "sp24_gemm_fwd", "sp24_gemm_dgrad",
+                "sp24_masked_decay", "sp24_flip_rate"}
+    assert expected <= set(names)
+
+
+def test_status_strings():
+    for code, name in sp.STATUS.items():
+        assert sp.sp24_status_string(code) == name
+    assert sp.sp24_status_string(99) == "SP24_UNKNOWN_STATUS"
+
+
+def test_pattern_table_matches_oracle():
+    assert sp.sp24_pattern_table() == [int(b) for b in oracle.pattern_bits()]
+
+
+def test_compressed_size():
+    assert sp.sp24_compressed_size(6400, 1600) == (6400 * 800 * 2, 50 * 13 * 2048)
+    assert sp.sp24_compressed_size(1600, 6400) == (1600 * 3200 * 2, 13 * 50 * 2048)
+    assert sp.sp24_compressed_size(0, 0) == (0, 0)
+    with pytest.raises(sp.Sp24Error):
+        sp.sp24_compressed_size(6, 8)
+
+
+def _raw(name, *args):
+    return getattr(sp.lib(), name)(*args)
+
+
+def test_host_validation_rejects_bad_arguments_without_a_device():
+    fake = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks run first
+    odd = ctypes.c_void_p(0x10008)
+    E = {v: k for k, v in sp.STATUS.items()}
+    # mask search: shapes, dtype, alignment, null pointers
+    assert _raw("sp24_mask_search", fake, 0, 6, 8, 8, fake, None) == E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_mask_search", fake, 7, 8, 8, 8, fake, None) == E["SP24_ERR_UNSUPPORTED_DTYPE"]
+    assert _raw("sp24_mask_search", odd, 0, 8, 8, 8, fake, None) == E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_mask_search", fake, 0, 8, 8, 12, fake, None) == E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_mask_search", fake, 0, 8, 8, 4, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_mask_search", None, 0, 8, 8, 8, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    # compression needs multiples of 16
+    assert _raw("sp24_prune_compress", fake, 0, 8, 16, 16, fake, fake, fake, fake, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_mask_step", fake, 0, 16, 16, 16, fake, fake, None, None, None, None, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]
+    # GEMMs
+    assert _raw("sp24_gemm_fwd", fake, 8, 24, fake, fake, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 16, 0, fake, 1, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # GELU without aux
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 16, 0, fake, 2, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # DGELU is not a forward epilogue
+    assert _raw("sp24_gemm_dgrad", fake, 8, 32, fake, fake, 16, 0, fake, 1, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # GELU is not an input-gradient epilogue
+    assert _raw("sp24_gemm_fwd", odd, 8, 32, fake, fake, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_gemm_fwd", fake, -1, 32, fake, fake, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]
+    # decay and flip
+    assert _raw("sp24_masked_decay", fake, fake, 0, 6, 8, fake, ctypes.c_float(1.0), None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_flip_rate", fake, fake, -1, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_flip_rate", fake, fake, 4, None, None) == E["SP24_ERR_INVALID_ARG"]
+
+
+def test_valid_call_without_a_device_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    fake = ctypes.c_void_p(0x10000)
+    assert _raw("sp24_mask_search", fake, 0, 8, 8, 8, fake, None) == 7
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 16), (48, 80), (128, 256), (144, 400)])
+def test_meta_layout_roundtrip_and_padding(rows, cols):
+    w = si.normal((rows, cols), 0.02, seed=rows + cols, dtype="f16")
+    bits = si.bits16(w)
+    idx = oracle.mask_search(bits, "f16")
+    (_, canon_row), (_, canon_col) = oracle.compress_both(bits, idx)
+    for canon, r, c in ((canon_row, rows, cols), (canon_col, cols, rows)):
+        dev = sp.sp24_meta_from_canonical(canon, r, c)
+        assert dev.size == sp.sp24_compressed_size(r, c)[1]
+        back = sp.sp24_meta_to_canonical(dev.tobytes(), r, c)
+        assert np.array_equal(back, canon)
+        nibbles = np.stack([(dev >> 4) & 0xF, dev & 0xF]).reshape(-1)
+        assert set(np.unique(nibbles).tolist()) <= set(oracle.NIBBLE_CODES)
+        # every byte that no (row, group) maps to keeps the padding code 0x44
+        assert (dev == 0x44).sum() >= dev.size - r * (c // 4) // 2
+
+
+def test_meta_layout_is_a_permutation():
+    # Distinct canonical inputs map to distinct device bytes: the map is injective.
+    rows, cols = 128, 128
+    rng = np.random.default_rng(0)
+    codes = np.array(oracle.NIBBLE_CODES, dtype=np.uint16)
+    canon = np.zeros((rows, cols // 16), np.uint16)
+    for k in range(4):
+        canon |= codes[rng.integers(0, 6, canon.shape)] << (4 * k)
+    dev = sp.sp24_meta_from_canonical(canon, rows, cols)
+    assert dev.size == 2048
+    flipped = canon.copy()
+    flipped[37, 3] ^= 0x0040            # 0x4 <-> 0x0 in one nibble changes exactly one device nibble
+    dev2 = sp.sp24_meta_from_canonical(flipped, rows, cols)
+    assert np.count_nonzero(dev != dev2) == 1
