@@ -79,7 +79,8 @@ SP24_API sp24_status sp24_pattern_table(uint16_t *out);
  * values it keeps and writes the index of the best one; ties go to the lowest
  * index.  The result is bit-exact (scores are exact integer sums, never
  * rounded).
- *   W    device, dtype, [rows x ldw] row-major, 16-byte aligned, ldw % 8 == 0
+ *   W    device, dtype, [rows x ldw] row-major, 16-byte aligned, ldw % 4 == 0
+ *        (ldw % 8 == 0 lets every row be read with 128-bit loads)
  *   idx  device, uint8 [rows/4][cols/4]
  *   rows, cols multiples of 4 (>= 0; zero-sized calls return SP24_OK).
  */

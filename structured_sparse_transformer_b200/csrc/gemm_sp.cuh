@@ -9,47 +9,121 @@
 //     out[T x M] = B * A^T
 //   forward:        A = W   [N x K] compressed along K,  B = X  -> Y  [T x N]
 //   input gradient: A = W^T [K x N] compressed along N,  B = dY -> dX [T x K]
-// The sparse operand must be the MMA's A operand, so each CTA computes a
-// transposed tile out^T[128 x BN] in tensor memory (lane = output feature,
-// column = token) and the epilogue transposes it through shared memory into a
-// TMA store of row-major out.
+// The sparse operand must be the MMA's A operand, so the tensor-memory tile is
+// out^T (lane = output feature, column = token); each epilogue thread owns one
+// feature and writes it for consecutive tokens of row-major out.
 //
-// CTA = 6 warps: warp 0 issues TMA loads, warp 1 allocates TMEM and issues the
-// MMAs (one elected thread), warps 2-5 run the epilogue.  A 4-stage ring holds,
-// per 128-wide logical K step: A (128 x 64 kept values, 128B swizzle),
-// B (BN x 128, two 128B-swizzled boxes) and the 2 KB metadata chunk, which
-// tcgen05.cp moves into 4 TMEM columns before the four K=32 sparse MMAs of the
-// step read it.  Every wait is bounded; a wait that runs out records a timeout
-// in the device error word and the CTA drains its copies and exits.
+// CTA pairs (clusters of 2, tcgen05 cta_group::2).  A pair computes a tile of
+// 256 output features x 224 tokens: each CTA holds 128 rows of the compressed
+// operand and 112 token rows of the activations in its own shared memory, and
+// the pair's even (leader) CTA issues MMAs of M = 256, N = 224, K = 32 that
+// read both.  Per CTA and 128-wide K step this moves 46 KB (A 16 KB, B 28 KB,
+// metadata 2 KB) for 7.3 MFLOP dense-equivalent; a single-CTA 128 x 128 tile
+// moves 50 KB for 4.2 MFLOP and is bound by the latency of its L2 -> SM stream.
+// Persistent: each pair walks tiles pair, pair + npairs, ... (feature tiles
+// fastest, so the pairs running at once share token tiles through L2).
+//
+// Warps: 0 = TMA producer (both CTAs), 1 = TMEM allocation and, in the leader,
+// the MMA issuer, 2-13 = epilogue: three groups of four warps take alternate
+// 16-token chunks (warp w may read TMEM lanes 32*(w%4)..+31 only, so each group
+// covers the four lane quadrants).  Each epilogue warp works alone: TMEM ->
+// registers -> coalesced 64-byte global stores (32 consecutive features of one
+// token per store), with no shared-memory staging and no cross-warp barrier.
+// Shared memory: a 4-stage ring of {A 128x64 kept values, B 112x128 as two
+// boxes (both 128B-swizzled), the 2 KB metadata chunk}.
+// Tensor memory per CTA: two 224-column fp32 accumulators (tile i+1 runs its
+// MMAs while tile i drains) and 4 metadata columns per stage.
+// Protocol:
+//   - both producers TMA-load their halves, counting bytes on the leader's
+//     `full` barrier (the leader alone arms it with the pair's byte count);
+//   - the leader's MMA thread moves both metadata chunks into tensor memory
+//     (tcgen05.cp over the pair), issues the MMAs, and commits to `empty` and
+//     `acc_full` of both CTAs;
+//   - every epilogue warp of both CTAs arrives once on the leader's
+//     `acc_empty` when it has read its last chunk of a tile.
+// The dGELU epilogue loads a tile's pre-activation values into registers
+// before waiting for its accumulator, so the main loop hides their latency.
+// No load uses cluster multicast; each CTA reads its own tiles.
+// Every wait is bounded; a wait that runs out records a timeout in the device
+// error word, raises the CTA's abort flag, and the CTA drains and exits.
 #pragma once
 #include "sp24_common.cuh"
 
 namespace sp24 {
 
-constexpr int kGemmBM = 128;             // output features per CTA (MMA M)
-constexpr int kGemmBN = 128;             // tokens per CTA (MMA N)
-constexpr int kGemmBK = 128;             // logical K per pipeline stage
-constexpr int kGemmBKc = kGemmBK / 2;    // kept values per stage and row
-constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 192;
-constexpr int kSmemA = kGemmBM * kGemmBKc * 2;          // 16 KB
-constexpr int kSmemBBox = kGemmBN * 64 * 2;             // one 128-byte-wide box
-constexpr int kSmemB = 2 * kSmemBBox;                   // 32 KB
-constexpr int kSmemE = 2048;                            // metadata chunk
-constexpr int kStageBytes = kSmemA + kSmemB + kSmemE;
-constexpr int kEpiTokens = 32;                          // tokens per epilogue store
-constexpr int kSmemOut = kEpiTokens * kGemmBM * 2;      // 8 KB staging
-constexpr int kTmemCols = 256;                          // accumulator 128 + metadata 16
-constexpr int kTmemMetaCol = kGemmBN;
-constexpr int kGemmSmemBytes = kGemmStages * kStageBytes + 2 * kSmemOut + 256 + 1024;
+constexpr int kGemmBK = 128;                           // logical K per pipeline stage
+constexpr int kGemmBKc = kGemmBK / 2;                  // kept values per stage and row
+constexpr int kEpiWarps = 12;                          // epilogue warps: 3 per TMEM lane quadrant
+constexpr int kEpiGroups = kEpiWarps / 4;              // warp groups taking alternate chunks
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+constexpr int kSmemE = 2048;                           // metadata chunk (128 rows x 128 columns)
+constexpr int kEpiTokens = 16;                         // tokens per epilogue chunk
+constexpr int kTmemCols = 512;
 constexpr uint64_t kDrainBudget = 1ull << 26;
+
+constexpr int kPairRows = 128;                         // compressed-operand rows per CTA
+constexpr int kPairBN = 224;                           // tokens per pair tile
+constexpr int kPairBNh = kPairBN / 2;                  // token rows per CTA
+constexpr int kPairSmemA = kPairRows * kGemmBKc * 2;   // 16 KB
+constexpr int kPairSmemBBox = kPairBNh * 64 * 2;       // 14 KB
+constexpr int kPairSmemB = 2 * kPairSmemBBox;
+constexpr int kPairStageBytes = kPairSmemA + kPairSmemB + kSmemE;   // 46 KB
+constexpr int kPairStages = 4;
+constexpr int kPairChunks = kPairBN / kEpiTokens;      // 14
+constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at columns 0 and 224
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 256 + 1024;
+static_assert(kPairStageBytes % 1024 == 0 && kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
+              "128B-swizzled tiles need 1 KB aligned starts");
+static_assert(kPairMetaCol + 4 * kPairStages <= kTmemCols, "tensor memory budget");
 
 enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
 
-__device__ __forceinline__ float gelu_f(float x) { return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f)); }
+// GELU (exact erf form) and its derivative for the epilogues:
+//   gelu(x) = x Phi(x),  gelu'(x) = Phi(x) + x phi(x),
+//   Phi(x) = 1 - erfc(x/sqrt2)/2 (x >= 0),  erfc(|x|/sqrt2)/2 (x < 0),
+//   phi(x) = exp(-x^2/2) / sqrt(2 pi).
+// erfc(z) = exp(-z^2) R(z) with R(z) = erfc(z) exp(z^2); R is evaluated with a
+// degree-12 polynomial in u = z/2 - 1 from a Chebyshev least-squares fit on
+// z in [0, 4] (csrc/fit_gelu_poly.py derives the coefficients; the fp32 Horner
+// evaluation stays within 9.1e-6 relative of R there).  The tail is thus
+// accurate to ~1e-5 relative on both sides of 0, far inside the fp16/bf16
+// output rounding; beyond z = 4 (|x| > 5.66) z is clamped for R only, where
+// exp(-z^2) < 1.2e-7 makes the tail vanish against 1 or round to 0.  One
+// exponential serves both Phi and phi.
+struct GaussTail {
+  float phi_cdf;  // Phi(x)
+  float e;        // exp(-x^2 / 2)
+};
+
+__device__ __forceinline__ GaussTail gauss_tail(float x) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float u = fminf(z, 4.0f) * 0.5f - 1.0f;
+  float r = 3.716457635e-03f;
+  r = fmaf(r, u, -6.721057463e-03f);
+  r = fmaf(r, u, 1.157346880e-03f);
+  r = fmaf(r, u, -2.581665060e-03f);
+  r = fmaf(r, u, 1.679963246e-02f);
+  r = fmaf(r, u, -2.721724845e-02f);
+  r = fmaf(r, u, 3.703121841e-02f);
+  r = fmaf(r, u, -5.757917091e-02f);
+  r = fmaf(r, u, 8.719655871e-02f);
+  r = fmaf(r, u, -1.238107979e-01f);
+  r = fmaf(r, u, 1.672022939e-01f);
+  r = fmaf(r, u, -2.135886401e-01f);
+  r = fmaf(r, u, 2.553957701e-01f);
+  const float e = __expf(-z * z);
+  const float half_erfc = 0.5f * r * e;
+  GaussTail g;
+  g.phi_cdf = x >= 0.0f ? 1.0f - half_erfc : half_erfc;
+  g.e = e;
+  return g;
+}
+
+__device__ __forceinline__ float gelu_f(float x) { return x * gauss_tail(x).phi_cdf; }
 
 __device__ __forceinline__ float gelu_grad_f(float x) {
-  return 0.5f * (1.0f + erff(x * 0.70710678118654752f)) + x * expf(-0.5f * x * x) * 0.39894228040143268f;
+  const GaussTail g = gauss_tail(x);
+  return fmaf(x * 0.39894228040143268f, g.e, g.phi_cdf);
 }
 
 template <bool BF16>
@@ -64,148 +138,221 @@ __device__ __forceinline__ float bits_to_f32(uint32_t b) {
   return __half2float(__ushort_as_half((unsigned short)b));
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 template <bool BF16, int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    sp24_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_aux,
-                     const uint8_t *__restrict__ meta, const uint16_t *__restrict__ aux_in, int M, int T,
-                     int num_kt, uint64_t wait_budget) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                          const __grid_constant__ CUtensorMap tm_meta, uint16_t *__restrict__ out,
+                          uint16_t *__restrict__ aux, int M, int T, int num_kt, uint64_t wait_budget) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_base = smem;
-  uint16_t *s_out = reinterpret_cast<uint16_t *>(smem + kGemmStages * kStageBytes);
-  uint16_t *s_aux = s_out + kSmemOut / 2;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kGemmStages * kStageBytes + 2 * kSmemOut);
-  uint64_t *full = bars;                       // [kGemmStages]
-  uint64_t *empty = bars + kGemmStages;        // [kGemmStages]
-  uint64_t *acc_full = bars + 2 * kGemmStages;
-  uint64_t *drain = acc_full + 1;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kPairStages * kPairStageBytes);
+  uint64_t *full = bars;                          // [stages] leader: TMA (both CTAs) -> MMA
+  uint64_t *empty = bars + kPairStages;           // [stages] MMA -> this CTA's TMA
+  uint64_t *acc_full = bars + 2 * kPairStages;    // [2] MMA -> this CTA's epilogue
+  uint64_t *acc_empty = acc_full + 2;             // [2] leader: both epilogues -> MMA
+  uint64_t *drain = acc_empty + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mt = blockIdx.x;
-  const int m0 = mt * kGemmBM;
-  const int n0 = blockIdx.y * kGemmBN;
+  const uint32_t rank = cluster_ctarank();
+  const bool is_leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_mt = (M + 2 * kPairRows - 1) / (2 * kPairRows);
+  const int num_row_tiles = (M + kPairRows - 1) / kPairRows;
+  const int num_tiles = num_mt * ((T + kPairBN - 1) / kPairBN);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGemmStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
+    }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbarrier_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
-    prefetch_tensormap(&tm_out);
+    prefetch_tensormap(&tm_meta);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(s_tmem, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or byte count
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- producer
-    int issued = 0;
-    for (int kt = 0; kt < num_kt; ++kt) {
-      const int s = kt % kGemmStages;
-      const uint32_t it = (uint32_t)(kt / kGemmStages);
-      if (!mbar_wait_bounded(&empty[s], (it & 1u) ^ 1u, wait_budget, s_abort)) break;
-      uint8_t *st = stage_base + s * kStageBytes;
-      mbar_arrive_expect_tx(&full[s], kStageBytes);
-      tma_load_2d(st, &tm_a, &full[s], kt * kGemmBKc, m0);
-      tma_load_2d(st + kSmemA, &tm_b, &full[s], kt * kGemmBK, n0);
-      tma_load_2d(st + kSmemA + kSmemBBox, &tm_b, &full[s], kt * kGemmBK + 64, n0);
-      bulk_load(st + kSmemA + kSmemB, meta + ((size_t)mt * num_kt + kt) * kSmemE, kSmemE, &full[s]);
-      ++issued;
-    }
-    // Let every copy this thread started land before the CTA can exit.
-    for (int kt = issued > kGemmStages ? issued - kGemmStages : 0; kt < issued; ++kt) {
-      volatile int no_abort = 0;
-      mbar_wait_bounded(&full[kt % kGemmStages], (uint32_t)(kt / kGemmStages) & 1u, kDrainBudget, &no_abort);
-    }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = make_idesc_sparse(BF16, kGemmBM, kGemmBN);
+    // ------------------------------------------------------ producer (both CTAs)
+    uint32_t g = 0;
     bool ok = true;
-    for (int kt = 0; kt < num_kt && ok; ++kt) {
-      const int s = kt % kGemmStages;
-      const uint32_t it = (uint32_t)(kt / kGemmStages);
-      ok = mbar_wait_bounded(&full[s], it & 1u, wait_budget, s_abort);
-      if (!ok) break;
-      tc_fence_after();
-      const uint8_t *st = stage_base + s * kStageBytes;
-      const uint32_t a_addr = smem_u32(st);
-      const uint32_t b_addr = smem_u32(st + kSmemA);
-      const uint32_t e_addr = smem_u32(st + kSmemA + kSmemB);
-      const uint32_t t_meta = tmem_base + kTmemMetaCol + 4 * s;
-      tc_cp_128x128b(t_meta, smem_desc(e_addr, 128, 128, kSwizzleNone));
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t adesc = smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B);
-        const uint64_t bdesc = smem_desc(b_addr + (kk >> 1) * kSmemBBox + (kk & 1) * 64, 16, 1024, kSwizzle128B);
-        tc_mma_sp_f16(tmem_base, adesc, bdesc, t_meta + kk, idesc, (kt | kk) != 0 ? 1u : 0u);
+    for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+      const int mt = tile % num_mt;
+      const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
+      const int b_row = (tile / num_mt) * kPairBN + (int)rank * kPairBNh;
+      // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
+      // it the last real metadata chunk so every code the MMA sees is valid.
+      const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
+      for (int kt = 0; kt < num_kt; ++kt, ++g) {
+        const int s = (int)(g % kPairStages);
+        if (!mbar_wait_cluster_bounded(&empty[s], ((g / kPairStages) & 1u) ^ 1u, wait_budget, s_abort)) {
+          ok = false;
+          break;
+        }
+        uint8_t *st = stage_base + s * kPairStageBytes;
+        if (is_leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
+        tma_load_2d_pair(st, &tm_a, &full[s], kt * kGemmBKc, a_row);
+        tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * kGemmBK, b_row);
+        tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * kGemmBK + 64, b_row);
+        tma_load_2d_pair(st + kPairSmemA + kPairSmemB, &tm_meta, &full[s], 0, chunk_row + kt);
       }
-      tc_commit(&empty[s]);
     }
-    if (ok) {
-      tc_commit(acc_full);
-    } else {
-      tc_commit(drain);
+    // The leader's `full` barriers count both CTAs' bytes: let every copy land.
+    if (is_leader) {
+      for (uint32_t i = g > kPairStages ? g - kPairStages : 0; i < g; ++i) {
+        volatile int no_abort = 0;
+        mbar_wait_cluster_bounded(&full[i % kPairStages], (i / kPairStages) & 1u, kDrainBudget, &no_abort);
+      }
+    }
+  } else if (warp == 1 && lane == 0 && is_leader) {
+    // ----------------------------------------------------- MMA issuer (leader)
+    constexpr uint32_t idesc = make_idesc_sparse(BF16, 2 * kPairRows, kPairBN);
+    uint32_t g = 0;
+    bool ok = true;
+    int j = 0;
+    for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++j) {
+      const int b = j & 1;
+      const uint32_t use = (uint32_t)(j >> 1);
+      if (!(ok = mbar_wait_cluster_bounded(&acc_empty[b], (use & 1u) ^ 1u, wait_budget, s_abort))) break;
+      tc_fence_after();
+      const uint32_t acc = tmem_base + (uint32_t)(b * kPairBN);
+      for (int kt = 0; kt < num_kt; ++kt, ++g) {
+        const int s = (int)(g % kPairStages);
+        if (!(ok = mbar_wait_cluster_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
+        tc_fence_after();
+        const uint8_t *st = stage_base + s * kPairStageBytes;
+        const uint32_t a_addr = smem_u32(st);
+        const uint32_t b_addr = smem_u32(st + kPairSmemA);
+        const uint32_t e_addr = smem_u32(st + kPairSmemA + kPairSmemB);
+        const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
+        tc_cp_128x128b_pair(t_meta, smem_desc(e_addr, 128, 128, kSwizzleNone));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adesc = smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B);
+          const uint64_t bdesc = smem_desc(b_addr + (kk >> 1) * kPairSmemBBox + (kk & 1) * 64, 16, 1024, kSwizzle128B);
+          // The metadata operand address must be 2-column aligned; the low column
+          // bit travels in the descriptor's sparsity-selector field instead.
+          tc_mma_sp_f16_pair(acc, adesc, bdesc, t_meta + (kk & 2), idesc | (uint32_t)(kk & 1), (kt | kk) != 0 ? 1u : 0u);
+        }
+        tc_commit_pair(&empty[s], 0x3);
+      }
+      if (ok) tc_commit_pair(&acc_full[b], 0x3);
+    }
+    if (!ok) {
+      tc_commit_pair(drain, 0x1);
       volatile int no_abort = 0;
-      mbar_wait_bounded(drain, 0, kDrainBudget, &no_abort);
+      mbar_wait_cluster_bounded(drain, 0, kDrainBudget, &no_abort);
     }
   } else if (warp >= 2) {
-    // --------------------------------------------------------------- epilogue
-    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    // ---------------------------------------------------- epilogue (both CTAs)
+    // Warp w reads lane quadrant w%4 and takes chunks grp, grp + kEpiGroups, ...
+    // (grp = (w-2)/4) of every tile.  Decisions after a bounded wait are made
+    // per warp (__all_sync), so the .sync.aligned TMEM loads stay convergent.
+    // A warp releases the accumulator with one arrive (lane 0) after its lanes'
+    // TMEM reads have completed.
+    const int grp = (warp - 2) >> 2;
+    const int q = warp & 3;
     const int m_local = 32 * q + lane;
-    const int m = m0 + m_local;
-    const bool leader = threadIdx.x == 64;
-    if (mbar_wait_bounded(acc_full, 0, wait_budget, s_abort)) {
-      tc_fence_after();
-      for (int c = 0; c < kGemmBN / kEpiTokens; ++c) {
-        const int t0 = n0 + c * kEpiTokens;
-        if (t0 >= T) break;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(c * kEpiTokens), r);
-        tmem_wait_ld();
-        if (leader) bulk_wait_group_read<0>();
-        named_barrier_sync(1, 128);
+    constexpr int kMaxChunksPerWarp = (kPairChunks + kEpiGroups - 1) / kEpiGroups;
+    auto release = [&](int buf) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_leader(&acc_empty[buf]);
+    };
+    int j = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
+      const int b = j & 1;
+      const int m = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + m_local;
+      const int n0 = (tile / num_mt) * kPairBN;
+      const int nchunks = min(kPairChunks, (T - n0 + kEpiTokens - 1) / kEpiTokens);
+      const bool m_ok = m < M;
+      // dGELU: pre-activations, two tokens per register, fetched two chunks
+      // ahead of use; the first two before the accumulator is ready, so the
+      // main loop hides their latency.
+      uint32_t pk[2][kEpiTokens / 2];
+      auto fetch = [&](int k, uint32_t (&dstv)[kEpiTokens / 2]) {
+        const int t0 = n0 + (grp + k * kEpiGroups) * kEpiTokens;
+        const uint16_t *src = aux + (size_t)t0 * M + m;
 #pragma unroll
-        for (int j = 0; j < kEpiTokens; ++j) {
-          const float acc = __uint_as_float(r[j]);
-          float out = acc;
-          if (EPI == kEpiGelu) {
-            s_aux[j * kGemmBM + m_local] = (uint16_t)f32_to_bits<BF16>(acc);
-            out = gelu_f(acc);
-          } else if (EPI == kEpiDgelu) {
-            const int t = t0 + j;
-            const float pre = (t < T && m < M) ? bits_to_f32<BF16>(aux_in[(size_t)t * M + m]) : 0.0f;
-            out = acc * gelu_grad_f(pre);
-          }
-          s_out[j * kGemmBM + m_local] = (uint16_t)f32_to_bits<BF16>(out);
+        for (int jj = 0; jj < kEpiTokens / 2; ++jj) {
+          const int t = t0 + 2 * jj;
+          const uint32_t lo = (m_ok && t < T) ? src[(size_t)(2 * jj) * M] : 0u;
+          const uint32_t hi = (m_ok && t + 1 < T) ? src[(size_t)(2 * jj + 1) * M] : 0u;
+          dstv[jj] = lo | (hi << 16);
         }
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (leader) {
-          tma_store_2d(&tm_out, s_out, m0, t0);
-          if (EPI == kEpiGelu) tma_store_2d(&tm_aux, s_aux, m0, t0);
-          bulk_commit_group();
-        }
+      };
+      if (EPI == kEpiDgelu) {
+        fetch(0, pk[0]);
+        fetch(1, pk[1]);
       }
-      if (leader) bulk_wait_group<0>();
+      const bool got = mbar_wait_cluster_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
+      tc_fence_after();
+      if (grp >= nchunks) release(b);  // nothing to read in this (ragged) tile
+      const int my_last = grp + ((nchunks - 1 - grp) / kEpiGroups) * kEpiGroups;
+#pragma unroll
+      for (int k = 0; k < kMaxChunksPerWarp; ++k) {
+        const int c = grp + k * kEpiGroups;
+        if (c >= nchunks) break;
+        const int t0 = n0 + c * kEpiTokens;
+        const int tn = min(kEpiTokens, T - t0);     // tokens of this chunk inside T
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN + c * kEpiTokens), r);
+        tmem_wait_ld();
+        if (c == my_last) release(b);
+        uint16_t *dst = out + (size_t)t0 * M + m;
+        uint16_t *dst_aux = aux + (size_t)t0 * M + m;
+        const bool full_chunk = tn == kEpiTokens;
+#pragma unroll
+        for (int jj = 0; jj < kEpiTokens; ++jj) {
+          const float acc = __uint_as_float(r[jj]);
+          float y = acc;
+          if (EPI == kEpiGelu) y = gelu_f(acc);
+          else if (EPI == kEpiDgelu)
+            y = acc * gelu_grad_f(bits_to_f32<BF16>((pk[k & 1][jj >> 1] >> ((jj & 1) * 16)) & 0xFFFFu));
+          if (m_ok && (full_chunk || jj < tn)) {
+            if (EPI == kEpiGelu) dst_aux[(size_t)jj * M] = (uint16_t)f32_to_bits<BF16>(acc);
+            dst[(size_t)jj * M] = (uint16_t)f32_to_bits<BF16>(y);
+          }
+        }
+        if (EPI == kEpiDgelu && k + 2 < kMaxChunksPerWarp) fetch(k + 2, pk[k & 1]);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // the peer's MMAs, copies and arrivals into this CTA are over
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 

@@ -8,7 +8,9 @@
 //     search, pruning and masked decay kernels);
 //   - abstract (flip rate; masked decay term on gradients).
 //
-// Mask search is exact.  Each |w| becomes an integer multiple of its dtype's
+// Mask search is exact.  The fast path sums magnitudes in fp32 where the
+// block's magnitude range proves those sums exact (search_block_fast); the
+// remaining blocks take an integer search.  There each |w| becomes an integer multiple of its dtype's
 // smallest subnormal (fp16: always; bf16: relative to the block's largest
 // exponent, 32 binades deep), pre-shifted left by 12 bits.  The 12 low bits of
 // a pattern's key hold (35 - top rank) << 6 | (35 - bottom rank), so one
@@ -141,6 +143,64 @@ __device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], cons
   return s_index[(35 - (r >> 6)) * 36 + (35 - (r & 63))];
 }
 
+constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
+
+// Fast path of the search on fp32 arithmetic.  Every |w| converts to fp32
+// exactly.  A sum of eight of them is exact in fp32 when the block's smallest
+// nonzero magnitude is at least its largest times 2^-10 (fp16: 11-bit
+// significands, 3 carry bits, 24-bit fp32 significand) or 2^-13 (bf16); then
+// every partial sum below is exact, comparisons are exact, and the result
+// equals the exact search.  Blocks that fail the test return kNeedsExact.
+// Ranks: within a column-count state the first combo (lowest rank) reaching
+// the state's maximum wins (strict >); across states the smallest
+// (top rank, bottom rank) among the states reaching the global maximum wins.
+template <bool BF16>
+__device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2], const uint8_t *s_index) {
+  constexpr PatternTables T = make_pattern_tables();
+  float v[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t h = (w[c >> 2][(c >> 1) & 1] >> ((c & 1) << 4)) & 0x7FFFu;
+    v[c] = BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
+  }
+  float vmax = v[0], vmin = v[0] > 0.0f ? v[0] : __int_as_float(0x7F800000);
+#pragma unroll
+  for (int c = 1; c < 16; ++c) {
+    vmax = fmaxf(vmax, v[c]);
+    vmin = fminf(vmin, v[c] > 0.0f ? v[c] : __int_as_float(0x7F800000));
+  }
+  if (!(vmin >= vmax * (BF16 ? 0x1p-13f : 0x1p-10f))) return kNeedsExact;
+
+  float P[4][6];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < 6; ++q) P[i][q] = v[4 * i + pair_lo(q)] + v[4 * i + pair_hi(q)];
+  float top[kNumStates], bot[kNumStates];
+  uint32_t tr[kNumStates], br[kNumStates];
+  bool seen_t[kNumStates] = {}, seen_b[kNumStates] = {};
+#pragma unroll
+  for (int c = 0; c < 36; ++c) {
+    const int st = T.top_state[c];
+    const float kt = P[0][c / 6] + P[1][c % 6];
+    if (!seen_t[st]) { top[st] = kt; tr[st] = (uint32_t)c; seen_t[st] = true; }
+    else { const bool gt = kt > top[st]; top[st] = gt ? kt : top[st]; tr[st] = gt ? (uint32_t)c : tr[st]; }
+    const int sb = T.bot_state[c];
+    const float kb = P[2][c / 6] + P[3][c % 6];
+    if (!seen_b[sb]) { bot[sb] = kb; br[sb] = (uint32_t)c; seen_b[sb] = true; }
+    else { const bool gt = kb > bot[sb]; bot[sb] = gt ? kb : bot[sb]; br[sb] = gt ? (uint32_t)c : br[sb]; }
+  }
+  float tot[kNumStates];
+  float best = 0.0f;
+#pragma unroll
+  for (int st = 0; st < kNumStates; ++st) { tot[st] = top[st] + bot[st]; best = fmaxf(best, tot[st]); }
+  uint32_t key = 0xFFFFu;
+#pragma unroll
+  for (int st = 0; st < kNumStates; ++st)
+    if (tot[st] == best) key = min(key, (tr[st] << 6) | br[st]);
+  return s_index[(key >> 6) * 36 + (key & 63)];
+}
+
 __device__ __forceinline__ uint32_t half_of(const uint32_t (&row)[4], int blk, uint32_t k) {
   const uint32_t wd = (k & 2) ? row[2 * blk + 1] : row[2 * blk];
   return (wd >> ((k & 1) << 4)) & 0xFFFFu;
@@ -160,6 +220,30 @@ __device__ __forceinline__ int vcol_word(int c_local, int br_local) {
          ((br_local & 3) ^ (((c_local >> 6) & 1) << 1));
 }
 
+// Loads one unit (4 rows x 8 columns = two blocks) of W; columns past C read as 0.
+__device__ __forceinline__ void load_unit(const uint16_t *__restrict__ W, int64_t ldw, int64_t r0, int64_t c0,
+                                          int64_t R, int64_t C, bool vec16, uint32_t (&w)[4][4]) {
+  const bool row_ok = r0 < R;
+  const bool ok0 = row_ok && c0 + 4 <= C;
+  const bool ok1 = row_ok && c0 + 8 <= C;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[i][0] = w[i][1] = w[i][2] = w[i][3] = 0;
+    const uint16_t *src = W + (r0 + i) * ldw + c0;
+    if (ok1 && vec16) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src));
+      w[i][0] = q.x; w[i][1] = q.y; w[i][2] = q.z; w[i][3] = q.w;
+    } else if (ok1) {
+      const uint2 q0 = __ldg(reinterpret_cast<const uint2 *>(src));
+      const uint2 q1 = __ldg(reinterpret_cast<const uint2 *>(src + 4));
+      w[i][0] = q0.x; w[i][1] = q0.y; w[i][2] = q1.x; w[i][3] = q1.y;
+    } else if (ok0) {
+      const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src));
+      w[i][0] = q.x; w[i][1] = q.y;
+    }
+  }
+}
+
 constexpr int kTile = 128;       // W tile: 128 rows x 128 columns per CTA
 constexpr int kMaskThreads = 256;
 
@@ -170,7 +254,7 @@ constexpr int kMaskThreads = 256;
 //             (values + tensor-core metadata)
 //   FLIP:     add the number of mask bits that differ from idx_prev to *flip_count
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads) mask_tile_kernel(
+__global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
     const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
@@ -181,6 +265,8 @@ __global__ void __launch_bounds__(kMaskThreads) mask_tile_kernel(
   __shared__ uint8_t s_index[36 * 36];
   __shared__ uint8_t s_idx[32][36];
   __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kTile * 32 : 4];
+  __shared__ uint16_t s_queue[SEARCH ? 1024 : 2];
+  __shared__ int s_qn;
   __shared__ unsigned long long s_flip;
 
   const int tid = threadIdx.x;
@@ -190,72 +276,103 @@ __global__ void __launch_bounds__(kMaskThreads) mask_tile_kernel(
     s_colcode[i] = c_tables.colcode[i];
   }
   for (int i = tid; i < 36 * 36; i += kMaskThreads) s_index[i] = c_tables.index[i];
-  if (tid == 0) s_flip = 0;
+  if (tid == 0) { s_flip = 0; s_qn = 0; }
   __syncthreads();
 
   const int64_t tile_r = (int64_t)blockIdx.y * kTile;
   const int64_t tile_c = (int64_t)blockIdx.x * kTile;
   const int64_t bcols = C >> 2;
   const int uc = tid & 15;
-  unsigned long long flips = 0;
+  const bool vec16 = (ldw & 7) == 0;  // rows 16-byte aligned: one 128-bit load per row of a unit
 
-#pragma unroll 1
+  // Phase 1: load both units, search the blocks the fast path can certify,
+  // queue the others (SEARCH) or read the given mask (!SEARCH).
+  uint32_t w[2][4][4];
+#pragma unroll
+  for (int half = 0; half < 2; ++half)
+    load_unit(W, ldw, tile_r + 4 * ((tid >> 4) + 16 * half), tile_c + 8 * uc, R, C, vec16, w[half]);
+#pragma unroll
   for (int half = 0; half < 2; ++half) {
-    const int br = (tid >> 4) + 16 * half;  // block row within the tile
+    const int br = (tid >> 4) + 16 * half;
+    const int64_t r0 = tile_r + 4 * br;
+    const int64_t c0 = tile_c + 8 * uc;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const bool ok = r0 < R && c0 + 4 * (b + 1) <= C;
+      uint32_t p = kPadIndex;
+      if (ok) {
+        if (SEARCH) {
+          uint32_t blk[4][2];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { blk[i][0] = w[half][i][2 * b]; blk[i][1] = w[half][i][2 * b + 1]; }
+          p = search_block_fast<BF16>(blk, s_index);
+          if (p == kNeedsExact) {
+            const int slot = atomicAdd(&s_qn, 1);
+            s_queue[slot] = (uint16_t)(br * 32 + 2 * uc + b);
+          }
+        } else {
+          p = idx[(r0 >> 2) * bcols + (c0 >> 2) + b];
+        }
+      }
+      s_idx[br][2 * uc + b] = (uint8_t)p;
+    }
+  }
+
+  // Phase 1b: blocks the fast path could not certify take the exact integer search.
+  if (SEARCH) {
+    __syncthreads();
+    const int qn = s_qn;
+    for (int k = tid; k < qn; k += kMaskThreads) {
+      const int id = s_queue[k];
+      const int br = id >> 5, bc = id & 31;
+      const uint16_t *src = W + (tile_r + 4 * br) * ldw + tile_c + 4 * bc;
+      uint32_t blk[4][2];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src + i * ldw));
+        blk[i][0] = q.x; blk[i][1] = q.y;
+      }
+      s_idx[br][bc] = (uint8_t)search_block<BF16>(blk, s_index, s_bits);
+    }
+  }
+  if (SEARCH || COMPRESS || FLIP) __syncthreads();
+
+  // Phase 2: per-thread outputs of its own blocks.
+  unsigned long long flips = 0;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int br = (tid >> 4) + 16 * half;
     const int64_t r0 = tile_r + 4 * br;
     const int64_t c0 = tile_c + 8 * uc;
     const bool row_ok = r0 < R;
     const bool ok0 = row_ok && c0 + 4 <= C;
     const bool ok1 = row_ok && c0 + 8 <= C;
-    uint32_t w[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      w[i][0] = w[i][1] = w[i][2] = w[i][3] = 0;
-      const uint16_t *src = W + (r0 + i) * ldw + c0;
-      if (ok1) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src));
-        w[i][0] = q.x; w[i][1] = q.y; w[i][2] = q.z; w[i][3] = q.w;
-      } else if (ok0) {
-        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src));
-        w[i][0] = q.x; w[i][1] = q.y;
-      }
-    }
-    uint32_t p[2] = {kPadIndex, kPadIndex};
+    uint32_t p[2];
+    uint32_t x[4][4];  // the unit again (an L1 hit): keeps registers free during the search
+    if (COMPRESS) load_unit(W, ldw, r0, c0, R, C, vec16, x);
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
+      p[b] = s_idx[br][2 * uc + b];
       const bool ok = b ? ok1 : ok0;
       const int64_t bidx = (r0 >> 2) * bcols + (c0 >> 2) + b;
-      if (SEARCH) {
-        uint32_t blk[4][2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
-        if (ok) {
-          p[b] = search_block<BF16>(blk, s_index, s_bits);
-          idx[bidx] = (uint8_t)p[b];
-        }
-      } else if (ok) {
-        p[b] = idx[bidx];
-      }
-      if (FLIP && ok) {
-        const uint32_t prev = idx_prev[bidx];
-        flips += __popc((uint32_t)(s_bits[prev] ^ s_bits[p[b]]));
-      }
-      s_idx[br][2 * uc + b] = (uint8_t)p[b];
+      if (SEARCH && ok) idx[bidx] = (uint8_t)p[b];
+      if (FLIP && ok) flips += __popc((uint32_t)(s_bits[idx_prev[bidx]] ^ s_bits[p[b]]));
     }
-    if (COMPRESS && row_ok && ok0) {
+    if (COMPRESS && ok0) {
       // Forward operand: kept values of each row, in column order.
+      if (vals_row) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t packed[2];
+        for (int i = 0; i < 4; ++i) {
+          uint32_t packed[2];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const uint32_t nib = (s_rowcode[p[b]] >> (4 * i)) & 0xFu;
-          packed[b] = half_of(w[i], b, nib & 3u) | (half_of(w[i], b, nib >> 2) << 16);
+          for (int b = 0; b < 2; ++b) {
+            const uint32_t nib = (s_rowcode[p[b]] >> (4 * i)) & 0xFu;
+            packed[b] = half_of(x[i], b, nib & 3u) | (half_of(x[i], b, nib >> 2) << 16);
+          }
+          uint16_t *dst = vals_row + (r0 + i) * (C >> 1) + (c0 >> 1);
+          if (ok1) *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+          else *reinterpret_cast<uint32_t *>(dst) = packed[0];
         }
-        uint16_t *dst = vals_row + (r0 + i) * (C >> 1) + (c0 >> 1);
-        if (!vals_row) break;
-        if (ok1) *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
-        else *reinterpret_cast<uint32_t *>(dst) = packed[0];
       }
       // Input-gradient operand: kept values of each column, staged transposed.
 #pragma unroll
@@ -264,8 +381,8 @@ __global__ void __launch_bounds__(kMaskThreads) mask_tile_kernel(
         for (int j = 0; j < 4; ++j) {
           const uint32_t nib = (s_colcode[p[b]] >> (4 * j)) & 0xFu;
           const int word = 2 * b + (j >> 1);
-          const uint32_t lo = (pick_row(w, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
-          const uint32_t hi = (pick_row(w, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
+          const uint32_t lo = (pick_row(x, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
+          const uint32_t hi = (pick_row(x, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
           s_vcol[vcol_word(8 * uc + 4 * b + j, br)] = lo | (hi << 16);
         }
       }

@@ -70,16 +70,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map over a row-major [outer x inner] array of 16-bit elements.
+// 2-D map over a row-major [outer x inner] array of 16-bit (or `type`) elements.
 bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer, uint64_t pitch_bytes,
-                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle,
+                 CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_UINT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+  CUresult r = fn(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -87,33 +88,47 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 
 // ---------------------------------------------------------------- GEMM launch
 
+// CTA-pair kernel: clusters of two CTAs, 256 x 224 tiles (see gemm_sp.cuh).
 template <bool BF16, int EPI>
-sp24_status launch_gemm_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
-                          void *out, void *aux, cudaStream_t stream) {
-  CUtensorMap ta, tb, tout, taux;
-  if (!make_map_2d(&ta, vals, (uint64_t)(Kd / 2), (uint64_t)M, (uint64_t)Kd, kGemmBKc, kGemmBM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tout, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, kGemmBM, kEpiTokens,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
-    return SP24_ERR_CUDA;
-  taux = tout;
-  if (EPI == kEpiGelu &&
-      !make_map_2d(&taux, aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, kGemmBM, kEpiTokens,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
-    return SP24_ERR_CUDA;
-  auto kernel = sp24_gemm_kernel<BF16, EPI>;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
-      return SP24_ERR_CUDA;
-    configured = true;
-  }
+sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                               void *out, void *aux, cudaStream_t stream) {
   const int num_kt = (int)((Kd + kGemmBK - 1) / kGemmBK);
-  dim3 grid((unsigned)((M + kGemmBM - 1) / kGemmBM), (unsigned)((T + kGemmBN - 1) / kGemmBN));
-  kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(ta, tb, tout, taux, static_cast<const uint8_t *>(meta),
-                                                         static_cast<const uint16_t *>(aux), (int)M, (int)T,
-                                                         num_kt, g_wait_budget.load());
+  const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
+  CUtensorMap ta, tb, tm;
+  if (!make_map_2d(&ta, vals, (uint64_t)(Kd / 2), (uint64_t)M, (uint64_t)Kd, kGemmBKc, kPairRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT64))
+    return SP24_ERR_CUDA;
+  auto kernel = sp24_gemm_pair_kernel<BF16, EPI>;
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) != cudaSuccess)
+      return SP24_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    max_pairs = n;
+  }
+  const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + kPairBN - 1) / kPairBN);
+  const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  kernel<<<2 * pairs, kGemmThreads, kPairSmemBytes, stream>>>(ta, tb, tm, static_cast<uint16_t *>(out),
+                                                              static_cast<uint16_t *>(aux), (int)M, (int)T, num_kt,
+                                                              g_wait_budget.load());
   return launch_status();
 }
 
@@ -121,12 +136,12 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
                         sp24_dtype dt, void *out, int epi, void *aux, cudaStream_t s) {
   const bool bf = dt == SP24_BF16;
   switch (epi) {
-    case kEpiNone: return bf ? launch_gemm_t<true, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_t<false, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s);
-    case kEpiGelu: return bf ? launch_gemm_t<true, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_t<false, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s);
-    default: return bf ? launch_gemm_t<true, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s)
-                       : launch_gemm_t<false, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiNone: return bf ? launch_gemm_pair_t<true, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_pair_t<false, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_pair_t<false, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s);
+    default: return bf ? launch_gemm_pair_t<true, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s)
+                       : launch_gemm_pair_t<false, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s);
   }
 }
 
@@ -172,7 +187,7 @@ sp24_status validate_w(const void *W, sp24_dtype dt, int64_t rows, int64_t cols,
   if (rows % 4 || cols % 4) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (rows > 0 && cols > 0) {
     if (!W) return SP24_ERR_INVALID_ARG;
-    if (!aligned16(W) || ldw % 8) return SP24_ERR_MISALIGNED;
+    if (!aligned16(W) || ldw % 4) return SP24_ERR_MISALIGNED;
   }
   return SP24_OK;
 }

@@ -62,7 +62,7 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert _raw("sp24_mask_search", fake, 0, 6, 8, 8, fake, None) == E["SP24_ERR_UNSUPPORTED_SHAPE"]
     assert _raw("sp24_mask_search", fake, 7, 8, 8, 8, fake, None) == E["SP24_ERR_UNSUPPORTED_DTYPE"]
     assert _raw("sp24_mask_search", odd, 0, 8, 8, 8, fake, None) == E["SP24_ERR_MISALIGNED"]
-    assert _raw("sp24_mask_search", fake, 0, 8, 8, 12, fake, None) == E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_mask_search", fake, 0, 8, 8, 10, fake, None) == E["SP24_ERR_MISALIGNED"]
     assert _raw("sp24_mask_search", fake, 0, 8, 8, 4, fake, None) == E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_mask_search", None, 0, 8, 8, 8, fake, None) == E["SP24_ERR_INVALID_ARG"]
     # compression needs multiples of 16
