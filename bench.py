@@ -64,6 +64,30 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def kernel_source_hash(*names: str) -> str:
+    """Short hash of the CUDA sources a profile was taken from (stale profiles report null)."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "structured_sparse_transformer_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch measured by ncu for `kernel` on `workload`
+    (profiles/traffic.json), or None if absent or taken from other sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    entry = json.load(open(p)).get(kernel, {}).get(workload)
+    if not entry:
+        return None
+    if entry.get("source_hash") != kernel_source_hash(*entry.get("sources", [])):
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -75,53 +99,57 @@ def load_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
+    """Samples SM clock, power and throttle reasons of one GPU with nvidia-smi
+    every ~200 ms from a background thread (one query per sample, so nothing
+    is lost to output buffering when sampling stops)."""
+
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = f"/tmp/sp24_clocks_{os.getpid()}.csv"
+    def __init__(self, gpu_index: int, period_s: float = 0.2):
+        import threading
+        self.gpu, self.period = gpu_index, period_s
+        self.samples = []
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _query(self):
+        r = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                            "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
+        if r.returncode != 0:
+            raise RuntimeError(r.stderr.strip() or f"nvidia-smi exit {r.returncode}")
+        f = [x.strip() for x in r.stdout.strip().splitlines()[0].split(",")]
+        reasons = {n for n, v in zip(self.NAMES, f[5:9]) if v.lower().startswith("active")}
+        return float(f[1]), float(f[2]), reasons
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._query())
+            except Exception as e:  # nvidia-smi missing or a field unsupported
+                self.error = str(e)[:200]
+                return
+            self._stop.wait(self.period)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        self._thread.join(timeout=15)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted(set().union(*[x[2] for x in self.samples]))
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "samples": len(sm), "reasons": reasons,
+                "window": "warm-up through the end-to-end loop, one query per ~200 ms"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -219,24 +247,25 @@ def run_ours(args, wl, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
+    clk = ClockSampler(torch.cuda.current_device()).__enter__()
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
     st = sp.sp24_device_status()
     if st != 0:
+        clk.__exit__()
         raise RuntimeError(f"device status after warm-up: {sp.sp24_status_string(st)}")
 
     events, step_ev = {}, []
     barrier()
-    with ClockSampler(local_rank) as clk:
-        for _ in range(args.steps):
-            flush.fill_(1.0)
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
-            step.run(events)
-            e.record()
-            step_ev.append((s, e))
-        barrier()
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step.run(events)
+        e.record()
+        step_ev.append((s, e))
+    barrier()
     st = sp.sp24_device_status()
     if st != 0:
         raise RuntimeError(f"device status after timing: {sp.sp24_status_string(st)}")
@@ -264,13 +293,15 @@ def run_ours(args, wl, rank, world, local_rank):
     g_avg = g_time / g_launches * 1e-6
     g_ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
     roofline = {"bound": "tensor", "achieved": round(g_ach, 1), "peak": sparse_peak, "unit": "TFLOP/s",
-                "frac": round(g_ach / sparse_peak, 4), "traffic": args.gemm_traffic,
-                "kernel": "sp24_gemm_kernel (fwd + dgrad launches)",
+                "frac": round(g_ach / sparse_peak, 4),
+                "traffic": args.gemm_traffic or load_traffic("gemm", wl.name),
+                "kernel": "sp24_gemm_pair_kernel (fwd + dgrad launches)",
                 "peak_source": f"2 x {peak_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s), "
                                "the nominal 2:4 sparse ratio"}
     mask = kernels["mask_step"]
 
     e2e = run_e2e(args, step, wl, world, dev, barrier)
+    clk.__exit__()
     clocks = clk.summary()
     flips = [int(x) for x in step.flips.cpu().tolist()]
     line = {
@@ -282,7 +313,8 @@ def run_ours(args, wl, rank, world, local_rank):
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)"},
         "roofline": roofline,
         "mask_search_roofline": {"bound": "hbm", "achieved": mask["achieved"], "peak": peaks["hbm_gbs"],
-                                 "unit": "GB/s", "frac": mask["frac"], "traffic": args.mask_traffic,
+                                 "unit": "GB/s", "frac": mask["frac"],
+                                 "traffic": args.mask_traffic or load_traffic("mask_step", wl.name),
                                  "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
         "kernels": kernels,
         "e2e": e2e,

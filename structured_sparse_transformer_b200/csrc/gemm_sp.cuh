@@ -89,41 +89,53 @@ enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
 // accurate to ~1e-5 relative on both sides of 0, far inside the fp16/bf16
 // output rounding; beyond z = 4 (|x| > 5.66) z is clamped for R only, where
 // exp(-z^2) < 1.2e-7 makes the tail vanish against 1 or round to 0.  One
-// exponential serves both Phi and phi.
+// exponential serves both Phi and phi; the sign cases fold into a max and a
+// fused multiply-add, so the epilogue spends ~20 instructions per element.
+// 2^y with the hardware's approximate base-2 exponential (relative error ~2^-22).
+__device__ __forceinline__ float ex2_approx(float y) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+  return r;
+}
+
+// t = erfc(|x| / sqrt 2) / 2 (the normal tail beyond |x|) and e = exp(-x^2 / 2).
+// R's coefficients are the fitted ones scaled by 1/2 (exact), so r = R/2.
 struct GaussTail {
-  float phi_cdf;  // Phi(x)
-  float e;        // exp(-x^2 / 2)
+  float t;
+  float e;
 };
 
 __device__ __forceinline__ GaussTail gauss_tail(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float u = fminf(z, 4.0f) * 0.5f - 1.0f;
-  float r = 3.716457635e-03f;
-  r = fmaf(r, u, -6.721057463e-03f);
-  r = fmaf(r, u, 1.157346880e-03f);
-  r = fmaf(r, u, -2.581665060e-03f);
-  r = fmaf(r, u, 1.679963246e-02f);
-  r = fmaf(r, u, -2.721724845e-02f);
-  r = fmaf(r, u, 3.703121841e-02f);
-  r = fmaf(r, u, -5.757917091e-02f);
-  r = fmaf(r, u, 8.719655871e-02f);
-  r = fmaf(r, u, -1.238107979e-01f);
-  r = fmaf(r, u, 1.672022939e-01f);
-  r = fmaf(r, u, -2.135886401e-01f);
-  r = fmaf(r, u, 2.553957701e-01f);
-  const float e = __expf(-z * z);
-  const float half_erfc = 0.5f * r * e;
+  // u = z/2 - 1 with z = min(|x|, 4 sqrt 2) / sqrt 2
+  const float u = fmaf(fminf(fabsf(x), 5.65685424949238f), 0.353553390593274f, -1.0f);
+  float r = 1.858228817e-03f;
+  r = fmaf(r, u, -3.360528732e-03f);
+  r = fmaf(r, u, 5.786734400e-04f);
+  r = fmaf(r, u, -1.290832530e-03f);
+  r = fmaf(r, u, 8.399816230e-03f);
+  r = fmaf(r, u, -1.360862422e-02f);
+  r = fmaf(r, u, 1.851560920e-02f);
+  r = fmaf(r, u, -2.878958545e-02f);
+  r = fmaf(r, u, 4.359827935e-02f);
+  r = fmaf(r, u, -6.190539895e-02f);
+  r = fmaf(r, u, 8.360114695e-02f);
+  r = fmaf(r, u, -1.067943201e-01f);
+  r = fmaf(r, u, 1.276978850e-01f);
+  const float e = ex2_approx(x * (x * -0.721347520444482f));  // exp(-x^2/2) = 2^(-x^2 log2(e) / 2)
   GaussTail g;
-  g.phi_cdf = x >= 0.0f ? 1.0f - half_erfc : half_erfc;
+  g.t = r * e;
   g.e = e;
   return g;
 }
 
-__device__ __forceinline__ float gelu_f(float x) { return x * gauss_tail(x).phi_cdf; }
+// gelu(x) = x Phi(x) = max(x, 0) - |x| t.
+__device__ __forceinline__ float gelu_f(float x) { return fmaf(-fabsf(x), gauss_tail(x).t, fmaxf(x, 0.0f)); }
 
+// gelu'(x) = Phi(x) + x phi(x), Phi(x) = 1/2 + sign(x) (1/2 - t).
 __device__ __forceinline__ float gelu_grad_f(float x) {
   const GaussTail g = gauss_tail(x);
-  return fmaf(x * 0.39894228040143268f, g.e, g.phi_cdf);
+  const float phi_cdf = 0.5f + copysignf(0.5f - g.t, x);
+  return fmaf(x * 0.39894228040143268f, g.e, phi_cdf);
 }
 
 template <bool BF16>
@@ -148,6 +160,17 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+
+// Waits for this thread's outstanding TMEM loads.  The registers are passed
+// as in/out operands so the compiler cannot move their uses above the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
 }
 
 template <bool BF16, int EPI>
@@ -317,22 +340,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       if (grp >= nchunks) release(b);  // nothing to read in this (ragged) tile
       const int my_last = grp + ((nchunks - 1 - grp) / kEpiGroups) * kEpiGroups;
+      // TMEM loads run one chunk ahead: chunk k+1 is in flight while chunk k
+      // is converted and stored.
+      uint32_t r[2][16];
+      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN);
+      if (grp < nchunks) {
+        tmem_ld_32x32b_x16(t_row + (uint32_t)(grp * kEpiTokens), r[0]);
+        tmem_wait_ld_regs(r[0]);
+        if (grp == my_last) release(b);
+      }
 #pragma unroll
       for (int k = 0; k < kMaxChunksPerWarp; ++k) {
         const int c = grp + k * kEpiGroups;
         if (c >= nchunks) break;
+        const int cn = c + kEpiGroups;
+        if (k + 1 < kMaxChunksPerWarp && cn < nchunks)
+          tmem_ld_32x32b_x16(t_row + (uint32_t)(cn * kEpiTokens), r[(k + 1) & 1]);
         const int t0 = n0 + c * kEpiTokens;
         const int tn = min(kEpiTokens, T - t0);     // tokens of this chunk inside T
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN + c * kEpiTokens), r);
-        tmem_wait_ld();
-        if (c == my_last) release(b);
         uint16_t *dst = out + (size_t)t0 * M + m;
         uint16_t *dst_aux = aux + (size_t)t0 * M + m;
         const bool full_chunk = tn == kEpiTokens;
 #pragma unroll
         for (int jj = 0; jj < kEpiTokens; ++jj) {
-          const float acc = __uint_as_float(r[jj]);
+          const float acc = __uint_as_float(r[k & 1][jj]);
           float y = acc;
           if (EPI == kEpiGelu) y = gelu_f(acc);
           else if (EPI == kEpiDgelu)
@@ -343,6 +374,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
         if (EPI == kEpiDgelu && k + 2 < kMaxChunksPerWarp) fetch(k + 2, pk[k & 1]);
+        if (k + 1 < kMaxChunksPerWarp && cn < nchunks) {
+          tmem_wait_ld_regs(r[(k + 1) & 1]);
+          if (cn == my_last) release(b);
+        }
       }
     }
   }

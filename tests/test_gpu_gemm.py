@@ -158,3 +158,37 @@ def test_zero_tokens_is_a_no_op():
     y = torch.empty(0, 128, dtype=torch.float16, device="cuda")
     sp.sp24_gemm_fwd(x, vr, mr, 128, y)
     assert sp.sp24_device_status() == 0
+
+
+def test_metadata_layout_probe():
+    """The tensor cores read the metadata exactly where the host layout map says.
+
+    All-ones kept values and code 0x4 (keep offsets 0, 1) everywhere give
+    out[t][m] = 1 for t % 4 in {0, 1}.  Setting one nibble of the device buffer
+    to 0xE (keep 2, 3) must move exactly that row's group to offsets 2, 3, at the
+    (row, group) that sp24_meta_to_canonical assigns to that nibble."""
+    M = Kd = 128
+    vals = torch.ones(M, Kd // 2, dtype=torch.float16, device="cuda")
+    x = torch.eye(Kd, dtype=torch.float16, device="cuda")
+    base = np.full(2048, 0x44, dtype=np.uint8)
+    probes = [(L, 0, 0) for L in range(0, 128, 3)] + [(0, kk, e) for kk in range(4) for e in range(8)] + \
+             [(L, kk, e) for L in (5, 13, 21, 77, 126) for kk in (1, 3) for e in (3, 4, 7)]
+    for (L, kk, e) in probes:
+        meta = base.copy()
+        pos = L * 16 + kk * 4 + e // 2
+        meta[pos] = (meta[pos] & 0xF0) | 0x0E if e % 2 == 0 else (meta[pos] & 0x0F) | 0xE0
+        y = torch.empty(Kd, M, dtype=torch.float16, device="cuda")
+        sp.sp24_gemm_fwd(x, vals, torch.from_numpy(meta).cuda(), M, y)
+        torch.cuda.synchronize()
+        canon = sp.sp24_meta_to_canonical(meta.tobytes(), M, Kd)
+        rows, words = np.nonzero(canon != 0x4444)
+        assert len(rows) == 1
+        r, w = int(rows[0]), int(words[0])
+        nib = [k for k in range(4) if (canon[r, w] >> (4 * k)) & 0xF == 0xE]
+        assert len(nib) == 1
+        g = 4 * w + nib[0]
+        expect = np.zeros((Kd, M), np.float32)
+        expect[np.arange(Kd) % 4 < 2, :] = 1.0
+        expect[4 * g:4 * g + 2, r] = 0.0
+        expect[4 * g + 2:4 * g + 4, r] = 1.0
+        assert np.array_equal(y.float().cpu().numpy(), expect), (L, kk, e, r, g)
