@@ -235,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
       for (int kt = 0; kt < num_kt; ++kt, ++g) {
         const int s = (int)(g % kPairStages);
-        if (!mbar_wait_cluster_bounded(&empty[s], ((g / kPairStages) & 1u) ^ 1u, wait_budget, s_abort)) {
+        if (!mbar_wait_bounded(&empty[s], ((g / kPairStages) & 1u) ^ 1u, wait_budget, s_abort)) {
           ok = false;
           break;
         }
@@ -251,39 +251,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (is_leader) {
       for (uint32_t i = g > kPairStages ? g - kPairStages : 0; i < g; ++i) {
         volatile int no_abort = 0;
-        mbar_wait_cluster_bounded(&full[i % kPairStages], (i / kPairStages) & 1u, kDrainBudget, &no_abort);
+        mbar_wait_bounded(&full[i % kPairStages], (i / kPairStages) & 1u, kDrainBudget, &no_abort);
       }
     }
   } else if (warp == 1 && lane == 0 && is_leader) {
     // ----------------------------------------------------- MMA issuer (leader)
+    // Descriptors of stage 0; stage s and K step kk only move the 14-bit start
+    // address field (all of shared memory is below 2^18 bytes, so it never carries).
     constexpr uint32_t idesc = make_idesc_sparse(BF16, 2 * kPairRows, kPairBN);
+    const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
+    const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), 16, 1024, kSwizzle128B);
+    const uint64_t e_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA + kPairSmemB), 128, 128, kSwizzleNone);
     uint32_t g = 0;
     bool ok = true;
     int j = 0;
     for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++j) {
       const int b = j & 1;
       const uint32_t use = (uint32_t)(j >> 1);
-      if (!(ok = mbar_wait_cluster_bounded(&acc_empty[b], (use & 1u) ^ 1u, wait_budget, s_abort))) break;
+      if (!(ok = mbar_wait_bounded(&acc_empty[b], (use & 1u) ^ 1u, wait_budget, s_abort))) break;
       tc_fence_after();
       const uint32_t acc = tmem_base + (uint32_t)(b * kPairBN);
       for (int kt = 0; kt < num_kt; ++kt, ++g) {
         const int s = (int)(g % kPairStages);
-        if (!(ok = mbar_wait_cluster_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
+        if (!(ok = mbar_wait_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
         tc_fence_after();
-        const uint8_t *st = stage_base + s * kPairStageBytes;
-        const uint32_t a_addr = smem_u32(st);
-        const uint32_t b_addr = smem_u32(st + kPairSmemA);
-        const uint32_t e_addr = smem_u32(st + kPairSmemA + kPairSmemB);
+        const uint64_t so = (uint64_t)((s * kPairStageBytes) >> 4);
         const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
-        tc_cp_128x128b_pair(t_meta, smem_desc(e_addr, 128, 128, kSwizzleNone));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t adesc = smem_desc(a_addr + kk * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bdesc = smem_desc(b_addr + (kk >> 1) * kPairSmemBBox + (kk & 1) * 64, 16, 1024, kSwizzle128B);
-          // The metadata operand address must be 2-column aligned; the low column
-          // bit travels in the descriptor's sparsity-selector field instead.
-          tc_mma_sp_f16_pair(acc, adesc, bdesc, t_meta + (kk & 2), idesc | (uint32_t)(kk & 1), (kt | kk) != 0 ? 1u : 0u);
-        }
+        tc_cp_128x128b_pair(t_meta, e_desc0 + so);
+        const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
+        // The metadata operand address must be 2-column aligned; the low column
+        // bit travels in the descriptor's sparsity-selector field instead.
+        tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != 0 ? 1u : 0u);
+        tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
+        tc_mma_sp_f16_pair(acc, ad + 4, bd + (kPairSmemBBox >> 4), t_meta + 2, idesc, 1u);
+        tc_mma_sp_f16_pair(acc, ad + 6, bd + (kPairSmemBBox >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
         tc_commit_pair(&empty[s], 0x3);
       }
       if (ok) tc_commit_pair(&acc_full[b], 0x3);
@@ -291,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (!ok) {
       tc_commit_pair(drain, 0x1);
       volatile int no_abort = 0;
-      mbar_wait_cluster_bounded(drain, 0, kDrainBudget, &no_abort);
+      mbar_wait_bounded(drain, 0, kDrainBudget, &no_abort);
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------- epilogue (both CTAs)
@@ -335,7 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         fetch(0, pk[0]);
         fetch(1, pk[1]);
       }
-      const bool got = mbar_wait_cluster_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
+      const bool got = mbar_wait_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
       if (grp >= nchunks) release(b);  // nothing to read in this (ragged) tile

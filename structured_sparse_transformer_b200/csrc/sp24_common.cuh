@@ -54,21 +54,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-// Spins until the barrier's phase with `parity` has completed, the CTA-wide
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or `ns` nanoseconds pass, instead of spinning on issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return done != 0;
+}
+
+constexpr uint32_t kWaitSliceNs = 200000;  // one sleeping try_wait: 0.2 ms at most
+
+// Waits until the barrier's phase with `parity` has completed, the CTA-wide
 // abort flag is raised, or `budget` SM cycles pass.  Returns false on give-up;
 // a give-up caused by the budget raises the abort flag and records a timeout.
+// Also used for barriers that the CTA pair's other CTA arrives on (tcgen05
+// commits and TMA byte counts carry their own visibility).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t budget,
                                                   volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if ((uint64_t)(clock64() - t0) > budget) {
       *abort_flag = 1;
       record_device_error(kDevErrTimeout);
       return false;
     }
+    if (mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
   }
 }
 
@@ -158,34 +176,6 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void mbar_arrive_leader(uint64_t *bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(smem_u32(bar) & kPairLeaderMask)
                : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-// Bounded wait on a barrier that other CTAs of the cluster arrive on.
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity, uint64_t budget,
-                                                          volatile int *abort_flag) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if ((uint64_t)(clock64() - t0) > budget) {
-      *abort_flag = 1;
-      record_device_error(kDevErrTimeout);
-      return false;
-    }
-  }
 }
 
 // TMA tile load into this CTA's shared memory whose completion is counted on
