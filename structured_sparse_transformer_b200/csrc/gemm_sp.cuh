@@ -26,11 +26,14 @@
 // Warps: 0 = TMA producer (both CTAs), 1 = TMEM allocation and, in the leader,
 // the MMA issuer, 2-13 = epilogue: three groups of four warps take alternate
 // 16-token chunks (warp w may read TMEM lanes 32*(w%4)..+31 only, so each group
-// covers the four lane quadrants).  Each epilogue warp works alone: TMEM ->
-// registers -> coalesced 64-byte global stores (32 consecutive features of one
-// token per store), with no shared-memory staging and no cross-warp barrier.
+// covers the four lane quadrants).  Each epilogue warp works alone, with no
+// cross-warp barrier: TMEM -> registers (two adjacent tokens of one feature
+// per thread) -> packed 16-bit pairs -> stmatrix.trans into its own staging
+// tile [16 tokens x 32 features] -> one TMA store per chunk and output.
 // Shared memory: a 4-stage ring of {A 128x64 kept values, B 112x128 as two
-// boxes (both 128B-swizzled), the 2 KB metadata chunk}.
+// boxes (both 128B-swizzled), the 2 KB metadata chunk}, then 1 KB staging
+// tiles per epilogue warp (out; + aux for GELU; two pre-activation tiles for
+// dGELU).
 // Tensor memory per CTA: two 224-column fp32 accumulators (tile i+1 runs its
 // MMAs while tile i drains) and 4 metadata columns per stage.
 // Protocol:
@@ -41,8 +44,8 @@
 //     `acc_full` of both CTAs;
 //   - every epilogue warp of both CTAs arrives once on the leader's
 //     `acc_empty` when it has read its last chunk of a tile.
-// The dGELU epilogue loads a tile's pre-activation values into registers
-// before waiting for its accumulator, so the main loop hides their latency.
+// The dGELU epilogue TMA-loads its pre-activation tiles two chunks ahead (the
+// first two before waiting for the accumulator, so the main loop hides them).
 // No load uses cluster multicast; each CTA reads its own tiles.
 // Every wait is bounded; a wait that runs out records a timeout in the device
 // error word, raises the CTA's abort flag, and the CTA drains and exits.
@@ -71,12 +74,21 @@ constexpr int kPairStageBytes = kPairSmemA + kPairSmemB + kSmemE;   // 46 KB
 constexpr int kPairStages = 4;
 constexpr int kPairChunks = kPairBN / kEpiTokens;      // 14
 constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at columns 0 and 224
-constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 256 + 1024;
+constexpr int kEpiBufBytes = kEpiTokens * 32 * 2;      // staging tile: 16 tokens x 32 features, 64B-swizzled
+constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM address, abort flag
+
+enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
+
+// Staging tiles per epilogue warp: out; out + pre-activation; out + two
+// pre-activation inputs.
+__host__ __device__ constexpr int epi_bufs(int epi) { return epi == kEpiNone ? 1 : (epi == kEpiGelu ? 2 : 3); }
+__host__ __device__ constexpr int pair_smem_bytes(int epi) {
+  return kPairStages * kPairStageBytes + kEpiWarps * epi_bufs(epi) * kEpiBufBytes + kPairBarBytes + 1024;
+}
+static_assert(pair_smem_bytes(kEpiDgelu) <= 232448, "shared memory per CTA");
 static_assert(kPairStageBytes % 1024 == 0 && kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
 static_assert(kPairMetaCol + 4 * kPairStages <= kTmemCols, "tensor memory budget");
-
-enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
 
 // GELU (exact erf form) and its derivative for the epilogues:
 //   gelu(x) = x Phi(x),  gelu'(x) = Phi(x) + x phi(x),
@@ -151,37 +163,77 @@ __device__ __forceinline__ float bits_to_f32(uint32_t b) {
 }
 
 // 32 lanes x 16 consecutive 32-bit columns.
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+// 16 TMEM lanes x 16 columns (two 16x256b blocks).  Thread t receives, for
+// column block i (registers 4i..4i+3): lane t/4 at columns 8i + 2(t%4) + {0, 1},
+// then lane t/4 + 8 at the same two columns.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
 }
 
-// Waits for this thread's outstanding TMEM loads.  The registers are passed
-// as in/out operands so the compiler cannot move their uses above the wait.
-__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                 "+r"(r[14]), "+r"(r[15])
-               :
+// After tmem_wait_ld, reg_fence on the loaded registers keeps every use of
+// them below the wait.  Makes the compiler treat the registers as redefined
+// here (emits nothing).
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[8]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+}
+
+// Four 8x8 16-bit matrices, transposed on the way: register j of thread t
+// holds row t/4, columns 2(t%4) and 2(t%4)+1 of matrix j; lane 8j + r gives
+// the shared address of (stored) row r of matrix j.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, const uint32_t (&r)[4]) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
                : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// Byte offset of 16-byte column c of row `row` in a 64B-swizzled tile of
+// 64-byte rows (the TMA's 64B pattern: the column index is XORed with row/2 mod 4).
+__host__ __device__ constexpr uint32_t swz64(int row, int c) {
+  return (uint32_t)(row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
+}
+
+// Two floats -> one register of 16-bit values, lo in the low half (round to nearest even).
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  uint32_t d;
+  if (BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void unpack2(uint32_t v, float &lo, float &hi) {
+  if (BF16) {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xFFFF0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&v));
+    lo = f.x;
+    hi = f.y;
+  }
 }
 
 template <bool BF16, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                          const __grid_constant__ CUtensorMap tm_meta, uint16_t *__restrict__ out,
-                          uint16_t *__restrict__ aux, int M, int T, int num_kt, uint64_t wait_budget) {
+                          const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
+                          const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
+                          uint64_t wait_budget) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_base = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kPairStages * kPairStageBytes);
+  uint8_t *epi_smem = smem + kPairStages * kPairStageBytes;   // staging tiles, 1 KB aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(epi_smem + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes);
   uint64_t *full = bars;                          // [stages] leader: TMA (both CTAs) -> MMA
   uint64_t *empty = bars + kPairStages;           // [stages] MMA -> this CTA's TMA
   uint64_t *acc_full = bars + 2 * kPairStages;    // [2] MMA -> this CTA's epilogue
@@ -189,6 +241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t *drain = acc_empty + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+  uint64_t *aux_bars = bars + 16;                 // [kEpiWarps][2] dGELU pre-activation tiles
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -206,11 +259,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
+    if (EPI == kEpiDgelu)
+      for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(&aux_bars[i], 1);
     *s_abort = 0;
     fence_mbarrier_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
     prefetch_tensormap(&tm_meta);
+    prefetch_tensormap(&tm_out);
+    if (EPI != kEpiNone) prefetch_tensormap(&tm_aux);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, kTmemCols);
@@ -296,89 +353,143 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------- epilogue (both CTAs)
-    // Warp w reads lane quadrant w%4 and takes chunks grp, grp + kEpiGroups, ...
-    // (grp = (w-2)/4) of every tile.  Decisions after a bounded wait are made
-    // per warp (__all_sync), so the .sync.aligned TMEM loads stay convergent.
-    // A warp releases the accumulator with one arrive (lane 0) after its lanes'
-    // TMEM reads have completed.
-    const int grp = (warp - 2) >> 2;
+    // Warp w reads TMEM lane quadrant q = w%4 (features 32q..32q+31 of this
+    // CTA's rows) and takes the 16-token chunks grp, grp + kEpiGroups, ...
+    // (grp = (w-2)/4) of every tile.  It issues all its TMEM loads of a tile
+    // at once and returns the accumulator to the MMA after one round trip; the
+    // math, packing and stores then overlap the next tiles' main loop.
+    // Decisions after a bounded wait are made per warp (__all_sync), so the
+    // .sync.aligned instructions stay convergent.
+    const int ew = warp - 2;
+    const int grp = ew >> 2;
     const int q = warp & 3;
-    const int m_local = 32 * q + lane;
     constexpr int kMaxChunksPerWarp = (kPairChunks + kEpiGroups - 1) / kEpiGroups;
+    uint8_t *stg = epi_smem + ew * epi_bufs(EPI) * kEpiBufBytes;   // [out][aux] or [out][pre 0][pre 1]
+    const uint32_t stg_u32 = smem_u32(stg);
+    uint64_t *pre_bar = aux_bars + 2 * ew;
+    // stmatrix/ldmatrix addressing: lane l names row l%8 of matrix l/8; matrix
+    // j holds tokens 8(j/2).. and features 8(j%2).. (+16 for the upper 16 TMEM lanes).
+    const int mrow = 8 * (lane >> 4) + (lane & 7);
+    const uint32_t lane_off0 = swz64(mrow, (lane >> 3) & 1);
+    const uint32_t lane_off1 = swz64(mrow, 2 + ((lane >> 3) & 1));
     auto release = [&](int buf) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&acc_empty[buf]);
     };
+    uint32_t pre_issued = 0, pre_used = 0;   // dGELU pre-activation tiles (tile s uses buffer s%2)
+    auto pre_load = [&](int x, int y) {
+      const uint32_t seq = pre_issued++;
+      if (lane == 0) {
+        uint64_t *bar = &pre_bar[seq & 1];
+        mbar_arrive_expect_tx(bar, kEpiBufBytes);
+        tma_load_2d(stg + kEpiBufBytes * (1 + (seq & 1)), &tm_aux, bar, x, y);
+      }
+    };
+    bool alive = true;
     int j = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
+    for (int tile = pair; tile < num_tiles && alive; tile += npairs, ++j) {
       const int b = j & 1;
-      const int m = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + m_local;
+      const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
       const int n0 = (tile / num_mt) * kPairBN;
       const int nchunks = min(kPairChunks, (T - n0 + kEpiTokens - 1) / kEpiTokens);
-      const bool m_ok = m < M;
-      // dGELU: pre-activations, two tokens per register, fetched two chunks
-      // ahead of use; the first two before the accumulator is ready, so the
-      // main loop hides their latency.
-      uint32_t pk[2][kEpiTokens / 2];
-      auto fetch = [&](int k, uint32_t (&dstv)[kEpiTokens / 2]) {
-        const int t0 = n0 + (grp + k * kEpiGroups) * kEpiTokens;
-        const uint16_t *src = aux + (size_t)t0 * M + m;
-#pragma unroll
-        for (int jj = 0; jj < kEpiTokens / 2; ++jj) {
-          const int t = t0 + 2 * jj;
-          const uint32_t lo = (m_ok && t < T) ? src[(size_t)(2 * jj) * M] : 0u;
-          const uint32_t hi = (m_ok && t + 1 < T) ? src[(size_t)(2 * jj + 1) * M] : 0u;
-          dstv[jj] = lo | (hi << 16);
-        }
-      };
-      if (EPI == kEpiDgelu) {
-        fetch(0, pk[0]);
-        fetch(1, pk[1]);
-      }
+      const int nk = grp < nchunks ? (nchunks - 1 - grp) / kEpiGroups + 1 : 0;   // this warp's chunks
+      if (EPI == kEpiDgelu)
+        for (int k = 0; k < 2 && k < nk; ++k) pre_load(m0, n0 + (grp + k * kEpiGroups) * kEpiTokens);
       const bool got = mbar_wait_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
-      if (!__all_sync(0xFFFFFFFFu, got)) break;
-      tc_fence_after();
-      if (grp >= nchunks) release(b);  // nothing to read in this (ragged) tile
-      const int my_last = grp + ((nchunks - 1 - grp) / kEpiGroups) * kEpiGroups;
-      // TMEM loads run one chunk ahead: chunk k+1 is in flight while chunk k
-      // is converted and stored.
-      uint32_t r[2][16];
-      const uint32_t t_row = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN);
-      if (grp < nchunks) {
-        tmem_ld_32x32b_x16(t_row + (uint32_t)(grp * kEpiTokens), r[0]);
-        tmem_wait_ld_regs(r[0]);
-        if (grp == my_last) release(b);
+      if (!__all_sync(0xFFFFFFFFu, got)) {
+        alive = false;
+        break;
       }
+      tc_fence_after();
+      uint32_t r[kMaxChunksPerWarp][2][8];
+      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN);
 #pragma unroll
       for (int k = 0; k < kMaxChunksPerWarp; ++k) {
-        const int c = grp + k * kEpiGroups;
-        if (c >= nchunks) break;
-        const int cn = c + kEpiGroups;
-        if (k + 1 < kMaxChunksPerWarp && cn < nchunks)
-          tmem_ld_32x32b_x16(t_row + (uint32_t)(cn * kEpiTokens), r[(k + 1) & 1]);
-        const int t0 = n0 + c * kEpiTokens;
-        const int tn = min(kEpiTokens, T - t0);     // tokens of this chunk inside T
-        uint16_t *dst = out + (size_t)t0 * M + m;
-        uint16_t *dst_aux = aux + (size_t)t0 * M + m;
-        const bool full_chunk = tn == kEpiTokens;
+        if (k < nk) {
+          const uint32_t col = (uint32_t)((grp + k * kEpiGroups) * kEpiTokens);
+          tmem_ld_16x256b_x2(t_base + col, r[k][0]);
+          tmem_ld_16x256b_x2(t_base + (16u << 16) + col, r[k][1]);
+        }
+      }
+      tmem_wait_ld();
 #pragma unroll
-        for (int jj = 0; jj < kEpiTokens; ++jj) {
-          const float acc = __uint_as_float(r[k & 1][jj]);
-          float y = acc;
-          if (EPI == kEpiGelu) y = gelu_f(acc);
-          else if (EPI == kEpiDgelu)
-            y = acc * gelu_grad_f(bits_to_f32<BF16>((pk[k & 1][jj >> 1] >> ((jj & 1) * 16)) & 0xFFFFu));
-          if (m_ok && (full_chunk || jj < tn)) {
-            if (EPI == kEpiGelu) dst_aux[(size_t)jj * M] = (uint16_t)f32_to_bits<BF16>(acc);
-            dst[(size_t)jj * M] = (uint16_t)f32_to_bits<BF16>(y);
+      for (int k = 0; k < kMaxChunksPerWarp; ++k) {
+        reg_fence(r[k][0]);
+        reg_fence(r[k][1]);
+      }
+      release(b);
+#pragma unroll
+      for (int k = 0; k < kMaxChunksPerWarp; ++k) {
+        if (k >= nk) break;
+        const int t0 = n0 + (grp + k * kEpiGroups) * kEpiTokens;
+        uint32_t hx[2][4];
+        if (EPI == kEpiDgelu) {
+          const uint32_t seq = pre_used;
+          const bool ready = mbar_wait_bounded(&pre_bar[seq & 1], (seq >> 1) & 1u, wait_budget, s_abort);
+          if (!__all_sync(0xFFFFFFFFu, ready)) {
+            alive = false;
+            break;
+          }
+          ++pre_used;
+          const uint32_t src = stg_u32 + kEpiBufBytes * (1 + (seq & 1));
+          ldmatrix_x4_trans(src + lane_off0, hx[0]);
+          ldmatrix_x4_trans(src + lane_off1, hx[1]);
+        }
+        // Register i of half h: tokens 8(i/2) + 2(lane%4) + {0, 1} of feature
+        // 16h + 8(i%2) + lane/4 (TMEM registers 4(i/2) + 2(i%2) + {0, 1}).
+        uint32_t po[2][4], pa[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int ri = 4 * (i >> 1) + 2 * (i & 1);
+            const float a0 = __uint_as_float(r[k][h][ri]);
+            const float a1 = __uint_as_float(r[k][h][ri + 1]);
+            float y0 = a0, y1 = a1;
+            if (EPI == kEpiGelu) {
+              y0 = gelu_f(a0);
+              y1 = gelu_f(a1);
+              pa[h][i] = pack2<BF16>(a0, a1);
+            } else if (EPI == kEpiDgelu) {
+              float h0, h1;
+              unpack2<BF16>(hx[h][i], h0, h1);
+              y0 = a0 * gelu_grad_f(h0);
+              y1 = a1 * gelu_grad_f(h1);
+            }
+            po[h][i] = pack2<BF16>(y0, y1);
           }
         }
-        if (EPI == kEpiDgelu && k + 2 < kMaxChunksPerWarp) fetch(k + 2, pk[k & 1]);
-        if (k + 1 < kMaxChunksPerWarp && cn < nchunks) {
-          tmem_wait_ld_regs(r[(k + 1) & 1]);
-          if (cn == my_last) release(b);
+        if (EPI == kEpiDgelu) {
+          // This warp's ldmatrix reads of the tile come before the TMA write
+          // that refills it.
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (k + 2 < nk) pre_load(m0, t0 + 2 * kEpiGroups * kEpiTokens);
         }
+        if (lane == 0) bulk_wait_group_read<0>();   // the previous chunk's stores have read the staging tiles
+        __syncwarp();
+        stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);
+        stmatrix_x4_trans(stg_u32 + lane_off1, po[1]);
+        if (EPI == kEpiGelu) {
+          stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off0, pa[0]);
+          stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off1, pa[1]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && m0 < M) {   // the TMA unit clips features >= M and tokens >= T
+          tma_store_2d(&tm_out, stg, m0, t0);
+          if (EPI == kEpiGelu) tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (lane == 0) {
+      bulk_wait_group<0>();
+      // After an abort, let the pre-activation loads still in flight land.
+      for (uint32_t seq = pre_used; seq < pre_issued; ++seq) {
+        volatile int no_abort = 0;
+        mbar_wait_bounded(&pre_bar[seq & 1], (seq >> 1) & 1u, kDrainBudget, &no_abort);
       }
     }
   }

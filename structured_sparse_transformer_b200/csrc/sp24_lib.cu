@@ -101,15 +101,22 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
       !make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT64))
     return SP24_ERR_CUDA;
+  // Epilogue staging tiles: 32 features x 16 tokens of row-major out / aux [T x M].
+  CUtensorMap to, tx;
+  if (!make_map_2d(&to, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_2d(&tx, EPI == kEpiNone ? out : aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return SP24_ERR_CUDA;
+  constexpr int smem_bytes = pair_smem_bytes(EPI);
   auto kernel = sp24_gemm_pair_kernel<BF16, EPI>;
   static int max_pairs = 0;
   if (max_pairs == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
       return SP24_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -126,9 +133,8 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   }
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + kPairBN - 1) / kPairBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
-  kernel<<<2 * pairs, kGemmThreads, kPairSmemBytes, stream>>>(ta, tb, tm, static_cast<uint16_t *>(out),
-                                                              static_cast<uint16_t *>(aux), (int)M, (int)T, num_kt,
-                                                              g_wait_budget.load());
+  kernel<<<2 * pairs, kGemmThreads, smem_bytes, stream>>>(ta, tb, tm, to, tx, (int)M, (int)T, num_kt,
+                                                         g_wait_budget.load());
   return launch_status();
 }
 
