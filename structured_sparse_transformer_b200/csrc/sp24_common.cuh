@@ -172,9 +172,13 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on the mbarrier at the same offset in the pair's leader CTA.
+// Arrive on the mbarrier at the same offset in the pair's leader CTA.  Relaxed:
+// it only reports tensor-memory reads that tcgen05.wait::ld has already
+// completed, so it need not wait for this thread's earlier memory traffic
+// (a release at cluster scope would hold the arrive until the outstanding
+// global stores are performed).
 __device__ __forceinline__ void mbar_arrive_leader(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(smem_u32(bar) & kPairLeaderMask)
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(smem_u32(bar) & kPairLeaderMask)
                : "memory");
 }
 
