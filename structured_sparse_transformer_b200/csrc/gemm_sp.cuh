@@ -110,44 +110,56 @@ __device__ __forceinline__ float ex2_approx(float y) {
   return r;
 }
 
-// t = erfc(|x| / sqrt 2) / 2 (the normal tail beyond |x|) and e = exp(-x^2 / 2).
-// R's coefficients are the fitted ones scaled by 1/2 (exact), so r = R/2.
-struct GaussTail {
-  float t;
-  float e;
-};
+// The epilogue evaluates elements in pairs (two adjacent tokens of one
+// feature) with the packed f32x2 FMA path: every add, multiply and fused
+// multiply-add below is the IEEE fp32 operation on each lane, two results per
+// instruction.
+__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
 
-__device__ __forceinline__ GaussTail gauss_tail(float x) {
-  // u = z/2 - 1 with z = min(|x|, 4 sqrt 2) / sqrt 2
-  const float u = fmaf(fminf(fabsf(x), 5.65685424949238f), 0.353553390593274f, -1.0f);
-  float r = 1.858228817e-03f;
-  r = fmaf(r, u, -3.360528732e-03f);
-  r = fmaf(r, u, 5.786734400e-04f);
-  r = fmaf(r, u, -1.290832530e-03f);
-  r = fmaf(r, u, 8.399816230e-03f);
-  r = fmaf(r, u, -1.360862422e-02f);
-  r = fmaf(r, u, 1.851560920e-02f);
-  r = fmaf(r, u, -2.878958545e-02f);
-  r = fmaf(r, u, 4.359827935e-02f);
-  r = fmaf(r, u, -6.190539895e-02f);
-  r = fmaf(r, u, 8.360114695e-02f);
-  r = fmaf(r, u, -1.067943201e-01f);
-  r = fmaf(r, u, 1.276978850e-01f);
-  const float e = ex2_approx(x * (x * -0.721347520444482f));  // exp(-x^2/2) = 2^(-x^2 log2(e) / 2)
-  GaussTail g;
-  g.t = r * e;
-  g.e = e;
-  return g;
+// R(z)/2 at z = min(|x|, 4 sqrt 2) / sqrt 2, in u = z/2 - 1 (the fitted
+// coefficients scaled by 1/2, exact).
+__device__ __forceinline__ float2 half_r2(float2 ax) {
+  const float2 zc = make_float2(fminf(ax.x, 5.65685424949238f), fminf(ax.y, 5.65685424949238f));
+  const float2 u = __ffma2_rn(zc, splat(0.353553390593274f), splat(-1.0f));
+  float2 r = splat(1.858228817e-03f);
+  r = __ffma2_rn(r, u, splat(-3.360528732e-03f));
+  r = __ffma2_rn(r, u, splat(5.786734400e-04f));
+  r = __ffma2_rn(r, u, splat(-1.290832530e-03f));
+  r = __ffma2_rn(r, u, splat(8.399816230e-03f));
+  r = __ffma2_rn(r, u, splat(-1.360862422e-02f));
+  r = __ffma2_rn(r, u, splat(1.851560920e-02f));
+  r = __ffma2_rn(r, u, splat(-2.878958545e-02f));
+  r = __ffma2_rn(r, u, splat(4.359827935e-02f));
+  r = __ffma2_rn(r, u, splat(-6.190539895e-02f));
+  r = __ffma2_rn(r, u, splat(8.360114695e-02f));
+  r = __ffma2_rn(r, u, splat(-1.067943201e-01f));
+  r = __ffma2_rn(r, u, splat(1.276978850e-01f));
+  return r;
 }
 
-// gelu(x) = x Phi(x) = max(x, 0) - |x| t.
-__device__ __forceinline__ float gelu_f(float x) { return fmaf(-fabsf(x), gauss_tail(x).t, fmaxf(x, 0.0f)); }
+// exp(-x^2/2) = 2^(-x^2 log2(e) / 2)
+__device__ __forceinline__ float2 gauss_e2(float2 x) {
+  const float2 a = __fmul2_rn(x, __fmul2_rn(x, splat(-0.721347520444482f)));
+  return make_float2(ex2_approx(a.x), ex2_approx(a.y));
+}
 
-// gelu'(x) = Phi(x) + x phi(x), Phi(x) = 1/2 + sign(x) (1/2 - t).
-__device__ __forceinline__ float gelu_grad_f(float x) {
-  const GaussTail g = gauss_tail(x);
-  const float phi_cdf = 0.5f + copysignf(0.5f - g.t, x);
-  return fmaf(x * 0.39894228040143268f, g.e, phi_cdf);
+// gelu(x) = x Phi(x) = max(x, 0) - |x| t with t = erfc(|x|/sqrt2)/2 = e R/2.
+__device__ __forceinline__ float2 gelu2(float2 x) {
+  const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+  const float2 t = __fmul2_rn(half_r2(ax), gauss_e2(x));
+  return __ffma2_rn(make_float2(-ax.x, -ax.y), t, make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f)));
+}
+
+// gelu'(x) = Phi(x) + x phi(x) with phi = e / sqrt(2 pi):
+//   x <  0:  t - |x| phi      = e (R/2 - |x|/sqrt(2 pi))
+//   x >= 0:  1 - t + |x| phi  = 1 - e (R/2 - |x|/sqrt(2 pi))
+// (both give 1/2 at x = 0, so -0 may take either side).
+__device__ __forceinline__ float2 gelu_grad2(float2 x) {
+  const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+  const float2 e = gauss_e2(x);
+  const float2 q = __ffma2_rn(make_float2(-ax.x, -ax.y), splat(0.39894228040143268f), half_r2(ax));
+  const bool p0 = x.x >= 0.0f, p1 = x.y >= 0.0f;
+  return __ffma2_rn(make_float2(p0 ? -e.x : e.x, p1 ? -e.y : e.y), q, make_float2(p0 ? 1.0f : 0.0f, p1 ? 1.0f : 0.0f));
 }
 
 template <bool BF16>
@@ -444,28 +456,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int ri = 4 * (i >> 1) + 2 * (i & 1);
-            const float a0 = __uint_as_float(r[k][h][ri]);
-            const float a1 = __uint_as_float(r[k][h][ri + 1]);
-            float y0 = a0, y1 = a1;
+            const float2 acc = make_float2(__uint_as_float(r[k][h][ri]), __uint_as_float(r[k][h][ri + 1]));
+            float2 y = acc;
             if (EPI == kEpiGelu) {
-              y0 = gelu_f(a0);
-              y1 = gelu_f(a1);
-              pa[h][i] = pack2<BF16>(a0, a1);
+              y = gelu2(acc);
+              pa[h][i] = pack2<BF16>(acc.x, acc.y);
             } else if (EPI == kEpiDgelu) {
-              float h0, h1;
-              unpack2<BF16>(hx[h][i], h0, h1);
-              y0 = a0 * gelu_grad_f(h0);
-              y1 = a1 * gelu_grad_f(h1);
+              float2 hv;
+              unpack2<BF16>(hx[h][i], hv.x, hv.y);
+              y = __fmul2_rn(acc, gelu_grad2(hv));
             }
-            po[h][i] = pack2<BF16>(y0, y1);
+            po[h][i] = pack2<BF16>(y.x, y.y);
           }
-        }
-        if (EPI == kEpiDgelu) {
-          // This warp's ldmatrix reads of the tile come before the TMA write
-          // that refills it.
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (k + 2 < nk) pre_load(m0, t0 + 2 * kEpiGroups * kEpiTokens);
         }
         if (lane == 0) bulk_wait_group_read<0>();   // the previous chunk's stores have read the staging tiles
         __syncwarp();
@@ -475,6 +477,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off0, pa[0]);
           stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off1, pa[1]);
         }
+        // One proxy fence orders this warp's shared-memory accesses of the
+        // chunk (the stmatrix writes, and for dGELU the ldmatrix reads of the
+        // pre-activation tile) before the TMA store that reads the staging tile
+        // and the TMA load that refills the pre-activation tile.
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && m0 < M) {   // the TMA unit clips features >= M and tokens >= T
@@ -482,6 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (EPI == kEpiGelu) tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
           bulk_commit_group();
         }
+        if (EPI == kEpiDgelu && k + 2 < nk) pre_load(m0, t0 + 2 * kEpiGroups * kEpiTokens);
       }
     }
     if (lane == 0) {
