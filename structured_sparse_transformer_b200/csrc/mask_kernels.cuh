@@ -27,7 +27,10 @@ namespace sp24 {
 
 using u64 = unsigned long long;
 
-__constant__ PatternTables c_tables = make_pattern_tables();
+// The pattern tables in global memory: threads index them with per-thread
+// pattern numbers, which the L1 cache serves without the serialisation that
+// divergent reads of __constant__ memory would take, and without a per-CTA copy.
+__device__ const PatternTables g_tables = make_pattern_tables();
 
 __device__ __forceinline__ u64 umax64(u64 a, u64 b) { return a > b ? a : b; }
 
@@ -62,13 +65,13 @@ __device__ __forceinline__ uint32_t dp_argmax_ranks(const u64 (&v)[16]) {
 // so the fast path keeps everything in registers.
 __device__ __noinline__ uint32_t exact_search_wide_bf16(uint32_t w00, uint32_t w01, uint32_t w10, uint32_t w11,
                                                         uint32_t w20, uint32_t w21, uint32_t w30, uint32_t w31,
-                                                        const uint16_t *s_bits) {
+                                                        const uint16_t *bits_tab) {
   const uint32_t words[8] = {w00, w01, w10, w11, w20, w21, w30, w31};
   u64 best[5] = {0, 0, 0, 0, 0};
   uint32_t best_p = 0;
   for (int p = 0; p < kNumPatterns; ++p) {
     u64 acc[5] = {0, 0, 0, 0, 0};
-    const uint32_t bits = s_bits[p];
+    const uint32_t bits = bits_tab[p];
     for (int c = 0; c < 16; ++c) {
       if (!((bits >> c) & 1u)) continue;
       const uint32_t a = (words[c >> 1] >> ((c & 1) << 4)) & 0x7FFFu;
@@ -102,20 +105,68 @@ __device__ __noinline__ uint32_t exact_search_wide_bf16(uint32_t w00, uint32_t w
   return best_p;
 }
 
+// Dynamic program over column-count states on magnitudes v[4*i+j] = |w(i,j)|
+// in a type whose sums here are exact.  One state at a time, so only the pair
+// sums and the running best stay live: the state's best top and bottom combos
+// (the lowest rank among equal sums), then the pattern total against the best
+// so far (a larger total wins; an equal total keeps the smaller
+// (top rank, bottom rank) key).  Returns top rank << 6 | bottom rank.
+template <typename Real>
+__device__ __forceinline__ uint32_t dp_state_key(const Real (&v)[16]) {
+  constexpr PatternTables T = make_pattern_tables();
+  Real P[4][6];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int q = 0; q < 6; ++q) P[i][q] = v[4 * i + pair_lo(q)] + v[4 * i + pair_hi(q)];
+  Real best = (Real)-1;  // every total is >= 0, so the first state is taken
+  uint32_t bkey = 0;
+#pragma unroll
+  for (int st = 0; st < kNumStates; ++st) {
+    Real tv = 0, bv = 0;
+    uint32_t tr = 0, br = 0;
+    bool tseen = false, bseen = false;
+#pragma unroll
+    for (int c = 0; c < 36; ++c) {
+      if (T.top_state[c] == st) {
+        const Real k = P[0][c / 6] + P[1][c % 6];
+        if (!tseen) { tv = k; tr = (uint32_t)c; tseen = true; }
+        else { const bool gt = k > tv; tv = gt ? k : tv; tr = gt ? (uint32_t)c : tr; }
+      }
+      if (T.bot_state[c] == st) {
+        const Real k = P[2][c / 6] + P[3][c % 6];
+        if (!bseen) { bv = k; br = (uint32_t)c; bseen = true; }
+        else { const bool gt = k > bv; bv = gt ? k : bv; br = gt ? (uint32_t)c : br; }
+      }
+    }
+    const Real tot = tv + bv;
+    const uint32_t key = (tr << 6) | br;
+    const bool take = tot > best || (tot == best && key < bkey);
+    best = take ? tot : best;
+    bkey = take ? key : bkey;
+  }
+  return bkey;
+}
+
 // Pattern index of one 4x4 block given as 4 rows x 2 words (two 16-bit values each).
 template <bool BF16>
-__device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], const uint8_t *s_index,
-                                                 const uint16_t *s_bits) {
+__device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], const uint8_t *index_tab,
+                                                 const uint16_t *bits_tab) {
   u64 v[16];
   if (!BF16) {
+    // fp16: |w| = sig * 2^ep units of 2^-24 is below 2^41; a sum of eight is
+    // below 2^44 and exact in fp64.
+    double d[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
       const uint32_t a = (w[c >> 2][(c >> 1) & 1] >> ((c & 1) << 4)) & 0x7FFFu;
       const uint32_t e = a >> 10;
       const uint32_t sig = e ? ((a & 0x3FFu) | 0x400u) : a;
       const uint32_t ep = e ? e - 1 : 0;
-      v[c] = (u64)sig << (ep + 12);
+      d[c] = __ull2double_rn((u64)sig << ep);
     }
+    const uint32_t key = dp_state_key<double>(d);
+    return index_tab[(key >> 6) * 36 + (key & 63)];
   } else {
     uint32_t sig[16], ep[16];
     uint32_t emax = 0;
@@ -137,10 +188,10 @@ __device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], cons
     }
     if (!exact)
       return exact_search_wide_bf16(w[0][0], w[0][1], w[1][0], w[1][1], w[2][0], w[2][1], w[3][0], w[3][1],
-                                    s_bits);
+                                    bits_tab);
   }
   const uint32_t r = dp_argmax_ranks(v);
-  return s_index[(35 - (r >> 6)) * 36 + (35 - (r & 63))];
+  return index_tab[(35 - (r >> 6)) * 36 + (35 - (r & 63))];
 }
 
 constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
@@ -155,7 +206,7 @@ constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 // the state's maximum wins (strict >); across states the smallest
 // (top rank, bottom rank) among the states reaching the global maximum wins.
 template <bool BF16>
-__device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2], const uint8_t *s_index) {
+__device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2], const uint8_t *index_tab) {
   constexpr PatternTables T = make_pattern_tables();
   float v[16];
 #pragma unroll
@@ -170,35 +221,8 @@ __device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2],
     vmin = fminf(vmin, v[c] > 0.0f ? v[c] : __int_as_float(0x7F800000));
   }
   if (!(vmin >= vmax * (BF16 ? 0x1p-13f : 0x1p-10f))) return kNeedsExact;
-
-  float P[4][6];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int q = 0; q < 6; ++q) P[i][q] = v[4 * i + pair_lo(q)] + v[4 * i + pair_hi(q)];
-  float top[kNumStates], bot[kNumStates];
-  uint32_t tr[kNumStates], br[kNumStates];
-  bool seen_t[kNumStates] = {}, seen_b[kNumStates] = {};
-#pragma unroll
-  for (int c = 0; c < 36; ++c) {
-    const int st = T.top_state[c];
-    const float kt = P[0][c / 6] + P[1][c % 6];
-    if (!seen_t[st]) { top[st] = kt; tr[st] = (uint32_t)c; seen_t[st] = true; }
-    else { const bool gt = kt > top[st]; top[st] = gt ? kt : top[st]; tr[st] = gt ? (uint32_t)c : tr[st]; }
-    const int sb = T.bot_state[c];
-    const float kb = P[2][c / 6] + P[3][c % 6];
-    if (!seen_b[sb]) { bot[sb] = kb; br[sb] = (uint32_t)c; seen_b[sb] = true; }
-    else { const bool gt = kb > bot[sb]; bot[sb] = gt ? kb : bot[sb]; br[sb] = gt ? (uint32_t)c : br[sb]; }
-  }
-  float tot[kNumStates];
-  float best = 0.0f;
-#pragma unroll
-  for (int st = 0; st < kNumStates; ++st) { tot[st] = top[st] + bot[st]; best = fmaxf(best, tot[st]); }
-  uint32_t key = 0xFFFFu;
-#pragma unroll
-  for (int st = 0; st < kNumStates; ++st)
-    if (tot[st] == best) key = min(key, (tr[st] << 6) | br[st]);
-  return s_index[(key >> 6) * 36 + (key & 63)];
+  const uint32_t key = dp_state_key<float>(v);
+  return index_tab[(key >> 6) * 36 + (key & 63)];
 }
 
 __device__ __forceinline__ uint32_t half_of(const uint32_t (&row)[4], int blk, uint32_t k) {
@@ -213,11 +237,12 @@ __device__ __forceinline__ uint32_t pick_row(const uint32_t (&w)[4][4], uint32_t
 }
 
 // Physical word of (W column c_local, block row br_local) in the transposed
-// values tile: 16-byte chunks XOR-swizzled by c_local/8, words inside a chunk
-// by c_local/64, so the writes of a warp hit 32 distinct banks.
+// values tile (64 columns x 16 words): the 16-byte chunk of four block rows
+// is XOR-swizzled by c_local/8, the word inside it by c_local/32, so the
+// staging stores of a warp spread over the banks.
 __device__ __forceinline__ int vcol_word(int c_local, int br_local) {
-  return c_local * 32 + ((((br_local >> 2) ^ (c_local >> 3)) & 7) << 2) +
-         ((br_local & 3) ^ (((c_local >> 6) & 1) << 1));
+  return c_local * 16 + ((((br_local >> 2) ^ (c_local >> 3)) & 3) << 2) +
+         ((br_local & 3) ^ (((c_local >> 5) & 1) << 1));
 }
 
 // Loads one unit (4 rows x 8 columns = two blocks) of W; columns past C read as 0.
@@ -244,121 +269,132 @@ __device__ __forceinline__ void load_unit(const uint16_t *__restrict__ W, int64_
   }
 }
 
-constexpr int kTile = 128;       // W tile: 128 rows x 128 columns per CTA
-constexpr int kMaskThreads = 256;
+constexpr int kTile = 64;           // W tile: 64 rows x 64 columns per CTA
+constexpr int kTileBlocks = kTile / 4;
+constexpr int kMaskThreads = 128;   // one unit (4 rows x 8 columns = two blocks) per thread
 
-// One CTA per 128x128 tile of W.  Thread t owns units (4 rows x 8 columns =
-// two blocks) at unit column t%16 and block rows t/16 and t/16 + 16.
+// Nibble (4 * shift) of each of the four 16-bit codes in v, packed 4 bits apart.
+__device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
+  const uint32_t lo = (v.x >> (4 * shift)) & 0x000F000Fu;   // codes 0, 1
+  const uint32_t hi = (v.y >> (4 * shift)) & 0x000F000Fu;   // codes 2, 3
+  return (lo & 0xFu) | ((lo >> 12) & 0xF0u) | ((hi & 0xFu) << 8) | ((hi >> 4) & 0xF000u);
+}
+
+// One CTA per 64x64 tile of W; thread t owns the unit at unit column t%8 and
+// block row t/8.  The tensor-core metadata comes in 2048-byte chunks of
+// 128x128 (see the GEMM); a tile writes its quadrant of the chunk, and with
+// COMPRESS the grid is rounded up to whole chunks so that rows and columns
+// past the matrix get the padding code.
 //   SEARCH:   compute the mask (else read it from idx)
 //   COMPRESS: write the compressed orientations whose pointers are non-null
 //             (values + tensor-core metadata)
 //   FLIP:     add the number of mask bits that differ from idx_prev to *flip_count
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
+__global__ void __launch_bounds__(kMaskThreads, 8) mask_tile_kernel(
     const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
     uint8_t *__restrict__ meta_col) {
-  __shared__ uint16_t s_bits[256];
-  __shared__ uint16_t s_rowcode[256];
-  __shared__ uint16_t s_colcode[256];
-  __shared__ uint8_t s_index[36 * 36];
-  __shared__ uint8_t s_idx[32][36];
-  __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kTile * 32 : 4];
-  __shared__ uint16_t s_queue[SEARCH ? 1024 : 2];
+  __shared__ uint8_t s_idx[kTileBlocks][kTileBlocks];
+  __shared__ __align__(8) uint16_t s_rc[kTileBlocks][kTileBlocks];   // row codes, [block row][block col]
+  __shared__ __align__(8) uint16_t s_cc[kTileBlocks][kTileBlocks];   // column codes, [block col][block row]
+  __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kTile * 16 : 4];
+  __shared__ uint16_t s_queue[SEARCH ? kTileBlocks * kTileBlocks : 2];
   __shared__ int s_qn;
   __shared__ unsigned long long s_flip;
 
   const int tid = threadIdx.x;
-  for (int i = tid; i < 256; i += kMaskThreads) {
-    s_bits[i] = c_tables.bits[i];
-    s_rowcode[i] = c_tables.rowcode[i];
-    s_colcode[i] = c_tables.colcode[i];
-  }
-  for (int i = tid; i < 36 * 36; i += kMaskThreads) s_index[i] = c_tables.index[i];
+  const uint16_t *bits_tab = g_tables.bits;
+  const uint8_t *index_tab = g_tables.index;
   if (tid == 0) { s_flip = 0; s_qn = 0; }
-  __syncthreads();
 
   const int64_t tile_r = (int64_t)blockIdx.y * kTile;
   const int64_t tile_c = (int64_t)blockIdx.x * kTile;
   const int64_t bcols = C >> 2;
-  const int uc = tid & 15;
+  const int uc = tid & 7;
+  const int br = tid >> 3;
+  const int64_t r0 = tile_r + 4 * br;
+  const int64_t c0 = tile_c + 8 * uc;
+  const bool row_ok = r0 < R;
+  const bool ok0 = row_ok && c0 + 4 <= C;
+  const bool ok1 = row_ok && c0 + 8 <= C;
   const bool vec16 = (ldw & 7) == 0;  // rows 16-byte aligned: one 128-bit load per row of a unit
+  const int64_t bidx0 = (r0 >> 2) * bcols + (c0 >> 2);
 
-  // Phase 1: load both units, search the blocks the fast path can certify,
-  // queue the others (SEARCH) or read the given mask (!SEARCH).
-  uint32_t w[2][4][4];
+  // Every global load of the thread is issued before the first barrier.
+  uint32_t w[4][4];
+  load_unit(W, ldw, r0, c0, R, C, vec16, w);
+  uint32_t prev[2] = {0, 0}, given[2] = {kPadIndex, kPadIndex};
+  if (FLIP) {
+    if (ok0) prev[0] = idx_prev[bidx0];
+    if (ok1) prev[1] = idx_prev[bidx0 + 1];
+  }
+  if (!SEARCH) {
+    if (ok0) given[0] = idx[bidx0];
+    if (ok1) given[1] = idx[bidx0 + 1];
+  }
+  __syncthreads();
+
+  // Phase 1: search the blocks the fast path can certify and queue the others
+  // (SEARCH), or take the given mask (!SEARCH).
 #pragma unroll
-  for (int half = 0; half < 2; ++half)
-    load_unit(W, ldw, tile_r + 4 * ((tid >> 4) + 16 * half), tile_c + 8 * uc, R, C, vec16, w[half]);
+  for (int b = 0; b < 2; ++b) {
+    const bool ok = b ? ok1 : ok0;
+    uint32_t p = given[b];
+    if (SEARCH && ok) {
+      uint32_t blk[4][2];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int br = (tid >> 4) + 16 * half;
-    const int64_t r0 = tile_r + 4 * br;
-    const int64_t c0 = tile_c + 8 * uc;
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const bool ok = r0 < R && c0 + 4 * (b + 1) <= C;
-      uint32_t p = kPadIndex;
-      if (ok) {
-        if (SEARCH) {
-          uint32_t blk[4][2];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) { blk[i][0] = w[half][i][2 * b]; blk[i][1] = w[half][i][2 * b + 1]; }
-          p = search_block_fast<BF16>(blk, s_index);
-          if (p == kNeedsExact) {
-            const int slot = atomicAdd(&s_qn, 1);
-            s_queue[slot] = (uint16_t)(br * 32 + 2 * uc + b);
-          }
-        } else {
-          p = idx[(r0 >> 2) * bcols + (c0 >> 2) + b];
-        }
+      for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
+      p = search_block_fast<BF16>(blk, index_tab);
+      if (p == kNeedsExact) {
+        const int slot = atomicAdd(&s_qn, 1);
+        s_queue[slot] = (uint16_t)(br * kTileBlocks + 2 * uc + b);
       }
-      s_idx[br][2 * uc + b] = (uint8_t)p;
     }
+    s_idx[br][2 * uc + b] = (uint8_t)p;
   }
 
   // Phase 1b: blocks the fast path could not certify take the exact integer search.
   if (SEARCH) {
     __syncthreads();
+    // Queue entry k goes to lane k/4 of warp k%4, so a few entries run on
+    // different schedulers instead of side by side in one warp.
     const int qn = s_qn;
-    for (int k = tid; k < qn; k += kMaskThreads) {
+    for (int k = (tid >> 5) + 4 * (tid & 31); k < qn; k += kMaskThreads) {
       const int id = s_queue[k];
-      const int br = id >> 5, bc = id & 31;
-      const uint16_t *src = W + (tile_r + 4 * br) * ldw + tile_c + 4 * bc;
+      const int qbr = id / kTileBlocks, qbc = id % kTileBlocks;
+      const uint16_t *src = W + (tile_r + 4 * qbr) * ldw + tile_c + 4 * qbc;
       uint32_t blk[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src + i * ldw));
         blk[i][0] = q.x; blk[i][1] = q.y;
       }
-      s_idx[br][bc] = (uint8_t)search_block<BF16>(blk, s_index, s_bits);
+      s_idx[qbr][qbc] = (uint8_t)search_block<BF16>(blk, index_tab, bits_tab);
     }
   }
-  if (SEARCH || COMPRESS || FLIP) __syncthreads();
+  if (SEARCH) __syncthreads();
 
-  // Phase 2: per-thread outputs of its own blocks.
-  unsigned long long flips = 0;
+  // Phase 2: outputs of this thread's two blocks.
+  uint32_t p[2];
+  unsigned flips = 0;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int br = (tid >> 4) + 16 * half;
-    const int64_t r0 = tile_r + 4 * br;
-    const int64_t c0 = tile_c + 8 * uc;
-    const bool row_ok = r0 < R;
-    const bool ok0 = row_ok && c0 + 4 <= C;
-    const bool ok1 = row_ok && c0 + 8 <= C;
-    uint32_t p[2];
-    uint32_t x[4][4];  // the unit again (an L1 hit): keeps registers free during the search
-    if (COMPRESS) load_unit(W, ldw, r0, c0, R, C, vec16, x);
+  for (int b = 0; b < 2; ++b) {
+    p[b] = SEARCH ? s_idx[br][2 * uc + b] : given[b];
+    const bool ok = b ? ok1 : ok0;
+    if (SEARCH && ok) idx[bidx0 + b] = (uint8_t)p[b];
+    if (FLIP && ok) flips += __popc((uint32_t)(bits_tab[prev[b]] ^ bits_tab[p[b]]));
+  }
+  if (COMPRESS) {
+    uint32_t rc[2], cc[2];
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      p[b] = s_idx[br][2 * uc + b];
-      const bool ok = b ? ok1 : ok0;
-      const int64_t bidx = (r0 >> 2) * bcols + (c0 >> 2) + b;
-      if (SEARCH && ok) idx[bidx] = (uint8_t)p[b];
-      if (FLIP && ok) flips += __popc((uint32_t)(s_bits[idx_prev[bidx]] ^ s_bits[p[b]]));
+      rc[b] = g_tables.rowcode[p[b]];
+      cc[b] = g_tables.colcode[p[b]];
+      s_rc[br][2 * uc + b] = (uint16_t)rc[b];
+      s_cc[2 * uc + b][br] = (uint16_t)cc[b];
     }
-    if (COMPRESS && ok0) {
+    if (ok0) {
       // Forward operand: kept values of each row, in column order.
       if (vals_row) {
 #pragma unroll
@@ -366,8 +402,8 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
           uint32_t packed[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
-            const uint32_t nib = (s_rowcode[p[b]] >> (4 * i)) & 0xFu;
-            packed[b] = half_of(x[i], b, nib & 3u) | (half_of(x[i], b, nib >> 2) << 16);
+            const uint32_t nib = (rc[b] >> (4 * i)) & 0xFu;
+            packed[b] = half_of(w[i], b, nib & 3u) | (half_of(w[i], b, nib >> 2) << 16);
           }
           uint16_t *dst = vals_row + (r0 + i) * (C >> 1) + (c0 >> 1);
           if (ok1) *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
@@ -379,10 +415,10 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
       for (int b = 0; b < 2; ++b) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint32_t nib = (s_colcode[p[b]] >> (4 * j)) & 0xFu;
+          const uint32_t nib = (cc[b] >> (4 * j)) & 0xFu;
           const int word = 2 * b + (j >> 1);
-          const uint32_t lo = (pick_row(x, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
-          const uint32_t hi = (pick_row(x, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
+          const uint32_t lo = (pick_row(w, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
+          const uint32_t hi = (pick_row(w, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
           s_vcol[vcol_word(8 * uc + 4 * b + j, br)] = lo | (hi << 16);
         }
       }
@@ -390,56 +426,52 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
   }
 
   if (FLIP) {
-    const unsigned long long warp_sum = __reduce_add_sync(0xFFFFFFFFu, (unsigned)flips);
-    if ((tid & 31) == 0 && warp_sum) atomicAdd(&s_flip, warp_sum);
+    const unsigned warp_sum = __reduce_add_sync(0xFFFFFFFFu, flips);
+    if ((tid & 31) == 0 && warp_sum) atomicAdd(&s_flip, (unsigned long long)warp_sum);
   }
   if (COMPRESS || FLIP) __syncthreads();
   if (FLIP && tid == 0 && s_flip) atomicAdd(flip_count, s_flip);
 
   if (COMPRESS) {
-    // Transposed values: W column c (a row of W^T) holds 64 kept values per tile.
+    // Transposed values: W column c (a row of W^T) holds 32 kept values per tile.
     const int64_t half_rows = R >> 1;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < (kTile * 4) / kMaskThreads; ++k) {
       const int id = tid + kMaskThreads * k;
-      const int c_local = id >> 3, q = id & 7;
+      const int c_local = id >> 2, q = id & 3;
       if (vals_col && tile_c + c_local < C && tile_r + 16 * q + 16 <= R) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(
-            &s_vcol[c_local * 32 + (((q ^ (c_local >> 3)) & 7) << 2)]);
-        const bool swap = (c_local >> 6) & 1;
+        const uint4 v = *reinterpret_cast<const uint4 *>(&s_vcol[c_local * 16 + (((q ^ (c_local >> 3)) & 3) << 2)]);
+        const bool swap = (c_local >> 5) & 1;
         const uint4 o = swap ? make_uint4(v.z, v.w, v.x, v.y) : v;
         *reinterpret_cast<uint4 *>(vals_col + (tile_c + c_local) * half_rows + (tile_r >> 1) + 8 * q) = o;
       }
     }
-    // Metadata: one 2048-byte chunk per 128x128 tile and orientation.  Lane L,
+    // Metadata: one 2048-byte chunk per 128x128 region and orientation.  Lane L,
     // word kk (one 32-column K step of the MMA) holds rows m and m+8,
     // m = (L%8) + 16*(L/16), groups 4*((L/8)%2) .. +3 of that K step; the
     // low 16 bits are row m, the high 16 bits row m+8, one nibble per group.
-    const bool col_side = tid >= 128;
-    const int L = tid & 127;
-    const int m_lo = (L & 7) + ((L >> 4) << 4);
-    uint32_t words[4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int g = kk * 8 + ((L >> 3) & 1) * 4 + e;
-#pragma unroll
-        for (int hsel = 0; hsel < 2; ++hsel) {
-          const int m = m_lo + 8 * hsel;
-          uint32_t nib;
-          if (!col_side) nib = (s_rowcode[s_idx[m >> 2][g]] >> (4 * (m & 3))) & 0xFu;
-          else nib = (s_colcode[s_idx[g][m >> 2]] >> (4 * (m & 3))) & 0xFu;
-          word |= nib << (16 * hsel + 4 * e);
-        }
-      }
-      words[kk] = word;
+    // This tile is quadrant (rh, kh) of its chunk: lanes 64*rh.., words 2*kh..
+    // for the rows of W, lanes 64*kh.., words 2*rh.. for its columns.  Thread
+    // t builds word t%2 of lane t/2 of the quadrant on each side.
+    const int rh = (int)(blockIdx.y & 1), kh = (int)(blockIdx.x & 1);
+    const int lq = tid >> 1, kx = tid & 1;
+    const int m_lo = (lq & 7) + ((lq >> 4) << 4);   // row of the quadrant (0..55)
+    const int gq = kx * 8 + ((lq >> 3) & 1) * 4;     // first of four groups, in blocks of the quadrant
+    const int shift = m_lo & 3;
+    if (meta_row) {
+      const uint2 a = *reinterpret_cast<const uint2 *>(&s_rc[m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&s_rc[(m_lo >> 2) + 2][gq]);
+      const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
+      const size_t chunk = (size_t)(blockIdx.y >> 1) * (gridDim.x >> 1) + (blockIdx.x >> 1);
+      *reinterpret_cast<uint32_t *>(meta_row + chunk * 2048 + (64 * rh + lq) * 16 + 4 * (2 * kh + kx)) = word;
     }
-    uint8_t *dst = col_side
-                       ? (meta_col ? meta_col + ((size_t)blockIdx.x * gridDim.y + blockIdx.y) * 2048 + L * 16 : nullptr)
-                       : (meta_row ? meta_row + ((size_t)blockIdx.y * gridDim.x + blockIdx.x) * 2048 + L * 16 : nullptr);
-    if (dst) *reinterpret_cast<uint4 *>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+    if (meta_col) {
+      const uint2 a = *reinterpret_cast<const uint2 *>(&s_cc[m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&s_cc[(m_lo >> 2) + 2][gq]);
+      const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
+      const size_t chunk = (size_t)(blockIdx.x >> 1) * (gridDim.y >> 1) + (blockIdx.y >> 1);
+      *reinterpret_cast<uint32_t *>(meta_col + chunk * 2048 + (64 * kh + lq) * 16 + 4 * (2 * rh + kx)) = word;
+    }
   }
 }
 
@@ -447,9 +479,7 @@ __global__ void __launch_bounds__(kMaskThreads, 2) mask_tile_kernel(
 __global__ void __launch_bounds__(256) flip_count_kernel(const uint8_t *__restrict__ a,
                                                          const uint8_t *__restrict__ b, int64_t n,
                                                          unsigned long long *__restrict__ count) {
-  __shared__ uint16_t s_bits[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bits[i] = c_tables.bits[i];
-  __syncthreads();
+  const uint16_t *bits_tab = g_tables.bits;
   unsigned long long local = 0;
   const int64_t nvec = ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15) ? 0 : n / 16;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -462,46 +492,52 @@ __global__ void __launch_bounds__(256) flip_count_kernel(const uint8_t *__restri
     for (int k = 0; k < 16; ++k) {
       const uint32_t pa = (wa[k >> 2] >> (8 * (k & 3))) & 0xFFu;
       const uint32_t pb = (wb[k >> 2] >> (8 * (k & 3))) & 0xFFu;
-      local += __popc((uint32_t)(s_bits[pa] ^ s_bits[pb]));
+      local += __popc((uint32_t)(bits_tab[pa] ^ bits_tab[pb]));
     }
   }
   for (int64_t i = nvec * 16 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
-    local += __popc((uint32_t)(s_bits[a[i]] ^ s_bits[b[i]]));
+    local += __popc((uint32_t)(bits_tab[a[i]] ^ bits_tab[b[i]]));
   const unsigned warp_sum = __reduce_add_sync(0xFFFFFFFFu, (unsigned)local);
   if ((threadIdx.x & 31) == 0 && warp_sum) atomicAdd(count, (unsigned long long)warp_sum);
 }
 
-// Masked decay: one thread per 4x4 block; g <- fmaf(lambda, w, g) on pruned entries.
+// Masked decay: one thread per 4x4 block; g <- fmaf(lambda, w, g) on pruned
+// entries.  Grid: x covers the block columns in 256-thread strips, y walks the
+// block rows, so no thread divides.  A thread issues all nine loads of its
+// block (four 16-byte rows of g, four 8-byte rows of W, the pattern index)
+// before it computes, so each block costs one memory round trip.
 template <bool BF16>
 __global__ void __launch_bounds__(256) masked_decay_kernel(float *__restrict__ g,
                                                            const uint16_t *__restrict__ W,
                                                            const uint8_t *__restrict__ idx, int64_t R,
                                                            int64_t C, float lambda) {
-  __shared__ uint16_t s_bits[256];
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bits[i] = c_tables.bits[i];
-  __syncthreads();
+  const uint16_t *bits_tab = g_tables.bits;
   const int64_t bcols = C >> 2;
-  const int64_t nblocks = (R >> 2) * bcols;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
-    const int64_t r0 = (b / bcols) * 4, c0 = (b % bcols) * 4;
-    const uint32_t keep = s_bits[idx[b]];
+  const int64_t brows = R >> 2;
+  const int64_t bc = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (bc >= bcols) return;
+  for (int64_t br = blockIdx.y; br < brows; br += gridDim.y) {
+    const int64_t r0 = br * 4, c0 = bc * 4;
+    float4 gv[4];
+    uint2 wv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float4 *gp = reinterpret_cast<float4 *>(g + (r0 + i) * C + c0);
-      float4 gv = *gp;
-      const uint2 wv = __ldg(reinterpret_cast<const uint2 *>(W + (r0 + i) * C + c0));
-      const uint32_t hw[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
-      float wf[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        wf[j] = BF16 ? __uint_as_float(hw[j] << 16) : __half2float(__ushort_as_half((unsigned short)hw[j]));
-      float *gs = reinterpret_cast<float *>(&gv);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (!((keep >> (4 * i + j)) & 1u)) gs[j] = fmaf(lambda, wf[j], gs[j]);
-      *gp = gv;
+      gv[i] = *reinterpret_cast<const float4 *>(g + (r0 + i) * C + c0);
+      wv[i] = __ldg(reinterpret_cast<const uint2 *>(W + (r0 + i) * C + c0));
     }
+    const uint32_t keep = bits_tab[__ldg(idx + br * bcols + bc)];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t hw[4] = {wv[i].x & 0xFFFFu, wv[i].x >> 16, wv[i].y & 0xFFFFu, wv[i].y >> 16};
+      float *gs = reinterpret_cast<float *>(&gv[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float wf = BF16 ? __uint_as_float(hw[j] << 16) : __half2float(__ushort_as_half((unsigned short)hw[j]));
+        if (!((keep >> (4 * i + j)) & 1u)) gs[j] = fmaf(lambda, wf, gs[j]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) *reinterpret_cast<float4 *>(g + (r0 + i) * C + c0) = gv[i];
   }
 }
 

@@ -172,7 +172,9 @@ sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
 sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint8_t *idx, const uint8_t *prev,
                           unsigned long long *flip, void *vr, void *mr, void *vc, void *mc, cudaStream_t s) {
-  dim3 grid((unsigned)((C + kTile - 1) / kTile), (unsigned)((R + kTile - 1) / kTile));
+  // With COMPRESS the grid covers whole 128x128 metadata chunks (two tiles each way).
+  const int64_t g = COMPRESS ? 2 * kTile : kTile;
+  dim3 grid((unsigned)((C + g - 1) / g * (g / kTile)), (unsigned)((R + g - 1) / g * (g / kTile)));
   mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP><<<grid, kMaskThreads, 0, s>>>(
       static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
       static_cast<uint8_t *>(mr), static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc));
@@ -337,9 +339,9 @@ sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int6
   if (rows > 0 && cols > 0 && !aligned16(grad)) return SP24_ERR_MISALIGNED;
   if ((st = check_device()) != SP24_OK) return st;
   if (rows == 0 || cols == 0) return SP24_OK;
-  const int64_t nblocks = (rows / 4) * (cols / 4);
-  const int64_t want = (nblocks + 255) / 256;
-  const int grid = (int)(want < (int64_t)sm_count() * 16 ? want : (int64_t)sm_count() * 16);
+  const int64_t strips = (cols / 4 + 255) / 256;
+  const int64_t brows = rows / 4;
+  const dim3 grid((unsigned)strips, (unsigned)(brows < 65535 ? brows : 65535));
   cudaStream_t s = as_stream(stream);
   if (dtype == SP24_BF16)
     masked_decay_kernel<true><<<grid, 256, 0, s>>>(grad, static_cast<const uint16_t *>(W), idx, rows, cols, lambda);
