@@ -290,6 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or byte count
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  pdl_launch_dependents();
+  pdl_wait();  // the previous kernel's outputs (operands, pre-activations) are complete
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ producer (both CTAs)

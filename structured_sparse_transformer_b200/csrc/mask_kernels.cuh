@@ -207,7 +207,6 @@ constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 // (top rank, bottom rank) among the states reaching the global maximum wins.
 template <bool BF16>
 __device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2], const uint8_t *index_tab) {
-  constexpr PatternTables T = make_pattern_tables();
   float v[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
@@ -307,6 +306,8 @@ __global__ void __launch_bounds__(kMaskThreads, 8) mask_tile_kernel(
   const uint16_t *bits_tab = g_tables.bits;
   const uint8_t *index_tab = g_tables.index;
   if (tid == 0) { s_flip = 0; s_qn = 0; }
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int64_t tile_r = (int64_t)blockIdx.y * kTile;
   const int64_t tile_c = (int64_t)blockIdx.x * kTile;
@@ -480,6 +481,8 @@ __global__ void __launch_bounds__(256) flip_count_kernel(const uint8_t *__restri
                                                          const uint8_t *__restrict__ b, int64_t n,
                                                          unsigned long long *__restrict__ count) {
   const uint16_t *bits_tab = g_tables.bits;
+  pdl_launch_dependents();
+  pdl_wait();
   unsigned long long local = 0;
   const int64_t nvec = ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15) ? 0 : n / 16;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -512,6 +515,8 @@ __global__ void __launch_bounds__(256) masked_decay_kernel(float *__restrict__ g
                                                            const uint8_t *__restrict__ idx, int64_t R,
                                                            int64_t C, float lambda) {
   const uint16_t *bits_tab = g_tables.bits;
+  pdl_launch_dependents();
+  pdl_wait();
   const int64_t bcols = C >> 2;
   const int64_t brows = R >> 2;
   const int64_t bc = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;

@@ -90,6 +90,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// ------------------------------------------ programmatic dependent launch
+// Every kernel here is launched with programmatic stream serialisation: the
+// next kernel in the stream may be scheduled (and run its prologue) while
+// this one drains.  pdl_wait blocks until the preceding kernel in the stream
+// has completed and its memory is visible, so it comes before the first
+// global-memory access; without a programmatic predecessor it returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------ TMA and bulk copy
 
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,

@@ -36,8 +36,27 @@ sp24_status check_device() {
   return major == 10 ? SP24_OK : SP24_ERR_NO_DEVICE;
 }
 
-sp24_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while its predecessor in the stream drains; each kernel here calls
+// griddepcontrol.wait before its first global-memory access.
+template <typename... KArgs, typename... Args>
+sp24_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return SP24_ERR_CUDA;
+  }
+  return SP24_OK;
 }
 
 int sm_count() {
@@ -133,9 +152,8 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   }
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + kPairBN - 1) / kPairBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
-  kernel<<<2 * pairs, kGemmThreads, smem_bytes, stream>>>(ta, tb, tm, to, tx, (int)M, (int)T, num_kt,
-                                                         g_wait_budget.load());
-  return launch_status();
+  return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
+                    (int)T, num_kt, (uint64_t)g_wait_budget.load());
 }
 
 sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
@@ -175,10 +193,9 @@ sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint
   // With COMPRESS the grid covers whole 128x128 metadata chunks (two tiles each way).
   const int64_t g = COMPRESS ? 2 * kTile : kTile;
   dim3 grid((unsigned)((C + g - 1) / g * (g / kTile)), (unsigned)((R + g - 1) / g * (g / kTile)));
-  mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP><<<grid, kMaskThreads, 0, s>>>(
-      static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
-      static_cast<uint8_t *>(mr), static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc));
-  return launch_status();
+  return launch_pdl(mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP>, grid, dim3(kMaskThreads), 0, s,
+                    static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
+                    static_cast<uint8_t *>(mr), static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc));
 }
 
 template <bool SEARCH, bool COMPRESS, bool FLIP>
@@ -343,11 +360,9 @@ sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int6
   const int64_t brows = rows / 4;
   const dim3 grid((unsigned)strips, (unsigned)(brows < 65535 ? brows : 65535));
   cudaStream_t s = as_stream(stream);
-  if (dtype == SP24_BF16)
-    masked_decay_kernel<true><<<grid, 256, 0, s>>>(grad, static_cast<const uint16_t *>(W), idx, rows, cols, lambda);
-  else
-    masked_decay_kernel<false><<<grid, 256, 0, s>>>(grad, static_cast<const uint16_t *>(W), idx, rows, cols, lambda);
-  return launch_status();
+  const uint16_t *w16 = static_cast<const uint16_t *>(W);
+  return dtype == SP24_BF16 ? launch_pdl(masked_decay_kernel<true>, grid, dim3(256), 0, s, grad, w16, idx, rows, cols, lambda)
+                            : launch_pdl(masked_decay_kernel<false>, grid, dim3(256), 0, s, grad, w16, idx, rows, cols, lambda);
 }
 
 sp24_status sp24_flip_rate(const uint8_t *idx_prev, const uint8_t *idx_cur, int64_t nblocks,
@@ -360,8 +375,7 @@ sp24_status sp24_flip_rate(const uint8_t *idx_prev, const uint8_t *idx_cur, int6
   if (nblocks == 0) return SP24_OK;
   const int64_t want = (nblocks / 16 + 255) / 256 + 1;
   const int grid = (int)(want < (int64_t)sm_count() * 8 ? want : (int64_t)sm_count() * 8);
-  flip_count_kernel<<<grid, 256, 0, s>>>(idx_prev, idx_cur, nblocks, d_count);
-  return launch_status();
+  return launch_pdl(flip_count_kernel, dim3(grid), dim3(256), 0, s, idx_prev, idx_cur, nblocks, d_count);
 }
 
 sp24_status sp24_meta_to_canonical(const void *meta_dev_layout_host, int64_t rows, int64_t cols, uint16_t *canon) {
