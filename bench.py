@@ -344,14 +344,18 @@ def run_e2e(args, step, wl, world, dev, barrier):
     memory and D2H of its results inside the timed region."""
     import torch
     h = {k: v.pin_memory() for k, v in step.host.items()}
+    # The weights a host would send change every step: alternate the seeded
+    # weights with their perturbed copies, so the masks flip as in training.
+    hw = [[h["W1"], step.W[0][1].cpu().pin_memory()], [h["W2"], step.W[1][1].cpu().pin_memory()]]
     out_y = torch.empty(step.Y.shape, dtype=step.Y.dtype).pin_memory()
     out_dx = torch.empty(step.dX.shape, dtype=step.dX.dtype).pin_memory()
     out_g = [torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in step.G]
     out_f = torch.empty(2, dtype=torch.int64).pin_memory()
 
     def one():
-        step.W[0][step.step_no % 2].copy_(h["W1"], non_blocking=True)
-        step.W[1][step.step_no % 2].copy_(h["W2"], non_blocking=True)
+        slot = step.step_no % 2
+        step.W[0][slot].copy_(hw[0][slot], non_blocking=True)
+        step.W[1][slot].copy_(hw[1][slot], non_blocking=True)
         step.X.copy_(h["X"], non_blocking=True)
         step.dY.copy_(h["dY"], non_blocking=True)
         step.G[0].copy_(h["G1"], non_blocking=True)

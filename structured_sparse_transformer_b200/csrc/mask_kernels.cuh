@@ -8,17 +8,18 @@
 //     search, pruning and masked decay kernels);
 //   - abstract (flip rate; masked decay term on gradients).
 //
-// Mask search is exact.  The fast path sums magnitudes in fp32 where the
-// block's magnitude range proves those sums exact (search_block_fast); the
-// remaining blocks take an integer search.  There each |w| becomes an integer multiple of its dtype's
-// smallest subnormal (fp16: always; bf16: relative to the block's largest
-// exponent, 32 binades deep), pre-shifted left by 12 bits.  The 12 low bits of
-// a pattern's key hold (35 - top rank) << 6 | (35 - bottom rank), so one
-// unsigned 64-bit max picks the largest exact sum and, among equal sums, the
-// lowest pattern index.  The max over the 90 patterns is taken by a dynamic
-// program over column-count states (top rows 0-1 and bottom rows 2-3, see
-// sp24_tables.cuh) instead of enumerating all 90.  bf16 blocks whose nonzero
-// magnitudes span more than 32 binades take an exact multi-word brute force.
+// Mask search is exact.  The fast path sums magnitudes in fp64, which holds
+// every pattern sum of a fp16 block exactly, and of a bf16 block whose nonzero
+// magnitudes span at most 42 binades (search_block_fast).  The remaining bf16
+// blocks take an integer search: each |w| becomes an integer multiple of the
+// smallest subnormal relative to the block's largest exponent (32 binades
+// deep), pre-shifted left by 12 bits; the 12 low bits of a pattern's key hold
+// (35 - top rank) << 6 | (35 - bottom rank), so one unsigned 64-bit max picks
+// the largest exact sum and, among equal sums, the lowest pattern index.
+// Both take the max over the 90 patterns by a dynamic program over
+// column-count states (top rows 0-1 and bottom rows 2-3, see sp24_tables.cuh)
+// instead of enumerating all 90.  bf16 blocks whose nonzero magnitudes span
+// more than 32 binades take an exact multi-word brute force.
 #pragma once
 #include "sp24_common.cuh"
 #include "sp24_tables.cuh"
@@ -150,7 +151,7 @@ __device__ __forceinline__ uint32_t dp_state_key(const Real (&v)[16]) {
 
 // Pattern index of one 4x4 block given as 4 rows x 2 words (two 16-bit values each).
 template <bool BF16>
-__device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], const uint8_t *index_tab,
+__device__ __noinline__ uint32_t search_block(const uint32_t (&w)[4][2], const uint8_t *index_tab,
                                                  const uint16_t *bits_tab) {
   u64 v[16];
   if (!BF16) {
@@ -196,12 +197,14 @@ __device__ __forceinline__ uint32_t search_block(const uint32_t (&w)[4][2], cons
 
 constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 
-// Fast path of the search on fp32 arithmetic.  Every |w| converts to fp32
-// exactly.  A sum of eight of them is exact in fp32 when the block's smallest
-// nonzero magnitude is at least its largest times 2^-10 (fp16: 11-bit
-// significands, 3 carry bits, 24-bit fp32 significand) or 2^-13 (bf16); then
-// every partial sum below is exact, comparisons are exact, and the result
-// equals the exact search.  Blocks that fail the test return kNeedsExact.
+// Fast path of the search, on fp64 sums.  fp16: every |w| is an integer
+// multiple of 2^-24 below 2^17, so a sum of eight needs at most 44
+// significant bits and fp64 holds every partial sum exactly: the search is
+// exact for every block.  bf16: 8-bit significands and 3 carry bits fit the
+// 53-bit fp64 significand when the block's smallest nonzero magnitude is at
+// least its largest times 2^-42 (when that bound underflows fp32, every
+// magnitude is below 2^-84 and the sums still fit above the 2^-133
+// subnormal step); blocks that fail return kNeedsExact for the integer search.
 // Ranks: within a column-count state the first combo (lowest rank) reaching
 // the state's maximum wins (strict >); across states the smallest
 // (top rank, bottom rank) among the states reaching the global maximum wins.
@@ -213,14 +216,19 @@ __device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2],
     const uint32_t h = (w[c >> 2][(c >> 1) & 1] >> ((c & 1) << 4)) & 0x7FFFu;
     v[c] = BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
   }
-  float vmax = v[0], vmin = v[0] > 0.0f ? v[0] : __int_as_float(0x7F800000);
+  if (BF16) {
+    float vmax = v[0], vmin = v[0] > 0.0f ? v[0] : __int_as_float(0x7F800000);
 #pragma unroll
-  for (int c = 1; c < 16; ++c) {
-    vmax = fmaxf(vmax, v[c]);
-    vmin = fminf(vmin, v[c] > 0.0f ? v[c] : __int_as_float(0x7F800000));
+    for (int c = 1; c < 16; ++c) {
+      vmax = fmaxf(vmax, v[c]);
+      vmin = fminf(vmin, v[c] > 0.0f ? v[c] : __int_as_float(0x7F800000));
+    }
+    if (!(vmin >= vmax * 0x1p-42f)) return kNeedsExact;
   }
-  if (!(vmin >= vmax * (BF16 ? 0x1p-13f : 0x1p-10f))) return kNeedsExact;
-  const uint32_t key = dp_state_key<float>(v);
+  double d[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) d[c] = (double)v[c];
+  const uint32_t key = dp_state_key<double>(d);
   return index_tab[(key >> 6) * 36 + (key & 63)];
 }
 
@@ -289,7 +297,7 @@ __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
 //             (values + tensor-core metadata)
 //   FLIP:     add the number of mask bits that differ from idx_prev to *flip_count
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, 8) mask_tile_kernel(
+__global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
     const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
@@ -336,27 +344,28 @@ __global__ void __launch_bounds__(kMaskThreads, 8) mask_tile_kernel(
   }
   __syncthreads();
 
-  // Phase 1: search the blocks the fast path can certify and queue the others
-  // (SEARCH), or take the given mask (!SEARCH).
+  // Phase 1: search (SEARCH), or take the given mask (!SEARCH).  bf16 blocks
+  // the fast path cannot certify are queued for the exact integer search.
+  uint32_t p[2];
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     const bool ok = b ? ok1 : ok0;
-    uint32_t p = given[b];
+    p[b] = given[b];
     if (SEARCH && ok) {
       uint32_t blk[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
-      p = search_block_fast<BF16>(blk, index_tab);
-      if (p == kNeedsExact) {
+      p[b] = search_block_fast<BF16>(blk, index_tab);
+      if (BF16 && p[b] == kNeedsExact) {
         const int slot = atomicAdd(&s_qn, 1);
         s_queue[slot] = (uint16_t)(br * kTileBlocks + 2 * uc + b);
       }
     }
-    s_idx[br][2 * uc + b] = (uint8_t)p;
+    if (SEARCH && BF16) s_idx[br][2 * uc + b] = (uint8_t)p[b];
   }
 
-  // Phase 1b: blocks the fast path could not certify take the exact integer search.
-  if (SEARCH) {
+  // Phase 1b (bf16): blocks the fast path could not certify take the exact integer search.
+  if (SEARCH && BF16) {
     __syncthreads();
     // Queue entry k goes to lane k/4 of warp k%4, so a few entries run on
     // different schedulers instead of side by side in one warp.
@@ -373,15 +382,15 @@ __global__ void __launch_bounds__(kMaskThreads, 8) mask_tile_kernel(
       }
       s_idx[qbr][qbc] = (uint8_t)search_block<BF16>(blk, index_tab, bits_tab);
     }
+    __syncthreads();
+#pragma unroll
+    for (int b = 0; b < 2; ++b) p[b] = s_idx[br][2 * uc + b];
   }
-  if (SEARCH) __syncthreads();
 
   // Phase 2: outputs of this thread's two blocks.
-  uint32_t p[2];
   unsigned flips = 0;
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
-    p[b] = SEARCH ? s_idx[br][2 * uc + b] : given[b];
     const bool ok = b ? ok1 : ok0;
     if (SEARCH && ok) idx[bidx0 + b] = (uint8_t)p[b];
     if (FLIP && ok) flips += __popc((uint32_t)(bits_tab[prev[b]] ^ bits_tab[p[b]]));
