@@ -513,45 +513,59 @@ __global__ void __launch_bounds__(256) flip_count_kernel(const uint8_t *__restri
   if ((threadIdx.x & 31) == 0 && warp_sum) atomicAdd(count, (unsigned long long)warp_sum);
 }
 
-// Masked decay: one thread per 4x4 block; g <- fmaf(lambda, w, g) on pruned
-// entries.  Grid: x covers the block columns in 256-thread strips, y walks the
-// block rows, so no thread divides.  A thread issues all nine loads of its
-// block (four 16-byte rows of g, four 8-byte rows of W, the pattern index)
-// before it computes, so each block costs one memory round trip.
+// Masked decay: g <- fmaf(lambda, w, g) on pruned entries.  Thread t of
+// CTA (x, y) owns the 4x4 block at block column 256x + t of block rows
+// y, y + gridDim.y, ...; no thread divides.  The block's four 16-byte rows of
+// g and 8-byte rows of W travel by cp.async into the thread's own shared
+// slots, so the bytes in flight do not occupy registers and every block of a
+// 355M-size weight is in flight in one wave.  A thread reads back only its
+// own slots, so no barrier is needed.
+__device__ __forceinline__ void cp_async(void *smem_dst, const void *gmem_src, int bytes16or8) {
+  if (bytes16or8 == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(256) masked_decay_kernel(float *__restrict__ g,
                                                            const uint16_t *__restrict__ W,
                                                            const uint8_t *__restrict__ idx, int64_t R,
                                                            int64_t C, float lambda) {
+  __shared__ __align__(16) float4 s_g[4][256];
+  __shared__ __align__(16) uint2 s_w[4][256];
   const uint16_t *bits_tab = g_tables.bits;
   pdl_launch_dependents();
   pdl_wait();
+  const int t = threadIdx.x;
   const int64_t bcols = C >> 2;
   const int64_t brows = R >> 2;
-  const int64_t bc = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t bc = (int64_t)blockIdx.x * blockDim.x + t;
   if (bc >= bcols) return;
   for (int64_t br = blockIdx.y; br < brows; br += gridDim.y) {
-    const int64_t r0 = br * 4, c0 = bc * 4;
-    float4 gv[4];
-    uint2 wv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      gv[i] = *reinterpret_cast<const float4 *>(g + (r0 + i) * C + c0);
-      wv[i] = __ldg(reinterpret_cast<const uint2 *>(W + (r0 + i) * C + c0));
+      const int64_t off = (4 * br + i) * C + 4 * bc;
+      cp_async(&s_g[i][t], g + off, 16);
+      cp_async(&s_w[i][t], W + off, 8);
     }
-    const uint32_t keep = bits_tab[__ldg(idx + br * bcols + bc)];
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const uint32_t p = __ldg(idx + br * bcols + bc);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    const uint32_t keep = bits_tab[p];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t hw[4] = {wv[i].x & 0xFFFFu, wv[i].x >> 16, wv[i].y & 0xFFFFu, wv[i].y >> 16};
-      float *gs = reinterpret_cast<float *>(&gv[i]);
+      float4 gv = s_g[i][t];
+      const uint2 wv = s_w[i][t];
+      const uint32_t hw[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
+      float *gs = reinterpret_cast<float *>(&gv);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float wf = BF16 ? __uint_as_float(hw[j] << 16) : __half2float(__ushort_as_half((unsigned short)hw[j]));
         if (!((keep >> (4 * i + j)) & 1u)) gs[j] = fmaf(lambda, wf, gs[j]);
       }
+      *reinterpret_cast<float4 *>(g + (4 * br + i) * C + 4 * bc) = gv;
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) *reinterpret_cast<float4 *>(g + (r0 + i) * C + c0) = gv[i];
   }
 }
 
