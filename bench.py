@@ -218,6 +218,34 @@ class FFNStep:
                                                                       wl.lam))
         self.step_no += 1
 
+    def run_dense(self, events=None):
+        """One step of the dense fine-tuning phase (the last 1/6 of the steps):
+        W^T of both weights (they change every step), the four FFN products on
+        the dense tensor-core path; no mask, compression or decay."""
+        sp, torch = self.sp, self.torch
+        cur = self.step_no % 2
+        if not hasattr(self, "Wt"):
+            self.Wt = [torch.empty(w[0].shape[1], w[0].shape[0], dtype=w[0].dtype, device="cuda") for w in self.W]
+
+        def timed(name, fn):
+            if events is None:
+                fn()
+                return
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn()
+            e.record()
+            events.setdefault(name, []).append((s, e))
+
+        for li in range(2):
+            timed("transpose", lambda li=li: sp.sp24_transpose(self.W[li][cur], self.Wt[li]))
+        W1, W2 = self.W[0][cur], self.W[1][cur]
+        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu", self.Hpre))
+        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
+        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "dgelu", self.Hpre))
+        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
+        self.step_no += 1
+
     # algorithmic bytes / flops per launch of each kernel
     def work(self):
         wl = self.wl
@@ -280,6 +308,7 @@ def run_ours(args, wl, rank, world, local_rank):
         flush.fill_(1.0)
         step.run(events)
     barrier()
+    dense = run_dense_phase(args, step, wl, world, dev, flush, barrier)
     total_ms = max_over_ranks(step_ms, world, dev)
     ms_per_step = total_ms / args.steps
     flops = wl.gemm_flops()
@@ -328,6 +357,7 @@ def run_ours(args, wl, rank, world, local_rank):
                                  "traffic": args.mask_traffic or load_traffic("mask_step", wl.name),
                                  "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
         "kernels": kernels,
+        "dense_finetune_step": dense,
         "e2e": e2e,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
@@ -337,6 +367,50 @@ def run_ours(args, wl, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_tokens)
     return line
+
+
+def run_dense_phase(args, step, wl, world, dev, flush, barrier):
+    """The dense fine-tuning step, timed like the 2:4 step (back to back, L2
+    flushed outside the step events), and its GEMMs from an instrumented pass."""
+    import torch
+    import structured_sparse_transformer_b200 as sp
+    for _ in range(args.warmup):
+        step.run_dense()
+    step_ev = []
+    barrier()
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step.run_dense()
+        e.record()
+        step_ev.append((s, e))
+    barrier()
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), world, dev) / args.steps
+    events = {}
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        step.run_dense(events)
+    barrier()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the dense phase: {sp.sp24_status_string(st)}")
+    peaks, _ = load_peaks()
+    g = [s.elapsed_time(e) * 1e-3 for s, e in events["gemm_dense"]]
+    t = [s.elapsed_time(e) * 1e-3 for s, e in events["transpose"]]
+    g_avg = sum(g) / len(g)
+    ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
+    n_el = wl.d * wl.ff
+    t_avg = sum(t) / len(t)
+    return {"ms_per_step": round(ms, 4),
+            "value": round(wl.gemm_flops() * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "gemm": {"launches": len(g), "avg_us": round(g_avg * 1e6, 2), "achieved": round(ach, 1),
+                     "peak": peaks["bf16_tflops"], "frac": round(ach / peaks["bf16_tflops"], 4)},
+            "transpose": {"launches": len(t), "avg_us": round(t_avg * 1e6, 2),
+                          "achieved": round(4 * n_el / t_avg / 1e9, 1), "unit": "GB/s",
+                          "peak": peaks["hbm_gbs"], "frac": round(4 * n_el / t_avg / 1e9 / peaks["hbm_gbs"], 4)},
+            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights and the four FFN "
+                    "products on the dense tcgen05 path, same workload"}
 
 
 def run_e2e(args, step, wl, world, dev, barrier):

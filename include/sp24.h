@@ -157,6 +157,30 @@ SP24_API sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const
                             sp24_epilogue epi, const void *aux, void *stream);
 
 /*
+ * Dense GEMM for the dense fine-tuning phase (abstract: a dense fine-tuning
+ * procedure near the end of pre-training; Experiment Setup row: the last 1/6
+ * of the total steps), on the same tcgen05 pipeline as the 2:4 GEMMs:
+ *   out[T x M] = B[T x Kd] * A[M x Kd]^T
+ * forward:        B = X  [T x K], A = W   [N x K]  (epi NONE or GELU)
+ * input gradient: B = dY [T x N], A = W^T [K x N]  (epi NONE or DGELU;
+ *                 W^T from sp24_transpose)
+ *   B, A, out  device, row-major, contiguous; aux as in sp24_gemm_fwd (GELU:
+ *              written with the pre-activation) or sp24_gemm_dgrad (DGELU: read)
+ * fp32 accumulation; outputs rounded to dtype.  Kd % 16 == 0, M % 16 == 0,
+ * T >= 0.  All pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A, int64_t M,
+                            sp24_dtype dtype, void *out, sp24_epilogue epi, void *aux, void *stream);
+
+/*
+ * out[cols x rows] = in[rows x cols]^T for 16-bit elements (bit copy): the
+ * input-gradient operand W^T of the dense fine-tuning GEMM.
+ *   in, out  device, row-major, contiguous, not overlapping; rows, cols >= 0
+ */
+SP24_API sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtype dtype, void *out,
+                           void *stream);
+
+/*
  * Masked decay on gradients (abstract; masked decay kernel of the Software
  * Dependencies row): grad <- grad + lambda * W where the mask is 0, unchanged
  * where it is 1, as one fp32 fused multiply-add per pruned entry (in place).

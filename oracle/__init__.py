@@ -205,6 +205,19 @@ def sparse_dgrad(dy: np.ndarray, w: np.ndarray, keep: np.ndarray) -> np.ndarray:
     return np.asarray(dy, np.float64) @ np.where(keep, w, 0.0)
 
 
+def dense_fwd(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """fp64 ``Y = X W^T`` for X [T, K] and W [N, K]: the FFN forward product of
+    the dense fine-tuning phase ("Accelerating Transformer Pre-training with 2:4
+    Sparsity", abstract: dense fine-tuning near the end of pre-training;
+    Experiment Setup row: the last 1/6 of the total steps), where no mask applies."""
+    return np.asarray(x, np.float64) @ np.asarray(w, np.float64).T
+
+
+def dense_dgrad(dy: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """fp64 ``dX = dY W`` for dY [T, N] and W [N, K] (dense fine-tuning phase)."""
+    return np.asarray(dy, np.float64) @ np.asarray(w, np.float64)
+
+
 def gelu(x: np.ndarray) -> np.ndarray:
     """GELU, exact erf form ``0.5 x (1 + erf(x / sqrt 2))``, fp64."""
     from scipy.special import erf

@@ -6,12 +6,13 @@ helpers), passes their data pointers, sizes and the current CUDA stream, and
 raises ``Sp24Error`` on a non-OK status.  Every step of the computation runs in
 the library's kernels; there is no fallback of any kind.  Importing the package
 raises if ``libsp24.so`` is missing: build it with
-``python -m structured_sparse_transformer_b200.build``.
+``python structured_sparse_transformer_b200/build.py``.
 
 Operations from "Accelerating Transformer Pre-training with 2:4 Sparsity":
 transposable 2:4 mask search (reproducibility table, Pseudocode row,
 Algorithm 1), pruning/compression and the 2:4 sparse FFN GEMMs (Software
-Dependencies row), masked decay and flip rate (abstract).
+Dependencies row), masked decay and flip rate (abstract), and the dense GEMM
+of the dense fine-tuning phase (abstract; Experiment Setup row).
 """
 from __future__ import annotations
 
@@ -22,7 +23,7 @@ _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG_DIR, "libsp24.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing; build it with `python -m structured_sparse_transformer_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing; build it with `python structured_sparse_transformer_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -35,6 +36,8 @@ _SIGNATURES = {
     "sp24_mask_step": [P, I32, I64, I64, I64, P, P, P, P, P, P, P, P],
     "sp24_gemm_fwd": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
     "sp24_gemm_dgrad": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
+    "sp24_gemm_dense": [P, I64, I64, P, I64, I32, P, I32, P, P],
+    "sp24_transpose": [P, I64, I64, I32, P, P],
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
     "sp24_flip_rate": [P, P, I64, P, P],
     "sp24_meta_to_canonical": [P, I64, I64, P],
@@ -181,6 +184,23 @@ def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stre
     _check("sp24_gemm_dgrad",
            _lib.sp24_gemm_dgrad(_ptr(dY), T, N, _ptr(vals_col), _ptr(meta_col), K, _dtype_code(dY), _ptr(dX),
                                 EPILOGUES[epi], _ptr(aux), _stream(stream)))
+
+
+def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
+    """out[T, M] <- B[T, Kd] A[M, Kd]^T on the dense tensor-core path; epi None, 'gelu' or 'dgelu'."""
+    _need_cuda(B, A, out, aux)
+    T, Kd = B.shape
+    M = A.shape[0]
+    _check("sp24_gemm_dense",
+           _lib.sp24_gemm_dense(_ptr(B), T, Kd, _ptr(A), M, _dtype_code(B), _ptr(out), EPILOGUES[epi], _ptr(aux),
+                                _stream(stream)))
+
+
+def sp24_transpose(x, out, stream=None):
+    """out[C, R] <- x[R, C]^T (16-bit elements, bit copy)."""
+    _need_cuda(x, out)
+    R, C = x.shape
+    _check("sp24_transpose", _lib.sp24_transpose(_ptr(x), R, C, _dtype_code(x), _ptr(out), _stream(stream)))
 
 
 def sp24_masked_decay(grad, W, idx, lam: float, stream=None):

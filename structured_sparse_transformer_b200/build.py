@@ -1,6 +1,7 @@
 """Build step of libsp24.so: one nvcc invocation for sm_100a, output in-tree.
 
-Run as ``python -m structured_sparse_transformer_b200.build`` or call
+Run as ``python structured_sparse_transformer_b200/build.py`` (by path, so the
+package, which loads the library, is not imported first) or call
 ``build_library()``.  Rebuilds only when a source or the public header is newer
 than the library.
 """

@@ -54,8 +54,6 @@
 
 namespace sp24 {
 
-constexpr int kGemmBK = 128;                           // logical K per pipeline stage
-constexpr int kGemmBKc = kGemmBK / 2;                  // kept values per stage and row
 constexpr int kEpiWarps = 12;                          // epilogue warps: 3 per TMEM lane quadrant
 constexpr int kEpiGroups = kEpiWarps / 4;              // warp groups taking alternate chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
@@ -67,13 +65,24 @@ constexpr uint64_t kDrainBudget = 1ull << 26;
 constexpr int kPairRows = 128;                         // compressed-operand rows per CTA
 constexpr int kPairBN = 224;                           // tokens per pair tile
 constexpr int kPairBNh = kPairBN / 2;                  // token rows per CTA
-constexpr int kPairSmemA = kPairRows * kGemmBKc * 2;   // 16 KB
-constexpr int kPairSmemBBox = kPairBNh * 64 * 2;       // 14 KB
-constexpr int kPairSmemB = 2 * kPairSmemBBox;
-constexpr int kPairStageBytes = kPairSmemA + kPairSmemB + kSmemE;   // 46 KB
-constexpr int kPairStages = 4;
+constexpr int kPairSmemA = kPairRows * 64 * 2;        // 16 KB: 128 rows x 64 values (128B swizzle)
+constexpr int kPairSmemBBox = kPairBNh * 64 * 2;       // 14 KB: 112 token rows x 64 K
 constexpr int kPairChunks = kPairBN / kEpiTokens;      // 14
 constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at columns 0 and 224
+
+// Pipeline stage of the 2:4 GEMM (SPARSE) and of the dense GEMM of the dense
+// fine-tuning phase.  Sparse: 128 logical K per stage = 64 kept values of A,
+// two 64-K boxes of B and the 2 KB metadata chunk (46 KB), 4 stages.  Dense:
+// 64 K per stage, one box of A and one of B (30 KB), 6 stages.
+template <bool SPARSE>
+struct PairGeom {
+  static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
+  static constexpr int kAcols = 64;                      // A values per row and stage
+  static constexpr int kBBoxes = SPARSE ? 2 : 1;
+  static constexpr int kMeta = SPARSE ? kSmemE : 0;
+  static constexpr int kStageBytes = kPairSmemA + kBBoxes * kPairSmemBBox + kMeta;
+  static constexpr int kStages = SPARSE ? 4 : 6;
+};
 constexpr int kEpiBufBytes = kEpiTokens * 32 * 2;      // staging tile: 16 tokens x 32 features, 64B-swizzled
 constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM address, abort flag
 
@@ -82,13 +91,18 @@ enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
 // Staging tiles per epilogue warp: out; out + pre-activation; out + two
 // pre-activation inputs.
 __host__ __device__ constexpr int epi_bufs(int epi) { return epi == kEpiNone ? 1 : (epi == kEpiGelu ? 2 : 3); }
+template <bool SPARSE>
 __host__ __device__ constexpr int pair_smem_bytes(int epi) {
-  return kPairStages * kPairStageBytes + kEpiWarps * epi_bufs(epi) * kEpiBufBytes + kPairBarBytes + 1024;
+  return PairGeom<SPARSE>::kStages * PairGeom<SPARSE>::kStageBytes + kEpiWarps * epi_bufs(epi) * kEpiBufBytes +
+         kPairBarBytes + 1024;
 }
-static_assert(pair_smem_bytes(kEpiDgelu) <= 232448, "shared memory per CTA");
-static_assert(kPairStageBytes % 1024 == 0 && kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
+static_assert(pair_smem_bytes<true>(kEpiDgelu) <= 232448 && pair_smem_bytes<false>(kEpiDgelu) <= 232448,
+              "shared memory per CTA");
+static_assert(PairGeom<true>::kStageBytes % 1024 == 0 && PairGeom<false>::kStageBytes % 1024 == 0 &&
+                  kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
-static_assert(kPairMetaCol + 4 * kPairStages <= kTmemCols, "tensor memory budget");
+static_assert(kPairMetaCol + 4 * PairGeom<true>::kStages <= kTmemCols, "tensor memory budget");
+static_assert(2 * PairGeom<false>::kStages + 16 + 2 * kEpiWarps <= kPairBarBytes / 8, "barrier space");
 
 // GELU (exact erf form) and its derivative for the epilogues:
 //   gelu(x) = x Phi(x),  gelu'(x) = Phi(x) + x phi(x),
@@ -235,12 +249,15 @@ __device__ __forceinline__ void unpack2(uint32_t v, float &lo, float &hi) {
   }
 }
 
-template <bool BF16, int EPI>
+template <bool BF16, int EPI, bool SPARSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
                           const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
                           uint64_t wait_budget) {
+  using G = PairGeom<SPARSE>;
+  constexpr int kPairStages = G::kStages;
+  constexpr int kPairStageBytes = G::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *stage_base = smem;
@@ -253,7 +270,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t *drain = acc_empty + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
-  uint64_t *aux_bars = bars + 16;                 // [kEpiWarps][2] dGELU pre-activation tiles
+  uint64_t *aux_bars = bars + 2 * kPairStages + 8;  // [kEpiWarps][2] dGELU pre-activation tiles
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -277,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     fence_mbarrier_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
-    prefetch_tensormap(&tm_meta);
+    if (SPARSE) prefetch_tensormap(&tm_meta);
     prefetch_tensormap(&tm_out);
     if (EPI != kEpiNone) prefetch_tensormap(&tm_aux);
   }
@@ -312,10 +329,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         uint8_t *st = stage_base + s * kPairStageBytes;
         if (is_leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
-        tma_load_2d_pair(st, &tm_a, &full[s], kt * kGemmBKc, a_row);
-        tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * kGemmBK, b_row);
-        tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * kGemmBK + 64, b_row);
-        tma_load_2d_pair(st + kPairSmemA + kPairSmemB, &tm_meta, &full[s], 0, chunk_row + kt);
+        tma_load_2d_pair(st, &tm_a, &full[s], kt * G::kAcols, a_row);
+        tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
+        if (SPARSE) {
+          tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * G::kBK + 64, b_row);
+          tma_load_2d_pair(st + kPairSmemA + 2 * kPairSmemBBox, &tm_meta, &full[s], 0, chunk_row + kt);
+        }
       }
     }
     // The leader's `full` barriers count both CTAs' bytes: let every copy land.
@@ -329,10 +348,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------- MMA issuer (leader)
     // Descriptors of stage 0; stage s and K step kk only move the 14-bit start
     // address field (all of shared memory is below 2^18 bytes, so it never carries).
-    constexpr uint32_t idesc = make_idesc_sparse(BF16, 2 * kPairRows, kPairBN);
+    constexpr uint32_t idesc =
+        SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN) : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
     const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), 16, 1024, kSwizzle128B);
-    const uint64_t e_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA + kPairSmemB), 128, 128, kSwizzleNone);
+    const uint64_t e_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA + 2 * kPairSmemBBox), 128, 128, kSwizzleNone);
     uint32_t g = 0;
     bool ok = true;
     int j = 0;
@@ -347,15 +367,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (!(ok = mbar_wait_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((s * kPairStageBytes) >> 4);
-        const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
-        tc_cp_128x128b_pair(t_meta, e_desc0 + so);
         const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
-        // The metadata operand address must be 2-column aligned; the low column
-        // bit travels in the descriptor's sparsity-selector field instead.
-        tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != 0 ? 1u : 0u);
-        tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
-        tc_mma_sp_f16_pair(acc, ad + 4, bd + (kPairSmemBBox >> 4), t_meta + 2, idesc, 1u);
-        tc_mma_sp_f16_pair(acc, ad + 6, bd + (kPairSmemBBox >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
+        if (SPARSE) {
+          const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
+          tc_cp_128x128b_pair(t_meta, e_desc0 + so);
+          // The metadata operand address must be 2-column aligned; the low column
+          // bit travels in the descriptor's sparsity-selector field instead.
+          tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != 0 ? 1u : 0u);
+          tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
+          tc_mma_sp_f16_pair(acc, ad + 4, bd + (kPairSmemBBox >> 4), t_meta + 2, idesc, 1u);
+          tc_mma_sp_f16_pair(acc, ad + 6, bd + (kPairSmemBBox >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
+        } else {
+          // Four K = 16 steps through the 128-byte swizzled rows of A and B (32 bytes each).
+          tc_mma_f16_pair(acc, ad, bd, idesc, kt != 0 ? 1u : 0u);
+          tc_mma_f16_pair(acc, ad + 2, bd + 2, idesc, 1u);
+          tc_mma_f16_pair(acc, ad + 4, bd + 4, idesc, 1u);
+          tc_mma_f16_pair(acc, ad + 6, bd + 6, idesc, 1u);
+        }
         tc_commit_pair(&empty[s], 0x3);
       }
       if (ok) tc_commit_pair(&acc_full[b], 0x3);

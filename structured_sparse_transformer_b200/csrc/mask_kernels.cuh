@@ -569,4 +569,33 @@ __global__ void __launch_bounds__(256) masked_decay_kernel(float *__restrict__ g
   }
 }
 
+// Transpose of a row-major [rows x cols] 16-bit matrix into [cols x rows]:
+// the input-gradient operand of the dense fine-tuning GEMM (W^T).  32x32
+// tiles through padded shared memory; each thread moves kTransRows elements.
+constexpr int kTransTile = 32;
+constexpr int kTransRows = 4;
+
+__global__ void __launch_bounds__(kTransTile * kTransTile / kTransRows) transpose16_kernel(
+    const uint16_t *__restrict__ in, uint16_t *__restrict__ out, int64_t rows, int64_t cols) {
+  __shared__ uint16_t tile[kTransTile][kTransTile + 1];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int64_t c0 = (int64_t)blockIdx.x * kTransTile;
+  for (int64_t r0 = (int64_t)blockIdx.y * kTransTile; r0 < rows; r0 += (int64_t)gridDim.y * kTransTile) {
+#pragma unroll
+    for (int k = 0; k < kTransTile; k += kTransTile / kTransRows) {
+      const int64_t r = r0 + ty + k, c = c0 + tx;
+      if (r < rows && c < cols) tile[ty + k][tx] = in[r * cols + c];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kTransTile; k += kTransTile / kTransRows) {
+      const int64_t c = c0 + ty + k, r = r0 + tx;
+      if (r < rows && c < cols) out[c * rows + r] = tile[tx][ty + k];
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace sp24

@@ -243,6 +243,17 @@ __device__ __forceinline__ void tc_mma_sp_f16_pair(uint32_t d_tmem, uint64_t a_d
       : "memory");
 }
 
+// Dense MMA of the pair (kind::f16, K = 16), for the dense fine-tuning GEMM.
+__device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // --------------------------------------------------------------- tcgen05 / TMEM
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols) {
@@ -330,6 +341,15 @@ constexpr uint32_t kSwizzle128B = 2;
 // Instruction descriptor of kind::f16 with fp32 accumulation, both operands
 // K-major, 2:4 sparse A.  Bits 0-1 (sparsity selector) are left 0 here and set
 // per MMA to the low column bit of the metadata address.
+// Instruction descriptor of a dense kind::f16 MMA with fp32 accumulation.
+__host__ __device__ constexpr uint32_t make_idesc_dense(bool bf16, int m, int n) {
+  return (1u << 4)                      // D format fp32
+         | ((bf16 ? 1u : 0u) << 7)      // A format
+         | ((bf16 ? 1u : 0u) << 10)     // B format
+         | ((uint32_t)(n >> 3) << 17)   // N / 8
+         | ((uint32_t)(m >> 4) << 24);  // M / 16
+}
+
 __host__ __device__ constexpr uint32_t make_idesc_sparse(bool bf16, int m, int n) {
   return (1u << 2)                      // sparse
          | (1u << 4)                    // D format fp32

@@ -108,26 +108,33 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 // ---------------------------------------------------------------- GEMM launch
 
 // CTA-pair kernel: clusters of two CTAs, 256 x 224 tiles (see gemm_sp.cuh).
-template <bool BF16, int EPI>
+// SPARSE: A = kept values [M x Kd/2] + metadata chunks; dense: A = [M x Kd].
+template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream) {
-  const int num_kt = (int)((Kd + kGemmBK - 1) / kGemmBK);
+  using G = PairGeom<SPARSE>;
+  const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
+  const uint64_t a_cols = SPARSE ? (uint64_t)(Kd / 2) : (uint64_t)Kd;
   CUtensorMap ta, tb, tm;
-  if (!make_map_2d(&ta, vals, (uint64_t)(Kd / 2), (uint64_t)M, (uint64_t)Kd, kGemmBKc, kPairRows,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT64))
+  if (!make_map_2d(&ta, vals, a_cols, (uint64_t)M, a_cols * 2, G::kAcols, kPairRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh, CU_TENSOR_MAP_SWIZZLE_128B))
     return SP24_ERR_CUDA;
+  if (SPARSE) {
+    if (!make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT64))
+      return SP24_ERR_CUDA;
+  } else {
+    tm = ta;  // unused by the dense kernel
+  }
   // Epilogue staging tiles: 32 features x 16 tokens of row-major out / aux [T x M].
   CUtensorMap to, tx;
   if (!make_map_2d(&to, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map_2d(&tx, EPI == kEpiNone ? out : aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens,
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return SP24_ERR_CUDA;
-  constexpr int smem_bytes = pair_smem_bytes(EPI);
-  auto kernel = sp24_gemm_pair_kernel<BF16, EPI>;
+  constexpr int smem_bytes = pair_smem_bytes<SPARSE>(EPI);
+  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
   static int max_pairs = 0;
   if (max_pairs == 0) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
@@ -156,16 +163,17 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
                     (int)T, num_kt, (uint64_t)g_wait_budget.load());
 }
 
+template <bool SPARSE>
 sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                         sp24_dtype dt, void *out, int epi, void *aux, cudaStream_t s) {
   const bool bf = dt == SP24_BF16;
   switch (epi) {
-    case kEpiNone: return bf ? launch_gemm_pair_t<true, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_pair_t<false, kEpiNone>(B, T, Kd, vals, meta, M, out, aux, s);
-    case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_pair_t<false, kEpiGelu>(B, T, Kd, vals, meta, M, out, aux, s);
-    default: return bf ? launch_gemm_pair_t<true, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s)
-                       : launch_gemm_pair_t<false, kEpiDgelu>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiNone: return bf ? launch_gemm_pair_t<true, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_pair_t<false, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                             : launch_gemm_pair_t<false, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    default: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                       : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
   }
 }
 
@@ -335,7 +343,7 @@ sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const void *vals_
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;
-  return launch_gemm(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, as_stream(stream));
+  return launch_gemm<true>(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, as_stream(stream));
 }
 
 sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *vals_col, const void *meta_col,
@@ -345,7 +353,33 @@ sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *va
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;
-  return launch_gemm(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, const_cast<void *>(aux), as_stream(stream));
+  return launch_gemm<true>(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, const_cast<void *>(aux),
+                          as_stream(stream));
+}
+
+sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A, int64_t M, sp24_dtype dtype,
+                            void *out, sp24_epilogue epi, void *aux, void *stream) {
+  if (epi != SP24_EPI_NONE && epi != SP24_EPI_GELU && epi != SP24_EPI_DGELU) return SP24_ERR_INVALID_ARG;
+  sp24_status st = validate_gemm(B, T, Kd, A, A, M, dtype, out, epi, aux, epi == SP24_EPI_NONE ? SP24_EPI_GELU : epi);
+  if (st != SP24_OK) return st;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (T == 0) return SP24_OK;
+  return launch_gemm<false>(B, T, Kd, A, nullptr, M, dtype, out, epi, aux, as_stream(stream));
+}
+
+sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtype dtype, void *out, void *stream) {
+  if (rows < 0 || cols < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (rows == 0 || cols == 0) return SP24_OK;
+  if (!in || !out) return SP24_ERR_INVALID_ARG;
+  if (rows > INT32_MAX || cols > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  const dim3 grid((unsigned)((cols + kTransTile - 1) / kTransTile),
+                  (unsigned)((rows + kTransTile - 1) / kTransTile < 65535 ? (rows + kTransTile - 1) / kTransTile
+                                                                            : 65535));
+  return launch_pdl(transpose16_kernel, grid, dim3(kTransTile, kTransTile / kTransRows), 0, as_stream(stream),
+                    static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out), rows, cols);
 }
 
 sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,

@@ -29,13 +29,14 @@ BYTES_PER_ELEMENT = {
     "prune_compress": 2 + 1 / 16 + 2 + 0.25,         # read W and index, write both orientations
     "masked_decay": 4 + 2 + 1 / 16 + 4,              # read g, W, index; write g
     "flip": 2 / 16,                                  # read two indices
+    "transpose": 4,                                  # read W, write W^T
 }
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--kernel", required=True,
-                    choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad"])
+                    choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad", "gemm_dense_fwd", "gemm_dense_dgrad"])
     ap.add_argument("--rows", type=int, required=True)
     ap.add_argument("--cols", type=int, required=True)
     ap.add_argument("--tokens", type=int, default=8192)
@@ -82,6 +83,23 @@ def main(argv=None):
         aux = torch.empty(T, R, dtype=tdt, device=dev) if args.epi == "gelu" else None
         epi = "gelu" if args.epi == "gelu" else None
         fn = lambda: sp.sp24_gemm_fwd(x, bufs[0], bufs[1], R, y, epi, aux)
+    elif k == "transpose":
+        wt = torch.empty(C, R, dtype=tdt, device=dev)
+        fn = lambda: sp.sp24_transpose(w, wt)
+    elif k == "gemm_dense_fwd":
+        x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
+        y = torch.empty(T, R, dtype=tdt, device=dev)
+        aux = torch.empty(T, R, dtype=tdt, device=dev) if args.epi == "gelu" else None
+        epi = "gelu" if args.epi == "gelu" else None
+        fn = lambda: sp.sp24_gemm_dense(x, w, y, epi, aux)
+    elif k == "gemm_dense_dgrad":
+        dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
+        wt = torch.empty(C, R, dtype=tdt, device=dev)
+        sp.sp24_transpose(w, wt)
+        dx = torch.empty(T, C, dtype=tdt, device=dev)
+        aux = torch.randn(T, C, device=dev, generator=gen).to(tdt) if args.epi == "dgelu" else None
+        epi = "dgelu" if args.epi == "dgelu" else None
+        fn = lambda: sp.sp24_gemm_dense(dy, wt, dx, epi, aux)
     else:
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
         dx = torch.empty(T, C, dtype=tdt, device=dev)

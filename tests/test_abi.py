@@ -83,6 +83,18 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_MISALIGNED"]
     assert _raw("sp24_gemm_fwd", fake, -1, 32, fake, fake, 16, 0, fake, 0, None, None) == \
         E["SP24_ERR_INVALID_ARG"]
+    # dense fine-tuning GEMM and transpose
+    assert _raw("sp24_gemm_dense", fake, 8, 24, fake, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_gemm_dense", fake, 8, 32, fake, 16, 0, fake, 2, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # DGELU without aux
+    assert _raw("sp24_gemm_dense", fake, 8, 32, fake, 16, 0, fake, 3, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # no such epilogue
+    assert _raw("sp24_gemm_dense", fake, 8, 32, odd, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_transpose", fake, 8, 8, 5, fake, None) == E["SP24_ERR_UNSUPPORTED_DTYPE"]
+    assert _raw("sp24_transpose", None, 8, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_transpose", fake, -2, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
     # decay and flip
     assert _raw("sp24_masked_decay", fake, fake, 0, 6, 8, fake, ctypes.c_float(1.0), None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]

@@ -106,3 +106,25 @@ def test_gelu_closed_forms():
     fd = (oracle.gelu(x + h) - oracle.gelu(x - h)) / (2 * h)
     assert np.allclose(oracle.gelu_grad(x), fd, atol=1e-9)
     assert abs(oracle.gelu_grad(np.array([0.0]))[0] - 0.5) < 1e-15
+
+
+def test_dense_gemms_exact_on_small_integers_and_adjoint():
+    """Dense fine-tuning products: exact integer sums by explicit loops, the
+    adjoint identity, and the one-hot case returning W (and W^T) itself."""
+    rng = np.random.default_rng(3)
+    T, N, K = 4, 8, 12
+    x = rng.integers(-9, 10, (T, K)).astype(np.float64)
+    dy = rng.integers(-9, 10, (T, N)).astype(np.float64)
+    w = rng.integers(-9, 10, (N, K)).astype(np.float64)
+    y, dx = oracle.dense_fwd(x, w), oracle.dense_dgrad(dy, w)
+    for t in range(T):
+        for n in range(N):
+            assert y[t, n] == sum(int(x[t, k]) * int(w[n, k]) for k in range(K))
+        for k in range(K):
+            assert dx[t, k] == sum(int(dy[t, n]) * int(w[n, k]) for n in range(N))
+    xr, dyr, wr = rng.normal(size=(5, 24)), rng.normal(size=(5, 16)), rng.normal(size=(16, 24))
+    lhs = np.sum(dyr * oracle.dense_fwd(xr, wr))
+    rhs = np.sum(oracle.dense_dgrad(dyr, wr) * xr)
+    assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs))
+    assert np.array_equal(oracle.dense_fwd(np.eye(K), w), w.T)
+    assert np.array_equal(oracle.dense_dgrad(np.eye(N), w), w)
