@@ -175,7 +175,8 @@ SP24_API sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const
 /*
  * out[cols x rows] = in[rows x cols]^T for 16-bit elements (bit copy): the
  * input-gradient operand W^T of the dense fine-tuning GEMM.
- *   in, out  device, row-major, contiguous, not overlapping; rows, cols >= 0
+ *   in, out  device, row-major, contiguous, not overlapping, 16-byte aligned;
+ *            rows, cols >= 0 (any values)
  */
 SP24_API sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtype dtype, void *out,
                            void *stream);

@@ -570,29 +570,63 @@ __global__ void __launch_bounds__(256) masked_decay_kernel(float *__restrict__ g
 }
 
 // Transpose of a row-major [rows x cols] 16-bit matrix into [cols x rows]:
-// the input-gradient operand of the dense fine-tuning GEMM (W^T).  32x32
-// tiles through padded shared memory; each thread moves kTransRows elements.
-constexpr int kTransTile = 32;
-constexpr int kTransRows = 4;
+// the input-gradient operand W^T of the dense fine-tuning GEMM.  64x64 tiles,
+// 256 threads (16 x 16): every global access is 8 bytes (four elements), a
+// half-warp covers 128 contiguous bytes of a row.  The shared tile has a row
+// stride of 33 words, so the column reads of the store phase spread over the
+// banks.  Edges (rows or cols not multiples of 4 or 64) take element accesses.
+constexpr int kTransTile = 64;
+constexpr int kTransStride = 66;   // 16-bit elements per shared row (33 words)
 
-__global__ void __launch_bounds__(kTransTile * kTransTile / kTransRows) transpose16_kernel(
-    const uint16_t *__restrict__ in, uint16_t *__restrict__ out, int64_t rows, int64_t cols) {
-  __shared__ uint16_t tile[kTransTile][kTransTile + 1];
+__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t *__restrict__ in,
+                                                          uint16_t *__restrict__ out, int64_t rows, int64_t cols) {
+  __shared__ __align__(8) uint16_t tile[kTransTile * kTransStride];
   pdl_launch_dependents();
   pdl_wait();
-  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int64_t c0 = (int64_t)blockIdx.x * kTransTile;
+  const bool vec_in = (cols & 3) == 0, vec_out = (rows & 3) == 0;
   for (int64_t r0 = (int64_t)blockIdx.y * kTransTile; r0 < rows; r0 += (int64_t)gridDim.y * kTransTile) {
 #pragma unroll
-    for (int k = 0; k < kTransTile; k += kTransTile / kTransRows) {
-      const int64_t r = r0 + ty + k, c = c0 + tx;
-      if (r < rows && c < cols) tile[ty + k][tx] = in[r * cols + c];
+    for (int k = 0; k < 4; ++k) {
+      const int lr = ty + 16 * k;
+      const int64_t r = r0 + lr, c = c0 + 4 * tx;
+      uint32_t lo = 0, hi = 0;
+      if (r < rows) {
+        if (vec_in && c + 4 <= cols) {
+          const uint2 v = *reinterpret_cast<const uint2 *>(in + r * cols + c);
+          lo = v.x;
+          hi = v.y;
+        } else {
+          const uint16_t *src = in + r * cols;
+          const uint32_t e0 = c < cols ? src[c] : 0u, e1 = c + 1 < cols ? src[c + 1] : 0u;
+          const uint32_t e2 = c + 2 < cols ? src[c + 2] : 0u, e3 = c + 3 < cols ? src[c + 3] : 0u;
+          lo = e0 | (e1 << 16);
+          hi = e2 | (e3 << 16);
+        }
+      }
+      uint32_t *dst = reinterpret_cast<uint32_t *>(&tile[lr * kTransStride + 4 * tx]);
+      dst[0] = lo;
+      dst[1] = hi;
     }
     __syncthreads();
 #pragma unroll
-    for (int k = 0; k < kTransTile; k += kTransTile / kTransRows) {
-      const int64_t c = c0 + ty + k, r = r0 + tx;
-      if (r < rows && c < cols) out[c * rows + r] = tile[tx][ty + k];
+    for (int k = 0; k < 4; ++k) {
+      const int lc = ty + 16 * k;              // output row = input column c0 + lc
+      const int64_t c = c0 + lc, r = r0 + 4 * tx;
+      if (c < cols) {
+        const uint32_t e0 = tile[(4 * tx) * kTransStride + lc], e1 = tile[(4 * tx + 1) * kTransStride + lc];
+        const uint32_t e2 = tile[(4 * tx + 2) * kTransStride + lc], e3 = tile[(4 * tx + 3) * kTransStride + lc];
+        uint16_t *dst = out + c * rows;
+        if (vec_out && r + 4 <= rows) {
+          *reinterpret_cast<uint2 *>(dst + r) = make_uint2(e0 | (e1 << 16), e2 | (e3 << 16));
+        } else {
+          if (r < rows) dst[r] = (uint16_t)e0;
+          if (r + 1 < rows) dst[r + 1] = (uint16_t)e1;
+          if (r + 2 < rows) dst[r + 2] = (uint16_t)e2;
+          if (r + 3 < rows) dst[r + 3] = (uint16_t)e3;
+        }
+      }
     }
     __syncthreads();
   }

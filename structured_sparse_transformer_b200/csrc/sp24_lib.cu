@@ -372,13 +372,14 @@ sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtyp
   if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
   if (rows == 0 || cols == 0) return SP24_OK;
   if (!in || !out) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out)) return SP24_ERR_MISALIGNED;
   if (rows > INT32_MAX || cols > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
   sp24_status st = check_device();
   if (st != SP24_OK) return st;
   const dim3 grid((unsigned)((cols + kTransTile - 1) / kTransTile),
                   (unsigned)((rows + kTransTile - 1) / kTransTile < 65535 ? (rows + kTransTile - 1) / kTransTile
                                                                             : 65535));
-  return launch_pdl(transpose16_kernel, grid, dim3(kTransTile, kTransTile / kTransRows), 0, as_stream(stream),
+  return launch_pdl(transpose16_kernel, grid, dim3(256), 0, as_stream(stream),
                     static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out), rows, cols);
 }
 

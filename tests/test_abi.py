@@ -95,6 +95,7 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert _raw("sp24_transpose", fake, 8, 8, 5, fake, None) == E["SP24_ERR_UNSUPPORTED_DTYPE"]
     assert _raw("sp24_transpose", None, 8, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_transpose", fake, -2, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_transpose", odd, 8, 8, 0, fake, None) == E["SP24_ERR_MISALIGNED"]
     # decay and flip
     assert _raw("sp24_masked_decay", fake, fake, 0, 6, 8, fake, ctypes.c_float(1.0), None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]
