@@ -63,7 +63,14 @@ typedef enum sp24_dtype { SP24_F16 = 0, SP24_BF16 = 1 } sp24_dtype;
 typedef enum sp24_epilogue {
   SP24_EPI_NONE = 0,
   SP24_EPI_GELU = 1,  /* out = gelu(acc) (exact erf form); aux <- acc rounded to dtype */
-  SP24_EPI_DGELU = 2  /* out = acc * gelu'(aux); aux holds the pre-activation */
+  SP24_EPI_DGELU = 2, /* out = acc * gelu'(aux); aux holds the pre-activation */
+  /* Gated GELU (abstract: gated activation functions).  The stacked weight
+   * holds groups of 16 rows of W_gate and of W_up alternately (gate rows
+   * 16g..16g+15 at 32g.., up rows at 32g+16..), so the accumulator columns of
+   * one output feature sit 16 apart. */
+  SP24_EPI_GEGLU = 3, /* out[T x N/2] = gelu(gate) * up; aux[T x N] <- acc (both halves) */
+  SP24_EPI_DGEGLU = 4 /* out[T x 2K] = (acc*up*gelu'(gate), acc*gelu(gate)) interleaved as
+                         aux; aux[T x 2K] holds the gated pre-activations */
 } sp24_epilogue;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -134,8 +141,10 @@ SP24_API sp24_status sp24_mask_step(const void *W, sp24_dtype dtype, int64_t row
  *   X         device [T x K] row-major, contiguous
  *   vals_row, meta_row   device, W [N x K] compressed along K (sp24_prune_compress)
  *   Y         device [T x N] row-major, contiguous
- *   epi       SP24_EPI_NONE, or SP24_EPI_GELU: Y = gelu(acc) and aux[T x N] <- acc
- *   aux       device [T x N] for SP24_EPI_GELU, else ignored (may be NULL)
+ *   epi       SP24_EPI_NONE, or SP24_EPI_GELU: Y = gelu(acc) and aux[T x N] <- acc,
+ *             or SP24_EPI_GEGLU: Y is [T x N/2] = gelu(gate) * up for the stacked
+ *             gate/up weight (N % 32 == 0) and aux[T x N] <- acc
+ *   aux       device [T x N] for SP24_EPI_GELU / GEGLU, else ignored (may be NULL)
  * fp32 accumulation; outputs rounded to dtype.  K % 16 == 0, N % 16 == 0,
  * T >= 0.  All pointers 16-byte aligned.
  */
@@ -149,7 +158,10 @@ SP24_API sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const vo
  *   dY        device [T x N] row-major, contiguous
  *   vals_col, meta_col   device, W^T [K x N] compressed along N (sp24_prune_compress)
  *   dX        device [T x K]
- *   epi       SP24_EPI_NONE, or SP24_EPI_DGELU: dX = acc * gelu'(aux), aux [T x K]
+ *   epi       SP24_EPI_NONE, or SP24_EPI_DGELU: dX = acc * gelu'(aux), aux [T x K],
+ *             or SP24_EPI_DGEGLU (input gradient of the down projection of a
+ *             gated FFN, acc = dH): dX is [T x 2K], the gradients of the gate
+ *             and up pre-activations in the stacked layout of aux [T x 2K]
  * N % 16 == 0, K % 16 == 0.
  */
 SP24_API sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *vals_col,

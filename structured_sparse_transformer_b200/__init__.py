@@ -57,7 +57,7 @@ STATUS = {0: "SP24_OK", 1: "SP24_ERR_INVALID_ARG", 2: "SP24_ERR_UNSUPPORTED_SHAP
           6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE"}
 SP24_F16, SP24_BF16 = 0, 1
 SP24_EPI_NONE, SP24_EPI_GELU, SP24_EPI_DGELU = 0, 1, 2
-EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2}
+EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4}
 
 
 class Sp24Error(RuntimeError):
@@ -169,7 +169,8 @@ def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_r
 
 
 def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=None):
-    """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None or 'gelu' (aux <- pre-activation)."""
+    """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None, 'gelu' (aux <- pre-activation) or
+    'geglu' (W the stacked gate/up weight: Y[T, N/2] <- gelu(gate) * up, aux[T, N] <- pre-activations)."""
     _need_cuda(X, vals_row, meta_row, Y, aux)
     T, K = X.shape
     _check("sp24_gemm_fwd",
@@ -178,7 +179,8 @@ def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=N
 
 
 def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stream=None):
-    """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None or 'dgelu' (uses aux [T, K])."""
+    """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None, 'dgelu' (uses aux [T, K]) or
+    'dgeglu' (dX[T, 2K] <- gradients of the gated pre-activations in aux [T, 2K])."""
     _need_cuda(dY, vals_col, meta_col, dX, aux)
     T, N = dY.shape
     _check("sp24_gemm_dgrad",

@@ -70,39 +70,51 @@ constexpr int kPairSmemBBox = kPairBNh * 64 * 2;       // 14 KB: 112 token rows 
 constexpr int kPairChunks = kPairBN / kEpiTokens;      // 14
 constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at columns 0 and 224
 
+// Epilogues: none; GELU (aux <- pre-activation); GELU' (aux = pre-activation,
+// read); gated GELU on a gate/up-interleaved output (out = gelu(gate) * up at
+// half width, aux <- both pre-activations); and its input gradient (aux =
+// both pre-activations, read; out = (d gate, d up) interleaved at twice the
+// accumulator width).
+enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4 };
+constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in the stacked gated weight
+
 // Pipeline stage of the 2:4 GEMM (SPARSE) and of the dense GEMM of the dense
 // fine-tuning phase.  Sparse: 128 logical K per stage = 64 kept values of A,
-// two 64-K boxes of B and the 2 KB metadata chunk (46 KB), 4 stages.  Dense:
+// two 64-K boxes of B and the 2 KB metadata chunk (46 KB), 4 stages (3 when
+// the gated-GELU gradient epilogue takes 6 KB of staging per warp).  Dense:
 // 64 K per stage, one box of A and one of B (30 KB), 6 stages.
-template <bool SPARSE>
+template <bool SPARSE, int EPI>
 struct PairGeom {
   static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
   static constexpr int kAcols = 64;                      // A values per row and stage
   static constexpr int kBBoxes = SPARSE ? 2 : 1;
   static constexpr int kMeta = SPARSE ? kSmemE : 0;
   static constexpr int kStageBytes = kPairSmemA + kBBoxes * kPairSmemBBox + kMeta;
-  static constexpr int kStages = SPARSE ? 4 : 6;
+  static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
 };
 constexpr int kEpiBufBytes = kEpiTokens * 32 * 2;      // staging tile: 16 tokens x 32 features, 64B-swizzled
 constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM address, abort flag
 
-enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2 };
-
-// Staging tiles per epilogue warp: out; out + pre-activation; out + two
-// pre-activation inputs.
-__host__ __device__ constexpr int epi_bufs(int epi) { return epi == kEpiNone ? 1 : (epi == kEpiGelu ? 2 : 3); }
-template <bool SPARSE>
-__host__ __device__ constexpr int pair_smem_bytes(int epi) {
-  return PairGeom<SPARSE>::kStages * PairGeom<SPARSE>::kStageBytes + kEpiWarps * epi_bufs(epi) * kEpiBufBytes +
+// Staging per epilogue warp, in 1 KB tiles: out; out + pre-activation; out +
+// two pre-activation inputs; gated: half-width out (in a 1 KB tile) +
+// pre-activations; gated gradient: a 2 KB out tile + two 2 KB pre-activation
+// inputs.
+__host__ __device__ constexpr int epi_bufs(int epi) {
+  return epi == kEpiNone ? 1 : (epi == kEpiGelu || epi == kEpiGeglu) ? 2 : (epi == kEpiDgelu ? 3 : 6);
+}
+template <bool SPARSE, int EPI>
+__host__ __device__ constexpr int pair_smem_bytes() {
+  return PairGeom<SPARSE, EPI>::kStages * PairGeom<SPARSE, EPI>::kStageBytes + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
          kPairBarBytes + 1024;
 }
-static_assert(pair_smem_bytes<true>(kEpiDgelu) <= 232448 && pair_smem_bytes<false>(kEpiDgelu) <= 232448,
+static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<false, kEpiDgelu>() <= 232448 &&
+                  pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448,
               "shared memory per CTA");
-static_assert(PairGeom<true>::kStageBytes % 1024 == 0 && PairGeom<false>::kStageBytes % 1024 == 0 &&
+static_assert(PairGeom<true, kEpiNone>::kStageBytes % 1024 == 0 && PairGeom<false, kEpiNone>::kStageBytes % 1024 == 0 &&
                   kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
-static_assert(kPairMetaCol + 4 * PairGeom<true>::kStages <= kTmemCols, "tensor memory budget");
-static_assert(2 * PairGeom<false>::kStages + 16 + 2 * kEpiWarps <= kPairBarBytes / 8, "barrier space");
+static_assert(kPairMetaCol + 4 * PairGeom<true, kEpiNone>::kStages <= kTmemCols, "tensor memory budget");
+static_assert(2 * PairGeom<false, kEpiNone>::kStages + 16 + 2 * kEpiWarps <= kPairBarBytes / 8, "barrier space");
 
 // GELU (exact erf form) and its derivative for the epilogues:
 //   gelu(x) = x Phi(x),  gelu'(x) = Phi(x) + x phi(x),
@@ -176,6 +188,19 @@ __device__ __forceinline__ float2 gelu_grad2(float2 x) {
   return __ffma2_rn(make_float2(p0 ? -e.x : e.x, p1 ? -e.y : e.y), q, make_float2(p0 ? 1.0f : 0.0f, p1 ? 1.0f : 0.0f));
 }
 
+// gelu and gelu' of the same pair, sharing the exponential and the polynomial
+// (each result is computed exactly as gelu2 and gelu_grad2 compute it).
+__device__ __forceinline__ void gelu_and_grad2(float2 x, float2 &g, float2 &gp) {
+  const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+  const float2 nax = make_float2(-ax.x, -ax.y);
+  const float2 e = gauss_e2(x);
+  const float2 hr = half_r2(ax);
+  g = __ffma2_rn(nax, __fmul2_rn(hr, e), make_float2(fmaxf(x.x, 0.0f), fmaxf(x.y, 0.0f)));
+  const float2 q = __ffma2_rn(nax, splat(0.39894228040143268f), hr);
+  const bool p0 = x.x >= 0.0f, p1 = x.y >= 0.0f;
+  gp = __ffma2_rn(make_float2(p0 ? -e.x : e.x, p1 ? -e.y : e.y), q, make_float2(p0 ? 1.0f : 0.0f, p1 ? 1.0f : 0.0f));
+}
+
 template <bool BF16>
 __device__ __forceinline__ uint32_t f32_to_bits(float x) {
   if (BF16) return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
@@ -228,6 +253,11 @@ __host__ __device__ constexpr uint32_t swz64(int row, int c) {
   return (uint32_t)(row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
 }
 
+// The same for 128-byte rows and the TMA's 128B pattern (column index XOR row mod 8).
+__host__ __device__ constexpr uint32_t swz128(int row, int c) {
+  return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4));
+}
+
 // Two floats -> one register of 16-bit values, lo in the low half (round to nearest even).
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -255,7 +285,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
                           const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
                           uint64_t wait_budget) {
-  using G = PairGeom<SPARSE>;
+  using G = PairGeom<SPARSE, EPI>;
   constexpr int kPairStages = G::kStages;
   constexpr int kPairStageBytes = G::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -288,7 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
-    if (EPI == kEpiDgelu)
+    if (EPI == kEpiDgelu || EPI == kEpiDgeglu)
       for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(&aux_bars[i], 1);
     *s_abort = 0;
     fence_mbarrier_init();
@@ -406,26 +436,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int grp = ew >> 2;
     const int q = warp & 3;
     constexpr int kMaxChunksPerWarp = (kPairChunks + kEpiGroups - 1) / kEpiGroups;
-    uint8_t *stg = epi_smem + ew * epi_bufs(EPI) * kEpiBufBytes;   // [out][aux] or [out][pre 0][pre 1]
+    constexpr bool kPre = EPI == kEpiDgelu || EPI == kEpiDgeglu;       // TMA-loaded pre-activations
+    constexpr int kPreBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
+    constexpr int kOutBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
+    // Staging of warp ew: [out][aux] (GELU, gated), [out][pre 0][pre 1] (gradients).
+    uint8_t *stg = epi_smem + ew * epi_bufs(EPI) * kEpiBufBytes;
     const uint32_t stg_u32 = smem_u32(stg);
     uint64_t *pre_bar = aux_bars + 2 * ew;
     // stmatrix/ldmatrix addressing: lane l names row l%8 of matrix l/8; matrix
     // j holds tokens 8(j/2).. and features 8(j%2).. (+16 for the upper 16 TMEM lanes).
     const int mrow = 8 * (lane >> 4) + (lane & 7);
-    const uint32_t lane_off0 = swz64(mrow, (lane >> 3) & 1);
-    const uint32_t lane_off1 = swz64(mrow, 2 + ((lane >> 3) & 1));
+    const int mcol = (lane >> 3) & 1;
+    const uint32_t lane_off0 = swz64(mrow, mcol);
+    const uint32_t lane_off1 = swz64(mrow, 2 + mcol);
+    // Columns (features) of this warp in out and aux: the gated output has half
+    // the accumulator's width, the gated gradient twice it.
+    auto out_col = [&](int m0) { return EPI == kEpiGeglu ? m0 / 2 : (EPI == kEpiDgeglu ? 2 * m0 : m0); };
+    auto pre_col = [&](int m0) { return EPI == kEpiDgeglu ? 2 * m0 : m0; };
     auto release = [&](int buf) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(&acc_empty[buf]);
     };
-    uint32_t pre_issued = 0, pre_used = 0;   // dGELU pre-activation tiles (tile s uses buffer s%2)
+    uint32_t pre_issued = 0, pre_used = 0;   // pre-activation tiles (tile s uses buffer s%2)
     auto pre_load = [&](int x, int y) {
       const uint32_t seq = pre_issued++;
       if (lane == 0) {
         uint64_t *bar = &pre_bar[seq & 1];
-        mbar_arrive_expect_tx(bar, kEpiBufBytes);
-        tma_load_2d(stg + kEpiBufBytes * (1 + (seq & 1)), &tm_aux, bar, x, y);
+        mbar_arrive_expect_tx(bar, kPreBytes);
+        tma_load_2d(stg + kOutBytes + kPreBytes * (seq & 1), &tm_aux, bar, x, y);
       }
     };
     bool alive = true;
@@ -436,8 +475,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int n0 = (tile / num_mt) * kPairBN;
       const int nchunks = min(kPairChunks, (T - n0 + kEpiTokens - 1) / kEpiTokens);
       const int nk = grp < nchunks ? (nchunks - 1 - grp) / kEpiGroups + 1 : 0;   // this warp's chunks
-      if (EPI == kEpiDgelu)
-        for (int k = 0; k < 2 && k < nk; ++k) pre_load(m0, n0 + (grp + k * kEpiGroups) * kEpiTokens);
+      if (kPre)
+        for (int k = 0; k < 2 && k < nk; ++k) pre_load(pre_col(m0), n0 + (grp + k * kEpiGroups) * kEpiTokens);
       const bool got = mbar_wait_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) {
         alive = false;
@@ -465,8 +504,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int k = 0; k < kMaxChunksPerWarp; ++k) {
         if (k >= nk) break;
         const int t0 = n0 + (grp + k * kEpiGroups) * kEpiTokens;
-        uint32_t hx[2][4];
-        if (EPI == kEpiDgelu) {
+        uint32_t pre_src = 0;
+        if (kPre) {
           const uint32_t seq = pre_used;
           const bool ready = mbar_wait_bounded(&pre_bar[seq & 1], (seq >> 1) & 1u, wait_budget, s_abort);
           if (!__all_sync(0xFFFFFFFFu, ready)) {
@@ -474,51 +513,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           ++pre_used;
-          const uint32_t src = stg_u32 + kEpiBufBytes * (1 + (seq & 1));
-          ldmatrix_x4_trans(src + lane_off0, hx[0]);
-          ldmatrix_x4_trans(src + lane_off1, hx[1]);
-        }
-        // Register i of half h: tokens 8(i/2) + 2(lane%4) + {0, 1} of feature
-        // 16h + 8(i%2) + lane/4 (TMEM registers 4(i/2) + 2(i%2) + {0, 1}).
-        uint32_t po[2][4], pa[2][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int ri = 4 * (i >> 1) + 2 * (i & 1);
-            const float2 acc = make_float2(__uint_as_float(r[k][h][ri]), __uint_as_float(r[k][h][ri + 1]));
-            float2 y = acc;
-            if (EPI == kEpiGelu) {
-              y = gelu2(acc);
-              pa[h][i] = pack2<BF16>(acc.x, acc.y);
-            } else if (EPI == kEpiDgelu) {
-              float2 hv;
-              unpack2<BF16>(hx[h][i], hv.x, hv.y);
-              y = __fmul2_rn(acc, gelu_grad2(hv));
-            }
-            po[h][i] = pack2<BF16>(y.x, y.y);
-          }
+          pre_src = stg_u32 + kOutBytes + kPreBytes * (seq & 1);
         }
         if (lane == 0) bulk_wait_group_read<0>();   // the previous chunk's stores have read the staging tiles
         __syncwarp();
-        stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);
-        stmatrix_x4_trans(stg_u32 + lane_off1, po[1]);
-        if (EPI == kEpiGelu) {
+        // Register i of half h: tokens 8(i/2) + 2(lane%4) + {0, 1} of feature
+        // 16h + 8(i%2) + lane/4 (TMEM registers 4(i/2) + 2(i%2) + {0, 1}).
+        if (EPI == kEpiGeglu) {
+          // Half 0 holds the gate rows, half 1 the up rows of the same 16
+          // features: out = gelu(gate) * up [16 tokens x 16 features, 32-byte
+          // rows], aux <- both halves as accumulated.
+          uint32_t po[4], pa[2][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int ri = 4 * (i >> 1) + 2 * (i & 1);
+            const float2 g = make_float2(__uint_as_float(r[k][0][ri]), __uint_as_float(r[k][0][ri + 1]));
+            const float2 u = make_float2(__uint_as_float(r[k][1][ri]), __uint_as_float(r[k][1][ri + 1]));
+            const float2 y = __fmul2_rn(gelu2(g), u);
+            po[i] = pack2<BF16>(y.x, y.y);
+            pa[0][i] = pack2<BF16>(g.x, g.y);
+            pa[1][i] = pack2<BF16>(u.x, u.y);
+          }
+          stmatrix_x4_trans(stg_u32 + (uint32_t)(mrow * 32 + mcol * 16), po);
           stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off0, pa[0]);
           stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off1, pa[1]);
+        } else if (EPI == kEpiDgeglu) {
+          // The pre-activation tile is [16 tokens x 64 columns, 128B-swizzled]:
+          // the gate and up values of the warp's 32 features, in 16-column
+          // groups gate(h=0), up(h=0), gate(h=1), up(h=1).  The output has the
+          // same layout: (d gate, d up) = (acc * up * gelu'(gate), acc * gelu(gate)).
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t hg[4], hu[4], og[4], ou[4];
+            ldmatrix_x4_trans(pre_src + swz128(mrow, 4 * h + mcol), hg);
+            ldmatrix_x4_trans(pre_src + swz128(mrow, 4 * h + 2 + mcol), hu);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ri = 4 * (i >> 1) + 2 * (i & 1);
+              const float2 a = make_float2(__uint_as_float(r[k][h][ri]), __uint_as_float(r[k][h][ri + 1]));
+              float2 g, u, gel, gp;
+              unpack2<BF16>(hg[i], g.x, g.y);
+              unpack2<BF16>(hu[i], u.x, u.y);
+              gelu_and_grad2(g, gel, gp);
+              const float2 dg = __fmul2_rn(__fmul2_rn(a, u), gp);
+              const float2 du = __fmul2_rn(a, gel);
+              og[i] = pack2<BF16>(dg.x, dg.y);
+              ou[i] = pack2<BF16>(du.x, du.y);
+            }
+            stmatrix_x4_trans(stg_u32 + swz128(mrow, 4 * h + mcol), og);
+            stmatrix_x4_trans(stg_u32 + swz128(mrow, 4 * h + 2 + mcol), ou);
+          }
+        } else {
+          uint32_t hx[2][4];
+          if (EPI == kEpiDgelu) {
+            ldmatrix_x4_trans(pre_src + lane_off0, hx[0]);
+            ldmatrix_x4_trans(pre_src + lane_off1, hx[1]);
+          }
+          uint32_t po[2][4], pa[2][4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ri = 4 * (i >> 1) + 2 * (i & 1);
+              const float2 acc = make_float2(__uint_as_float(r[k][h][ri]), __uint_as_float(r[k][h][ri + 1]));
+              float2 y = acc;
+              if (EPI == kEpiGelu) {
+                y = gelu2(acc);
+                pa[h][i] = pack2<BF16>(acc.x, acc.y);
+              } else if (EPI == kEpiDgelu) {
+                float2 hv;
+                unpack2<BF16>(hx[h][i], hv.x, hv.y);
+                y = __fmul2_rn(acc, gelu_grad2(hv));
+              }
+              po[h][i] = pack2<BF16>(y.x, y.y);
+            }
+          }
+          stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);
+          stmatrix_x4_trans(stg_u32 + lane_off1, po[1]);
+          if (EPI == kEpiGelu) {
+            stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off0, pa[0]);
+            stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off1, pa[1]);
+          }
         }
         // One proxy fence orders this warp's shared-memory accesses of the
-        // chunk (the stmatrix writes, and for dGELU the ldmatrix reads of the
-        // pre-activation tile) before the TMA store that reads the staging tile
-        // and the TMA load that refills the pre-activation tile.
+        // chunk (the stmatrix writes, and for the gradients the ldmatrix reads
+        // of the pre-activation tile) before the TMA store that reads the
+        // staging tile and the TMA load that refills the pre-activation tile.
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && m0 < M) {   // the TMA unit clips features >= M and tokens >= T
-          tma_store_2d(&tm_out, stg, m0, t0);
-          if (EPI == kEpiGelu) tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
+        if (lane == 0 && m0 < M) {   // the TMA unit clips columns past the tensor and tokens >= T
+          tma_store_2d(&tm_out, stg, out_col(m0), t0);
+          if (EPI == kEpiGelu || EPI == kEpiGeglu) tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
           bulk_commit_group();
         }
-        if (EPI == kEpiDgelu && k + 2 < nk) pre_load(m0, t0 + 2 * kEpiGroups * kEpiTokens);
+        if (kPre && k + 2 < nk) pre_load(pre_col(m0), t0 + 2 * kEpiGroups * kEpiTokens);
       }
     }
     if (lane == 0) {

@@ -112,7 +112,7 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream) {
-  using G = PairGeom<SPARSE>;
+  using G = PairGeom<SPARSE, EPI>;
   const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
   const uint64_t a_cols = SPARSE ? (uint64_t)(Kd / 2) : (uint64_t)Kd;
@@ -127,13 +127,24 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   } else {
     tm = ta;  // unused by the dense kernel
   }
-  // Epilogue staging tiles: 32 features x 16 tokens of row-major out / aux [T x M].
+  // Epilogue staging tiles of row-major out / aux, 16 tokens high: 32 features
+  // (64B swizzle); gated: out 16 features (no swizzle), aux 32; gated
+  // gradient: out and aux 64 columns (128B swizzle) over twice the width.
   CUtensorMap to, tx;
-  if (!make_map_2d(&to, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_2d(&tx, EPI == kEpiNone ? out : aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens,
-                   CU_TENSOR_MAP_SWIZZLE_64B))
-    return SP24_ERR_CUDA;
-  constexpr int smem_bytes = pair_smem_bytes<SPARSE>(EPI);
+  bool maps_ok;
+  if (EPI == kEpiGeglu) {
+    maps_ok = make_map_2d(&to, out, (uint64_t)M / 2, (uint64_t)T, (uint64_t)M, 16, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map_2d(&tx, aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B);
+  } else if (EPI == kEpiDgeglu) {
+    maps_ok = make_map_2d(&to, out, (uint64_t)M * 2, (uint64_t)T, (uint64_t)M * 4, 64, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map_2d(&tx, aux, (uint64_t)M * 2, (uint64_t)T, (uint64_t)M * 4, 64, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    maps_ok = make_map_2d(&to, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B) &&
+              make_map_2d(&tx, EPI == kEpiNone ? out : aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens,
+                          CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  if (!maps_ok) return SP24_ERR_CUDA;
+  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
   auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
   static int max_pairs = 0;
   if (max_pairs == 0) {
@@ -172,9 +183,20 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
                              : launch_gemm_pair_t<false, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
     case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
                              : launch_gemm_pair_t<false, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
-    default: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                       : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiDgelu: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                              : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    default: break;
   }
+  if (SPARSE) {   // the gated epilogues serve the 2:4 GEMMs
+    switch (epi) {
+      case kEpiGeglu: return bf ? launch_gemm_pair_t<true, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s)
+                                : launch_gemm_pair_t<false, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s);
+      case kEpiDgeglu: return bf ? launch_gemm_pair_t<true, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s)
+                                 : launch_gemm_pair_t<false, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s);
+      default: break;
+    }
+  }
+  return SP24_ERR_INVALID_ARG;
 }
 
 sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
@@ -183,7 +205,8 @@ sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals
   if (!vals || !meta || (!out && T > 0)) return SP24_ERR_INVALID_ARG;
   if (T < 0 || Kd <= 0 || M <= 0) return SP24_ERR_INVALID_ARG;
   if (!valid_dtype(dt)) return SP24_ERR_UNSUPPORTED_DTYPE;
-  if (epi != SP24_EPI_NONE && epi != allowed_epi) return SP24_ERR_INVALID_ARG;
+  if (epi != SP24_EPI_NONE && epi != allowed_epi && epi != allowed_epi + 2) return SP24_ERR_INVALID_ARG;
+  if (epi == SP24_EPI_GEGLU && M % (2 * kGegluGroup)) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (epi != SP24_EPI_NONE && !aux) return SP24_ERR_INVALID_ARG;
   if (Kd % 16 || M % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (T > INT32_MAX || M > INT32_MAX || Kd > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
@@ -361,6 +384,7 @@ sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A,
                             void *out, sp24_epilogue epi, void *aux, void *stream) {
   if (epi != SP24_EPI_NONE && epi != SP24_EPI_GELU && epi != SP24_EPI_DGELU) return SP24_ERR_INVALID_ARG;
   sp24_status st = validate_gemm(B, T, Kd, A, A, M, dtype, out, epi, aux, epi == SP24_EPI_NONE ? SP24_EPI_GELU : epi);
+  if (st == SP24_OK && epi != SP24_EPI_NONE && epi != SP24_EPI_GELU && epi != SP24_EPI_DGELU) st = SP24_ERR_INVALID_ARG;
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;

@@ -79,6 +79,14 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_INVALID_ARG"]                       # DGELU is not a forward epilogue
     assert _raw("sp24_gemm_dgrad", fake, 8, 32, fake, fake, 16, 0, fake, 1, fake, None) == \
         E["SP24_ERR_INVALID_ARG"]                       # GELU is not an input-gradient epilogue
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 48, 0, fake, 3, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # GEGLU needs whole gate/up row groups
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 64, 0, fake, 4, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # DGEGLU is not a forward epilogue
+    assert _raw("sp24_gemm_dgrad", fake, 8, 32, fake, fake, 64, 0, fake, 3, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # GEGLU is not an input-gradient epilogue
+    assert _raw("sp24_gemm_dense", fake, 8, 32, fake, 64, 0, fake, 3, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # gated epilogues serve the 2:4 GEMMs
     assert _raw("sp24_gemm_fwd", odd, 8, 32, fake, fake, 16, 0, fake, 0, None, None) == \
         E["SP24_ERR_MISALIGNED"]
     assert _raw("sp24_gemm_fwd", fake, -1, 32, fake, fake, 16, 0, fake, 0, None, None) == \

@@ -128,3 +128,30 @@ def test_dense_gemms_exact_on_small_integers_and_adjoint():
     assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs))
     assert np.array_equal(oracle.dense_fwd(np.eye(K), w), w.T)
     assert np.array_equal(oracle.dense_dgrad(np.eye(N), w), w)
+
+
+def test_gate_up_interleave_and_split_are_inverse():
+    rng = np.random.default_rng(5)
+    wg, wu = rng.normal(size=(48, 8)), rng.normal(size=(48, 8))
+    w = oracle.interleave_gate_up(wg, wu)
+    assert np.array_equal(w[0:16], wg[0:16]) and np.array_equal(w[16:32], wu[0:16])
+    assert np.array_equal(w[32:48], wg[16:32]) and np.array_equal(w[80:96], wu[32:48])
+    # the columns of X W^T split back into X W_gate^T and X W_up^T
+    x = rng.normal(size=(5, 8))
+    g, u = oracle.split_gate_up(x @ w.T)
+    assert np.allclose(g, x @ wg.T, rtol=0, atol=1e-12) and np.allclose(u, x @ wu.T, rtol=0, atol=1e-12)
+
+
+def test_geglu_closed_forms_and_finite_differences():
+    assert oracle.geglu(np.array([0.0]), np.array([3.0]))[0] == 0.0
+    assert oracle.geglu(np.array([2.0]), np.array([0.0]))[0] == 0.0
+    dg, du = oracle.geglu_grad(np.array([1.0]), np.array([0.0]), np.array([3.0]))
+    assert dg[0] == 1.5 and du[0] == 0.0                  # gelu'(0) = 1/2, gelu(0) = 0
+    rng = np.random.default_rng(6)
+    g, u, dh = rng.normal(size=64) * 2, rng.normal(size=64), rng.normal(size=64)
+    eps = 1e-6
+    fd_g = (oracle.geglu(g + eps, u) - oracle.geglu(g - eps, u)) / (2 * eps)
+    fd_u = (oracle.geglu(g, u + eps) - oracle.geglu(g, u - eps)) / (2 * eps)
+    dg, du = oracle.geglu_grad(dh, g, u)
+    assert np.allclose(dg, dh * fd_g, rtol=1e-6, atol=1e-8)
+    assert np.allclose(du, dh * fd_u, rtol=1e-6, atol=1e-8)
