@@ -309,6 +309,7 @@ def run_ours(args, wl, rank, world, local_rank):
         step.run(events)
     barrier()
     dense = run_dense_phase(args, step, wl, world, dev, flush, barrier)
+    geglu = run_geglu_phase(args, step, wl, world, dev, flush, barrier)
     total_ms = max_over_ranks(step_ms, world, dev)
     ms_per_step = total_ms / args.steps
     flops = wl.gemm_flops()
@@ -358,6 +359,7 @@ def run_ours(args, wl, rank, world, local_rank):
                                  "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
         "kernels": kernels,
         "dense_finetune_step": dense,
+        "geglu_ffn_step": geglu,
         "e2e": e2e,
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": clocks,
@@ -411,6 +413,74 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier):
                           "peak": peaks["hbm_gbs"], "frac": round(4 * n_el / t_avg / 1e9 / peaks["hbm_gbs"], 4)},
             "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights and the four FFN "
                     "products on the dense tcgen05 path, same workload"}
+
+
+class GegluStep:
+    """The gated FFN of the same width on the 2:4 path: stacked gate/up weight
+    [2 ff, d] (16-row groups alternate), down projection [d, ff]; per step the
+    two mask steps, the GEGLU forward, the down projection, its input gradient
+    with the gated-gradient epilogue, the stacked input gradient and both decays."""
+
+    def __init__(self, step):
+        import torch
+        import structured_sparse_transformer_b200 as sp
+        self.sp, self.torch, self.step = sp, torch, step
+        wl = step.wl
+        tdt = si.DTYPES[wl.dtype]
+        T, d, ff = wl.tokens, wl.d, wl.ff
+        g = torch.Generator().manual_seed(300)
+        mk = lambda shape, std, dt: (torch.randn(*shape, generator=g) * std).to(dt).cuda()
+        self.Wgu, self.Wd = mk((2 * ff, d), 0.02, tdt), mk((d, ff), 0.02, tdt)
+        self.Ggu, self.Gd = mk((2 * ff, d), 1e-2, torch.float32), mk((d, ff), 1e-2, torch.float32)
+        self.idx = [torch.zeros(2 * ff // 4, d // 4, dtype=torch.uint8, device="cuda"),
+                    torch.zeros(d // 4, ff // 4, dtype=torch.uint8, device="cuda")]
+        self.c = [sp.alloc_compressed(2 * ff, d, tdt), sp.alloc_compressed(d, ff, tdt)]
+        self.H = torch.empty(T, ff, dtype=tdt, device="cuda")
+        self.GU = torch.empty(T, 2 * ff, dtype=tdt, device="cuda")
+        self.dGU = torch.empty(T, 2 * ff, dtype=tdt, device="cuda")
+        self.Y = torch.empty(T, d, dtype=tdt, device="cuda")
+        self.dX = torch.empty(T, d, dtype=tdt, device="cuda")
+        self.flops = 6 * 2.0 * T * d * ff
+
+    def run(self):
+        sp, st, wl = self.sp, self.step, self.step.wl
+        d, ff = wl.d, wl.ff
+        for w, i, c in ((self.Wgu, self.idx[0], self.c[0]), (self.Wd, self.idx[1], self.c[1])):
+            sp.sp24_mask_step(w, i, None, None, *c)
+        (vr_gu, mr_gu, vc_gu, mc_gu), (vr_d, mr_d, vc_d, mc_d) = self.c
+        sp.sp24_gemm_fwd(st.X, vr_gu, mr_gu, 2 * ff, self.H, "geglu", self.GU)
+        sp.sp24_gemm_fwd(self.H, vr_d, mr_d, d, self.Y)
+        sp.sp24_gemm_dgrad(st.dY, vc_d, mc_d, ff, self.dGU, "dgeglu", self.GU)
+        sp.sp24_gemm_dgrad(self.dGU, vc_gu, mc_gu, d, self.dX)
+        sp.sp24_masked_decay(self.Ggu, self.Wgu, self.idx[0], wl.lam)
+        sp.sp24_masked_decay(self.Gd, self.Wd, self.idx[1], wl.lam)
+
+
+def run_geglu_phase(args, step, wl, world, dev, flush, barrier):
+    """The gated FFN step, timed like the 2:4 step."""
+    import torch
+    import structured_sparse_transformer_b200 as sp
+    g = GegluStep(step)
+    for _ in range(args.warmup):
+        g.run()
+    ev = []
+    barrier()
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.run()
+        e.record()
+        ev.append((s, e))
+    barrier()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the gated step: {sp.sp24_status_string(st)}")
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world, dev) / args.steps
+    return {"ms_per_step": round(ms, 4), "value": round(g.flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "note": "gated FFN (GEGLU) of the same d and ff on the 2:4 path: stacked gate/up weight [2 ff, d], "
+                    "down projection [d, ff]; mask steps, the four GEMMs with the gated epilogues, both decays; "
+                    "FLOPs 6 x 2 T d ff dense-equivalent"}
 
 
 def run_e2e(args, step, wl, world, dev, barrier):
