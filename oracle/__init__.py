@@ -25,6 +25,11 @@ Pre-training with 2:4 Sparsity"):
   ``g + lambda * (not m) * W`` as one fp32 fused multiply-add (plain C).
 * ``flip_count`` -- abstract: the flip rate monitoring mask stability, read as
   the number of mask entries that differ between two masks.
+* ``mvue_sparsify_t`` / ``weight_grad`` -- the weight gradient ``dW = Yhat X``
+  with Yhat the minimum-variance unbiased 2:4 estimate of dY^T along tokens (the
+  MVUE kernel of the Software Dependencies row; the estimator is this project's
+  reading, see ``mvue_select``), drawn with ``philox4x64_10`` (Salmon et al.,
+  SC 2011) so that both sides use the same random numbers.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against exhaustive
 search, closed forms, invariants or exact rational arithmetic.
@@ -295,3 +300,180 @@ def flip_count(idx_prev: np.ndarray, idx_cur: np.ndarray) -> int:
 def flip_rate(idx_prev: np.ndarray, idx_cur: np.ndarray) -> float:
     """``flip_count / (R*C)``: the fraction of weights whose mask bit changed."""
     return flip_count(idx_prev, idx_cur) / (16.0 * idx_cur.size)
+
+
+# --------------------------------------- weight gradient with the MVUE of dY
+
+# Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as
+# easy as 1, 2, 3", SC 2011): the round multipliers and the key increments
+# (golden ratio and sqrt(3) - 1 in 0.64 fixed point) of the published definition.
+PHILOX_M = (0xD2E7470EE14C6C93, 0xCA5A826395121157)
+PHILOX_W = (0x9E3779B97F4A7C15, 0xBB67AE8584CAA73B)
+_U64 = (1 << 64) - 1
+
+
+def _mulhilo64(m: int, a: np.ndarray):
+    """(high, low) 64-bit halves of the 128-bit product m * a, from 32-bit pieces."""
+    a = np.asarray(a, np.uint64)
+    lo32 = np.uint64(0xFFFFFFFF)
+    s32 = np.uint64(32)
+    mlo, mhi = np.uint64(m & 0xFFFFFFFF), np.uint64(m >> 32)
+    alo, ahi = a & lo32, a >> s32
+    ll, lh, hl, hh = alo * mlo, alo * mhi, ahi * mlo, ahi * mhi
+    cross = (ll >> s32) + (lh & lo32) + (hl & lo32)
+    lo = (ll & lo32) | (cross << s32)
+    hi = hh + (lh >> s32) + (hl >> s32) + (cross >> s32)
+    return hi, lo
+
+
+def philox4x64_10(ctr: np.ndarray, key) -> np.ndarray:
+    """Philox4x64 with 10 rounds: uint64 counters [..., 4] and a two-word key -> uint64 [..., 4].
+
+    Round: (c0, c1, c2, c3) -> (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1, lo(M0 c0));
+    the key grows by the Weyl increments before every round but the first."""
+    ctr = np.asarray(ctr, np.uint64)
+    c = [ctr[..., i] for i in range(4)]
+    k0, k1 = int(key[0]) & _U64, int(key[1]) & _U64
+    for r in range(10):
+        if r:
+            k0, k1 = (k0 + PHILOX_W[0]) & _U64, (k1 + PHILOX_W[1]) & _U64
+        hi0, lo0 = _mulhilo64(PHILOX_M[0], c[0])
+        hi1, lo1 = _mulhilo64(PHILOX_M[1], c[2])
+        c = [hi1 ^ c[1] ^ np.uint64(k0), lo1, hi0 ^ c[3] ^ np.uint64(k1), lo0]
+    return np.stack(c, axis=-1)
+
+
+def mvue_uniforms(rows: int, groups: int, seed: int, offset: int) -> np.ndarray:
+    """The uniform draw of every group of four of the sparsified operand, float64 [rows, groups].
+
+    Group g of row n takes 32 bits of philox4x64_10(counter (g // 8, n, 0, 0), key (seed, offset)):
+    word (g % 8) // 2, low half for even g, high half for odd g.  The top 24 of those bits,
+    times 2^-24, give u in [0, 1 - 2^-24] (exact in fp32 and fp64)."""
+    n = np.arange(rows, dtype=np.uint64)[:, None]
+    blk = np.arange((groups + 7) // 8, dtype=np.uint64)[None, :]
+    ctr = np.zeros((rows, blk.shape[1], 4), np.uint64)
+    ctr[..., 0] = blk
+    ctr[..., 1] = n
+    words = philox4x64_10(ctr, (seed, offset))                   # [rows, blocks, 4]
+    g = np.arange(groups)
+    w = words[:, g // 8, (g % 8) // 2]                           # [rows, groups]
+    u32 = np.where((g % 2) == 0, w & np.uint64(0xFFFFFFFF), w >> np.uint64(32))
+    return (u32 >> np.uint64(8)).astype(np.float64) * 2.0 ** -24
+
+
+def mvue_select(v: np.ndarray, u: np.ndarray):
+    """Minimum-variance unbiased 2:4 estimate of each group of four values.
+
+    ``v`` float64 [..., 4] (exact fp16/bf16 values), ``u`` float64 [...] uniform draws.
+    Returns (pos [..., 2] kept positions ascending, est [..., 2] float64 estimates there).
+
+    Reading of the "MVUE kernel" the pages name (reproducibility table, Software
+    Dependencies row): an unbiased estimate with exactly two of four kept whose summed
+    variance sum_i v_i^2 (1/p_i - 1) is least.  That fixes the keep probabilities at
+    p_i = min(1, c |v_i|) with sum p_i = 2, and the estimate at v_i / p_i where kept.
+    Two kept values are drawn by systematic sampling with one uniform u:
+      * no |v_i| reaches half the group's sum S: points u S/2 and u S/2 + S/2 on the
+        cumulative sums of |v| in index order select two distinct entries, each with
+        probability 2 |v_i| / S, kept as sign(v_i) S/2;
+      * otherwise the largest |v_m| (lowest index among equal) is kept as is, and one
+        point u R on the cumulative sums of the other three (R their sum) selects the
+        second, kept as sign(v_k) R; if R = 0 the lowest other position is kept as +0.
+    Every step is an fp64 operation in the order written (each sum is exact for fp16
+    groups); an entry is selected by counting the cumulative sums at or below the point.
+    """
+    v = np.asarray(v, np.float64)
+    u = np.asarray(u, np.float64)
+    a = np.abs(v)
+    a0, a1, a2, a3 = a[..., 0], a[..., 1], a[..., 2], a[..., 3]
+    c1 = a0
+    c2 = c1 + a1
+    c3 = c2 + a2
+    s = c3 + a3
+    m = np.argmax(a, axis=-1)
+    am = np.take_along_axis(a, m[..., None], axis=-1)[..., 0]
+    capped = (am + am) >= s
+
+    # systematic sampling with two points half the total apart
+    h = s * 0.5
+    p1 = u * h
+    p2 = p1 + h
+    i1 = (c1 <= p1).astype(np.int64) + (c2 <= p1) + (c3 <= p1)
+    i2 = (c1 <= p2).astype(np.int64) + (c2 <= p2) + (c3 <= p2)
+    # Only a rounded cumulative sum can put both points in one entry; then the second
+    # goes to the next nonzero entry after the first, else the last nonzero one before it.
+    nz = a > 0
+    coll = i2 == i1
+    if np.any(coll & ~capped):
+        for ix in zip(*np.nonzero(coll & ~capped)):
+            j1 = int(i1[ix])
+            after = [j for j in range(j1 + 1, 4) if nz[ix][j]]
+            before = [j for j in range(j1 - 1, -1, -1) if nz[ix][j]]
+            i2[ix] = after[0] if after else before[0]
+
+    # the largest entry kept, one point over the other three
+    b = np.where(np.arange(4) == m[..., None], 0.0, a)
+    e1 = b[..., 0]
+    e2 = e1 + b[..., 1]
+    e3 = e2 + b[..., 2]
+    r = e3 + b[..., 3]
+    p = u * r
+    k = (e1 <= p).astype(np.int64) + (e2 <= p) + (e3 <= p)
+    k = np.where(r > 0, k, np.where(m == 0, 1, 0))
+
+    vm = np.take_along_axis(v, m[..., None], axis=-1)[..., 0]
+    vk = np.take_along_axis(v, k[..., None], axis=-1)[..., 0]
+    v1 = np.take_along_axis(v, i1[..., None], axis=-1)[..., 0]
+    v2 = np.take_along_axis(v, i2[..., None], axis=-1)[..., 0]
+    xk = np.where(r > 0, np.copysign(r, vk), 0.0)
+
+    pa = np.where(capped, m, i1)
+    pb = np.where(capped, k, i2)
+    xa = np.where(capped, vm, np.copysign(h, v1))
+    xb = np.where(capped, xk, np.copysign(h, v2))
+    swap = pa > pb
+    pos = np.stack([np.where(swap, pb, pa), np.where(swap, pa, pb)], axis=-1)
+    est = np.stack([np.where(swap, xb, xa), np.where(swap, xa, xb)], axis=-1)
+    return pos, est
+
+
+def _f64_to_bits_via_f32(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Storage bits of RNE_dtype(RNE_fp32(x))."""
+    x32 = np.asarray(x, np.float64).astype(np.float32)
+    if dtype == "f16":
+        return x32.astype(np.float16).view(np.uint16)
+    if dtype == "bf16":
+        import torch
+        return torch.from_numpy(np.ascontiguousarray(x32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    raise ValueError(dtype)
+
+
+def mvue_sparsify_t(dy_bits: np.ndarray, dtype: str, seed: int, offset: int):
+    """MVUE 2:4 sparsification of dY^T along the token axis.
+
+    ``dy_bits`` uint16 [T, N] (T % 4 == 0).  Row n of the result is column n of dY,
+    with every group of four consecutive tokens reduced to two kept estimates
+    (``mvue_select`` with the draws of ``mvue_uniforms(N, T/4, seed, offset)``),
+    each stored as RNE_dtype(RNE_fp32(estimate)).
+    Returns (bits [N, T] dense storage bits with +0 at dropped tokens, keep [N, T] bool,
+    est [N, T] float64 unrounded estimates with 0 at dropped tokens)."""
+    dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    T, N = dy_bits.shape
+    if T % 4:
+        raise ValueError("token count must be a multiple of 4")
+    v = to_f64(np.ascontiguousarray(dy_bits.T), dtype).reshape(N, T // 4, 4)
+    u = mvue_uniforms(N, T // 4, seed, offset)
+    pos, est = mvue_select(v, u)
+    keep = np.zeros((N, T // 4, 4), bool)
+    dense = np.zeros((N, T // 4, 4), np.float64)
+    nn, gg = np.meshgrid(np.arange(N), np.arange(T // 4), indexing="ij")
+    for j in range(2):
+        keep[nn, gg, pos[..., j]] = True
+        dense[nn, gg, pos[..., j]] = est[..., j]
+    bits = np.where(keep, _f64_to_bits_via_f32(dense, dtype), np.uint16(0)).astype(np.uint16)
+    return bits.reshape(N, T), keep.reshape(N, T), dense.reshape(N, T)
+
+
+def weight_grad(yhat: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """fp64 ``dW = Yhat X`` for the sparsified dY^T, Yhat [N, T], and the layer input X [T, K]
+    (the FFN weight gradient, dW [N, K] in the layout of W)."""
+    return np.asarray(yhat, np.float64) @ np.asarray(x, np.float64)
