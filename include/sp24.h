@@ -194,6 +194,49 @@ SP24_API sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, 
                            void *stream);
 
 /*
+ * MVUE 2:4 sparsification of dY^T along tokens (the MVUE kernel of the Software
+ * Dependencies row), the sparse operand of the weight-gradient GEMM.  The pages
+ * name the kernel without defining it; this call computes, per column n of dY
+ * and group g of four consecutive tokens, the minimum-variance unbiased
+ * estimate that keeps exactly two of the four: keep probabilities
+ * p_i = min(1, c |v_i|) with sum 2 and kept values v_i / p_i, drawn by
+ * systematic sampling with one uniform u.  If no |v_i| reaches half the
+ * group's magnitude sum S, the points u S/2 and u S/2 + S/2 on the cumulative
+ * |v| sums (index order) pick two entries, kept as sign(v_i) S/2; otherwise the
+ * largest |v_m| (lowest index among equal) is kept as is and the point u R on
+ * the cumulative sums of the other three (sum R) picks one more, kept as
+ * sign(v_k) R (R = 0: the lowest other position, as +0).  Decisions are fp64
+ * operations in that order; stored values are RNE_dtype(RNE_fp32(estimate)).
+ * u: the top 24 bits, times 2^-24, of the 32-bit half (g % 2) of word
+ * (g % 8) / 2 of Philox4x64-10 (Salmon et al., SC 2011) at counter
+ * (g / 8, n, 0, 0) and key (seed, offset): identical for a given
+ * (seed, offset) on every call and device.
+ *   dY    device [T x N] row-major, leading dimension ldy (ldy >= N, ldy % 8 == 0)
+ *   vals, meta  device: dY^T [N x T] compressed along T, in the layout of
+ *         sp24_prune_compress's row operand (sizes from
+ *         sp24_compressed_size(N, T)); whole metadata chunks are written,
+ *         padding with positions (0, 1)
+ * T % 16 == 0, N % 8 == 0; all pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_mvue_sparsify(const void *dY, int64_t T, int64_t N, int64_t ldy, sp24_dtype dtype,
+                               uint64_t seed, uint64_t offset, void *vals, void *meta, void *stream);
+
+/*
+ * Weight-gradient GEMM of an FFN layer with the MVUE-sparsified output
+ * gradient: dW[N x K] = Yhat[N x T] * X[T x K], Yhat = sp24_mvue_sparsify(dY)
+ * (2:4 along tokens), fp32 accumulation and fp32 output in W's layout (the
+ * gradient sp24_masked_decay takes).  Same tcgen05 pipeline as the other 2:4
+ * GEMMs, with X read as stored (token-major) by the tensor memory accelerator.
+ *   X     device [T x K] row-major, contiguous (the layer input: X for W1,
+ *         the hidden activation for W2)
+ *   vals, meta  device, from sp24_mvue_sparsify with the same T and N
+ *   dW    device fp32 [N x K] contiguous, overwritten (zeros when T == 0)
+ * T % 16 == 0, N % 16 == 0, K % 8 == 0; all pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
+                            int64_t N, sp24_dtype dtype, float *dW, void *stream);
+
+/*
  * Masked decay on gradients (abstract; masked decay kernel of the Software
  * Dependencies row): grad <- grad + lambda * W where the mask is 0, unchanged
  * where it is 1, as one fp32 fused multiply-add per pruned entry (in place).

@@ -38,6 +38,8 @@ _SIGNATURES = {
     "sp24_gemm_dgrad": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
     "sp24_gemm_dense": [P, I64, I64, P, I64, I32, P, I32, P, P],
     "sp24_transpose": [P, I64, I64, I32, P, P],
+    "sp24_mvue_sparsify": [P, I64, I64, I64, I32, U64, U64, P, P, P],
+    "sp24_gemm_wgrad": [P, I64, I64, P, P, I64, I32, P, P],
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
     "sp24_flip_rate": [P, P, I64, P, P],
     "sp24_meta_to_canonical": [P, I64, I64, P],
@@ -203,6 +205,24 @@ def sp24_transpose(x, out, stream=None):
     _need_cuda(x, out)
     R, C = x.shape
     _check("sp24_transpose", _lib.sp24_transpose(_ptr(x), R, C, _dtype_code(x), _ptr(out), _stream(stream)))
+
+
+def sp24_mvue_sparsify(dY, seed: int, offset: int, vals, meta, stream=None):
+    """vals/meta <- dY[T, N]^T compressed 2:4 along T with the MVUE draws of (seed, offset)."""
+    _need_cuda(dY, vals, meta)
+    T, N = dY.shape
+    _check("sp24_mvue_sparsify",
+           _lib.sp24_mvue_sparsify(_ptr(dY), T, N, dY.stride(0), _dtype_code(dY), int(seed) & (2**64 - 1),
+                                   int(offset) & (2**64 - 1), _ptr(vals), _ptr(meta), _stream(stream)))
+
+
+def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
+    """dW[N, K] (fp32) <- Yhat[N, T] X[T, K] with Yhat from sp24_mvue_sparsify."""
+    _need_cuda(X, vals, meta, dW)
+    T, K = X.shape
+    _check("sp24_gemm_wgrad",
+           _lib.sp24_gemm_wgrad(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(dW),
+                                _stream(stream)))
 
 
 def sp24_masked_decay(grad, W, idx, lam: float, stream=None):

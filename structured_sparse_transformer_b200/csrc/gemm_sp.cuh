@@ -75,7 +75,10 @@ constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at column
 // half width, aux <- both pre-activations); and its input gradient (aux =
 // both pre-activations, read; out = (d gate, d up) interleaved at twice the
 // accumulator width).
-enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4 };
+// The weight gradient (wgrad) is its own variant: A = the MVUE-sparsified dY^T
+// [N x T], B = the layer input [T x K] read MN-major, out = dW [N x K] fp32 in
+// the natural orientation (see PairGeom and the wgrad epilogue below).
+enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4, kEpiWgrad = 5 };
 constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in the stacked gated weight
 
 // Pipeline stage of the 2:4 GEMM (SPARSE) and of the dense GEMM of the dense
@@ -83,14 +86,29 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // two 64-K boxes of B and the 2 KB metadata chunk (46 KB), 4 stages (3 when
 // the gated-GELU gradient epilogue takes 6 KB of staging per warp).  Dense:
 // 64 K per stage, one box of A and one of B (30 KB), 6 stages.
+//
+// Weight gradient (EPI == kEpiWgrad, sparse): pair tiles of 256 rows of dW x
+// 256 columns.  B comes from the row-major layer input [T x K] (K contiguous),
+// i.e. MN-major for the MMA: per stage each CTA loads two 128B-swizzled atoms
+// of 64 columns x 128 tokens (16 KB each; atom a of CTA r holds columns
+// 128a + 64r .. +63 of the tile), so a stage is 50 KB and 4 stages fit.  Each
+// 32-token K step issues two MMAs of N = 128 (one per atom; the pair's two
+// 64-column halves make the 128), into accumulator columns 0 and 128: an MMA
+// never spans two atoms along N.  One 256-column accumulator (no double
+// buffering: the weight-gradient tiles run one per pair at the FFN sizes).
 template <bool SPARSE, int EPI>
 struct PairGeom {
+  static constexpr bool kWg = EPI == kEpiWgrad;
   static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
   static constexpr int kAcols = 64;                      // A values per row and stage
+  static constexpr int kBN = kWg ? 256 : kPairBN;        // B columns (tokens, or dW columns) per pair tile
   static constexpr int kBBoxes = SPARSE ? 2 : 1;
+  static constexpr int kBBoxBytes = kWg ? 64 * 128 * 2 : kPairSmemBBox;
   static constexpr int kMeta = SPARSE ? kSmemE : 0;
-  static constexpr int kStageBytes = kPairSmemA + kBBoxes * kPairSmemBBox + kMeta;
+  static constexpr int kStageBytes = kPairSmemA + kBBoxes * kBBoxBytes + kMeta;
   static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
+  static constexpr int kAccBufs = kWg ? 1 : 2;
+  static constexpr int kMetaCol = kAccBufs * kBN;        // metadata columns after the accumulators
 };
 constexpr int kEpiBufBytes = kEpiTokens * 32 * 2;      // staging tile: 16 tokens x 32 features, 64B-swizzled
 constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM address, abort flag
@@ -100,16 +118,24 @@ constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM addres
 // pre-activations; gated gradient: a 2 KB out tile + two 2 KB pre-activation
 // inputs.
 __host__ __device__ constexpr int epi_bufs(int epi) {
-  return epi == kEpiNone ? 1 : (epi == kEpiGelu || epi == kEpiGeglu) ? 2 : (epi == kEpiDgelu ? 3 : 6);
+  return epi == kEpiWgrad ? 0
+                          : epi == kEpiNone ? 1 : (epi == kEpiGelu || epi == kEpiGeglu) ? 2 : (epi == kEpiDgelu ? 3 : 6);
 }
+// The wgrad variant keeps 8 KB unused after its barriers, so that its MN-major
+// B reads stay inside the allocation under any reading of the descriptor strides.
 template <bool SPARSE, int EPI>
 __host__ __device__ constexpr int pair_smem_bytes() {
   return PairGeom<SPARSE, EPI>::kStages * PairGeom<SPARSE, EPI>::kStageBytes + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
-         kPairBarBytes + 1024;
+         kPairBarBytes + 1024 + (EPI == kEpiWgrad ? 8192 : 0);
 }
 static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<false, kEpiDgelu>() <= 232448 &&
-                  pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448,
+                  pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448 &&
+                  pair_smem_bytes<true, kEpiWgrad>() <= 232448,
               "shared memory per CTA");
+static_assert(PairGeom<true, kEpiWgrad>::kStageBytes % 1024 == 0 && PairGeom<true, kEpiWgrad>::kBBoxBytes % 1024 == 0,
+              "128B-swizzled tiles need 1 KB aligned starts");
+static_assert(PairGeom<true, kEpiWgrad>::kMetaCol + 4 * PairGeom<true, kEpiWgrad>::kStages <= kTmemCols,
+              "tensor memory budget (wgrad)");
 static_assert(PairGeom<true, kEpiNone>::kStageBytes % 1024 == 0 && PairGeom<false, kEpiNone>::kStageBytes % 1024 == 0 &&
                   kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
@@ -284,8 +310,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
                           const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
-                          uint64_t wait_budget) {
+                          uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out) {
+  // T counts the B operand's rows of the output: tokens, or for the weight
+  // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
   using G = PairGeom<SPARSE, EPI>;
+  constexpr bool WG = G::kWg;
   constexpr int kPairStages = G::kStages;
   constexpr int kPairStageBytes = G::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -309,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_mt = (M + 2 * kPairRows - 1) / (2 * kPairRows);
   const int num_row_tiles = (M + kPairRows - 1) / kPairRows;
-  const int num_tiles = num_mt * ((T + kPairBN - 1) / kPairBN);
+  const int num_tiles = num_mt * ((T + G::kBN - 1) / G::kBN);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -347,7 +376,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
       const int mt = tile % num_mt;
       const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
-      const int b_row = (tile / num_mt) * kPairBN + (int)rank * kPairBNh;
+      const int b_row = (tile / num_mt) * G::kBN + (int)rank * (WG ? 64 : kPairBNh);
       // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
       // it the last real metadata chunk so every code the MMA sees is valid.
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
@@ -360,11 +389,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         uint8_t *st = stage_base + s * kPairStageBytes;
         if (is_leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
         tma_load_2d_pair(st, &tm_a, &full[s], kt * G::kAcols, a_row);
-        tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
-        if (SPARSE) {
-          tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * G::kBK + 64, b_row);
-          tma_load_2d_pair(st + kPairSmemA + 2 * kPairSmemBBox, &tm_meta, &full[s], 0, chunk_row + kt);
+        if (WG) {
+          // MN-major atoms: x = dW column (b_row, b_row + 128), y = token.
+          tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], b_row, kt * G::kBK);
+          tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 128, kt * G::kBK);
+        } else {
+          tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
+          if (SPARSE) tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * G::kBK + 64, b_row);
         }
+        if (SPARSE)
+          tma_load_2d_pair(st + kPairSmemA + 2 * G::kBBoxBytes, &tm_meta, &full[s], 0, chunk_row + kt);
       }
     }
     // The leader's `full` barriers count both CTAs' bytes: let every copy land.
@@ -378,27 +412,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------- MMA issuer (leader)
     // Descriptors of stage 0; stage s and K step kk only move the 14-bit start
     // address field (all of shared memory is below 2^18 bytes, so it never carries).
-    constexpr uint32_t idesc =
-        SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN) : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
+    // wgrad: N = 128 per MMA and B MN-major (instruction descriptor bit 16).
+    // Its B descriptor steps 8-token groups 1024 bytes apart (the stride field);
+    // an MMA reads a single 64-column atom per CTA, so the field for the stride
+    // between atoms along N is never used and is given the same 1024.
+    constexpr uint32_t idesc = WG ? (make_idesc_sparse(BF16, 2 * kPairRows, 128) | (1u << 16))
+                               : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN)
+                                        : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
     const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
-    const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), 16, 1024, kSwizzle128B);
-    const uint64_t e_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA + 2 * kPairSmemBBox), 128, 128, kSwizzleNone);
+    const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
+    const uint64_t e_desc0 =
+        smem_desc(smem_u32(stage_base + kPairSmemA + 2 * G::kBBoxBytes), 128, 128, kSwizzleNone);
     uint32_t g = 0;
     bool ok = true;
     int j = 0;
     for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++j) {
-      const int b = j & 1;
-      const uint32_t use = (uint32_t)(j >> 1);
+      const int b = j % G::kAccBufs;
+      const uint32_t use = (uint32_t)(j / G::kAccBufs);
       if (!(ok = mbar_wait_bounded(&acc_empty[b], (use & 1u) ^ 1u, wait_budget, s_abort))) break;
       tc_fence_after();
-      const uint32_t acc = tmem_base + (uint32_t)(b * kPairBN);
+      const uint32_t acc = tmem_base + (uint32_t)(b * G::kBN);
       for (int kt = 0; kt < num_kt; ++kt, ++g) {
         const int s = (int)(g % kPairStages);
         if (!(ok = mbar_wait_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
         tc_fence_after();
         const uint64_t so = (uint64_t)((s * kPairStageBytes) >> 4);
         const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
-        if (SPARSE) {
+        if (WG) {
+          const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;
+          tc_cp_128x128b_pair(t_meta, e_desc0 + so);
+          // K step kk: A advances 32 bytes along its swizzled rows, B 32 tokens
+          // (4096 bytes); atom 1 of B sits 16 KB after atom 0.
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t tm = t_meta + 2 * (kk >> 1);
+            const uint32_t id = idesc | (uint32_t)(kk & 1);
+            const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
+            const uint64_t bk = bd + (uint64_t)(kk * (4096 >> 4));
+            tc_mma_sp_f16_pair(acc, ad + 2 * kk, bk, tm, id, accum);
+            tc_mma_sp_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), tm, id, accum);
+          }
+        } else if (SPARSE) {
           const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
           tc_cp_128x128b_pair(t_meta, e_desc0 + so);
           // The metadata operand address must be 2-column aligned; the low column
@@ -422,6 +476,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_commit_pair(drain, 0x1);
       volatile int no_abort = 0;
       mbar_wait_bounded(drain, 0, kDrainBudget, &no_abort);
+    }
+  } else if (warp >= 2 && WG) {
+    // ------------------------------------------ weight-gradient epilogue (both CTAs)
+    // Warp w drains TMEM lanes 32q..32q+31 (q = w%4; rows of dW) at the 16-column
+    // chunks grp, grp + kEpiGroups, ... of the accumulator, three chunks per
+    // round trip.  Register layout of tmem_ld_16x256b_x2: thread t holds row
+    // t/4 (+8) at columns 2(t%4), +1 of each 8-column block, so each float2
+    // store of a warp writes 8 rows x 32 contiguous bytes (whole sectors of dW).
+    const int grp = (warp - 2) >> 2;
+    const int q = warp & 3;
+    constexpr int kChunks = G::kBN / 16;
+    constexpr int kPerWarp = (kChunks + kEpiGroups - 1) / kEpiGroups;
+    constexpr int kBatch = 3;
+    int j = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
+      const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
+      const int n0 = (tile / num_mt) * G::kBN;
+      const bool got = mbar_wait_bounded(&acc_full[0], (uint32_t)j & 1u, wait_budget, s_abort);
+      if (!__all_sync(0xFFFFFFFFu, got)) break;
+      tc_fence_after();
+      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16);
+#pragma unroll
+      for (int k0 = 0; k0 < kPerWarp; k0 += kBatch) {
+        uint32_t r[kBatch][2][8];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+          const int ch = grp + (k0 + k) * kEpiGroups;
+          if (ch < kChunks) {
+            tmem_ld_16x256b_x2(t_base + (uint32_t)(16 * ch), r[k][0]);
+            tmem_ld_16x256b_x2(t_base + (16u << 16) + (uint32_t)(16 * ch), r[k][1]);
+          }
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+          reg_fence(r[k][0]);
+          reg_fence(r[k][1]);
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+          const int ch = grp + (k0 + k) * kEpiGroups;
+          if (ch >= kChunks) break;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int sub = 0; sub < 2; ++sub) {
+                const int row = m0 + 16 * h + 8 * sub + (lane >> 2);
+                const int col = n0 + 16 * ch + 8 * i + 2 * (lane & 3);
+                if (row < M && col < T)
+                  *reinterpret_cast<float2 *>(out_f32 + (int64_t)row * ld_out + col) =
+                      make_float2(__uint_as_float(r[k][h][4 * i + 2 * sub]),
+                                  __uint_as_float(r[k][h][4 * i + 2 * sub + 1]));
+              }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_leader(&acc_empty[0]);
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------- epilogue (both CTAs)

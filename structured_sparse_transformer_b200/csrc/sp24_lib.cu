@@ -14,6 +14,7 @@
 #include "sp24.h"
 #include "gemm_sp.cuh"
 #include "mask_kernels.cuh"
+#include "mvue.cuh"
 
 namespace {
 
@@ -109,6 +110,8 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 
 // CTA-pair kernel: clusters of two CTAs, 256 x 224 tiles (see gemm_sp.cuh).
 // SPARSE: A = kept values [M x Kd/2] + metadata chunks; dense: A = [M x Kd].
+// Weight gradient (kEpiWgrad): B = the layer input [Kd tokens x T columns]
+// read MN-major, out = fp32 [M x T]; tiles of 256 x 256.
 template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream) {
@@ -117,8 +120,12 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
   const uint64_t a_cols = SPARSE ? (uint64_t)(Kd / 2) : (uint64_t)Kd;
   CUtensorMap ta, tb, tm;
+  const bool b_ok = G::kWg ? make_map_2d(&tb, B, (uint64_t)T, (uint64_t)Kd, (uint64_t)T * 2, 64, (uint32_t)G::kBK,
+                                         CU_TENSOR_MAP_SWIZZLE_128B)
+                           : make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh,
+                                         CU_TENSOR_MAP_SWIZZLE_128B);
   if (!make_map_2d(&ta, vals, a_cols, (uint64_t)M, a_cols * 2, G::kAcols, kPairRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh, CU_TENSOR_MAP_SWIZZLE_128B))
+      !b_ok)
     return SP24_ERR_CUDA;
   if (SPARSE) {
     if (!make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
@@ -132,7 +139,11 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   // gradient: out and aux 64 columns (128B swizzle) over twice the width.
   CUtensorMap to, tx;
   bool maps_ok;
-  if (EPI == kEpiGeglu) {
+  if (G::kWg) {   // direct fp32 stores: no staging maps
+    to = ta;
+    tx = ta;
+    maps_ok = true;
+  } else if (EPI == kEpiGeglu) {
     maps_ok = make_map_2d(&to, out, (uint64_t)M / 2, (uint64_t)T, (uint64_t)M, 16, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               make_map_2d(&tx, aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B);
   } else if (EPI == kEpiDgeglu) {
@@ -168,10 +179,11 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
     }
     max_pairs = n;
   }
-  const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + kPairBN - 1) / kPairBN);
+  const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
-                    (int)T, num_kt, (uint64_t)g_wait_budget.load());
+                    (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
+                    (int64_t)(G::kWg ? T : 0));
 }
 
 template <bool SPARSE>
@@ -405,6 +417,47 @@ sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtyp
                                                                             : 65535));
   return launch_pdl(transpose16_kernel, grid, dim3(256), 0, as_stream(stream),
                     static_cast<const uint16_t *>(in), static_cast<uint16_t *>(out), rows, cols);
+}
+
+sp24_status sp24_mvue_sparsify(const void *dY, int64_t T, int64_t N, int64_t ldy, sp24_dtype dtype, uint64_t seed,
+                               uint64_t offset, void *vals, void *meta, void *stream) {
+  if (T < 0 || N < 0 || ldy < N) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (T % 16 || N % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || N > (int64_t)65535 / 2 * 128) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0 || N == 0) return SP24_OK;
+  if (!dY || !vals || !meta) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dY) || !aligned16(vals) || !aligned16(meta) || ldy % 8) return SP24_ERR_MISALIGNED;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  // Whole metadata chunks: 128 tokens x 128 columns, two CTAs per chunk.
+  const dim3 grid((unsigned)((T + kMvueTokens - 1) / kMvueTokens), (unsigned)(2 * ((N + 127) / 128)));
+  cudaStream_t s = as_stream(stream);
+  const uint16_t *d16 = static_cast<const uint16_t *>(dY);
+  uint16_t *v16 = static_cast<uint16_t *>(vals);
+  uint8_t *m8 = static_cast<uint8_t *>(meta);
+  return dtype == SP24_BF16
+             ? launch_pdl(mvue_sparsify_kernel<true>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, seed, offset, v16, m8)
+             : launch_pdl(mvue_sparsify_kernel<false>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, seed, offset, v16, m8);
+}
+
+sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *vals, const void *meta, int64_t N,
+                            sp24_dtype dtype, float *dW, void *stream) {
+  if (T < 0 || K < 0 || N < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (T % 16 || N % 16 || K % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!dW || (T > 0 && (!X || !vals || !meta))) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (T > 0 && (!aligned16(X) || !aligned16(vals) || !aligned16(meta)))) return SP24_ERR_MISALIGNED;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {   // an empty sum over tokens
+    return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  }
+  return dtype == SP24_BF16 ? launch_gemm_pair_t<true, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s)
+                            : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s);
 }
 
 sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,

@@ -7,7 +7,9 @@
 W is [rows x cols] (N(0, 0.02), or the 8-level tie-heavy variant with
 --dist tie), drawn on the device from a seeded generator.  GEMMs use
 T = --tokens rows of N(0, 1) activations: gemm_fwd computes [T x rows] from
-[T x cols], gemm_dgrad [T x cols] from [T x rows].  Each timed launch follows an
+[T x cols], gemm_dgrad [T x cols] from [T x rows], gemm_wgrad the fp32
+[rows x cols] weight gradient from dY [T x rows] (MVUE-sparsified) and
+X [T x cols]; mvue sparsifies dY [T x rows] (bytes per dY element).  Each timed launch follows an
 L2 flush (256 MiB write) and is timed alone with CUDA events on the current
 stream.  Prints one JSON line: average microseconds per launch and the
 algorithmic throughput (bytes for the memory-bound kernels, dense-equivalent
@@ -30,13 +32,15 @@ BYTES_PER_ELEMENT = {
     "masked_decay": 4 + 2 + 1 / 16 + 4,              # read g, W, index; write g
     "flip": 2 / 16,                                  # read two indices
     "transpose": 4,                                  # read W, write W^T
+    "mvue": 2 + 1 + 1 / 8,                           # read dY; write kept values and metadata
 }
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--kernel", required=True,
-                    choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad", "gemm_dense_fwd", "gemm_dense_dgrad"])
+                    choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad", "gemm_dense_fwd", "gemm_dense_dgrad",
+                                                         "gemm_wgrad"])
     ap.add_argument("--rows", type=int, required=True)
     ap.add_argument("--cols", type=int, required=True)
     ap.add_argument("--tokens", type=int, default=8192)
@@ -83,6 +87,17 @@ def main(argv=None):
         aux = torch.empty(T, R, dtype=tdt, device=dev) if args.epi == "gelu" else None
         epi = "gelu" if args.epi == "gelu" else None
         fn = lambda: sp.sp24_gemm_fwd(x, bufs[0], bufs[1], R, y, epi, aux)
+    elif k in ("mvue", "gemm_wgrad"):
+        dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
+        yv = torch.empty(R, T // 2, dtype=tdt, device=dev)
+        ym = torch.empty(sp.sp24_compressed_size(R, T)[1], dtype=torch.uint8, device=dev)
+        sp.sp24_mvue_sparsify(dy, 200, 0, yv, ym)
+        if k == "mvue":
+            fn = lambda: sp.sp24_mvue_sparsify(dy, 200, 1, yv, ym)
+        else:
+            x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
+            dw = torch.empty(R, C, dtype=torch.float32, device=dev)
+            fn = lambda: sp.sp24_gemm_wgrad(x, yv, ym, R, dw)
     elif k == "transpose":
         wt = torch.empty(C, R, dtype=tdt, device=dev)
         fn = lambda: sp.sp24_transpose(w, wt)
@@ -123,6 +138,8 @@ def main(argv=None):
     avg_s = total / args.iters * 1e-3
     if k.startswith("gemm"):
         amount, unit = 2.0 * T * R * C / avg_s / 1e12, "TFLOP/s"
+    elif k == "mvue":
+        amount, unit = T * R * BYTES_PER_ELEMENT[k] / avg_s / 1e9, "GB/s"
     else:
         amount, unit = R * C * BYTES_PER_ELEMENT[k] / avg_s / 1e9, "GB/s"
     print(json.dumps({"kernel": k, "rows": R, "cols": C, "tokens": T if k.startswith("gemm") else None,

@@ -71,7 +71,8 @@ class FFNWorkload:
     steps: int = 1
     lam: float = 6e-5
     seeds: dict = field(default_factory=lambda: {
-        "W1": 0, "W2": 1, "X": 2, "dY": 3, "G1": 4, "G2": 5, "perturb": 100})
+        "W1": 0, "W2": 1, "X": 2, "dY": 3, "G1": 4, "G2": 5, "H": 6, "dH": 7, "perturb": 100,
+        "mvue": 200})
 
     def weights(self):
         return (normal((self.ff, self.d), 0.02, self.seeds["W1"], self.dtype),
@@ -80,6 +81,12 @@ class FFNWorkload:
     def activations(self):
         return (normal((self.tokens, self.d), 1.0, self.seeds["X"], self.dtype),
                 normal((self.tokens, self.d), 1.0, self.seeds["dY"], self.dtype))
+
+    def hidden(self):
+        """Stand-ins for the hidden activation H and its gradient dH [T x ff], N(0, 1): the
+        operands of the weight-gradient products when they are tested on their own."""
+        return (normal((self.tokens, self.ff), 1.0, self.seeds["H"], self.dtype),
+                normal((self.tokens, self.ff), 1.0, self.seeds["dH"], self.dtype))
 
     def grads(self):
         return (normal((self.ff, self.d), 1e-2, self.seeds["G1"], "f32"),

@@ -104,6 +104,29 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert _raw("sp24_transpose", None, 8, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_transpose", fake, -2, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_transpose", odd, 8, 8, 0, fake, None) == E["SP24_ERR_MISALIGNED"]
+    # MVUE sparsification and the weight-gradient GEMM
+    assert _raw("sp24_mvue_sparsify", fake, 24, 64, 64, 0, 1, 2, fake, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # tokens must be a multiple of 16
+    assert _raw("sp24_mvue_sparsify", fake, 32, 12, 16, 0, 1, 2, fake, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # columns must be a multiple of 8
+    assert _raw("sp24_mvue_sparsify", fake, 32, 64, 32, 0, 1, 2, fake, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # ldy < N
+    assert _raw("sp24_mvue_sparsify", fake, 32, 64, 68, 0, 1, 2, fake, fake, None) == \
+        E["SP24_ERR_MISALIGNED"]                        # ldy not a multiple of 8
+    assert _raw("sp24_mvue_sparsify", fake, 32, 64, 64, 9, 1, 2, fake, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_DTYPE"]
+    assert _raw("sp24_mvue_sparsify", fake, 32, 64, 64, 0, 1, 2, None, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_gemm_wgrad", fake, 24, 64, fake, fake, 64, 0, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # tokens (the contraction) % 16
+    assert _raw("sp24_gemm_wgrad", fake, 32, 60, fake, fake, 64, 0, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # dW columns % 8
+    assert _raw("sp24_gemm_wgrad", fake, 32, 64, fake, fake, 40, 0, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # dW rows % 16
+    assert _raw("sp24_gemm_wgrad", fake, 32, 64, fake, fake, 64, 0, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_gemm_wgrad", fake, 32, 64, odd, fake, 64, 0, fake, None) == \
+        E["SP24_ERR_MISALIGNED"]
     # decay and flip
     assert _raw("sp24_masked_decay", fake, fake, 0, 6, 8, fake, ctypes.c_float(1.0), None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]

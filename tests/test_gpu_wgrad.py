@@ -1,0 +1,156 @@
+"""GPU parity of the MVUE sparsification of dY^T and of the weight-gradient GEMM.
+
+"Accelerating Transformer Pre-training with 2:4 Sparsity", reproducibility
+table, Software Dependencies row (the MVUE kernel, the 2:4 sparse matrix
+multiplications).  The sparsified operand is integer-decided work (which two
+of four tokens, in fp64 on both sides, from the same Philox draws), so its
+values and metadata must equal the oracle's bit for bit.  The weight gradient
+dW = Yhat X is fp32 out of fp32 tensor-core accumulation over T tokens; it is
+compared with the fp64 product of the GPU's own Yhat with a relative Frobenius
+error <= 1e-4 and a largest entry error <= 1e-3 of the largest |dW| (fp16/bf16
+products are exact in fp32, so only the accumulation rounds: about
+sqrt(T) * 2^-24 relative, 5e-6 at T = 8192).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic_inputs as si
+import structured_sparse_transformer_b200 as sp
+
+pytestmark = pytest.mark.gpu
+
+FRO_TOL = 1e-4
+MAX_TOL = 1e-3
+
+
+def _alloc(N, T, dtype):
+    vb, mb = sp.sp24_compressed_size(N, T)
+    return (torch.empty(N, T // 2, dtype=si.DTYPES[dtype], device="cuda"),
+            torch.empty(mb, dtype=torch.uint8, device="cuda"))
+
+
+def _yhat_of(vals, meta, N, T, dtype):
+    """Dense bits [N, T] of the GPU's compressed operand (host index maps only)."""
+    canon = sp.sp24_meta_to_canonical(meta.cpu().numpy().tobytes(), N, T)
+    return oracle.decompress_rows(si.bits16(vals.cpu()), canon, T), canon
+
+
+def _mixed_dy(T, N, dtype, seed):
+    """N(0, 1) with planted special groups: all zero, one, two or three nonzeros,
+    one dominant entry (the capped case) and equal magnitudes (ties)."""
+    x = si.normal((T, N), 1.0, seed, dtype).float()
+    g = torch.Generator().manual_seed(seed + 1)
+    kind = torch.randint(0, 7, (T // 4, N), generator=g)
+    grp = x.reshape(T // 4, 4, N).permute(0, 2, 1)          # [group, column, 4], a view of x
+    grp[kind == 1] = 0.0
+    grp[..., 1:][kind == 2] = 0.0
+    grp[..., 2:][kind == 3] = 0.0
+    grp[..., 0][kind == 4] *= 50.0
+    grp[kind == 5] = 0.5 * torch.sign(grp[kind == 5])
+    grp[..., 3][kind == 6] = 0.0
+    return x.to(si.DTYPES[dtype]).contiguous()
+
+
+@pytest.mark.parametrize("T,N,dtype", [(128, 64, "f16"), (256, 128, "f16"), (144, 200, "bf16"), (16, 8, "f16"),
+                                       (1040, 776, "f16"), (512, 256, "bf16")])
+def test_mvue_bit_exact(T, N, dtype):
+    dy = _mixed_dy(T, N, dtype, T + N)
+    vals, meta = _alloc(N, T, dtype)
+    sp.sp24_mvue_sparsify(dy.cuda(), 17, 5, vals, meta)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    bits, keep, _ = oracle.mvue_sparsify_t(si.bits16(dy), dtype, 17, 5)
+    ovals, ometa = oracle.compress_rows(bits, keep)
+    assert np.array_equal(si.bits16(vals.cpu()), ovals)
+    got, canon = _yhat_of(vals, meta, N, T, dtype)
+    assert np.array_equal(canon, ometa)
+    assert np.array_equal(got, bits)
+
+
+def test_mvue_leading_dimension_and_wide_bf16_groups():
+    T, N, ld = 64, 16, 40
+    base = torch.zeros(T, ld)
+    base[:, :N] = torch.randn(T, N, generator=torch.Generator().manual_seed(3))
+    base[0::4, :N] *= 1e30        # groups spanning ~100 binades
+    base[1::4, :N] *= 1e-30
+    dy = base.to(torch.bfloat16)
+    vals, meta = _alloc(N, T, "bf16")
+    sp.sp24_mvue_sparsify(dy.cuda()[:, :N], 1, 2, vals, meta)
+    torch.cuda.synchronize()
+    bits, keep, _ = oracle.mvue_sparsify_t(si.bits16(dy[:, :N].contiguous()), "bf16", 1, 2)
+    got, _ = _yhat_of(vals, meta, N, T, "bf16")
+    assert np.array_equal(got, bits)
+
+
+def test_mvue_draws_depend_on_seed_and_offset_only():
+    T, N = 256, 64
+    dy = si.normal((T, N), 1.0, 9, "f16").cuda()
+    outs = []
+    for seed, off in ((1, 1), (1, 1), (1, 2), (2, 1)):
+        vals, meta = _alloc(N, T, "f16")
+        sp.sp24_mvue_sparsify(dy, seed, off, vals, meta)
+        torch.cuda.synchronize()
+        outs.append(meta.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])
+    assert not np.array_equal(outs[0], outs[2]) and not np.array_equal(outs[0], outs[3])
+
+
+def _check_wgrad(dw, ref, what=""):
+    got = dw.double().cpu().numpy()
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    mx = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-300)
+    assert fro <= FRO_TOL, f"{what}: relative Frobenius error {fro:.3e}"
+    assert mx <= MAX_TOL, f"{what}: largest entry error {mx:.3e} of max |dW|"
+
+
+@pytest.mark.parametrize("T,N,K,dtype", [(128, 256, 256, "f16"), (256, 272, 200, "f16"), (144, 160, 520, "bf16"),
+                                         (16, 16, 8, "f16"), (2048, 512, 1024, "f16"), (400, 1040, 264, "bf16")])
+def test_wgrad_small(T, N, K, dtype):
+    dy = si.normal((T, N), 1.0, T + 3, dtype)
+    x = si.normal((T, K), 1.0, T + 4, dtype)
+    vals, meta = _alloc(N, T, dtype)
+    dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    sp.sp24_mvue_sparsify(dy.cuda(), 11, 0, vals, meta)
+    sp.sp24_gemm_wgrad(x.cuda(), vals, meta, N, dw)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    yhat, _ = _yhat_of(vals, meta, N, T, dtype)
+    ref = oracle.weight_grad(oracle.to_f64(yhat, dtype), oracle.to_f64(si.bits16(x), dtype))
+    _check_wgrad(dw, ref, f"wgrad {T}x{N}x{K}")
+
+
+def test_wgrad_zero_tokens_gives_zeros():
+    N, K = 32, 16
+    dw = torch.full((N, K), 7.0, device="cuda")
+    x = torch.empty(0, K, dtype=torch.float16, device="cuda")
+    vals, meta = _alloc(N, 16, "f16")
+    sp.sp24_gemm_wgrad(x, vals, meta, N, dw)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dw).item() == 0
+
+
+@pytest.mark.parametrize("wl", [si.GPT2_355M], ids=lambda w: w.name)
+def test_ffn_weight_grads_full_size_sampled(wl):
+    """Both weight gradients of the FFN at full size: dW2 = MVUE(dY^T) H and
+    dW1 = MVUE(dH^T) X.  The sparsified operands are compared in full; dW on
+    96 sampled rows (all columns) against the fp64 oracle."""
+    dt = wl.dtype
+    X, dY = wl.activations()
+    H, dH = wl.hidden()
+    T = wl.tokens
+    rng = np.random.default_rng(0)
+    for (g, b, N, K, off) in ((dY, H, wl.d, wl.ff, 1), (dH, X, wl.ff, wl.d, 2)):
+        vals, meta = _alloc(N, T, dt)
+        dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+        sp.sp24_mvue_sparsify(g.cuda(), wl.seeds["mvue"], off, vals, meta)
+        sp.sp24_gemm_wgrad(b.cuda(), vals, meta, N, dw)
+        torch.cuda.synchronize()
+        assert sp.sp24_device_status() == 0
+        bits, keep, _ = oracle.mvue_sparsify_t(si.bits16(g), dt, wl.seeds["mvue"], off)
+        ovals, _ = oracle.compress_rows(bits, keep)
+        assert np.array_equal(si.bits16(vals.cpu()), ovals)
+        rows = np.sort(rng.choice(N, 96, replace=False))
+        ref = oracle.weight_grad(oracle.to_f64(bits[rows], dt), oracle.to_f64(si.bits16(b), dt))
+        _check_wgrad(dw[torch.from_numpy(rows).cuda()], ref, f"dW [{N}x{K}] sampled rows")
