@@ -43,6 +43,18 @@ constexpr int kMvueTokens = 128;
 constexpr int kMvueCols = 64;
 constexpr int kMvueThreads = 128;
 
+// Both 64-bit halves of the 128-bit product a * b from three 32 x 32 -> 64
+// partial products and one more for the top (schoolbook, carries folded into
+// the wide multiply-adds: each partial sum stays below 2^64).
+__device__ __forceinline__ void mulhilo64(uint64_t a, uint64_t b, uint64_t &hi, uint64_t &lo) {
+  const uint32_t al = (uint32_t)a, ah = (uint32_t)(a >> 32), bl = (uint32_t)b, bh = (uint32_t)(b >> 32);
+  const uint64_t t0 = (uint64_t)al * bl;
+  const uint64_t t1 = (uint64_t)al * bh + (t0 >> 32);
+  const uint64_t t2 = (uint64_t)ah * bl + (uint32_t)t1;
+  hi = (uint64_t)ah * bh + (t1 >> 32) + (t2 >> 32);
+  lo = (t2 << 32) | (uint32_t)t0;
+}
+
 __device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], uint64_t k0, uint64_t k1) {
   constexpr uint64_t kM0 = 0xD2E7470EE14C6C93ull, kM1 = 0xCA5A826395121157ull;
   constexpr uint64_t kW0 = 0x9E3779B97F4A7C15ull, kW1 = 0xBB67AE8584CAA73Bull;
@@ -52,8 +64,9 @@ __device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], uint64_t k0, uin
       k0 += kW0;
       k1 += kW1;
     }
-    const uint64_t hi0 = __umul64hi(kM0, c[0]), lo0 = kM0 * c[0];
-    const uint64_t hi1 = __umul64hi(kM1, c[2]), lo1 = kM1 * c[2];
+    uint64_t hi0, lo0, hi1, lo1;
+    mulhilo64(c[0], kM0, hi0, lo0);
+    mulhilo64(c[2], kM1, hi1, lo1);
     const uint64_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
     c[0] = n0;
     c[1] = lo1;
@@ -62,77 +75,9 @@ __device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], uint64_t k0, uin
   }
 }
 
-__device__ __forceinline__ double pick4(const double (&x)[4], int i) {
-  return i == 0 ? x[0] : (i == 1 ? x[1] : (i == 2 ? x[2] : x[3]));
-}
-
 // Number of the cumulative sums c1, c2, c3 at or below the point: the entry it falls in.
 __device__ __forceinline__ int count_le(double c1, double c2, double c3, double p) {
   return (int)(c1 <= p) + (int)(c2 <= p) + (int)(c3 <= p);
-}
-
-// One group: kept positions pa < pb and their fp64 estimates.
-__device__ __forceinline__ void mvue_group(const double (&v)[4], double u, int &pa, int &pb, double &xa,
-                                           double &xb) {
-  double a[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = fabs(v[i]);
-  const double c1 = a[0];
-  const double c2 = __dadd_rn(c1, a[1]);
-  const double c3 = __dadd_rn(c2, a[2]);
-  const double s = __dadd_rn(c3, a[3]);
-  int m = 0;
-  double am = a[0];
-#pragma unroll
-  for (int i = 1; i < 4; ++i)
-    if (a[i] > am) {
-      am = a[i];
-      m = i;
-    }
-  int p0, p1;
-  double x0, x1;
-  if (__dadd_rn(am, am) >= s) {
-    const double b0 = m == 0 ? 0.0 : a[0], b1 = m == 1 ? 0.0 : a[1];
-    const double b2 = m == 2 ? 0.0 : a[2], b3 = m == 3 ? 0.0 : a[3];
-    const double e1 = b0;
-    const double e2 = __dadd_rn(e1, b1);
-    const double e3 = __dadd_rn(e2, b2);
-    const double r = __dadd_rn(e3, b3);
-    p0 = m;
-    x0 = pick4(v, m);
-    if (r > 0.0) {
-      p1 = count_le(e1, e2, e3, __dmul_rn(u, r));
-      x1 = copysign(r, pick4(v, p1));
-    } else {
-      p1 = m == 0 ? 1 : 0;
-      x1 = 0.0;
-    }
-  } else {
-    const double h = __dmul_rn(s, 0.5);
-    const double q1 = __dmul_rn(u, h);
-    const double q2 = __dadd_rn(q1, h);
-    p0 = count_le(c1, c2, c3, q1);
-    p1 = count_le(c1, c2, c3, q2);
-    if (p1 == p0) {
-      // Only a rounded cumulative sum puts both points in one entry: the second
-      // goes to the next nonzero entry after it, else the last nonzero one before.
-      int nxt = -1, prv = -1;
-#pragma unroll
-      for (int j = 3; j >= 0; --j)
-        if (j > p0 && a[j] > 0.0) nxt = j;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (j < p0 && a[j] > 0.0) prv = j;
-      p1 = nxt >= 0 ? nxt : prv;
-    }
-    x0 = copysign(h, pick4(v, p0));
-    x1 = copysign(h, pick4(v, p1));
-  }
-  if (p0 > p1) {
-    pa = p1; pb = p0; xa = x1; xb = x0;
-  } else {
-    pa = p0; pb = p1; xa = x0; xb = x1;
-  }
 }
 
 template <bool BF16>
@@ -143,9 +88,69 @@ __device__ __forceinline__ uint32_t mvue_bits(double x) {
 }
 
 template <bool BF16>
-__device__ __forceinline__ double half_bits_to_f64(uint32_t b) {
-  if (BF16) return (double)__uint_as_float(b << 16);
-  return (double)__half2float(__ushort_as_half((unsigned short)b));
+__device__ __forceinline__ double mag_f64(uint32_t b) {   // |v| of 16-bit storage bits, exact
+  if (BF16) return (double)__uint_as_float((b & 0x7FFFu) << 16);
+  return (double)__half2float(__ushort_as_half((unsigned short)(b & 0x7FFFu)));
+}
+
+__device__ __forceinline__ uint32_t pick_raw(uint64_t raw4, int i) { return (uint32_t)(raw4 >> (16 * i)) & 0xFFFFu; }
+
+// One group of four (16-bit storage bits packed in raw4, entry i at bits 16i),
+// without branches on the group's case: the cumulative sums run over
+// w = |v| with the largest entry zeroed when it is kept outright, which are the
+// sums of |v| (first case) or of the other three (second case) in the same
+// operation order.  Both kept estimates have the magnitude `step` (S/2, or R)
+// except the entry kept as is, so one rounding RNE_dtype(RNE_fp32(step)) serves
+// both and the signs come from the stored bits.  Returns the kept positions
+// pa < pb and their output bits.
+template <bool BF16>
+__device__ __forceinline__ void mvue_group(uint64_t raw4, double u, int &pa, int &pb, uint32_t &ba, uint32_t &bb) {
+  double a[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] = mag_f64<BF16>(pick_raw(raw4, i));
+  const double s = __dadd_rn(__dadd_rn(__dadd_rn(a[0], a[1]), a[2]), a[3]);
+  int m = 0;
+  double am = a[0];
+#pragma unroll
+  for (int i = 1; i < 4; ++i)
+    if (a[i] > am) {
+      am = a[i];
+      m = i;
+    }
+  const bool capped = __dadd_rn(am, am) >= s;
+  double w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = (capped && i == m) ? 0.0 : a[i];
+  const double e1 = w[0];
+  const double e2 = __dadd_rn(e1, w[1]);
+  const double e3 = __dadd_rn(e2, w[2]);
+  const double tot = __dadd_rn(e3, w[3]);
+  const double step = capped ? tot : __dmul_rn(tot, 0.5);
+  const double q1 = __dmul_rn(u, step);
+  int i1 = count_le(e1, e2, e3, q1);
+  int i2 = capped ? m : count_le(e1, e2, e3, __dadd_rn(q1, step));
+  const bool empty = capped && !(tot > 0.0);        // at most one nonzero entry
+  if (empty) i1 = m == 0 ? 1 : 0;
+  if (!capped && i2 == i1) {
+    // Only a rounded cumulative sum puts both points in one entry: the second
+    // goes to the next nonzero entry after it, else the last nonzero one before.
+    int nxt = -1, prv = -1;
+#pragma unroll
+    for (int j = 3; j >= 0; --j)
+      if (j > i1 && a[j] > 0.0) nxt = j;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (j < i1 && a[j] > 0.0) prv = j;
+    i2 = nxt >= 0 ? nxt : prv;
+  }
+  const uint32_t mag = empty ? 0u : mvue_bits<BF16>(step);
+  const uint32_t b1 = empty ? 0u : (mag | (pick_raw(raw4, i1) & 0x8000u));
+  const uint32_t b2 = capped ? pick_raw(raw4, m) : (mag | (pick_raw(raw4, i2) & 0x8000u));
+  if (i1 < i2) {
+    pa = i1; pb = i2; ba = b1; bb = b2;
+  } else {
+    pa = i2; pb = i1; ba = b2; bb = b1;
+  }
 }
 
 template <bool BF16>
@@ -176,43 +181,57 @@ __global__ void __launch_bounds__(kMvueThreads) mvue_sparsify_kernel(
   const int64_t tseg = t0 + 32 * w;                         // first token of this thread's segment
   const int ngroups = (int)max((int64_t)0, min((int64_t)8, (T - tseg) / 4));
   const int rh = (int)(blockIdx.y & 1);
+  uint64_t rnd[2][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    rnd[c][0] = (uint64_t)(tseg >> 5);
+    rnd[c][1] = (uint64_t)(n0 + 2 * p + c);
+    rnd[c][2] = 0ull;
+    rnd[c][3] = 0ull;
+    philox4x64_10(rnd[c], seed, offset);
+  }
+  uint32_t nib[2] = {0x44444444u, 0x44444444u};               // padding: positions 0, 1
+  uint32_t packed[2][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    packed[0][j] = 0u;
+    packed[1][j] = 0u;
+    if (j < ngroups) {
+      uint32_t wd[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wd[i] = s_tile[32 * w + 4 * j + i][p];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint64_t raw4 = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) raw4 |= (uint64_t)((wd[i] >> (16 * c)) & 0xFFFFu) << (16 * i);
+        const uint32_t u32 = (uint32_t)(rnd[c][j >> 1] >> (32 * (j & 1)));
+        const double u = (double)(u32 >> 8) * 0x1p-24;
+        int pa, pb;
+        uint32_t ba, bb;
+        mvue_group<BF16>(raw4, u, pa, pb, ba, bb);
+        nib[c] = (nib[c] & ~(0xFu << (4 * j))) | ((uint32_t)(pa | (pb << 2)) << (4 * j));
+        packed[c][j] = ba | (bb << 16);
+      }
+    }
+  }
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     const int64_t n = n0 + 2 * p + c;
-    uint32_t nib = 0x44444444u;                             // padding: positions 0, 1
     if (n < N && ngroups > 0) {
-      uint64_t ctr[4] = {(uint64_t)(tseg >> 5), (uint64_t)n, 0ull, 0ull};
-      philox4x64_10(ctr, seed, offset);
-      uint32_t packed[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < ngroups) {
-          const uint64_t word = ctr[j >> 1];
-          const uint32_t u32 = (uint32_t)(word >> (32 * (j & 1)));
-          const double u = (double)(u32 >> 8) * 0x1p-24;
-          double v[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) v[i] = half_bits_to_f64<BF16>((s_tile[32 * w + 4 * j + i][p] >> (16 * c)) & 0xFFFFu);
-          int pa, pb;
-          double xa, xb;
-          mvue_group(v, u, pa, pb, xa, xb);
-          nib = (nib & ~(0xFu << (4 * j))) | ((uint32_t)(pa | (pb << 2)) << (4 * j));
-          packed[j] = mvue_bits<BF16>(xa) | (mvue_bits<BF16>(xb) << 16);
-        } else {
-          packed[j] = 0u;
-        }
-      }
       uint16_t *dst = vals + n * (T >> 1) + (tseg >> 1);
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      if (ngroups > 4) *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[c][0], packed[c][1], packed[c][2], packed[c][3]);
+      if (ngroups > 4)
+        *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(packed[c][4], packed[c][5], packed[c][6], packed[c][7]);
     }
+    const uint32_t nb = n < N ? nib[c] : 0x44444444u;
     // Metadata: row r of the chunk, K step w; groups 0-3 go to lane
     // (r % 8) + 16 (r / 16), groups 4-7 to that lane + 8; the 16-bit half is (r / 8) % 2.
     const int r = 64 * rh + 2 * p + c;
     const int lane0 = (r & 7) + 16 * (r >> 4) - 64 * rh;
     const int half = (r >> 3) & 1;
-    s_meta[(lane0 * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nib & 0xFFFFu);
-    s_meta[((lane0 + 8) * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nib >> 16);
+    s_meta[(lane0 * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nb & 0xFFFFu);
+    s_meta[((lane0 + 8) * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nb >> 16);
   }
   __syncthreads();
   if (tid < 64) {
