@@ -28,11 +28,10 @@
 // [N x T] operand (2048 bytes per 128 rows x 128 tokens, chunk index
 // (n / 128) * ceil(T / 128) + t / 128), exactly as the forward operand of W.
 // One CTA per 128 tokens x 64 columns (half a chunk's rows): the tile is staged
-// in shared memory (16-byte loads along the columns), then thread (warp w,
-// lane p) takes columns 2p, 2p+1 and tokens 32w..32w+31 (one Philox block per
-// column: eight groups), writes 32 bytes of each of its two output rows and
-// its metadata nibbles into the CTA's 1 KB half of the chunk, which the CTA
-// then stores with 16-byte writes.  Groups past T and rows past N get the
+// in shared memory (16-byte loads along the columns), then each of 256 threads
+// takes one column and 32 tokens (eight groups: one Philox block), writes 32
+// bytes of its output row and its metadata nibbles into the CTA's 1 KB half of
+// the chunk, which the CTA then stores with 16-byte writes.  Groups past T and rows past N get the
 // padding code (positions 0, 1), so whole chunks are always written.
 #pragma once
 #include "sp24_common.cuh"
@@ -41,7 +40,7 @@ namespace sp24 {
 
 constexpr int kMvueTokens = 128;
 constexpr int kMvueCols = 64;
-constexpr int kMvueThreads = 128;
+constexpr int kMvueThreads = 256;
 
 // Both 64-bit halves of the 128-bit product a * b from three 32 x 32 -> 64
 // partial products and one more for the top (schoolbook, carries folded into
@@ -55,19 +54,30 @@ __device__ __forceinline__ void mulhilo64(uint64_t a, uint64_t b, uint64_t &hi, 
   lo = (t2 << 32) | (uint32_t)t0;
 }
 
-__device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], uint64_t k0, uint64_t k1) {
+// The ten round keys of Philox4x64-10 for key (k0, k1): round r uses
+// (k0 + r W0, k1 + r W1) mod 2^64 with the Weyl increments W0, W1.  The same
+// for every thread, so the host computes them once per launch.
+struct PhiloxKeys {
+  uint64_t k0[10], k1[10];
+};
+
+__host__ __device__ inline PhiloxKeys philox4x64_keys(uint64_t k0, uint64_t k1) {
+  PhiloxKeys ks;
+  for (int r = 0; r < 10; ++r) {
+    ks.k0[r] = k0 + (uint64_t)r * 0x9E3779B97F4A7C15ull;
+    ks.k1[r] = k1 + (uint64_t)r * 0xBB67AE8584CAA73Bull;
+  }
+  return ks;
+}
+
+__device__ __forceinline__ void philox4x64_10(uint64_t (&c)[4], const PhiloxKeys &ks) {
   constexpr uint64_t kM0 = 0xD2E7470EE14C6C93ull, kM1 = 0xCA5A826395121157ull;
-  constexpr uint64_t kW0 = 0x9E3779B97F4A7C15ull, kW1 = 0xBB67AE8584CAA73Bull;
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r) {
-      k0 += kW0;
-      k1 += kW1;
-    }
     uint64_t hi0, lo0, hi1, lo1;
     mulhilo64(c[0], kM0, hi0, lo0);
     mulhilo64(c[2], kM1, hi1, lo1);
-    const uint64_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    const uint64_t n0 = hi1 ^ c[1] ^ ks.k0[r], n2 = hi0 ^ c[3] ^ ks.k1[r];
     c[0] = n0;
     c[1] = lo1;
     c[2] = n2;
@@ -87,36 +97,60 @@ __device__ __forceinline__ uint32_t mvue_bits(double x) {
   return (uint32_t)__half_as_ushort(__float2half_rn(f));
 }
 
+// |v| of two 16-bit values packed in one word (sign bits cleared), exact in fp64.
 template <bool BF16>
-__device__ __forceinline__ double mag_f64(uint32_t b) {   // |v| of 16-bit storage bits, exact
-  if (BF16) return (double)__uint_as_float((b & 0x7FFFu) << 16);
-  return (double)__half2float(__ushort_as_half((unsigned short)(b & 0x7FFFu)));
+__device__ __forceinline__ void mag2_f64(uint32_t m2, double &lo, double &hi) {
+  if (BF16) {
+    lo = (double)__uint_as_float(m2 << 16);
+    hi = (double)__uint_as_float(m2 & 0xFFFF0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&m2));
+    lo = (double)f.x;
+    hi = (double)f.y;
+  }
 }
 
-__device__ __forceinline__ uint32_t pick_raw(uint64_t raw4, int i) { return (uint32_t)(raw4 >> (16 * i)) & 0xFFFFu; }
-
-// One group of four (16-bit storage bits packed in raw4, entry i at bits 16i),
-// without branches on the group's case: the cumulative sums run over
-// w = |v| with the largest entry zeroed when it is kept outright, which are the
-// sums of |v| (first case) or of the other three (second case) in the same
-// operation order.  Both kept estimates have the magnitude `step` (S/2, or R)
-// except the entry kept as is, so one rounding RNE_dtype(RNE_fp32(step)) serves
-// both and the signs come from the stored bits.  Returns the kept positions
-// pa < pb and their output bits.
 template <bool BF16>
-__device__ __forceinline__ void mvue_group(uint64_t raw4, double u, int &pa, int &pb, uint32_t &ba, uint32_t &bb) {
+__device__ __forceinline__ double mag_f64(uint32_t m) {
+  if (BF16) return (double)__uint_as_float(m << 16);
+  return (double)__half2float(__ushort_as_half((unsigned short)m));
+}
+
+// Entry i (0..3) of a group held as lo = v0 | v1 << 16, hi = v2 | v3 << 16.
+__device__ __forceinline__ uint32_t pick_raw(uint32_t lo, uint32_t hi, int i) {
+  return ((i < 2 ? lo : hi) >> (16 * (i & 1))) & 0xFFFFu;
+}
+
+// Sign bit (as bit 15) of entry i, from the group's 4-bit sign mask.
+__device__ __forceinline__ uint32_t sign_of(uint32_t sgn4, int i) { return ((sgn4 >> i) & 1u) << 15; }
+
+// One group of four (16-bit storage bits in lo/hi), without branches on the
+// group's case: the cumulative sums run over w = |v| with the largest entry
+// zeroed when it is kept outright, which are the sums of |v| (first case) or of
+// the other three (second case) in the same operation order.  Both kept
+// estimates have the magnitude `step` (S/2, or R) except the entry kept as is,
+// so one rounding RNE_dtype(RNE_fp32(step)) serves both and the signs come from
+// the stored bits.  The largest |v| is found on the magnitude bits (for finite
+// values their order is that of the magnitudes; equal magnitudes, equal bits).
+// Returns the kept positions pa < pb and their output bits.
+template <bool BF16>
+__device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, int &pa, int &pb, uint32_t &ba,
+                                           uint32_t &bb) {
+  const uint32_t lm = lo & 0x7FFF7FFFu, hm = hi & 0x7FFF7FFFu;
   double a[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = mag_f64<BF16>(pick_raw(raw4, i));
+  mag2_f64<BF16>(lm, a[0], a[1]);
+  mag2_f64<BF16>(hm, a[2], a[3]);
   const double s = __dadd_rn(__dadd_rn(__dadd_rn(a[0], a[1]), a[2]), a[3]);
+  const uint32_t q[4] = {lm & 0xFFFFu, lm >> 16, hm & 0xFFFFu, hm >> 16};
   int m = 0;
-  double am = a[0];
+  uint32_t qm = q[0];
 #pragma unroll
   for (int i = 1; i < 4; ++i)
-    if (a[i] > am) {
-      am = a[i];
+    if (q[i] > qm) {
+      qm = q[i];
       m = i;
     }
+  const double am = mag_f64<BF16>(qm);
   const bool capped = __dadd_rn(am, am) >= s;
   double w[4];
 #pragma unroll
@@ -131,21 +165,24 @@ __device__ __forceinline__ void mvue_group(uint64_t raw4, double u, int &pa, int
   int i2 = capped ? m : count_le(e1, e2, e3, __dadd_rn(q1, step));
   const bool empty = capped && !(tot > 0.0);        // at most one nonzero entry
   if (empty) i1 = m == 0 ? 1 : 0;
-  if (!capped && i2 == i1) {
-    // Only a rounded cumulative sum puts both points in one entry: the second
-    // goes to the next nonzero entry after it, else the last nonzero one before.
+  // Only a rounded cumulative sum puts both points in one entry: the second
+  // goes to the next nonzero entry after it, else the last nonzero one before.
+  // (Warp-uniform branch: all 32 lanes of the warp call this function.)
+  const bool collide = !capped && i2 == i1;
+  if (__any_sync(0xFFFFFFFFu, collide) && collide) {
     int nxt = -1, prv = -1;
 #pragma unroll
     for (int j = 3; j >= 0; --j)
-      if (j > i1 && a[j] > 0.0) nxt = j;
+      if (j > i1 && q[j] != 0u) nxt = j;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      if (j < i1 && a[j] > 0.0) prv = j;
+      if (j < i1 && q[j] != 0u) prv = j;
     i2 = nxt >= 0 ? nxt : prv;
   }
+  const uint32_t sgn4 = ((lo >> 15) & 1u) | ((lo >> 30) & 2u) | ((hi >> 13) & 4u) | ((hi >> 28) & 8u);
   const uint32_t mag = empty ? 0u : mvue_bits<BF16>(step);
-  const uint32_t b1 = empty ? 0u : (mag | (pick_raw(raw4, i1) & 0x8000u));
-  const uint32_t b2 = capped ? pick_raw(raw4, m) : (mag | (pick_raw(raw4, i2) & 0x8000u));
+  const uint32_t b1 = empty ? 0u : (mag | sign_of(sgn4, i1));
+  const uint32_t b2 = capped ? pick_raw(lo, hi, m) : (mag | sign_of(sgn4, i2));
   if (i1 < i2) {
     pa = i1; pb = i2; ba = b1; bb = b2;
   } else {
@@ -155,7 +192,7 @@ __device__ __forceinline__ void mvue_group(uint64_t raw4, double u, int &pa, int
 
 template <bool BF16>
 __global__ void __launch_bounds__(kMvueThreads) mvue_sparsify_kernel(
-    const uint16_t *__restrict__ dy, int64_t T, int64_t N, int64_t ldy, uint64_t seed, uint64_t offset,
+    const uint16_t *__restrict__ dy, int64_t T, int64_t N, int64_t ldy, const __grid_constant__ PhiloxKeys keys,
     uint16_t *__restrict__ vals, uint8_t *__restrict__ meta) {
   __shared__ __align__(16) uint32_t s_tile[kMvueTokens][kMvueCols / 2];   // [token][column pair]
   __shared__ __align__(16) uint16_t s_meta[512];                           // this CTA's half chunk
@@ -177,61 +214,48 @@ __global__ void __launch_bounds__(kMvueThreads) mvue_sparsify_kernel(
   }
   __syncthreads();
 
-  const int w = tid >> 5, p = tid & 31;
+  // Thread (segment w, column p): column n0 + p, tokens 32w .. 32w + 31 (eight groups,
+  // one Philox block).  A warp takes 32 consecutive columns of one segment.
+  const int p = tid & 63, w = tid >> 6;
   const int64_t tseg = t0 + 32 * w;                         // first token of this thread's segment
   const int ngroups = (int)max((int64_t)0, min((int64_t)8, (T - tseg) / 4));
   const int rh = (int)(blockIdx.y & 1);
-  uint64_t rnd[2][4];
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    rnd[c][0] = (uint64_t)(tseg >> 5);
-    rnd[c][1] = (uint64_t)(n0 + 2 * p + c);
-    rnd[c][2] = 0ull;
-    rnd[c][3] = 0ull;
-    philox4x64_10(rnd[c], seed, offset);
-  }
-  uint32_t nib[2] = {0x44444444u, 0x44444444u};               // padding: positions 0, 1
-  uint32_t packed[2][8];
+  const int64_t n = n0 + p;
+  uint64_t rnd[4] = {(uint64_t)(tseg >> 5), (uint64_t)n, 0ull, 0ull};
+  philox4x64_10(rnd, keys);
+  uint32_t nib = 0x44444444u;                               // padding: positions 0, 1
+  uint32_t packed[8];
+  const uint32_t sel = (p & 1) ? 0x7632u : 0x5410u;         // this column's halves of the staged words
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    packed[0][j] = 0u;
-    packed[1][j] = 0u;
+    packed[j] = 0u;
     if (j < ngroups) {
-      uint32_t wd[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) wd[i] = s_tile[32 * w + 4 * j + i][p];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint64_t raw4 = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) raw4 |= (uint64_t)((wd[i] >> (16 * c)) & 0xFFFFu) << (16 * i);
-        const uint32_t u32 = (uint32_t)(rnd[c][j >> 1] >> (32 * (j & 1)));
-        const double u = (double)(u32 >> 8) * 0x1p-24;
-        int pa, pb;
-        uint32_t ba, bb;
-        mvue_group<BF16>(raw4, u, pa, pb, ba, bb);
-        nib[c] = (nib[c] & ~(0xFu << (4 * j))) | ((uint32_t)(pa | (pb << 2)) << (4 * j));
-        packed[c][j] = ba | (bb << 16);
-      }
+      const uint32_t *col = &s_tile[32 * w + 4 * j][p >> 1];
+      const uint32_t lo = __byte_perm(col[0], col[kMvueCols / 2], sel);
+      const uint32_t hi = __byte_perm(col[kMvueCols], col[3 * kMvueCols / 2], sel);
+      const uint32_t u32 = (uint32_t)(rnd[j >> 1] >> (32 * (j & 1)));
+      const double u = (double)(u32 >> 8) * 0x1p-24;
+      int pa, pb;
+      uint32_t ba, bb;
+      mvue_group<BF16>(lo, hi, u, pa, pb, ba, bb);
+      nib = (nib & ~(0xFu << (4 * j))) | ((uint32_t)(pa | (pb << 2)) << (4 * j));
+      packed[j] = ba | (bb << 16);
     }
   }
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const int64_t n = n0 + 2 * p + c;
-    if (n < N && ngroups > 0) {
-      uint16_t *dst = vals + n * (T >> 1) + (tseg >> 1);
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[c][0], packed[c][1], packed[c][2], packed[c][3]);
-      if (ngroups > 4)
-        *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(packed[c][4], packed[c][5], packed[c][6], packed[c][7]);
-    }
-    const uint32_t nb = n < N ? nib[c] : 0x44444444u;
+  if (n < N && ngroups > 0) {
+    uint16_t *dst = vals + n * (T >> 1) + (tseg >> 1);
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (ngroups > 4) *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  }
+  if (n >= N) nib = 0x44444444u;
+  {
     // Metadata: row r of the chunk, K step w; groups 0-3 go to lane
     // (r % 8) + 16 (r / 16), groups 4-7 to that lane + 8; the 16-bit half is (r / 8) % 2.
-    const int r = 64 * rh + 2 * p + c;
+    const int r = 64 * rh + p;
     const int lane0 = (r & 7) + 16 * (r >> 4) - 64 * rh;
     const int half = (r >> 3) & 1;
-    s_meta[(lane0 * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nb & 0xFFFFu);
-    s_meta[((lane0 + 8) * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nb >> 16);
+    s_meta[(lane0 * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nib & 0xFFFFu);
+    s_meta[((lane0 + 8) * 16 + 4 * w + 2 * half) >> 1] = (uint16_t)(nib >> 16);
   }
   __syncthreads();
   if (tid < 64) {

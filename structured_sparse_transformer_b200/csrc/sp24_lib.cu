@@ -436,9 +436,10 @@ sp24_status sp24_mvue_sparsify(const void *dY, int64_t T, int64_t N, int64_t ldy
   const uint16_t *d16 = static_cast<const uint16_t *>(dY);
   uint16_t *v16 = static_cast<uint16_t *>(vals);
   uint8_t *m8 = static_cast<uint8_t *>(meta);
+  const PhiloxKeys keys = philox4x64_keys(seed, offset);
   return dtype == SP24_BF16
-             ? launch_pdl(mvue_sparsify_kernel<true>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, seed, offset, v16, m8)
-             : launch_pdl(mvue_sparsify_kernel<false>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, seed, offset, v16, m8);
+             ? launch_pdl(mvue_sparsify_kernel<true>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, keys, v16, m8)
+             : launch_pdl(mvue_sparsify_kernel<false>, grid, dim3(kMvueThreads), 0, s, d16, T, N, ldy, keys, v16, m8);
 }
 
 sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *vals, const void *meta, int64_t N,
