@@ -343,13 +343,14 @@ def philox4x64_10(ctr: np.ndarray, key) -> np.ndarray:
     return np.stack(c, axis=-1)
 
 
-def mvue_uniforms(rows: int, groups: int, seed: int, offset: int) -> np.ndarray:
-    """The uniform draw of every group of four of the sparsified operand, float64 [rows, groups].
+def mvue_uniforms(rows: int, groups: int, seed: int, offset: int, row0: int = 0) -> np.ndarray:
+    """The uniform draw of every group of four of the sparsified operand, float64 [rows, groups],
+    for rows row0 .. row0 + rows - 1 of it.
 
     Group g of row n takes 32 bits of philox4x64_10(counter (g // 8, n, 0, 0), key (seed, offset)):
     word (g % 8) // 2, low half for even g, high half for odd g.  The top 24 of those bits,
     times 2^-24, give u in [0, 1 - 2^-24] (exact in fp32 and fp64)."""
-    n = np.arange(rows, dtype=np.uint64)[:, None]
+    n = np.arange(row0, row0 + rows, dtype=np.uint64)[:, None]
     blk = np.arange((groups + 7) // 8, dtype=np.uint64)[None, :]
     ctr = np.zeros((rows, blk.shape[1], 4), np.uint64)
     ctr[..., 0] = blk
@@ -447,10 +448,11 @@ def _f64_to_bits_via_f32(x: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
-def mvue_sparsify_t(dy_bits: np.ndarray, dtype: str, seed: int, offset: int):
+def mvue_sparsify_t(dy_bits: np.ndarray, dtype: str, seed: int, offset: int, col0: int = 0):
     """MVUE 2:4 sparsification of dY^T along the token axis.
 
-    ``dy_bits`` uint16 [T, N] (T % 4 == 0).  Row n of the result is column n of dY,
+    ``dy_bits`` uint16 [T, N] (T % 4 == 0): columns col0 .. col0 + N - 1 of dY (the draws
+    depend on the column's index in the full dY).  Row n of the result is column n of dY,
     with every group of four consecutive tokens reduced to two kept estimates
     (``mvue_select`` with the draws of ``mvue_uniforms(N, T/4, seed, offset)``),
     each stored as RNE_dtype(RNE_fp32(estimate)).
@@ -461,7 +463,7 @@ def mvue_sparsify_t(dy_bits: np.ndarray, dtype: str, seed: int, offset: int):
     if T % 4:
         raise ValueError("token count must be a multiple of 4")
     v = to_f64(np.ascontiguousarray(dy_bits.T), dtype).reshape(N, T // 4, 4)
-    u = mvue_uniforms(N, T // 4, seed, offset)
+    u = mvue_uniforms(N, T // 4, seed, offset, col0)
     pos, est = mvue_select(v, u)
     keep = np.zeros((N, T // 4, 4), bool)
     dense = np.zeros((N, T // 4, 4), np.float64)

@@ -154,3 +154,37 @@ def test_ffn_weight_grads_full_size_sampled(wl):
         rows = np.sort(rng.choice(N, 96, replace=False))
         ref = oracle.weight_grad(oracle.to_f64(bits[rows], dt), oracle.to_f64(si.bits16(b), dt))
         _check_wgrad(dw[torch.from_numpy(rows).cuda()], ref, f"dW [{N}x{K}] sampled rows")
+
+
+@pytest.mark.parametrize("wl", [si.GPT2_774M], ids=lambda w: w.name)
+def test_ffn_weight_grads_full_size_column_sample(wl):
+    """Both weight gradients of the 774M FFN (bf16, 16384 tokens) at full size; the
+    sparsified operands are compared on 160 sampled columns of dY / dH (the oracle draws
+    from the columns' indices in the full matrices), dW on the same 160 rows."""
+    dt = wl.dtype
+    X, dY = wl.activations()
+    H, dH = wl.hidden()
+    T = wl.tokens
+    rng = np.random.default_rng(1)
+    for (g, b, N, K, off) in ((dY, H, wl.d, wl.ff, 3), (dH, X, wl.ff, wl.d, 4)):
+        vals, meta = _alloc(N, T, dt)
+        dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+        sp.sp24_mvue_sparsify(g.cuda(), wl.seeds["mvue"], off, vals, meta)
+        sp.sp24_gemm_wgrad(b.cuda(), vals, meta, N, dw)
+        torch.cuda.synchronize()
+        assert sp.sp24_device_status() == 0
+        start = int(rng.integers(0, N // 32)) * 32
+        rows = np.arange(start, start + 160) % N
+        gb = si.bits16(g)
+        bf = oracle.to_f64(si.bits16(b), dt)
+        got_vals = si.bits16(vals.cpu())
+        for r0 in range(0, 160, 32):
+            cols = rows[r0:r0 + 32]
+            if cols[-1] < cols[0]:
+                continue
+            bits, keep, _ = oracle.mvue_sparsify_t(np.ascontiguousarray(gb[:, cols[0]:cols[-1] + 1]), dt,
+                                                   wl.seeds["mvue"], off, col0=int(cols[0]))
+            ovals, _ = oracle.compress_rows(bits, keep)
+            assert np.array_equal(got_vals[cols[0]:cols[-1] + 1], ovals)
+            ref = oracle.weight_grad(oracle.to_f64(bits, dt), bf)
+            _check_wgrad(dw[int(cols[0]):int(cols[-1]) + 1], ref, f"dW [{N}x{K}] rows {cols[0]}..")

@@ -17,7 +17,6 @@ oracle's own code:
   or two nonzeros reproduced exactly);
 * the weight-gradient product's orientation with one-hot inputs.
 """
-from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -178,6 +177,14 @@ def test_sparsify_invariants():
     bits2, _, _ = oracle.mvue_sparsify_t(si.bits16(dy), "f16", seed=9, offset=1)
     bits3, _, _ = oracle.mvue_sparsify_t(si.bits16(dy), "f16", seed=9, offset=2)
     assert np.array_equal(bits, bits2) and not np.array_equal(bits, bits3)
+
+
+def test_column_sample_matches_the_full_matrix():
+    t, n = 64, 40
+    dy = si.normal((t, n), 1.0, 12, "bf16")
+    full, _, _ = oracle.mvue_sparsify_t(si.bits16(dy), "bf16", 4, 9)
+    part, _, _ = oracle.mvue_sparsify_t(si.bits16(dy[:, 17:29].contiguous()), "bf16", 4, 9, col0=17)
+    assert np.array_equal(part, full[17:29])
 
 
 def test_sparsify_bf16_exact_keeps():
