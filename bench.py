@@ -101,24 +101,57 @@ def load_peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """Samples SM clock, power and throttle reasons of one GPU with nvidia-smi
-    every ~200 ms from a background thread (one query per sample, so nothing
-    is lost to output buffering when sampling stops)."""
+    """Samples the SM clock and the clock-event (throttle) reasons of the GPU the
+    process runs on from a background thread: through NVML in-process every
+    ~5 ms (read-only queries), else with nvidia-smi every ~200 ms."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    NVML_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4}
 
     def __init__(self, gpu_index: int, period_s: float = 0.2):
         import threading
         self.gpu, self.period = gpu_index, period_s
         self.samples = []
         self.error = None
+        self.source = None
+        self._nvml = self._open_nvml()
         self._stop = threading.Event()
         self._thread = threading.Thread(target=self._run, daemon=True)
 
-    def _query(self):
+    def _open_nvml(self):
+        """NVML handle of the torch device (by UUID, then PCI bus id), or None."""
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(self.gpu)
+            handle = None
+            for uid in (f"GPU-{props.uuid}", str(props.uuid)):
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(uid)
+                    break
+                except Exception:
+                    continue
+            if handle is None:
+                bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+                handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            return pynvml, handle
+        except Exception as e:  # no NVML binding or no match: fall back to nvidia-smi
+            self.error = f"nvml: {str(e)[:120]}"
+            return None
+
+    def _query_nvml(self):
+        pynvml, h = self._nvml
+        sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+        smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+        bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+        return sm, smax, {n for n, b in self.NVML_BITS.items() if bits & b}
+
+    def _query_smi(self):
         r = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
                             "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10)
         if r.returncode != 0:
@@ -128,13 +161,15 @@ class ClockSampler:
         return float(f[1]), float(f[2]), reasons
 
     def _run(self):
+        query, period = ((self._query_nvml, 0.005) if self._nvml else (self._query_smi, self.period))
+        self.source = "nvml" if self._nvml else "nvidia-smi"
         while not self._stop.is_set():
             try:
-                self.samples.append(self._query())
-            except Exception as e:  # nvidia-smi missing or a field unsupported
+                self.samples.append(query())
+            except Exception as e:  # a field unsupported: stop sampling, keep what was read
                 self.error = str(e)[:200]
                 return
-            self._stop.wait(self.period)
+            self._stop.wait(period)
 
     def __enter__(self):
         self._thread.start()
@@ -149,9 +184,10 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
         sm = [x[0] for x in self.samples]
         reasons = sorted(set().union(*[x[2] for x in self.samples]))
+        period = "~5 ms" if self.source == "nvml" else "~200 ms"
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
-                "samples": len(sm), "reasons": reasons,
-                "window": "warm-up through the end-to-end loop, one query per ~200 ms"}
+                "sm_min_mhz": min(sm), "samples": len(sm), "reasons": reasons, "source": self.source,
+                "window": f"warm-up through the end-to-end loop, one query per {period}"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -258,12 +294,15 @@ class FFNStep:
 
     def run_dense(self, events=None):
         """One step of the dense fine-tuning phase (the last 1/6 of the steps):
-        W^T of both weights (they change every step), the four FFN products on
-        the dense tensor-core path; no mask, compression or decay."""
+        W^T of both weights (they change every step), the six FFN products on
+        the dense tensor-core path (the weight gradients take dY^T and dH^T from
+        the transpose kernel); no mask, compression or decay."""
         sp, torch = self.sp, self.torch
         cur = self.step_no % 2
         if not hasattr(self, "Wt"):
             self.Wt = [torch.empty(w[0].shape[1], w[0].shape[0], dtype=w[0].dtype, device="cuda") for w in self.W]
+            self.dYt = torch.empty(self.dY.shape[1], self.dY.shape[0], dtype=self.dY.dtype, device="cuda")
+            self.dHt = torch.empty(self.dH.shape[1], self.dH.shape[0], dtype=self.dH.dtype, device="cuda")
 
         def timed(name, fn):
             if events is None:
@@ -281,6 +320,10 @@ class FFNStep:
         timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu", self.Hpre))
         timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
         timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "dgelu", self.Hpre))
+        timed("transpose_act", lambda: sp.sp24_transpose(self.dY, self.dYt))
+        timed("gemm_dense_wgrad", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dYt, self.G[1]))
+        timed("transpose_act", lambda: sp.sp24_transpose(self.dH, self.dHt))
+        timed("gemm_dense_wgrad", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dHt, self.G[0]))
         timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
         self.step_no += 1
 
@@ -442,23 +485,27 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier):
     if st != 0:
         raise RuntimeError(f"device status after the dense phase: {sp.sp24_status_string(st)}")
     peaks, _ = load_peaks()
-    g = [s.elapsed_time(e) * 1e-3 for s, e in events["gemm_dense"]]
+    g = [s.elapsed_time(e) * 1e-3 for s, e in events["gemm_dense"] + events["gemm_dense_wgrad"]]
     t = [s.elapsed_time(e) * 1e-3 for s, e in events["transpose"]]
+    ta = [s.elapsed_time(e) * 1e-3 for s, e in events["transpose_act"]]
     g_avg = sum(g) / len(g)
     ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
     n_el = wl.d * wl.ff
     t_avg = sum(t) / len(t)
     return {"ms_per_step": round(ms, 4),
-            "value": round(4 * 2.0 * wl.tokens * wl.d * wl.ff * world / (ms * 1e-3) / 1e12, 2),
+            "value": round(wl.gemm_flops() * world / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s",
             "gemm": {"launches": len(g), "avg_us": round(g_avg * 1e6, 2), "achieved": round(ach, 1),
                      "peak": peaks["bf16_tflops"], "frac": round(ach / peaks["bf16_tflops"], 4)},
             "transpose": {"launches": len(t), "avg_us": round(t_avg * 1e6, 2),
                           "achieved": round(4 * n_el / t_avg / 1e9, 1), "unit": "GB/s",
                           "peak": peaks["hbm_gbs"], "frac": round(4 * n_el / t_avg / 1e9 / peaks["hbm_gbs"], 4)},
-            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights and the four FFN "
-                    "forward and input-gradient products on the dense tcgen05 path, same workload (no "
-                    "weight-gradient products: FLOPs 4 x 2 T d ff)"}
+            "transpose_act": {"launches": len(ta), "avg_us": round(sum(ta) / len(ta) * 1e6, 2),
+                              "achieved": round(4 * wl.tokens * (wl.d + wl.ff) / 2 / (sum(ta) / len(ta)) / 1e9, 1),
+                              "unit": "GB/s"},
+            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights, dY^T and dH^T, and "
+                    "the six FFN products (forward, input gradient, weight gradient) on the dense tcgen05 "
+                    "path, same workload; FLOPs 6 x 2 T d ff"}
 
 
 class GegluStep:

@@ -237,6 +237,20 @@ SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const 
                             int64_t N, sp24_dtype dtype, float *dW, void *stream);
 
 /*
+ * Dense weight-gradient GEMM for the dense fine-tuning phase (abstract: dense
+ * fine-tuning; Experiment Setup row: the last 1/6 of the steps):
+ * dW[N x K] = dY^T[N x T] * X[T x K], fp32 accumulation and fp32 output in W's
+ * layout, on the same tcgen05 pipeline (X read as stored, dY^T from
+ * sp24_transpose of dY).
+ *   X     device [T x K] row-major, contiguous
+ *   dYt   device [N x T] row-major, contiguous (dY transposed)
+ *   dW    device fp32 [N x K] contiguous, overwritten (zeros when T == 0)
+ * T % 16 == 0, N % 16 == 0, K % 8 == 0; all pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N,
+                                  sp24_dtype dtype, float *dW, void *stream);
+
+/*
  * Masked decay on gradients (abstract; masked decay kernel of the Software
  * Dependencies row): grad <- grad + lambda * W where the mask is 0, unchanged
  * where it is 1, as one fp32 fused multiply-add per pruned entry (in place).

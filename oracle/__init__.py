@@ -260,6 +260,12 @@ def dense_dgrad(dy: np.ndarray, w: np.ndarray) -> np.ndarray:
     return np.asarray(dy, np.float64) @ np.asarray(w, np.float64)
 
 
+def dense_weight_grad(dy: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """fp64 ``dW = dY^T X`` for dY [T, N] and X [T, K]: the weight gradient of the dense
+    fine-tuning phase, [N, K] in the layout of W."""
+    return np.asarray(dy, np.float64).T @ np.asarray(x, np.float64)
+
+
 def gelu(x: np.ndarray) -> np.ndarray:
     """GELU, exact erf form ``0.5 x (1 + erf(x / sqrt 2))``, fp64."""
     from scipy.special import erf

@@ -40,6 +40,7 @@ _SIGNATURES = {
     "sp24_transpose": [P, I64, I64, I32, P, P],
     "sp24_mvue_sparsify": [P, I64, I64, I64, I32, U64, U64, P, P, P],
     "sp24_gemm_wgrad": [P, I64, I64, P, P, I64, I32, P, P],
+    "sp24_gemm_wgrad_dense": [P, I64, I64, P, I64, I32, P, P],
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
     "sp24_flip_rate": [P, P, I64, P, P],
     "sp24_meta_to_canonical": [P, I64, I64, P],
@@ -223,6 +224,15 @@ def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
     _check("sp24_gemm_wgrad",
            _lib.sp24_gemm_wgrad(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(dW),
                                 _stream(stream)))
+
+
+def sp24_gemm_wgrad_dense(X, dYt, dW, stream=None):
+    """dW[N, K] (fp32) <- dYt[N, T] X[T, K] on the dense tensor-core path (dYt = dY transposed)."""
+    _need_cuda(X, dYt, dW)
+    T, K = X.shape
+    N = dYt.shape[0]
+    _check("sp24_gemm_wgrad_dense",
+           _lib.sp24_gemm_wgrad_dense(_ptr(X), T, K, _ptr(dYt), N, _dtype_code(X), _ptr(dW), _stream(stream)))
 
 
 def sp24_masked_decay(grad, W, idx, lam: float, stream=None):

@@ -96,14 +96,17 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // 64-column halves make the 128), into accumulator columns 0 and 128: an MMA
 // never spans two atoms along N.  One 256-column accumulator (no double
 // buffering: the weight-gradient tiles run one per pair at the FFN sizes).
+// The dense variant (dense fine-tuning) takes A = dY^T [N x T] dense, 64 tokens
+// per stage: A 16 KB + two 8 KB atoms, 6 stages; each 16-token K step issues
+// two dense MMAs of N = 128.
 template <bool SPARSE, int EPI>
 struct PairGeom {
   static constexpr bool kWg = EPI == kEpiWgrad;
   static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
   static constexpr int kAcols = 64;                      // A values per row and stage
   static constexpr int kBN = kWg ? 256 : kPairBN;        // B columns (tokens, or dW columns) per pair tile
-  static constexpr int kBBoxes = SPARSE ? 2 : 1;
-  static constexpr int kBBoxBytes = kWg ? 64 * 128 * 2 : kPairSmemBBox;
+  static constexpr int kBBoxes = (SPARSE || kWg) ? 2 : 1;  // wgrad: two 64-column atoms
+  static constexpr int kBBoxBytes = kWg ? 64 * kBK * 2 : kPairSmemBBox;
   static constexpr int kMeta = SPARSE ? kSmemE : 0;
   static constexpr int kStageBytes = kPairSmemA + kBBoxes * kBBoxBytes + kMeta;
   static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
@@ -132,7 +135,15 @@ static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<fa
                   pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448 &&
                   pair_smem_bytes<true, kEpiWgrad>() <= 232448,
               "shared memory per CTA");
-static_assert(PairGeom<true, kEpiWgrad>::kStageBytes % 1024 == 0 && PairGeom<true, kEpiWgrad>::kBBoxBytes % 1024 == 0,
+static_assert(pair_smem_bytes<false, kEpiWgrad>() <= 232448, "shared memory per CTA (dense wgrad)");
+// The producer loads A and two B atoms (and, sparse, the metadata chunk) per stage of a
+// weight-gradient pipeline: the stage, and the byte count armed on its barrier, hold all of them.
+static_assert(PairGeom<true, kEpiWgrad>::kStageBytes == kPairSmemA + 2 * (64 * 128 * 2) + kSmemE &&
+                  PairGeom<false, kEpiWgrad>::kStageBytes == kPairSmemA + 2 * (64 * 64 * 2),
+              "wgrad stage = A + two B atoms (+ metadata)");
+static_assert(PairGeom<true, kEpiWgrad>::kStageBytes % 1024 == 0 && PairGeom<true, kEpiWgrad>::kBBoxBytes % 1024 == 0 &&
+                  PairGeom<false, kEpiWgrad>::kStageBytes % 1024 == 0 &&
+                  PairGeom<false, kEpiWgrad>::kBBoxBytes % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
 static_assert(PairGeom<true, kEpiWgrad>::kMetaCol + 4 * PairGeom<true, kEpiWgrad>::kStages <= kTmemCols,
               "tensor memory budget (wgrad)");
@@ -416,7 +427,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // Its B descriptor steps 8-token groups 1024 bytes apart (the stride field);
     // an MMA reads a single 64-column atom per CTA, so the field for the stride
     // between atoms along N is never used and is given the same 1024.
-    constexpr uint32_t idesc = WG ? (make_idesc_sparse(BF16, 2 * kPairRows, 128) | (1u << 16))
+    constexpr uint32_t idesc = WG ? ((SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, 128)
+                                             : make_idesc_dense(BF16, 2 * kPairRows, 128)) |
+                                    (1u << 16))
                                : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN)
                                         : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
     const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
@@ -438,7 +451,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint64_t so = (uint64_t)((s * kPairStageBytes) >> 4);
         const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
-        if (WG) {
+        if (WG && !SPARSE) {
+          // Dense weight gradient: K step kk of 16 tokens moves A 32 bytes along its
+          // swizzled rows and B 16 tokens (2048 bytes); atom 1 of B sits 8 KB after atom 0.
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
+            const uint64_t bk = bd + (uint64_t)(kk * (2048 >> 4));
+            tc_mma_f16_pair(acc, ad + 2 * kk, bk, idesc, accum);
+            tc_mma_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
+          }
+        } else if (WG) {
           const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;
           tc_cp_128x128b_pair(t_meta, e_desc0 + so);
           // K step kk: A advances 32 bytes along its swizzled rows, B 32 tokens

@@ -461,6 +461,25 @@ sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *val
                             : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s);
 }
 
+sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N, sp24_dtype dtype,
+                                  float *dW, void *stream) {
+  if (T < 0 || K < 0 || N < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (T % 16 || N % 16 || K % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!dW || (T > 0 && (!X || !dYt))) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (T > 0 && (!aligned16(X) || !aligned16(dYt)))) return SP24_ERR_MISALIGNED;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {   // an empty sum over tokens
+    return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  }
+  return dtype == SP24_BF16 ? launch_gemm_pair_t<true, kEpiWgrad, false>(X, K, T, dYt, nullptr, N, dW, nullptr, s)
+                            : launch_gemm_pair_t<false, kEpiWgrad, false>(X, K, T, dYt, nullptr, N, dW, nullptr, s);
+}
+
 sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,
                               const uint8_t *idx, float lambda, void *stream) {
   sp24_status st = validate_w(W, dtype, rows, cols, cols);

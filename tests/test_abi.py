@@ -127,6 +127,10 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_gemm_wgrad", fake, 32, 64, odd, fake, 64, 0, fake, None) == \
         E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_gemm_wgrad_dense", fake, 24, 64, fake, 64, 0, fake, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]
+    assert _raw("sp24_gemm_wgrad_dense", fake, 32, 64, None, 64, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
+    assert _raw("sp24_gemm_wgrad_dense", fake, 32, 64, fake, 64, 0, odd, None) == E["SP24_ERR_MISALIGNED"]
     # decay and flip
     assert _raw("sp24_masked_decay", fake, fake, 0, 6, 8, fake, ctypes.c_float(1.0), None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]

@@ -89,3 +89,46 @@ def test_dense_zero_tokens_is_a_no_op():
     y = torch.empty(0, 128, dtype=torch.float16, device="cuda")
     sp.sp24_gemm_dense(x, w, y)
     assert sp.sp24_device_status() == 0
+
+
+def _check_wgrad(dw, ref, what=""):
+    """fp32 weight gradient against the fp64 product: relative Frobenius <= 1e-4 and the
+    largest entry error <= 1e-3 of max |dW| (only the fp32 accumulation rounds)."""
+    got = dw.double().cpu().numpy()
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    mx = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-300)
+    assert fro <= 1e-4, f"{what}: relative Frobenius error {fro:.3e}"
+    assert mx <= 1e-3, f"{what}: largest entry error {mx:.3e}"
+
+
+@pytest.mark.parametrize("T,N,K,dtype", [(128, 256, 256, "f16"), (256, 272, 200, "f16"), (144, 160, 520, "bf16"),
+                                         (16, 16, 8, "f16"), (2048, 512, 1024, "f16")])
+def test_dense_weight_grad(T, N, K, dtype):
+    """dW = dY^T X with dY^T from the transpose kernel (ragged M, N and K tiles)."""
+    dy = si.normal((T, N), 1.0, T + 5, dtype)
+    x = si.normal((T, K), 1.0, T + 6, dtype)
+    dyt = _transpose(dy.cuda())
+    dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    sp.sp24_gemm_wgrad_dense(x.cuda(), dyt, dw)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    ref = oracle.dense_weight_grad(oracle.to_f64(si.bits16(dy), dtype), oracle.to_f64(si.bits16(x), dtype))
+    _check_wgrad(dw, ref, f"dense wgrad {T}x{N}x{K}")
+
+
+def test_dense_weight_grads_355m_sampled_rows():
+    wl = si.GPT2_355M
+    X, dY = wl.activations()
+    H, dH = wl.hidden()
+    rng = np.random.default_rng(2)
+    for g, b in ((dY, H), (dH, X)):
+        N, K = g.shape[1], b.shape[1]
+        gt = _transpose(g.cuda())
+        dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+        sp.sp24_gemm_wgrad_dense(b.cuda(), gt, dw)
+        torch.cuda.synchronize()
+        assert sp.sp24_device_status() == 0
+        rows = np.sort(rng.choice(N, 64, replace=False))
+        gf = oracle.to_f64(si.bits16(g), wl.dtype)[:, rows]
+        ref = oracle.dense_weight_grad(gf, oracle.to_f64(si.bits16(b), wl.dtype))
+        _check_wgrad(dw[torch.from_numpy(rows).cuda()], ref, f"dense dW [{N}x{K}] sampled rows")

@@ -130,6 +130,23 @@ def test_dense_gemms_exact_on_small_integers_and_adjoint():
     assert np.array_equal(oracle.dense_dgrad(np.eye(N), w), w)
 
 
+def test_dense_weight_grad_is_the_adjoint_of_the_forward_product():
+    """<dW, W> = <dY, X W^T> for any W: the weight gradient of the dense phase is the
+    gradient of <dY, Y> with respect to W.  Exact on small integers; explicit loops too."""
+    rng = np.random.default_rng(7)
+    T, N, K = 6, 5, 7
+    x = rng.integers(-9, 10, (T, K)).astype(np.float64)
+    dy = rng.integers(-9, 10, (T, N)).astype(np.float64)
+    dw = oracle.dense_weight_grad(dy, x)
+    assert dw.shape == (N, K)
+    for n in range(N):
+        for k in range(K):
+            assert dw[n, k] == sum(int(dy[t, n]) * int(x[t, k]) for t in range(T))
+    for _ in range(3):
+        w = rng.integers(-9, 10, (N, K)).astype(np.float64)
+        assert np.sum(dw * w) == np.sum(dy * oracle.dense_fwd(x, w))
+
+
 def test_gate_up_interleave_and_split_are_inverse():
     rng = np.random.default_rng(5)
     wg, wu = rng.normal(size=(48, 8)), rng.normal(size=(48, 8))
