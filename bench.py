@@ -512,7 +512,10 @@ class GegluStep:
     """The gated FFN of the same width on the 2:4 path: stacked gate/up weight
     [2 ff, d] (16-row groups alternate), down projection [d, ff]; per step the
     two mask steps, the GEGLU forward, the down projection, its input gradient
-    with the gated-gradient epilogue, the stacked input gradient and both decays."""
+    with the gated-gradient epilogue, the stacked input gradient, the weight
+    gradients of both weights on the MVUE sparsification of dY and of the stacked
+    gate/up gradient (which is already in the stacked weight's row order), and
+    the decays of those gradients."""
 
     def __init__(self, step):
         import torch
@@ -533,7 +536,11 @@ class GegluStep:
         self.dGU = torch.empty(T, 2 * ff, dtype=tdt, device="cuda")
         self.Y = torch.empty(T, d, dtype=tdt, device="cuda")
         self.dX = torch.empty(T, d, dtype=tdt, device="cuda")
-        self.flops = 6 * 2.0 * T * d * ff
+        # MVUE-sparsified dY^T [d x T] and dGU^T [2 ff x T]
+        self.yh = [(torch.empty(n, T // 2, dtype=tdt, device="cuda"),
+                    torch.empty(sp.sp24_compressed_size(n, T)[1], dtype=torch.uint8, device="cuda")) for n in (d, 2 * ff)]
+        self.step_no = 0
+        self.flops = 9 * 2.0 * T * d * ff
 
     def run(self):
         sp, st, wl = self.sp, self.step, self.step.wl
@@ -544,9 +551,16 @@ class GegluStep:
         sp.sp24_gemm_fwd(st.X, vr_gu, mr_gu, 2 * ff, self.H, "geglu", self.GU)
         sp.sp24_gemm_fwd(self.H, vr_d, mr_d, d, self.Y)
         sp.sp24_gemm_dgrad(st.dY, vc_d, mc_d, ff, self.dGU, "dgeglu", self.GU)
+        seed = wl.seeds["mvue"] + 1
+        (ydv, ydm), (ygv, ygm) = self.yh
+        sp.sp24_mvue_sparsify(st.dY, seed, 2 * self.step_no + 1, ydv, ydm)
+        sp.sp24_gemm_wgrad(self.H, ydv, ydm, d, self.Gd)
+        sp.sp24_mvue_sparsify(self.dGU, seed, 2 * self.step_no, ygv, ygm)
+        sp.sp24_gemm_wgrad(st.X, ygv, ygm, 2 * ff, self.Ggu)
         sp.sp24_gemm_dgrad(self.dGU, vc_gu, mc_gu, d, self.dX)
         sp.sp24_masked_decay(self.Ggu, self.Wgu, self.idx[0], wl.lam)
         sp.sp24_masked_decay(self.Gd, self.Wd, self.idx[1], wl.lam)
+        self.step_no += 1
 
 
 def run_geglu_phase(args, step, wl, world, dev, flush, barrier):
@@ -572,8 +586,9 @@ def run_geglu_phase(args, step, wl, world, dev, flush, barrier):
     ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world, dev) / args.steps
     return {"ms_per_step": round(ms, 4), "value": round(g.flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "note": "gated FFN (GEGLU) of the same d and ff on the 2:4 path: stacked gate/up weight [2 ff, d], "
-                    "down projection [d, ff]; mask steps, the four GEMMs with the gated epilogues, both decays; "
-                    "FLOPs 6 x 2 T d ff dense-equivalent"}
+                    "down projection [d, ff]; mask steps, the forward and input-gradient GEMMs with the gated "
+                    "epilogues, both weight gradients on the MVUE sparsification of dY and of the stacked "
+                    "gate/up gradient, both decays; FLOPs 9 x 2 T d ff dense-equivalent"}
 
 
 def run_e2e(args, step, wl, world, dev, barrier):

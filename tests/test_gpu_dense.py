@@ -116,8 +116,8 @@ def test_dense_weight_grad(T, N, K, dtype):
     _check_wgrad(dw, ref, f"dense wgrad {T}x{N}x{K}")
 
 
-def test_dense_weight_grads_355m_sampled_rows():
-    wl = si.GPT2_355M
+@pytest.mark.parametrize("wl", [si.GPT2_355M, si.GPT2_774M], ids=lambda w: w.name)
+def test_dense_weight_grads_full_size_sampled_rows(wl):
     X, dY = wl.activations()
     H, dH = wl.hidden()
     rng = np.random.default_rng(2)
