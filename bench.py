@@ -5,12 +5,14 @@ One step = the whole path on one GPT-2 FFN (default: the 355M shape, fp16,
   mask step on W1 and W2 (transposable 2:4 search, flip count against the
   previous mask, compression of both orientations), forward GEMMs
   (X -> gelu(X W1m^T) -> H W2m^T), input-gradient GEMMs (dY -> dH with the
-  gelu' epilogue -> dX), weight-gradient GEMMs on the MVUE 2:4 sparsification
-  of the output gradients (dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X, fp32),
-  masked decay on both weight gradients.
+  gelu' epilogue -> dX), masked decay on both weights' gradients (lambda = 6e-5).
 The weights alternate between W and a N(0, 1e-4)-perturbed copy each step, so
-the flip count is live.  The metric is the dense-equivalent FLOPs of the six
+the flip count is live.  The metric is the dense-equivalent FLOPs of the four
 GEMMs divided by the step time (TFLOP/s); per-kernel times give the roofline.
+Further lines of the same JSON object time, on the same workload, the training
+step with the weight gradients (MVUE 2:4 sparsification of dY^T and dH^T, then
+dW2 = MVUE(dY^T) H and dW1 = MVUE(dH^T) X in fp32, decayed in place), the dense
+fine-tuning step and the gated (GEGLU) FFN step.
 
 Multi-GPU: one process per GPU (torchrun), data-parallel replicas with their
 own token batch; masks are computed redundantly and bit-identically, so no
@@ -195,7 +197,8 @@ class ClockSampler:
 class FFNStep:
     """Device buffers and the launch sequence of one step (kernel launches only)."""
 
-    KERNELS = ("mask_step", "gemm_fwd", "gemm_dgrad", "mvue_dy", "mvue_dh", "gemm_wgrad", "masked_decay")
+    KERNELS = ("mask_step", "gemm_fwd", "gemm_dgrad", "masked_decay")
+    WGRAD_KERNELS = ("mvue_dy", "mvue_dh", "gemm_wgrad")
 
     def __init__(self, wl: si.FFNWorkload, rank: int):
         import torch
@@ -227,14 +230,16 @@ class FFNStep:
         self.yh = [(torch.empty(n, T // 2, dtype=tdt, device=dev),
                     torch.empty(sp.sp24_compressed_size(n, T)[1], dtype=torch.uint8, device=dev)) for n in (d, ff)]
         self.step_no = 0
-        self.launches_per_step = 12
+        self.launches_per_step = 8
 
-    def run(self, events=None):
+    def run(self, events=None, wgrad=False):
         """Enqueue one step; if `events` is a dict, record (start, end) CUDA events per kernel.
         The two layers' mask steps, and their decays, are independent: the second of each
         pair runs on a side stream, concurrently with the first (the step forks before the
         mask steps and joins before the second layer's forward GEMM and after the decays);
-        with `events` everything runs on one stream."""
+        with `events` everything runs on one stream.  With `wgrad` the step also computes
+        both weight gradients into the gradient buffers (MVUE + weight-gradient GEMM)
+        before they are decayed."""
         sp, torch, wl = self.sp, self.torch, self.wl
         d, ff = wl.d, wl.ff
         cur, prev = self.step_no % 2, (self.step_no + 1) % 2
@@ -276,14 +281,15 @@ class FFNStep:
         join()
         timed("gemm_fwd", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y), main)
         timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre), main)
-        # Weight gradients into the gradient buffers: dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X;
-        # fresh draws every step and layer (offset 2 * step + layer).
-        seed = wl.seeds["mvue"]
-        (y2v, y2m), (y1v, y1m) = self.yh
-        timed("mvue_dy", lambda: sp.sp24_mvue_sparsify(self.dY, seed, 2 * self.step_no + 1, y2v, y2m), main)
-        timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.H, y2v, y2m, d, self.G[1]), main)
-        timed("mvue_dh", lambda: sp.sp24_mvue_sparsify(self.dH, seed, 2 * self.step_no, y1v, y1m), main)
-        timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.X, y1v, y1m, ff, self.G[0]), main)
+        if wgrad:
+            # Weight gradients into the gradient buffers: dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X;
+            # fresh draws every step and layer (offset 2 * step + layer).
+            seed = wl.seeds["mvue"]
+            (y2v, y2m), (y1v, y1m) = self.yh
+            timed("mvue_dy", lambda: sp.sp24_mvue_sparsify(self.dY, seed, 2 * self.step_no + 1, y2v, y2m), main)
+            timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.H, y2v, y2m, d, self.G[1]), main)
+            timed("mvue_dh", lambda: sp.sp24_mvue_sparsify(self.dH, seed, 2 * self.step_no, y1v, y1m), main)
+            timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.X, y1v, y1m, ff, self.G[0]), main)
         timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dH, c1[2], c1[3], d, self.dX), main)
         fork()
         for li, stream in ((0, main), (1, side)):
@@ -337,6 +343,7 @@ class FFNStep:
             "mask_step": ("GB/s", n_el * (2 + 1 / 16 + 1 / 16 + 2 + 0.25)),
             "gemm_fwd": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
             "gemm_dgrad": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
+            # the training step with the weight gradients
             "gemm_wgrad": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
             # read dY (2 B/el), write the kept values (1 B/el) and their metadata (1/8 B/el)
             "mvue_dy": ("GB/s", wl.tokens * wl.d * (2 + 1 + 1 / 8)),
@@ -393,6 +400,7 @@ def run_ours(args, wl, rank, world, local_rank):
         flush.fill_(1.0)
         step.run(events)
     barrier()
+    wgrad = run_wgrad_phase(args, step, wl, world, dev, flush, barrier)
     dense = run_dense_phase(args, step, wl, world, dev, flush, barrier)
     geglu = run_geglu_phase(args, step, wl, world, dev, flush, barrier)
     total_ms = max_over_ranks(step_ms, world, dev)
@@ -412,7 +420,7 @@ def run_ours(args, wl, rank, world, local_rank):
         peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
         kernels[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
                          "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
-    g = {k: kernels[k] for k in ("gemm_fwd", "gemm_dgrad", "gemm_wgrad")}
+    g = {k: kernels[k] for k in ("gemm_fwd", "gemm_dgrad")}
     g_time = sum(v["avg_us"] * v["launches"] for v in g.values())
     g_launches = sum(v["launches"] for v in g.values())
     g_avg = g_time / g_launches * 1e-6
@@ -420,7 +428,7 @@ def run_ours(args, wl, rank, world, local_rank):
     roofline = {"bound": "tensor", "achieved": round(g_ach, 1), "peak": sparse_peak, "unit": "TFLOP/s",
                 "frac": round(g_ach / sparse_peak, 4),
                 "traffic": args.gemm_traffic or load_traffic("gemm", wl.name),
-                "kernel": "sp24_gemm_pair_kernel (fwd + dgrad + wgrad launches)",
+                "kernel": "sp24_gemm_pair_kernel (fwd + dgrad launches)",
                 "peak_source": f"2 x {peak_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s), "
                                "the nominal 2:4 sparse ratio"}
     mask = kernels["mask_step"]
@@ -445,6 +453,7 @@ def run_ours(args, wl, rank, world, local_rank):
                                  "traffic": args.mask_traffic or load_traffic("mask_step", wl.name),
                                  "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
         "kernels": kernels,
+        "ffn_step_with_weight_gradients": wgrad,
         "dense_finetune_step": dense,
         "geglu_ffn_step": geglu,
         "e2e": e2e,
@@ -456,6 +465,53 @@ def run_ours(args, wl, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_tokens)
     return line
+
+
+def run_wgrad_phase(args, step, wl, world, dev, flush, barrier):
+    """The 2:4 training step with both weight gradients (MVUE + weight-gradient GEMM, then the
+    decay of the computed gradients), timed like the headline step, and its MVUE and
+    weight-gradient kernels from an instrumented pass."""
+    import torch
+    import structured_sparse_transformer_b200 as sp
+    for _ in range(args.warmup):
+        step.run(wgrad=True)
+    step_ev = []
+    barrier()
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step.run(wgrad=True)
+        e.record()
+        step_ev.append((s, e))
+    barrier()
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), world, dev) / args.steps
+    events = {}
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        step.run(events, wgrad=True)
+    barrier()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the weight-gradient step: {sp.sp24_status_string(st)}")
+    peaks, _ = load_peaks()
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    work = step.work()
+    kernels = {}
+    for name in FFNStep.WGRAD_KERNELS:
+        unit, amount = work[name]
+        times = [s.elapsed_time(e) * 1e-3 for s, e in events[name]]
+        avg = sum(times) / len(times)
+        achieved = amount / avg / (1e12 if unit == "TFLOP/s" else 1e9)
+        peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
+        kernels[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
+                         "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
+    flops = 6 * 2.0 * wl.tokens * wl.d * wl.ff
+    return {"ms_per_step": round(ms, 4), "value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "launches_per_step": 12, "kernels": kernels,
+            "note": "the headline step plus both weight gradients: MVUE 2:4 sparsification of dY^T and dH^T "
+                    "(Philox4x64-10 draws), dW2 = MVUE(dY^T) H and dW1 = MVUE(dH^T) X on the sparse tensor "
+                    "cores in fp32, then the masked decay of those gradients; FLOPs 6 x 2 T d ff"}
 
 
 def run_dense_phase(args, step, wl, world, dev, flush, barrier):
@@ -493,7 +549,7 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier):
     n_el = wl.d * wl.ff
     t_avg = sum(t) / len(t)
     return {"ms_per_step": round(ms, 4),
-            "value": round(wl.gemm_flops() * world / (ms * 1e-3) / 1e12, 2),
+            "value": round(6 * 2.0 * wl.tokens * wl.d * wl.ff * world / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s",
             "gemm": {"launches": len(g), "avg_us": round(g_avg * 1e6, 2), "achieved": round(ach, 1),
                      "peak": peaks["bf16_tflops"], "frac": round(ach / peaks["bf16_tflops"], 4)},
@@ -593,8 +649,8 @@ def run_geglu_phase(args, step, wl, world, dev, flush, barrier):
 
 def run_e2e(args, step, wl, world, dev, barrier):
     """Same metric through the C ABI with host buffers: H2D of the step's inputs (both weights,
-    X, dY) from pinned memory and D2H of its results (Y, dX, both decayed weight gradients,
-    the flip counts) inside the timed region.  Copies run on their own streams
+    X, dY, both gradients) from pinned memory and D2H of its results (Y, dX, both decayed
+    gradients, the flip counts) inside the timed region.  Copies run on their own streams
     and overlap the neighbouring steps' kernels: step k's inputs land in slot k % 2 while
     step k-1 computes, and its results leave while step k+1 computes."""
     import torch
@@ -623,6 +679,8 @@ def run_e2e(args, step, wl, world, dev, barrier):
             step.W[1][b].copy_(hw[1][b], non_blocking=True)
             sl["X"].copy_(h["X"], non_blocking=True)
             sl["dY"].copy_(h["dY"], non_blocking=True)
+            sl["G"][0].copy_(h["G1"], non_blocking=True)
+            sl["G"][1].copy_(h["G2"], non_blocking=True)
             landed = ev()
             landed.record(hs)
         cs.wait_event(landed)
@@ -656,7 +714,7 @@ def run_e2e(args, step, wl, world, dev, barrier):
     e.record(cs)
     barrier()
     ms = max_over_ranks(s.elapsed_time(e), world, dev)
-    h2d = sum(v.numel() * v.element_size() for v in (hw[0][0], hw[1][0], h["X"], h["dY"]))
+    h2d = sum(v.numel() * v.element_size() for v in (hw[0][0], hw[1][0], h["X"], h["dY"], h["G1"], h["G2"]))
     d2h = sum(t.numel() * t.element_size() for t in (out_y, out_dx, *out_g, out_f))
     return {"value": round(wl.gemm_flops() * world * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / args.steps, 4),
@@ -668,11 +726,9 @@ def run_e2e(args, step, wl, world, dev, barrier):
 
 def oracle_step(wl, host, rows):
     """One step of the CPU oracle on a token sample: both mask searches, both compressions,
-    the six GEMMs on `rows` token rows (forward, input gradient, MVUE sparsification and
-    weight gradient of both layers), GELU, masked decay on both gradients, flip counts.
+    the four GEMMs on `rows` token rows, GELU, masked decay on both gradients, flip counts.
     Returns the GEMM FLOPs it processed."""
     import oracle
-    import torch
     dt = wl.dtype
     b1, b2 = si.bits16(host["W1"]), si.bits16(host["W2"])
     i1, i2 = oracle.mask_search(b1, dt), oracle.mask_search(b2, dt)
@@ -687,17 +743,11 @@ def oracle_step(wl, host, rows):
     oracle.sparse_fwd(h, w2, k2)
     dh = oracle.sparse_dgrad(dy, w2, k2) * oracle.gelu_grad(pre)
     oracle.sparse_dgrad(dh, w1, k1)
-    seed = wl.seeds["mvue"]
-    y2 = oracle.mvue_sparsify_t(si.bits16(host["dY"])[:rows], dt, seed, 1)[0]
-    oracle.weight_grad(oracle.to_f64(y2, dt), oracle.round_to(h, dt))
-    dh_bits = si.bits16(torch.from_numpy(oracle.round_to(dh, dt)).to(si.DTYPES[dt]))
-    y1 = oracle.mvue_sparsify_t(dh_bits, dt, seed, 0)[0]
-    oracle.weight_grad(oracle.to_f64(y1, dt), x)
     oracle.masked_decay(host["G1"].numpy(), b1, dt, i1, wl.lam)
     oracle.masked_decay(host["G2"].numpy(), b2, dt, i2, wl.lam)
     oracle.flip_count(i1, i1)
     oracle.flip_count(i2, i2)
-    return 6 * 2.0 * rows * wl.d * wl.ff
+    return 4 * 2.0 * rows * wl.d * wl.ff
 
 
 def cpu_baseline(wl, rows):
@@ -712,9 +762,8 @@ def cpu_baseline(wl, rows):
     dt = time.perf_counter() - t0
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"one full oracle step of {wl.name} with the six GEMMs (and the MVUE sparsification) "
-                      f"on the first {rows} of {wl.tokens} token rows (mask search, compression, decay and "
-                      f"flips in full)"}
+            "sample": f"one full oracle step of {wl.name} with the four GEMMs on the first {rows} of "
+                      f"{wl.tokens} token rows (mask search, compression, decay and flips in full)"}
 
 
 def run_reference(args, wl):
@@ -733,8 +782,8 @@ def run_reference(args, wl):
         flops += oracle_step(wl, host, rows)
     sec = time.perf_counter() - t0
     value = flops / sec / 1e12
-    sample = (f"each step: the oracle's full {wl.name} step with the six GEMMs (and the MVUE "
-              f"sparsification) on the first {rows} of {wl.tokens} token rows")
+    sample = (f"each step: the oracle's full {wl.name} step with the four GEMMs on the first {rows} of "
+              f"{wl.tokens} token rows")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -97,9 +97,8 @@ class FFNWorkload:
         return self.seeds["perturb"] + 2 * step + which
 
     def gemm_flops(self) -> int:
-        """Dense-equivalent FLOPs of the six FFN GEMMs of a training step (forward,
-        input gradient and weight gradient of both layers)."""
-        return 6 * 2 * self.tokens * self.d * self.ff
+        """Dense-equivalent FLOPs of the four FFN GEMMs (fwd and dX for both layers)."""
+        return 4 * 2 * self.tokens * self.d * self.ff
 
 
 # The workloads: PR1 (one weight, fwd only) and three GPT-2 FFN shapes.
