@@ -4,7 +4,7 @@
 // table, Software Dependencies row (2:4 sparse matrix multiplications) and the
 // abstract (transposable masks make the input-gradient product 2:4 as well).
 //
-// One kernel serves both products.  With A the 2:4-compressed operand
+// One kernel serves the FFN products.  With A the 2:4-compressed operand
 // [M x Kd] (2 of every 4 values along Kd kept) and B = activations [T x Kd]:
 //     out[T x M] = B * A^T
 //   forward:        A = W   [N x K] compressed along K,  B = X  -> Y  [T x N]
@@ -12,6 +12,11 @@
 // The sparse operand must be the MMA's A operand, so the tensor-memory tile is
 // out^T (lane = output feature, column = token); each epilogue thread owns one
 // feature and writes it for consecutive tokens of row-major out.
+// The weight-gradient variant (EPI = kEpiWgrad) contracts over tokens instead:
+// A = MVUE(dY^T) [N x T] compressed along T (or, dense, dY^T), B = the layer
+// input [T x K] read as stored (MN-major), out = dW [N x K] fp32 in the natural
+// orientation (see PairGeom and the weight-gradient epilogue).  The same kernel
+// with SPARSE = false runs the dense fine-tuning products.
 //
 // CTA pairs (clusters of 2, tcgen05 cta_group::2).  A pair computes a tile of
 // 256 output features x 224 tokens: each CTA holds 128 rows of the compressed

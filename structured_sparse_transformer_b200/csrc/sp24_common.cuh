@@ -338,10 +338,8 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 constexpr uint32_t kSwizzleNone = 0;
 constexpr uint32_t kSwizzle128B = 2;
 
-// Instruction descriptor of kind::f16 with fp32 accumulation, both operands
-// K-major, 2:4 sparse A.  Bits 0-1 (sparsity selector) are left 0 here and set
-// per MMA to the low column bit of the metadata address.
-// Instruction descriptor of a dense kind::f16 MMA with fp32 accumulation.
+// Instruction descriptor of a dense kind::f16 MMA with fp32 accumulation, both
+// operands K-major (bit 16 set by the caller makes B MN-major).
 __host__ __device__ constexpr uint32_t make_idesc_dense(bool bf16, int m, int n) {
   return (1u << 4)                      // D format fp32
          | ((bf16 ? 1u : 0u) << 7)      // A format
@@ -350,6 +348,9 @@ __host__ __device__ constexpr uint32_t make_idesc_dense(bool bf16, int m, int n)
          | ((uint32_t)(m >> 4) << 24);  // M / 16
 }
 
+// Instruction descriptor of kind::f16 with fp32 accumulation, both operands
+// K-major, 2:4 sparse A.  Bits 0-1 (sparsity selector) are left 0 here and set
+// per MMA to the low column bit of the metadata address.
 __host__ __device__ constexpr uint32_t make_idesc_sparse(bool bf16, int m, int n) {
   return (1u << 2)                      // sparse
          | (1u << 4)                    // D format fp32
