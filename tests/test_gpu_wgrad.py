@@ -188,3 +188,32 @@ def test_ffn_weight_grads_full_size_column_sample(wl):
             assert np.array_equal(got_vals[cols[0]:cols[-1] + 1], ovals)
             ref = oracle.weight_grad(oracle.to_f64(bits, dt), bf)
             _check_wgrad(dw[int(cols[0]):int(cols[-1]) + 1], ref, f"dW [{N}x{K}] rows {cols[0]}..")
+
+
+def test_ffn_weight_grads_1p5b_sampled_rows_and_columns():
+    """Both weight gradients of the 1.5B FFN (fp16, 32768 tokens) at full size: dW1 [6400 x 1600]
+    has a ragged last column tile (1600 = 6 x 256 + 64).  The sparsified operand is compared on
+    64 columns of dY / dH, dW on those 64 rows x 96 columns (the last 32 in the ragged tile)."""
+    wl = si.GPT2_1P5B
+    dt = wl.dtype
+    X, dY = wl.activations()
+    H, dH = wl.hidden()
+    T = wl.tokens
+    rng = np.random.default_rng(5)
+    for (g, b, N, K, off) in ((dY, H, wl.d, wl.ff, 5), (dH, X, wl.ff, wl.d, 6)):
+        vals, meta = _alloc(N, T, dt)
+        dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+        sp.sp24_mvue_sparsify(g.cuda(), wl.seeds["mvue"], off, vals, meta)
+        sp.sp24_gemm_wgrad(b.cuda(), vals, meta, N, dw)
+        torch.cuda.synchronize()
+        assert sp.sp24_device_status() == 0
+        r0 = int(rng.integers(0, (N - 64) // 32)) * 32
+        cols = np.concatenate([np.sort(rng.choice(K - 32, 64, replace=False)), np.arange(K - 32, K)])
+        bits, keep, _ = oracle.mvue_sparsify_t(np.ascontiguousarray(si.bits16(g)[:, r0:r0 + 64]), dt,
+                                               wl.seeds["mvue"], off, col0=r0)
+        ovals, _ = oracle.compress_rows(bits, keep)
+        assert np.array_equal(si.bits16(vals[r0:r0 + 64].cpu()), ovals)
+        bf = oracle.to_f64(np.ascontiguousarray(si.bits16(b)[:, cols]), dt)
+        ref = oracle.weight_grad(oracle.to_f64(bits, dt), bf)
+        got = dw[r0:r0 + 64][:, torch.from_numpy(cols).cuda()]
+        _check_wgrad(got, ref, f"dW [{N}x{K}] rows {r0}.. sampled columns")
