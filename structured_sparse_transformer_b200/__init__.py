@@ -102,8 +102,17 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need_cuda(*ts):
+def _need_cuda(*ts, pitched=()):
+    """The library reads every buffer as row-major: contiguous tensors, except those in
+    `pitched` (2-D, unit stride along rows, the row pitch passed as a leading dimension).
+    Layout is checked first, then that every tensor lives on a CUDA device."""
     for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("sp24 takes contiguous (row-major) tensors")
+    for t in pitched:
+        if t is not None and (t.dim() != 2 or t.stride(1) != 1):
+            raise ValueError("sp24 takes 2-D row-major tensors with unit stride along rows")
+    for t in (*ts, *pitched):
         if t is not None and not t.is_cuda:
             raise ValueError("sp24 kernels take CUDA tensors only")
 
@@ -147,14 +156,14 @@ def sp24_meta_from_canonical(canon, rows: int, cols: int):
 
 def sp24_mask_search(W, idx, stream=None):
     """idx[R/4, C/4] (uint8, CUDA) <- Algorithm 1 on W [R, C] (fp16/bf16, CUDA, row-major)."""
-    _need_cuda(W, idx)
+    _need_cuda(idx, pitched=(W,))
     R, C = W.shape
     _check("sp24_mask_search", _lib.sp24_mask_search(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx),
                                                      _stream(stream)))
 
 
 def sp24_prune_compress(W, idx, vals_row, meta_row, vals_col, meta_col, stream=None):
-    _need_cuda(W, idx, vals_row, meta_row, vals_col, meta_col)
+    _need_cuda(idx, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
     R, C = W.shape
     _check("sp24_prune_compress",
            _lib.sp24_prune_compress(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(vals_row),
@@ -163,7 +172,7 @@ def sp24_prune_compress(W, idx, vals_row, meta_row, vals_col, meta_col, stream=N
 
 def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_row=None, vals_col=None,
                    meta_col=None, stream=None):
-    _need_cuda(W, idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col)
+    _need_cuda(idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
     R, C = W.shape
     _check("sp24_mask_step",
            _lib.sp24_mask_step(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(idx_prev),
@@ -210,7 +219,7 @@ def sp24_transpose(x, out, stream=None):
 
 def sp24_mvue_sparsify(dY, seed: int, offset: int, vals, meta, stream=None):
     """vals/meta <- dY[T, N]^T compressed 2:4 along T with the MVUE draws of (seed, offset)."""
-    _need_cuda(dY, vals, meta)
+    _need_cuda(vals, meta, pitched=(dY,))
     T, N = dY.shape
     _check("sp24_mvue_sparsify",
            _lib.sp24_mvue_sparsify(_ptr(dY), T, N, dY.stride(0), _dtype_code(dY), int(seed) & (2**64 - 1),

@@ -138,6 +138,24 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
     assert _raw("sp24_flip_rate", fake, fake, 4, None, None) == E["SP24_ERR_INVALID_ARG"]
 
 
+def test_binding_rejects_views_that_are_not_row_major():
+    """Layout is checked before anything else (here on CPU tensors, so no device is needed)."""
+    import torch
+    w = torch.zeros(64, 64, dtype=torch.float16)
+    idx = torch.zeros(16, 16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="row-major"):
+        sp.sp24_mask_search(w.t(), idx)                     # column-major view of W
+    with pytest.raises(ValueError, match="contiguous"):
+        sp.sp24_gemm_fwd(w[:, ::2], w, idx, 64, w)          # strided activations
+    with pytest.raises(ValueError, match="contiguous"):
+        sp.sp24_masked_decay(torch.zeros(64, 64).t(), w, idx, 1e-4)
+    with pytest.raises(ValueError, match="row-major"):
+        sp.sp24_mvue_sparsify(w[:, ::2], 0, 0, w, idx)
+    # a row-pitched W passes the layout check and stops at the device check
+    with pytest.raises(ValueError, match="CUDA"):
+        sp.sp24_mask_search(torch.zeros(64, 96, dtype=torch.float16)[:, :64], idx)
+
+
 def test_valid_call_without_a_device_reports_no_device():
     import torch
     if torch.cuda.is_available():
