@@ -1,0 +1,47 @@
+"""The benchmark's JSON contract, on the CPU: the reference arm (the oracle timed on
+the host cores) prints one line with the keys the measurement contract requires,
+for the same metric and workload as the GPU arm; the clock sampler summarises to
+the `clocks` object even where no GPU or NVML is present."""
+import contextlib
+import io
+import json
+
+import bench
+import synthetic_inputs as si
+
+REQUIRED = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+            "scaling", "vs_baseline", "dtype", "data", "config"}
+
+
+def test_reference_arm_prints_one_contract_line():
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0", "--cpu-tokens", "32"])
+    assert rc == 0
+    lines = [line for line in out.getvalue().splitlines() if line.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert REQUIRED <= set(d)
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"]["workload"] == si.GPT2_355M.name
+    assert d["config"]["d_model"] == 1024 and d["config"]["d_ff"] == 4096 and d["config"]["tokens_per_gpu"] == 8192
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "32 of 8192" in cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_clock_sampler_summary_without_a_gpu():
+    c = bench.ClockSampler(0, period_s=0.01)
+    with c:
+        pass
+    s = c.summary()
+    assert set(s) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+    if not c.samples:
+        assert s["sm_mhz"] is None and s["reasons"]
+
+
+def test_headline_flops_are_the_four_ffn_gemms():
+    wl = si.GPT2_355M
+    assert wl.gemm_flops() == 4 * 2 * 8192 * 1024 * 4096
