@@ -9,7 +9,13 @@
  *   - reproducibility table, Software Dependencies row: the pruning kernel and
  *     the 2:4 sparse matrix multiplications, the masked decay kernel;
  *   - abstract: masked decay on gradients, the flip rate that monitors mask
- *     stability, and transposable masks so the backward product is 2:4 too.
+ *     stability, and transposable masks so the backward product is 2:4 too;
+ *   - Software Dependencies row: the MVUE kernel (here the minimum-variance
+ *     unbiased 2:4 estimate of dY^T, sp24_mvue_sparsify) feeding the 2:4
+ *     weight-gradient product (sp24_gemm_wgrad), and the GEGLU kernel (the gated
+ *     epilogues of sp24_gemm_fwd / sp24_gemm_dgrad);
+ *   - abstract and Experiment Setup row: dense fine-tuning for the last 1/6 of
+ *     the steps (sp24_gemm_dense, sp24_gemm_wgrad_dense, sp24_transpose).
  *
  * Conventions shared by every call
  *   - Matrices are row-major.  W is [rows x cols] with leading dimension ldw
