@@ -156,6 +156,19 @@ def test_special_groups():
     assert pos.tolist() == [[0, 2], [0, 2], [1, 3], [1, 3]]
 
 
+def test_golden_groups():
+    """Hand-derived cases (tests/golden/mvue_groups.txt, derivations in the file)."""
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "mvue_groups.txt")
+    cases = [line.split("|") for line in open(path) if line.strip() and not line.startswith("#")]
+    assert len(cases) == 8
+    for v, u, pos, est in cases:
+        v = np.array([float(x) for x in v.split()])
+        p, e = oracle.mvue_select(v[None], np.array([float(u)]))
+        assert p[0].tolist() == [int(x) for x in pos.split()], (v, u)
+        assert e[0].tolist() == [float(x) for x in est.split()], (v, u)
+
+
 def test_sparsify_invariants():
     t, n = 256, 64
     dy = si.normal((t, n), 1.0, 3, "f16")
