@@ -174,7 +174,11 @@ static float to_float(uint16_t bits, int dtype) {
   }
   uint64_t sig;
   int shift;
-  decode_magnitude(bits, DT_F16, &sig, &shift);
+  if (decode_magnitude(bits, DT_F16, &sig, &shift) != ORACLE_OK) {
+    /* exponent all ones: infinity (zero fraction) or NaN, outside the finite-weight contract */
+    float inf = (bits & 0x3FFu) ? NAN : INFINITY;
+    return (bits & 0x8000u) ? -inf : inf;
+  }
   float mag = ldexpf((float)sig, shift - 24); /* exact: sig < 2^11 */
   return (bits & 0x8000u) ? -mag : mag;
 }
