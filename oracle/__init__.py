@@ -368,6 +368,20 @@ def mvue_uniforms(rows: int, groups: int, seed: int, offset: int, row0: int = 0)
     return (u32 >> np.uint64(8)).astype(np.float64) * 2.0 ** -24
 
 
+def _check_two_entries(i1: np.ndarray, i2: np.ndarray, a: np.ndarray, capped: np.ndarray) -> None:
+    """Raises unless, in every uncapped group, the systematic-sampling points select two
+    different entries in increasing order, both with a nonzero magnitude (see mvue_select)."""
+    free = ~np.asarray(capped, bool)
+    if not np.any(free):
+        return
+    j1, j2 = np.asarray(i1)[free], np.asarray(i2)[free]
+    af = np.asarray(a)[free]
+    nz1 = np.take_along_axis(af, j1[..., None], axis=-1)[..., 0] > 0
+    nz2 = np.take_along_axis(af, j2[..., None], axis=-1)[..., 0] > 0
+    if not (np.all(j1 < j2) and np.all(nz1) and np.all(nz2)):
+        raise ArithmeticError("MVUE systematic sampling selected one entry twice or a zero entry")
+
+
 def mvue_select(v: np.ndarray, u: np.ndarray):
     """Minimum-variance unbiased 2:4 estimate of each group of four values.
 
@@ -387,6 +401,22 @@ def mvue_select(v: np.ndarray, u: np.ndarray):
         second, kept as sign(v_k) R; if R = 0 the lowest other position is kept as +0.
     Every step is an fp64 operation in the order written (each sum is exact for fp16
     groups); an entry is selected by counting the cumulative sums at or below the point.
+
+    The two points always select two different nonzero entries, although the cumulative
+    sums c1 <= c2 <= c3 and the total s are rounded (fp64 round-to-nearest-even is
+    monotone).  With h = s/2 and no |v_i| reaching h, let the first point p1 = fl(u h)
+    select entry j, i.e. c_j <= p1 < c_(j+1) (c_0 = 0):
+      * j < 3: c_(j+1) = fl(c_j + a_j) <= fl(p1 + h) = p2, so p2 selects an entry after j;
+      * j = 3 would need c3 <= p1 <= h and a3 < h with s = fl(c3 + a3) = 2h, so the sum
+        rounds up by at least h - a3 and at most half an ulp of s, i.e. ulp(h): then a3 is
+        h - ulp(h) (h not a power of two; a format of at most 51 significant bits has no
+        value in [2^k - 2^(k-52), 2^k)), c3 = h, and c3 + a3 is halfway between 2a3 and 2h.
+        2a3 has the even significand (a3 has trailing zeros), so s = 2a3 and the group is
+        capped after all.
+    An entry j < 3 is selected only if c_(j+1) > c_j, so a_j > 0; the second point selects
+    the last entry only if a3 > 0 (else s = c3, and p2 < 2h = c3 since u <= 1 - 2^-24).
+    Hence `_check_two_entries` never raises; it is kept so that a slip in this function
+    cannot pass unnoticed.
     """
     v = np.asarray(v, np.float64)
     u = np.asarray(u, np.float64)
@@ -406,16 +436,7 @@ def mvue_select(v: np.ndarray, u: np.ndarray):
     p2 = p1 + h
     i1 = (c1 <= p1).astype(np.int64) + (c2 <= p1) + (c3 <= p1)
     i2 = (c1 <= p2).astype(np.int64) + (c2 <= p2) + (c3 <= p2)
-    # Only a rounded cumulative sum can put both points in one entry; then the second
-    # goes to the next nonzero entry after the first, else the last nonzero one before it.
-    nz = a > 0
-    coll = i2 == i1
-    if np.any(coll & ~capped):
-        for ix in zip(*np.nonzero(coll & ~capped)):
-            j1 = int(i1[ix])
-            after = [j for j in range(j1 + 1, 4) if nz[ix][j]]
-            before = [j for j in range(j1 - 1, -1, -1) if nz[ix][j]]
-            i2[ix] = after[0] if after else before[0]
+    _check_two_entries(i1, i2, a, capped)
 
     # the largest entry kept, one point over the other three
     b = np.where(np.arange(4) == m[..., None], 0.0, a)

@@ -161,12 +161,66 @@ def test_golden_groups():
     import os
     path = os.path.join(os.path.dirname(__file__), "golden", "mvue_groups.txt")
     cases = [line.split("|") for line in open(path) if line.strip() and not line.startswith("#")]
-    assert len(cases) == 8
+    assert len(cases) == 10
+
+    def num(x):
+        return float.fromhex(x) if "0x" in x else float(x)
+
     for v, u, pos, est in cases:
-        v = np.array([float(x) for x in v.split()])
-        p, e = oracle.mvue_select(v[None], np.array([float(u)]))
+        v = np.array([num(x) for x in v.split()])
+        p, e = oracle.mvue_select(v[None], np.array([num(u)]))
         assert p[0].tolist() == [int(x) for x in pos.split()], (v, u)
-        assert e[0].tolist() == [float(x) for x in est.split()], (v, u)
+        assert e[0].tolist() == [num(x) for x in est.split()], (v, u)
+
+
+def _bf16_values(rng, shape, emin, emax):
+    """Random bf16 values (as float64) with exponents uniform in [emin, emax], random signs."""
+    e = rng.integers(emin, emax + 1, size=shape)
+    m = rng.integers(0, 128, size=shape)
+    v = np.ldexp(1.0 + m / 128.0, e) * rng.choice([-1.0, 1.0], size=shape)
+    return v
+
+
+def test_systematic_points_always_select_two_nonzero_entries():
+    """The two sampling points of an uncapped group select two different nonzero entries for
+    every input, although the fp64 cumulative sums round (the proof is in mvue_select's
+    docstring); the oracle raises otherwise.  Groups here are built to stress the rounding:
+    bf16 magnitudes spread over up to 250 binades, entries just below half the group's sum,
+    tiny entries at rounding distance of the running sums, and the extreme draws."""
+    rng = np.random.default_rng(7)
+    us = np.array([0.0, 2.0**-24, 0.5, 1 - 2.0**-24])
+    groups = [_bf16_values(rng, (40000, 4), -126, 124),
+              _bf16_values(rng, (40000, 4), -10, 10)]
+    # one entry just below half of the sum: x + y ~ z, plus a tiny entry t at or near the
+    # rounding boundary of the running sums
+    x = _bf16_values(rng, (40000,), -2, 2)
+    y = _bf16_values(rng, (40000,), -2, 2)
+    z = torch.from_numpy(np.abs(x) + np.abs(y)).to(torch.bfloat16).double().numpy()
+    t = np.ldexp(1.0 + rng.integers(0, 128, 40000) / 128.0, rng.integers(-60, -45, 40000))
+    for perm in ([0, 1, 2, 3], [3, 2, 1, 0], [1, 3, 0, 2]):
+        groups.append(np.stack([t, x, y, z], axis=-1)[:, perm])
+    checked = 0
+    for g in groups:
+        for u in us:
+            pos, est = oracle.mvue_select(g, np.full(len(g), u))
+            assert np.all(pos[:, 0] < pos[:, 1])
+            kept = np.take_along_axis(g, pos, axis=-1)
+            a = np.abs(g)
+            capped = 2 * a.max(-1) >= a[:, 0] + a[:, 1] + a[:, 2] + a[:, 3]
+            assert np.all(kept[~capped] != 0)
+            checked += int((~capped).sum())
+    assert checked > 100000
+
+
+def test_two_entry_check_rejects_a_planted_slip():
+    a = np.array([[1.0, 1.0, 1.0, 0.0]])
+    capped = np.array([False])
+    oracle._check_two_entries(np.array([0]), np.array([2]), a, capped)
+    with pytest.raises(ArithmeticError):
+        oracle._check_two_entries(np.array([1]), np.array([1]), a, capped)     # one entry twice
+    with pytest.raises(ArithmeticError):
+        oracle._check_two_entries(np.array([0]), np.array([3]), a, capped)     # a zero entry
+    oracle._check_two_entries(np.array([1]), np.array([1]), a, np.array([True]))  # capped: not checked
 
 
 def test_sparsify_invariants():
