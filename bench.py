@@ -1,18 +1,21 @@
 """Benchmark of the 2:4 sparse FFN hot path on B200.
 
-One step = the whole path on one GPT-2 FFN (default: the 355M shape, fp16,
-8192 tokens):
-  mask step on W1 and W2 (transposable 2:4 search, flip count against the
-  previous mask, compression of both orientations), forward GEMMs
-  (X -> gelu(X W1m^T) -> H W2m^T), input-gradient GEMMs (dY -> dH with the
-  gelu' epilogue -> dX), masked decay on both weights' gradients (lambda = 6e-5).
-The weights alternate between W and a N(0, 1e-4)-perturbed copy each step, so
-the flip count is live.  The metric is the dense-equivalent FLOPs of the four
-GEMMs divided by the step time (TFLOP/s); per-kernel times give the roofline.
-Further lines of the same JSON object time, on the same workload, the training
-step with the weight gradients (MVUE 2:4 sparsification of dY^T and dH^T, then
-dW2 = MVUE(dY^T) H and dW1 = MVUE(dH^T) X in fp32, decayed in place), the dense
-fine-tuning step and the gated (GEGLU) FFN step.
+One step = the whole path on one GPT-2 FFN (default: the 1.5B shape, d = 1600,
+ff = 6400, fp16, 32768 tokens), as simulated training steps: the weights
+W_0 .. W_S of both layers follow W_(t+1) = round(W_t + N(0, 1e-4)) (S = 8 for
+the 1.5B shape), and step t runs
+  mask step on W1 and W2 at W_(t+1) (transposable 2:4 search, flip count against
+  the mask of W_t, compression of both orientations), forward GEMMs
+  (X -> gelu(X W1m^T) -> H W2m^T), input-gradient GEMMs (dY -> dH with the gelu'
+  epilogue -> dX), masked decay on both weights' gradients (lambda = 6e-5).
+Timed steps cycle through t = 0 .. S-1.  The metric is the dense-equivalent
+FLOPs of the four GEMMs divided by the step time (TFLOP/s); per-kernel times
+give the roofline.  The same JSON line carries the mask-search bandwidth sweep
+(fused mask step and search alone on fp16 16384 x 16384 and 16384 x 65536,
+Gaussian and 8-level tie-heavy), the GPT-2 355M step, and, on the headline
+workload, the training step with the weight gradients (MVUE 2:4 sparsification
+of dY^T and dH^T, then dW2 = MVUE(dY^T) H and dW1 = MVUE(dH^T) X in fp32,
+decayed in place), the dense fine-tuning step and the gated (GEGLU) FFN step.
 
 Multi-GPU: one process per GPU (torchrun), data-parallel replicas with their
 own token batch; masks are computed redundantly and bit-identically, so no
@@ -194,13 +197,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 
+def weight_sequence(wl: si.FFNWorkload, W1, W2):
+    """[[W1_0 .. W1_S], [W2_0 .. W2_S]] (host tensors) with W_(t+1) = round(W_t + N(0, 1e-4)),
+    the simulated training steps of the workload (S = max(1, wl.steps))."""
+    seq = [[W1], [W2]]
+    for t in range(max(1, wl.steps)):
+        for li in range(2):
+            seq[li].append(si.perturb(seq[li][-1], wl.perturb_seed(t, li)))
+    return seq
+
+
 class FFNStep:
     """Device buffers and the launch sequence of one step (kernel launches only)."""
 
-    KERNELS = ("mask_step", "gemm_fwd", "gemm_dgrad", "masked_decay")
-    WGRAD_KERNELS = ("mvue_dy", "mvue_dh", "gemm_wgrad")
+    GEMMS = ("gemm_fwd1_gelu", "gemm_fwd2", "gemm_dgrad2_dgelu", "gemm_dgrad1")
+    KERNELS = ("mask_step",) + GEMMS + ("masked_decay",)
+    WGRAD_KERNELS = ("mvue_dy", "mvue_dh", "gemm_wgrad2", "gemm_wgrad1")
 
-    def __init__(self, wl: si.FFNWorkload, rank: int):
+    def __init__(self, wl: si.FFNWorkload, rank: int, with_host=True):
         import torch
         import structured_sparse_transformer_b200 as sp
         self.sp, self.torch, self.wl = sp, torch, wl
@@ -211,16 +225,21 @@ class FFNStep:
         W1, W2 = wl_r.weights()
         X, dY = wl_r.activations()
         G1, G2 = wl_r.grads()
-        self.host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
         dev = "cuda"
-        self.W = [[W1.to(dev), si.perturb(W1, wl.perturb_seed(0, 0)).to(dev)],
-                  [W2.to(dev), si.perturb(W2, wl.perturb_seed(0, 1)).to(dev)]]
+        # The simulated training steps: W_(t+1) = round(W_t + N(0, 1e-4)), t = 0 .. S-1.
+        self.S = max(1, wl.steps)
+        hostW = weight_sequence(wl, W1, W2)
+        self.host = {"W": hostW, "X": X, "dY": dY, "G1": G1, "G2": G2} if with_host else None
+        self.W = [[w.to(dev) for w in hostW[li]] for li in range(2)]
         self.X, self.dY = X.to(dev), dY.to(dev)
         self.G = [G1.to(dev), G2.to(dev)]
-        self.idx = [[torch.zeros(ff // 4, d // 4, dtype=torch.uint8, device=dev) for _ in range(2)],
-                    [torch.zeros(d // 4, ff // 4, dtype=torch.uint8, device=dev) for _ in range(2)]]
-        self.flips = torch.zeros(2, dtype=torch.int64, device=dev)
+        shapes = ((ff // 4, d // 4), (d // 4, ff // 4))
+        self.idx = [[torch.zeros(*shapes[li], dtype=torch.uint8, device=dev) for _ in range(self.S + 1)]
+                    for li in range(2)]
+        self.flips = torch.zeros(self.S, 2, dtype=torch.int64, device=dev)
         self.c = [sp.alloc_compressed(ff, d, tdt), sp.alloc_compressed(d, ff, tdt)]
+        for li in range(2):   # the mask of W_0, against which step 0 counts its flips
+            sp.sp24_mask_search(self.W[li][0], self.idx[li][0])
         self.H = torch.empty(T, ff, dtype=tdt, device=dev)
         self.Hpre = torch.empty(T, ff, dtype=tdt, device=dev)
         self.dH = torch.empty(T, ff, dtype=tdt, device=dev)
@@ -242,7 +261,8 @@ class FFNStep:
         before they are decayed."""
         sp, torch, wl = self.sp, self.torch, self.wl
         d, ff = wl.d, wl.ff
-        cur, prev = self.step_no % 2, (self.step_no + 1) % 2
+        t = self.step_no % self.S
+        cur, prev = t + 1, t
         main = torch.cuda.current_stream()
         if not hasattr(self, "side"):
             self.side = torch.cuda.Stream()
@@ -275,26 +295,27 @@ class FFNStep:
         for li, stream in ((0, main), (1, side)):
             c = self.c[li]
             timed("mask_step", lambda li=li, c=c: sp.sp24_mask_step(
-                self.W[li][cur], self.idx[li][cur], self.idx[li][prev], self.flips[li:li + 1], *c), stream)
+                self.W[li][cur], self.idx[li][cur], self.idx[li][prev], self.flips[t, li:li + 1], *c), stream)
         c1, c2 = self.c
-        timed("gemm_fwd", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu", self.Hpre), main)
+        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu", self.Hpre), main)
         join()
-        timed("gemm_fwd", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y), main)
-        timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre), main)
+        timed("gemm_fwd2", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y), main)
+        timed("gemm_dgrad2_dgelu",
+              lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre), main)
         if wgrad:
             # Weight gradients into the gradient buffers: dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X;
             # fresh draws every step and layer (offset 2 * step + layer).
             seed = wl.seeds["mvue"]
             (y2v, y2m), (y1v, y1m) = self.yh
             timed("mvue_dy", lambda: sp.sp24_mvue_sparsify(self.dY, seed, 2 * self.step_no + 1, y2v, y2m), main)
-            timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.H, y2v, y2m, d, self.G[1]), main)
+            timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad(self.H, y2v, y2m, d, self.G[1]), main)
             timed("mvue_dh", lambda: sp.sp24_mvue_sparsify(self.dH, seed, 2 * self.step_no, y1v, y1m), main)
-            timed("gemm_wgrad", lambda: sp.sp24_gemm_wgrad(self.X, y1v, y1m, ff, self.G[0]), main)
-        timed("gemm_dgrad", lambda: sp.sp24_gemm_dgrad(self.dH, c1[2], c1[3], d, self.dX), main)
+            timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad(self.X, y1v, y1m, ff, self.G[0]), main)
+        timed("gemm_dgrad1", lambda: sp.sp24_gemm_dgrad(self.dH, c1[2], c1[3], d, self.dX), main)
         fork()
         for li, stream in ((0, main), (1, side)):
-            timed("masked_decay", lambda li=li: sp.sp24_masked_decay(self.G[li], self.W[li][cur], self.idx[li][cur],
-                                                                      wl.lam), stream)
+            timed("masked_decay", lambda li=li: sp.sp24_masked_decay(self.G[li], self.W[li][cur],
+                                                                      self.idx[li][cur], wl.lam), stream)
         join()
         self.step_no += 1
 
@@ -304,7 +325,7 @@ class FFNStep:
         the dense tensor-core path (the weight gradients take dY^T and dH^T from
         the transpose kernel); no mask, compression or decay."""
         sp, torch = self.sp, self.torch
-        cur = self.step_no % 2
+        cur = self.step_no % self.S + 1
         if not hasattr(self, "Wt"):
             self.Wt = [torch.empty(w[0].shape[1], w[0].shape[0], dtype=w[0].dtype, device="cuda") for w in self.W]
             self.dYt = torch.empty(self.dY.shape[1], self.dY.shape[0], dtype=self.dY.dtype, device="cuda")
@@ -323,34 +344,68 @@ class FFNStep:
         for li in range(2):
             timed("transpose", lambda li=li: sp.sp24_transpose(self.W[li][cur], self.Wt[li]))
         W1, W2 = self.W[0][cur], self.W[1][cur]
-        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu", self.Hpre))
-        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
-        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "dgelu", self.Hpre))
+        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu", self.Hpre))
+        timed("gemm_fwd2", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
+        timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "dgelu", self.Hpre))
         timed("transpose_act", lambda: sp.sp24_transpose(self.dY, self.dYt))
-        timed("gemm_dense_wgrad", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dYt, self.G[1]))
+        timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dYt, self.G[1]))
         timed("transpose_act", lambda: sp.sp24_transpose(self.dH, self.dHt))
-        timed("gemm_dense_wgrad", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dHt, self.G[0]))
-        timed("gemm_dense", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
+        timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dHt, self.G[0]))
+        timed("gemm_dgrad1", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
         self.step_no += 1
 
     # algorithmic bytes / flops per launch of each kernel
     def work(self):
         wl = self.wl
         n_el = wl.d * wl.ff
-        return {
+        gemm = ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff)
+        w = {
             # read W (2 B/el), idx_prev (1/16), write idx (1/16), values of both orientations (2 B/el),
             # metadata of both orientations (2 x 1/8 B/el)
             "mask_step": ("GB/s", n_el * (2 + 1 / 16 + 1 / 16 + 2 + 0.25)),
-            "gemm_fwd": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
-            "gemm_dgrad": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
-            # the training step with the weight gradients
-            "gemm_wgrad": ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff),
             # read dY (2 B/el), write the kept values (1 B/el) and their metadata (1/8 B/el)
             "mvue_dy": ("GB/s", wl.tokens * wl.d * (2 + 1 + 1 / 8)),
             "mvue_dh": ("GB/s", wl.tokens * wl.ff * (2 + 1 + 1 / 8)),
             # read g (4), W (2), idx (1/16), write g (4)
             "masked_decay": ("GB/s", n_el * (10 + 1 / 16)),
         }
+        for g in self.GEMMS + ("gemm_wgrad2", "gemm_wgrad1"):
+            w[g] = gemm
+        return w
+
+
+def kernel_table(events, work, peaks, names):
+    """Per-kernel launches, average duration and roofline fraction from the instrumented pass."""
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    out = {}
+    for name in names:
+        if name not in events:
+            continue
+        unit, amount = work[name]
+        times = [s.elapsed_time(e) * 1e-3 for s, e in events[name]]
+        avg = sum(times) / len(times)
+        achieved = amount / avg / (1e12 if unit == "TFLOP/s" else 1e9)
+        peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
+        out[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
+                     "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
+    return out
+
+
+def timed_steps(step_fn, steps, flush, barrier):
+    """Runs `steps` steps back to back, each bracketed by CUDA events after an L2 flush;
+    returns the summed step time in ms."""
+    import torch
+    ev = []
+    barrier()
+    for _ in range(steps):
+        flush.fill_(1.0)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        step_fn()
+        e.record()
+        ev.append((s, e))
+    barrier()
+    return sum(s.elapsed_time(e) for s, e in ev)
 
 
 def run_ours(args, wl, rank, world, local_rank):
@@ -367,99 +422,93 @@ def run_ours(args, wl, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
-    clk = ClockSampler(torch.cuda.current_device()).__enter__()
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    st = sp.sp24_device_status()
-    if st != 0:
-        clk.__exit__()
-        raise RuntimeError(f"device status after warm-up: {sp.sp24_status_string(st)}")
+    def status(where):
+        st = sp.sp24_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {where}: {sp.sp24_status_string(st)}")
 
-    # Timed region: the step's launches back to back (each kernel may start
-    # while its predecessor drains: programmatic dependent launch).
-    step_ev = []
-    barrier()
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        step.run()
-        e.record()
-        step_ev.append((s, e))
-    barrier()
-    st = sp.sp24_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {sp.sp24_status_string(st)}")
-    step_ms = sum(s.elapsed_time(e) for s, e in step_ev)
-    # Per-kernel durations: a second pass of the same steps with events around
-    # every launch (an event between two launches serialises them).
-    events = {}
-    barrier()
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        step.run(events)
-    barrier()
-    wgrad = run_wgrad_phase(args, step, wl, world, dev, flush, barrier)
-    dense = run_dense_phase(args, step, wl, world, dev, flush, barrier)
-    geglu = run_geglu_phase(args, step, wl, world, dev, flush, barrier)
+    clk = ClockSampler(torch.cuda.current_device()).__enter__()
+    try:
+        for _ in range(args.warmup):
+            step.run()
+        torch.cuda.synchronize()
+        status("after warm-up")
+        # Timed region: the step's launches back to back (each kernel may start
+        # while its predecessor drains: programmatic dependent launch).
+        step_ms = timed_steps(step.run, args.steps, flush, barrier)
+        status("after timing")
+        flips = step.flips.cpu().tolist()
+        # Per-kernel durations: a second pass of the same steps with events around
+        # every launch (an event between two launches serialises them).
+        events = {}
+        barrier()
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            step.run(events)
+        barrier()
+        peaks, peak_kind = load_peaks()
+        kernels = kernel_table(events, step.work(), peaks, FFNStep.KERNELS)
+        wgrad = run_wgrad_phase(args, step, wl, world, dev, flush, barrier, peaks)
+        dense = run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks)
+        geglu = run_geglu_phase(args, step, wl, world, dev, flush, barrier)
+        e2e = run_e2e(args, step, wl, world, dev, barrier)
+        del step
+        torch.cuda.empty_cache()
+        secondary = run_secondary(args, si.GPT2_355M, rank, world, dev, flush, barrier, peaks)
+        sweep = None if args.no_sweep else run_sweep(args, dev, flush, barrier, peaks)
+    finally:
+        clk.__exit__()
     total_ms = max_over_ranks(step_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    flops = wl.gemm_flops()
-    value = flops * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = wl.gemm_flops() * world * args.steps / (total_ms * 1e-3) / 1e12
 
-    peaks, peak_kind = load_peaks()
     sparse_peak = 2.0 * peaks["bf16_tflops"]
-    kernels = {}
-    for name, (unit, amount) in step.work().items():
-        times = [s.elapsed_time(e) * 1e-3 for s, e in events.get(name, [])]
-        if not times:
-            continue
-        avg = sum(times) / len(times)
-        achieved = amount / avg / (1e12 if unit == "TFLOP/s" else 1e9)
-        peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
-        kernels[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
-                         "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
-    g = {k: kernels[k] for k in ("gemm_fwd", "gemm_dgrad")}
-    g_time = sum(v["avg_us"] * v["launches"] for v in g.values())
-    g_launches = sum(v["launches"] for v in g.values())
-    g_avg = g_time / g_launches * 1e-6
+    g = [kernels[k] for k in FFNStep.GEMMS]
+    g_avg = sum(v["avg_us"] * v["launches"] for v in g) / sum(v["launches"] for v in g) * 1e-6
     g_ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
     roofline = {"bound": "tensor", "achieved": round(g_ach, 1), "peak": sparse_peak, "unit": "TFLOP/s",
                 "frac": round(g_ach / sparse_peak, 4),
                 "traffic": args.gemm_traffic or load_traffic("gemm", wl.name),
-                "kernel": "sp24_gemm_pair_kernel (fwd + dgrad launches)",
+                "kernel": "sp24_gemm_pair_kernel (the four forward and input-gradient launches)",
                 "peak_source": f"2 x {peak_kind} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s), "
                                "the nominal 2:4 sparse ratio"}
+    # 2:4 over dense, per product, from the two instrumented passes on the same workload
+    ratio = {k: round(dense["kernels"][k]["avg_us"] / kernels[k]["avg_us"], 3) for k in FFNStep.GEMMS}
+    for k in ("gemm_wgrad2", "gemm_wgrad1"):
+        ratio[k] = round(dense["kernels"][k]["avg_us"] / wgrad["kernels"][k]["avg_us"], 3)
     mask = kernels["mask_step"]
-
-    e2e = run_e2e(args, step, wl, world, dev, barrier)
-    clk.__exit__()
+    gate = sweep["16384x65536"]["normal"]["mask_step"] if sweep else None
     clocks = clk.summary()
-    flips = [int(x) for x in step.flips.cpu().tolist()]
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
         "config": {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff, "tokens_per_gpu": wl.tokens,
-                   "global_tokens": wl.tokens * world, "parallelism": f"dp{world} replicas, no collective",
+                   "global_tokens": wl.tokens * world, "simulated_steps": max(1, wl.steps),
+                   "perturbation": "W_(t+1) = round(W_t + N(0, 1e-4)) per weight; timed steps cycle t = 0..S-1",
+                   "parallelism": f"dp{world} replicas, no collective",
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)",
                    "kernel_times": "second pass of the same steps with events around each launch, all on "
                                    "one stream (the timed steps run the second layer's mask step and "
                                    "decay concurrently on a side stream)"},
         "roofline": roofline,
-        "mask_search_roofline": {"bound": "hbm", "achieved": mask["achieved"], "peak": peaks["hbm_gbs"],
-                                 "unit": "GB/s", "frac": mask["frac"],
-                                 "traffic": args.mask_traffic or load_traffic("mask_step", wl.name),
-                                 "kernel": "mask_tile_kernel (search + flip + compress, both weights)"},
+        "mask_search_roofline": (
+            {"bound": "hbm", "achieved": gate["achieved"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": gate["frac"], "traffic": args.mask_traffic or load_traffic("mask_step", "sweep-16384x65536"),
+             "kernel": "mask_tile_kernel (search + flip + both compressions), fp16 16384 x 65536 N(0, 0.02) "
+                       "(2 GiB of weights, beyond L2)"} if gate else None),
         "kernels": kernels,
+        "sparse_over_dense": ratio,
+        "flip_counts_per_step": flips,
+        "flip_rate_per_step": [[round(c / (wl.d * wl.ff), 6) for c in row] for row in flips],
+        "mask_search_sweep": sweep,
         "ffn_step_with_weight_gradients": wgrad,
         "dense_finetune_step": dense,
         "geglu_ffn_step": geglu,
+        "gpt2_355m": secondary,
         "e2e": e2e,
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": 8 * args.steps,
         "clocks": clocks,
-        "last_flip_counts": flips,
         "peaks": peak_kind,
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -467,25 +516,100 @@ def run_ours(args, wl, rank, world, local_rank):
     return line
 
 
-def run_wgrad_phase(args, step, wl, world, dev, flush, barrier):
+def run_secondary(args, wl, rank, world, dev, flush, barrier, peaks):
+    """The headline step on a second workload (timed the same way), with its kernels."""
+    import torch
+    import structured_sparse_transformer_b200 as sp
+    step = FFNStep(wl, rank, with_host=False)
+    for _ in range(args.warmup):
+        step.run()
+    ms = max_over_ranks(timed_steps(step.run, args.steps, flush, barrier), world, dev) / args.steps
+    events = {}
+    for _ in range(args.steps):
+        flush.fill_(1.0)
+        step.run(events)
+    barrier()
+    st = sp.sp24_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the {wl.name} step: {sp.sp24_status_string(st)}")
+    kernels = kernel_table(events, step.work(), peaks, FFNStep.KERNELS)
+    del step
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff, "tokens_per_gpu": wl.tokens,
+            "ms_per_step": round(ms, 4), "value": round(wl.gemm_flops() * world / (ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "kernels": kernels}
+
+
+def run_sweep(args, dev, flush, barrier, peaks):
+    """Mask-search bandwidth sweep at the sizes beyond L2: the fused mask step (search + flip
+    count against the mask before an N(0, 1e-4) update + both compressions) and the search
+    alone, on fp16 Gaussian N(0, 0.02) and 8-level tie-heavy weights.  Inputs are drawn on
+    the device from seeded generators; each launch follows an L2 flush and is timed alone."""
+    import torch
+    import structured_sparse_transformer_b200 as sp
+    out = {}
+    per_el = {"mask_step": 2 + 1 / 16 + 1 / 16 + 2 + 0.25, "search": 2 + 1 / 16}
+    for R, C in args.sweep_shapes:
+        key = f"{R}x{C}"
+        out[key] = {}
+        idx = torch.empty(R // 4, C // 4, dtype=torch.uint8, device=dev)
+        prev = torch.empty_like(idx)
+        count = torch.zeros(1, dtype=torch.int64, device=dev)
+        bufs = sp.alloc_compressed(R, C, torch.float16, device=dev)
+        for dist_name in ("normal", "tie"):
+            g = torch.Generator(device=dev)
+            g.manual_seed(400 + (dist_name == "tie"))
+            w = torch.empty(R, C, dtype=torch.float16, device=dev)
+            for r0 in range(0, R, 1024):   # fp32 draws in row slabs (bounded temporaries)
+                x = torch.randn(min(1024, R - r0), C, device=dev, generator=g) * 0.02
+                if dist_name == "tie":
+                    x = torch.clamp(torch.round(x / 2.0**-6), -4, 3) * 2.0**-6
+                w[r0:r0 + x.shape[0]] = x.to(torch.float16)
+            sp.sp24_mask_search(w, prev)
+            for r0 in range(0, R, 1024):   # one simulated update, so that the flip count is live
+                sl = w[r0:r0 + 1024]
+                sl.copy_((sl.float() + torch.randn(sl.shape, device=dev, generator=g) * 1e-4).to(torch.float16))
+            fns = {"mask_step": lambda: sp.sp24_mask_step(w, idx, prev, count, *bufs),
+                   "search": lambda: sp.sp24_mask_search(w, idx)}
+            res = {}
+            for name, fn in fns.items():
+                for _ in range(2):
+                    fn()
+                barrier()
+                ev = []
+                for _ in range(args.sweep_iters):
+                    flush.fill_(1.0)
+                    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    s.record()
+                    fn()
+                    e.record()
+                    ev.append((s, e))
+                barrier()
+                avg = sum(s.elapsed_time(e) for s, e in ev) / len(ev) * 1e-3
+                gbs = R * C * per_el[name] / avg / 1e9
+                res[name] = {"avg_us": round(avg * 1e6, 2), "achieved": round(gbs, 1), "unit": "GB/s",
+                             "peak": peaks["hbm_gbs"], "frac": round(gbs / peaks["hbm_gbs"], 4),
+                             "bytes_per_element": round(per_el[name], 4)}
+            res["flips"] = int(count.item())
+            st = sp.sp24_device_status()
+            if st != 0:
+                raise RuntimeError(f"device status after the sweep at {key}: {sp.sp24_status_string(st)}")
+            out[key][dist_name] = res
+            del w
+        del idx, prev, bufs
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_wgrad_phase(args, step, wl, world, dev, flush, barrier, peaks):
     """The 2:4 training step with both weight gradients (MVUE + weight-gradient GEMM, then the
     decay of the computed gradients), timed like the headline step, and its MVUE and
     weight-gradient kernels from an instrumented pass."""
-    import torch
     import structured_sparse_transformer_b200 as sp
     for _ in range(args.warmup):
         step.run(wgrad=True)
-    step_ev = []
-    barrier()
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        step.run(wgrad=True)
-        e.record()
-        step_ev.append((s, e))
-    barrier()
-    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), world, dev) / args.steps
+    ms = max_over_ranks(timed_steps(lambda: step.run(wgrad=True), args.steps, flush, barrier), world, dev)
+    ms /= args.steps
     events = {}
     for _ in range(args.steps):
         flush.fill_(1.0)
@@ -494,18 +618,7 @@ def run_wgrad_phase(args, step, wl, world, dev, flush, barrier):
     st = sp.sp24_device_status()
     if st != 0:
         raise RuntimeError(f"device status after the weight-gradient step: {sp.sp24_status_string(st)}")
-    peaks, _ = load_peaks()
-    sparse_peak = 2.0 * peaks["bf16_tflops"]
-    work = step.work()
-    kernels = {}
-    for name in FFNStep.WGRAD_KERNELS:
-        unit, amount = work[name]
-        times = [s.elapsed_time(e) * 1e-3 for s, e in events[name]]
-        avg = sum(times) / len(times)
-        achieved = amount / avg / (1e12 if unit == "TFLOP/s" else 1e9)
-        peak = sparse_peak if unit == "TFLOP/s" else peaks["hbm_gbs"]
-        kernels[name] = {"launches": len(times), "avg_us": round(avg * 1e6, 2), "achieved": round(achieved, 1),
-                         "unit": unit, "peak": peak, "frac": round(achieved / peak, 4)}
+    kernels = kernel_table(events, step.work(), peaks, FFNStep.WGRAD_KERNELS)
     flops = 6 * 2.0 * wl.tokens * wl.d * wl.ff
     return {"ms_per_step": round(ms, 4), "value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "launches_per_step": 12, "kernels": kernels,
@@ -514,24 +627,13 @@ def run_wgrad_phase(args, step, wl, world, dev, flush, barrier):
                     "cores in fp32, then the masked decay of those gradients; FLOPs 6 x 2 T d ff"}
 
 
-def run_dense_phase(args, step, wl, world, dev, flush, barrier):
+def run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks):
     """The dense fine-tuning step, timed like the 2:4 step (back to back, L2
-    flushed outside the step events), and its GEMMs from an instrumented pass."""
-    import torch
+    flushed outside the step events), and its kernels from an instrumented pass."""
     import structured_sparse_transformer_b200 as sp
     for _ in range(args.warmup):
         step.run_dense()
-    step_ev = []
-    barrier()
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s.record()
-        step.run_dense()
-        e.record()
-        step_ev.append((s, e))
-    barrier()
-    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in step_ev), world, dev) / args.steps
+    ms = max_over_ranks(timed_steps(step.run_dense, args.steps, flush, barrier), world, dev) / args.steps
     events = {}
     for _ in range(args.steps):
         flush.fill_(1.0)
@@ -540,28 +642,19 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier):
     st = sp.sp24_device_status()
     if st != 0:
         raise RuntimeError(f"device status after the dense phase: {sp.sp24_status_string(st)}")
-    peaks, _ = load_peaks()
-    g = [s.elapsed_time(e) * 1e-3 for s, e in events["gemm_dense"] + events["gemm_dense_wgrad"]]
-    t = [s.elapsed_time(e) * 1e-3 for s, e in events["transpose"]]
-    ta = [s.elapsed_time(e) * 1e-3 for s, e in events["transpose_act"]]
-    g_avg = sum(g) / len(g)
-    ach = 2.0 * wl.tokens * wl.d * wl.ff / g_avg / 1e12
     n_el = wl.d * wl.ff
-    t_avg = sum(t) / len(t)
+    work = {k: ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff) for k in FFNStep.GEMMS + ("gemm_wgrad2", "gemm_wgrad1")}
+    work["transpose"] = ("GB/s", 4 * n_el)
+    work["transpose_act"] = ("GB/s", 4 * wl.tokens * (wl.d + wl.ff) / 2)
+    dense_peaks = dict(peaks)
+    dense_peaks["bf16_tflops"] = peaks["bf16_tflops"] / 2.0   # kernel_table doubles it for the 2:4 peak
+    kernels = kernel_table(events, work, dense_peaks, list(work))
     return {"ms_per_step": round(ms, 4),
             "value": round(6 * 2.0 * wl.tokens * wl.d * wl.ff * world / (ms * 1e-3) / 1e12, 2),
-            "unit": "TFLOP/s",
-            "gemm": {"launches": len(g), "avg_us": round(g_avg * 1e6, 2), "achieved": round(ach, 1),
-                     "peak": peaks["bf16_tflops"], "frac": round(ach / peaks["bf16_tflops"], 4)},
-            "transpose": {"launches": len(t), "avg_us": round(t_avg * 1e6, 2),
-                          "achieved": round(4 * n_el / t_avg / 1e9, 1), "unit": "GB/s",
-                          "peak": peaks["hbm_gbs"], "frac": round(4 * n_el / t_avg / 1e9 / peaks["hbm_gbs"], 4)},
-            "transpose_act": {"launches": len(ta), "avg_us": round(sum(ta) / len(ta) * 1e6, 2),
-                              "achieved": round(4 * wl.tokens * (wl.d + wl.ff) / 2 / (sum(ta) / len(ta)) / 1e9, 1),
-                              "unit": "GB/s"},
+            "unit": "TFLOP/s", "kernels": kernels,
             "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights, dY^T and dH^T, and "
                     "the six FFN products (forward, input gradient, weight gradient) on the dense tcgen05 "
-                    "path, same workload; FLOPs 6 x 2 T d ff"}
+                    "path, same workload; FLOPs 6 x 2 T d ff; GEMM peak = the dense bf16 burst"}
 
 
 class GegluStep:
@@ -654,14 +747,14 @@ def run_e2e(args, step, wl, world, dev, barrier):
     and overlap the neighbouring steps' kernels: step k's inputs land in slot k % 2 while
     step k-1 computes, and its results leave while step k+1 computes."""
     import torch
-    h = {k: v.pin_memory() for k, v in step.host.items()}
-    # The weights a host would send change every step: alternate the seeded
-    # weights with their perturbed copies, so the masks flip as in training.
-    hw = [[h["W1"], step.W[0][1].cpu().pin_memory()], [h["W2"], step.W[1][1].cpu().pin_memory()]]
+    h = {k: step.host[k].pin_memory() for k in ("X", "dY", "G1", "G2")}
+    # The weights a host sends change every step: step t sends W_(t+1) of both layers
+    # (the simulated updates), so the masks flip as in training.
+    hw = [[w.pin_memory() for w in step.host["W"][li]] for li in range(2)]
     out_y = torch.empty(step.Y.shape, dtype=step.Y.dtype).pin_memory()
     out_dx = torch.empty(step.dX.shape, dtype=step.dX.dtype).pin_memory()
     out_g = [torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in step.G]
-    out_f = torch.empty(2, dtype=torch.int64).pin_memory()
+    out_f = torch.empty(step.flips.shape, dtype=torch.int64).pin_memory()
     slots = [{"X": step.X, "dY": step.dY, "G": step.G, "Y": step.Y, "dX": step.dX, "flips": step.flips}]
     slots.append({k: ([t.clone() for t in v] if isinstance(v, list) else v.clone()) for k, v in slots[0].items()})
     cs = torch.cuda.current_stream()
@@ -675,8 +768,9 @@ def run_e2e(args, step, wl, world, dev, barrier):
         with torch.cuda.stream(hs):
             if d2h_done[b] is not None:
                 hs.wait_event(d2h_done[b])     # slot b's previous results have left
-            step.W[0][b].copy_(hw[0][b], non_blocking=True)
-            step.W[1][b].copy_(hw[1][b], non_blocking=True)
+            cur = k % step.S + 1
+            step.W[0][cur].copy_(hw[0][cur], non_blocking=True)
+            step.W[1][cur].copy_(hw[1][cur], non_blocking=True)
             sl["X"].copy_(h["X"], non_blocking=True)
             sl["dY"].copy_(h["dY"], non_blocking=True)
             sl["G"][0].copy_(h["G1"], non_blocking=True)
@@ -714,7 +808,7 @@ def run_e2e(args, step, wl, world, dev, barrier):
     e.record(cs)
     barrier()
     ms = max_over_ranks(s.elapsed_time(e), world, dev)
-    h2d = sum(v.numel() * v.element_size() for v in (hw[0][0], hw[1][0], h["X"], h["dY"], h["G1"], h["G2"]))
+    h2d = sum(v.numel() * v.element_size() for v in (hw[0][1], hw[1][1], h["X"], h["dY"], h["G1"], h["G2"]))
     d2h = sum(t.numel() * t.element_size() for t in (out_y, out_dx, *out_g, out_f))
     return {"value": round(wl.gemm_flops() * world * args.steps / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / args.steps, 4),
@@ -724,18 +818,37 @@ def run_e2e(args, step, wl, world, dev, barrier):
 
 # ---------------------------------------------------------- oracle (CPU) arm
 
-def oracle_step(wl, host, rows):
-    """One step of the CPU oracle on a token sample: both mask searches, both compressions,
-    the four GEMMs on `rows` token rows, GELU, masked decay on both gradients, flip counts.
-    Returns the GEMM FLOPs it processed."""
+def oracle_host(wl):
+    """Host inputs of the oracle arm: the weight sequence, activations, gradients, and the
+    masks of W_0 (step 0 counts its flips against them)."""
+    import oracle
+    W1, W2 = wl.weights()
+    X, dY = wl.activations()
+    G1, G2 = wl.grads()
+    seq = weight_sequence(wl, W1, W2)
+    masks = [[oracle.mask_search(si.bits16(seq[li][0]), wl.dtype)] + [None] * max(1, wl.steps) for li in range(2)]
+    return {"W": seq, "X": X, "dY": dY, "G1": G1, "G2": G2, "masks": masks}
+
+
+def oracle_step(wl, host, rows, t):
+    """Simulated step t of the CPU oracle on a token sample: both mask searches on W_(t+1),
+    both compressions, the flip counts against the masks of W_t, the four GEMMs on `rows`
+    token rows with GELU between, masked decay on both gradients.  Returns the GEMM FLOPs
+    it processed."""
     import oracle
     dt = wl.dtype
-    b1, b2 = si.bits16(host["W1"]), si.bits16(host["W2"])
-    i1, i2 = oracle.mask_search(b1, dt), oracle.mask_search(b2, dt)
-    oracle.compress_both(b1, i1)
-    oracle.compress_both(b2, i2)
-    k1, k2 = oracle.dense_mask(i1), oracle.dense_mask(i2)
-    w1, w2 = oracle.to_f64(b1, dt), oracle.to_f64(b2, dt)
+    cur = t % max(1, wl.steps) + 1
+    b = [si.bits16(host["W"][li][cur]) for li in range(2)]
+    idx = [oracle.mask_search(b[li], dt) for li in range(2)]
+    for li in range(2):
+        oracle.compress_both(b[li], idx[li])
+        prev = host["masks"][li][cur - 1]
+        if prev is None:   # an earlier step's mask the sample has not computed yet
+            prev = host["masks"][li][cur - 1] = oracle.mask_search(si.bits16(host["W"][li][cur - 1]), dt)
+        oracle.flip_count(prev, idx[li])
+        host["masks"][li][cur] = idx[li]
+    k1, k2 = oracle.dense_mask(idx[0]), oracle.dense_mask(idx[1])
+    w1, w2 = oracle.to_f64(b[0], dt), oracle.to_f64(b[1], dt)
     x = oracle.to_f64(si.bits16(host["X"])[:rows], dt)
     dy = oracle.to_f64(si.bits16(host["dY"])[:rows], dt)
     pre = oracle.sparse_fwd(x, w1, k1)
@@ -743,47 +856,40 @@ def oracle_step(wl, host, rows):
     oracle.sparse_fwd(h, w2, k2)
     dh = oracle.sparse_dgrad(dy, w2, k2) * oracle.gelu_grad(pre)
     oracle.sparse_dgrad(dh, w1, k1)
-    oracle.masked_decay(host["G1"].numpy(), b1, dt, i1, wl.lam)
-    oracle.masked_decay(host["G2"].numpy(), b2, dt, i2, wl.lam)
-    oracle.flip_count(i1, i1)
-    oracle.flip_count(i2, i2)
+    oracle.masked_decay(host["G1"].numpy(), b[0], dt, idx[0], wl.lam)
+    oracle.masked_decay(host["G2"].numpy(), b[1], dt, idx[1], wl.lam)
     return 4 * 2.0 * rows * wl.d * wl.ff
 
 
 def cpu_baseline(wl, rows):
     import oracle
     oracle.build()
-    W1, W2 = wl.weights()
-    X, dY = wl.activations()
-    G1, G2 = wl.grads()
-    host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
+    host = oracle_host(wl)
     t0 = time.perf_counter()
-    flops = oracle_step(wl, host, rows)
+    flops = oracle_step(wl, host, rows, 0)
     dt = time.perf_counter() - t0
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"one full oracle step of {wl.name} with the four GEMMs on the first {rows} of "
-                      f"{wl.tokens} token rows (mask search, compression, decay and flips in full)"}
+            "sample": f"one simulated step of {wl.name} on the oracle with the four GEMMs on the first {rows} "
+                      f"of {wl.tokens} token rows (both mask searches, compressions, flip counts and decays "
+                      f"in full)"}
 
 
 def run_reference(args, wl):
     import oracle
     oracle.build()
-    W1, W2 = wl.weights()
-    X, dY = wl.activations()
-    G1, G2 = wl.grads()
-    host = {"W1": W1, "W2": W2, "X": X, "dY": dY, "G1": G1, "G2": G2}
+    host = oracle_host(wl)
     rows = args.cpu_tokens
-    for _ in range(args.warmup):
-        oracle_step(wl, host, rows)
+    for k in range(args.warmup):
+        oracle_step(wl, host, rows, k)
     t0 = time.perf_counter()
     flops = 0.0
-    for _ in range(args.steps):
-        flops += oracle_step(wl, host, rows)
+    for k in range(args.steps):
+        flops += oracle_step(wl, host, rows, args.warmup + k)
     sec = time.perf_counter() - t0
     value = flops / sec / 1e12
-    sample = (f"each step: the oracle's full {wl.name} step with the four GEMMs on the first {rows} of "
-              f"{wl.tokens} token rows")
+    sample = (f"each step: one simulated step of {wl.name} on the oracle with the four GEMMs on the first "
+              f"{rows} of {wl.tokens} token rows (mask searches, compressions, flips, decays in full)")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -800,12 +906,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=si.GPT2_355M.name, choices=sorted(si.FFN_WORKLOADS))
+    ap.add_argument("--workload", default=si.GPT2_1P5B.name, choices=sorted(si.FFN_WORKLOADS))
+    ap.add_argument("--no-sweep", action="store_true", help="skip the mask-search bandwidth sweep")
+    ap.add_argument("--sweep-iters", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=256, help="token rows of the oracle's GEMM sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-traffic", type=float, default=None, help="ncu DRAM bytes per GEMM launch")
     ap.add_argument("--mask-traffic", type=float, default=None, help="ncu DRAM bytes per mask-step launch")
     args = ap.parse_args(argv)
+    args.sweep_shapes = [(16384, 16384), (16384, 65536)]
     wl = si.FFN_WORKLOADS[args.workload]
     rank, world, local_rank = dist_env()
 

@@ -102,19 +102,49 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need_cuda(*ts, pitched=()):
+def _need_rowmajor(*ts, pitched=()):
     """The library reads every buffer as row-major: contiguous tensors, except those in
-    `pitched` (2-D, unit stride along rows, the row pitch passed as a leading dimension).
-    Layout is checked first, then that every tensor lives on a CUDA device."""
+    `pitched` (2-D, unit stride along rows, the row pitch passed as a leading dimension)."""
     for t in ts:
         if t is not None and not t.is_contiguous():
             raise ValueError("sp24 takes contiguous (row-major) tensors")
     for t in pitched:
         if t is not None and (t.dim() != 2 or t.stride(1) != 1):
             raise ValueError("sp24 takes 2-D row-major tensors with unit stride along rows")
-    for t in (*ts, *pitched):
+
+
+def _need_device(*ts):
+    """Every tensor passed to a kernel lives on a CUDA device (checked after layout, dtype and
+    size, so those checks also run on CPU tensors)."""
+    for t in ts:
         if t is not None and not t.is_cuda:
             raise ValueError("sp24 kernels take CUDA tensors only")
+
+
+def _expect(t, name: str, dtype, numel: int, exact: bool = True):
+    """Raises ValueError unless tensor `t` has `dtype` and holds `numel` elements (at least
+    `numel` when not `exact`): the kernels read and write exactly the sizes passed to the C
+    call, so a short or mistyped buffer would be accessed out of bounds."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    n = t.numel()
+    if (n != numel) if exact else (n < numel):
+        raise ValueError(f"{name}: expected {'' if exact else 'at least '}{numel} elements, got {n}")
+
+
+def _expect_compressed(vals, meta, rows: int, cols: int, dtype, what: str):
+    """vals [rows x cols/2] of `dtype` and the metadata bytes of an [rows x cols] operand."""
+    import torch
+    _expect(vals, f"{what} values", dtype, rows * (cols // 2))
+    _expect(meta, f"{what} metadata", torch.uint8, sp24_compressed_size(rows, cols)[1], exact=False)
+
+
+def _shape2(t, name: str):
+    if t.dim() != 2:
+        raise ValueError(f"{name}: expected a 2-D tensor, got {t.dim()}-D")
+    return t.shape
 
 
 # ------------------------------------------------------------ host helpers
@@ -156,15 +186,25 @@ def sp24_meta_from_canonical(canon, rows: int, cols: int):
 
 def sp24_mask_search(W, idx, stream=None):
     """idx[R/4, C/4] (uint8, CUDA) <- Algorithm 1 on W [R, C] (fp16/bf16, CUDA, row-major)."""
-    _need_cuda(idx, pitched=(W,))
-    R, C = W.shape
+    import torch
+    _need_rowmajor(idx, pitched=(W,))
+    R, C = _shape2(W, "W")
+    _dtype_code(W)
+    _expect(idx, "idx", torch.uint8, (R // 4) * (C // 4))
+    _need_device(idx, W)
     _check("sp24_mask_search", _lib.sp24_mask_search(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx),
                                                      _stream(stream)))
 
 
 def sp24_prune_compress(W, idx, vals_row, meta_row, vals_col, meta_col, stream=None):
-    _need_cuda(idx, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
-    R, C = W.shape
+    import torch
+    _need_rowmajor(idx, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
+    R, C = _shape2(W, "W")
+    _dtype_code(W)
+    _expect(idx, "idx", torch.uint8, (R // 4) * (C // 4))
+    _expect_compressed(vals_row, meta_row, R, C, W.dtype, "row-compressed")
+    _expect_compressed(vals_col, meta_col, C, R, W.dtype, "column-compressed")
+    _need_device(idx, vals_row, meta_row, vals_col, meta_col, W)
     _check("sp24_prune_compress",
            _lib.sp24_prune_compress(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(vals_row),
                                     _ptr(meta_row), _ptr(vals_col), _ptr(meta_col), _stream(stream)))
@@ -172,8 +212,16 @@ def sp24_prune_compress(W, idx, vals_row, meta_row, vals_col, meta_col, stream=N
 
 def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_row=None, vals_col=None,
                    meta_col=None, stream=None):
-    _need_cuda(idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
-    R, C = W.shape
+    import torch
+    _need_rowmajor(idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col, pitched=(W,))
+    R, C = _shape2(W, "W")
+    _dtype_code(W)
+    _expect(idx, "idx", torch.uint8, (R // 4) * (C // 4))
+    _expect(idx_prev, "idx_prev", torch.uint8, (R // 4) * (C // 4))
+    _expect(flip_count, "flip_count", torch.int64, 1, exact=False)
+    _expect_compressed(vals_row, meta_row, R, C, W.dtype, "row-compressed")
+    _expect_compressed(vals_col, meta_col, C, R, W.dtype, "column-compressed")
+    _need_device(idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col, W)
     _check("sp24_mask_step",
            _lib.sp24_mask_step(_ptr(W), _dtype_code(W), R, C, W.stride(0), _ptr(idx), _ptr(idx_prev),
                                _ptr(flip_count), _ptr(vals_row), _ptr(meta_row), _ptr(vals_col),
@@ -183,8 +231,13 @@ def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_r
 def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=None):
     """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None, 'gelu' (aux <- pre-activation) or
     'geglu' (W the stacked gate/up weight: Y[T, N/2] <- gelu(gate) * up, aux[T, N] <- pre-activations)."""
-    _need_cuda(X, vals_row, meta_row, Y, aux)
-    T, K = X.shape
+    _need_rowmajor(X, vals_row, meta_row, Y, aux)
+    T, K = _shape2(X, "X")
+    _dtype_code(X)
+    _expect_compressed(vals_row, meta_row, N, K, X.dtype, "W")
+    _expect(Y, "Y", X.dtype, T * (N // 2 if epi == "geglu" else N))
+    _expect(aux, "aux", X.dtype, T * N)
+    _need_device(X, vals_row, meta_row, Y, aux)
     _check("sp24_gemm_fwd",
            _lib.sp24_gemm_fwd(_ptr(X), T, K, _ptr(vals_row), _ptr(meta_row), N, _dtype_code(X), _ptr(Y),
                               EPILOGUES[epi], _ptr(aux), _stream(stream)))
@@ -193,8 +246,14 @@ def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=N
 def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stream=None):
     """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None, 'dgelu' (uses aux [T, K]) or
     'dgeglu' (dX[T, 2K] <- gradients of the gated pre-activations in aux [T, 2K])."""
-    _need_cuda(dY, vals_col, meta_col, dX, aux)
-    T, N = dY.shape
+    _need_rowmajor(dY, vals_col, meta_col, dX, aux)
+    T, N = _shape2(dY, "dY")
+    _dtype_code(dY)
+    _expect_compressed(vals_col, meta_col, K, N, dY.dtype, "W^T")
+    width = 2 * K if epi == "dgeglu" else K
+    _expect(dX, "dX", dY.dtype, T * width)
+    _expect(aux, "aux", dY.dtype, T * width)
+    _need_device(dY, vals_col, meta_col, dX, aux)
     _check("sp24_gemm_dgrad",
            _lib.sp24_gemm_dgrad(_ptr(dY), T, N, _ptr(vals_col), _ptr(meta_col), K, _dtype_code(dY), _ptr(dX),
                                 EPILOGUES[epi], _ptr(aux), _stream(stream)))
@@ -202,9 +261,14 @@ def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stre
 
 def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
     """out[T, M] <- B[T, Kd] A[M, Kd]^T on the dense tensor-core path; epi None, 'gelu' or 'dgelu'."""
-    _need_cuda(B, A, out, aux)
-    T, Kd = B.shape
-    M = A.shape[0]
+    _need_rowmajor(B, A, out, aux)
+    T, Kd = _shape2(B, "B")
+    M = _shape2(A, "A")[0]
+    _dtype_code(B)
+    _expect(A, "A", B.dtype, M * Kd)
+    _expect(out, "out", B.dtype, T * M)
+    _expect(aux, "aux", B.dtype, T * M)
+    _need_device(B, A, out, aux)
     _check("sp24_gemm_dense",
            _lib.sp24_gemm_dense(_ptr(B), T, Kd, _ptr(A), M, _dtype_code(B), _ptr(out), EPILOGUES[epi], _ptr(aux),
                                 _stream(stream)))
@@ -212,15 +276,21 @@ def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
 
 def sp24_transpose(x, out, stream=None):
     """out[C, R] <- x[R, C]^T (16-bit elements, bit copy)."""
-    _need_cuda(x, out)
-    R, C = x.shape
+    _need_rowmajor(x, out)
+    R, C = _shape2(x, "x")
+    _dtype_code(x)
+    _expect(out, "out", x.dtype, R * C)
+    _need_device(x, out)
     _check("sp24_transpose", _lib.sp24_transpose(_ptr(x), R, C, _dtype_code(x), _ptr(out), _stream(stream)))
 
 
 def sp24_mvue_sparsify(dY, seed: int, offset: int, vals, meta, stream=None):
     """vals/meta <- dY[T, N]^T compressed 2:4 along T with the MVUE draws of (seed, offset)."""
-    _need_cuda(vals, meta, pitched=(dY,))
-    T, N = dY.shape
+    _need_rowmajor(vals, meta, pitched=(dY,))
+    T, N = _shape2(dY, "dY")
+    _dtype_code(dY)
+    _expect_compressed(vals, meta, N, T, dY.dtype, "MVUE(dY^T)")
+    _need_device(vals, meta, dY)
     _check("sp24_mvue_sparsify",
            _lib.sp24_mvue_sparsify(_ptr(dY), T, N, dY.stride(0), _dtype_code(dY), int(seed) & (2**64 - 1),
                                    int(offset) & (2**64 - 1), _ptr(vals), _ptr(meta), _stream(stream)))
@@ -228,8 +298,13 @@ def sp24_mvue_sparsify(dY, seed: int, offset: int, vals, meta, stream=None):
 
 def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
     """dW[N, K] (fp32) <- Yhat[N, T] X[T, K] with Yhat from sp24_mvue_sparsify."""
-    _need_cuda(X, vals, meta, dW)
-    T, K = X.shape
+    import torch
+    _need_rowmajor(X, vals, meta, dW)
+    T, K = _shape2(X, "X")
+    _dtype_code(X)
+    _expect_compressed(vals, meta, N, T, X.dtype, "MVUE(dY^T)")
+    _expect(dW, "dW", torch.float32, N * K)
+    _need_device(X, vals, meta, dW)
     _check("sp24_gemm_wgrad",
            _lib.sp24_gemm_wgrad(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(dW),
                                 _stream(stream)))
@@ -237,17 +312,27 @@ def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
 
 def sp24_gemm_wgrad_dense(X, dYt, dW, stream=None):
     """dW[N, K] (fp32) <- dYt[N, T] X[T, K] on the dense tensor-core path (dYt = dY transposed)."""
-    _need_cuda(X, dYt, dW)
-    T, K = X.shape
-    N = dYt.shape[0]
+    import torch
+    _need_rowmajor(X, dYt, dW)
+    T, K = _shape2(X, "X")
+    N = _shape2(dYt, "dYt")[0]
+    _dtype_code(X)
+    _expect(dYt, "dYt", X.dtype, N * T)
+    _expect(dW, "dW", torch.float32, N * K)
+    _need_device(X, dYt, dW)
     _check("sp24_gemm_wgrad_dense",
            _lib.sp24_gemm_wgrad_dense(_ptr(X), T, K, _ptr(dYt), N, _dtype_code(X), _ptr(dW), _stream(stream)))
 
 
 def sp24_masked_decay(grad, W, idx, lam: float, stream=None):
     """grad[R, C] (fp32, in place) <- grad + lam * W on pruned entries."""
-    _need_cuda(grad, W, idx)
-    R, C = W.shape
+    import torch
+    _need_rowmajor(grad, W, idx)
+    R, C = _shape2(W, "W")
+    _dtype_code(W)
+    _expect(grad, "grad", torch.float32, R * C)
+    _expect(idx, "idx", torch.uint8, (R // 4) * (C // 4))
+    _need_device(grad, W, idx)
     _check("sp24_masked_decay",
            _lib.sp24_masked_decay(_ptr(grad), _ptr(W), _dtype_code(W), R, C, _ptr(idx), float(lam),
                                   _stream(stream)))
@@ -255,7 +340,12 @@ def sp24_masked_decay(grad, W, idx, lam: float, stream=None):
 
 def sp24_flip_rate(idx_prev, idx_cur, count, stream=None):
     """count[0] (int64 CUDA tensor, read as uint64) <- number of mask entries that differ."""
-    _need_cuda(idx_prev, idx_cur, count)
+    import torch
+    _need_rowmajor(idx_prev, idx_cur, count)
+    _expect(idx_cur, "idx_cur", torch.uint8, idx_cur.numel())
+    _expect(idx_prev, "idx_prev", torch.uint8, idx_cur.numel())
+    _expect(count, "count", torch.int64, 1, exact=False)
+    _need_device(idx_prev, idx_cur, count)
     _check("sp24_flip_rate",
            _lib.sp24_flip_rate(_ptr(idx_prev), _ptr(idx_cur), idx_cur.numel(), _ptr(count), _stream(stream)))
 

@@ -60,15 +60,37 @@ sp24_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return SP24_OK;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+constexpr int kMaxDevices = 64;
+
+// A value computed once per device (under std::call_once, so concurrent host
+// threads and several devices in one process each see their own).
+struct PerDevice {
+  std::once_flag once[kMaxDevices];
+  int value[kMaxDevices] = {};
+};
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return -1;
   }
-  return n;
+  return dev;
+}
+
+int sm_count() {
+  static PerDevice cache;
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  std::call_once(cache.once[dev], [dev] {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    cache.value[dev] = n;
+  });
+  return cache.value[dev];
 }
 
 // --------------------------------------------------------- tensor maps (TMA)
@@ -157,10 +179,17 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   if (!maps_ok) return SP24_ERR_CUDA;
   constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
   auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
-  static int max_pairs = 0;
-  if (max_pairs == 0) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
-      return SP24_ERR_CUDA;
+  // Per device, once: the shared-memory opt-in of this instantiation and the number
+  // of CTA pairs that fit at once (0 marks a failed set-up).
+  static PerDevice pairs_cache;
+  const int dev = current_device();
+  if (dev < 0) return SP24_ERR_NO_DEVICE;
+  std::call_once(pairs_cache.once[dev], [&] {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess) {
+      cudaGetLastError();
+      pairs_cache.value[dev] = 0;
+      return;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
     cfg.blockDim = dim3(kGemmThreads);
@@ -177,8 +206,10 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
       cudaGetLastError();
       n = sm_count() / 2;
     }
-    max_pairs = n;
-  }
+    pairs_cache.value[dev] = n;
+  });
+  const int max_pairs = pairs_cache.value[dev];
+  if (max_pairs <= 0) return SP24_ERR_CUDA;
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,

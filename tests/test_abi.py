@@ -156,6 +156,72 @@ def test_binding_rejects_views_that_are_not_row_major():
         sp.sp24_mask_search(torch.zeros(64, 96, dtype=torch.float16)[:, :64], idx)
 
 
+def test_binding_rejects_wrong_dtype_and_short_buffers():
+    """Every buffer's dtype and size is checked against what the C call will touch, before the
+    call (CPU tensors: the checks run before the device check)."""
+    import torch
+    f16, u8, f32, i64 = torch.float16, torch.uint8, torch.float32, torch.int64
+    R, C, T = 64, 128, 32
+    w = torch.zeros(R, C, dtype=f16)
+    idx = torch.zeros(R // 4, C // 4, dtype=u8)
+    vr, mr = sp.sp24_compressed_size(R, C)
+    vc, mc = sp.sp24_compressed_size(C, R)
+    comp = [torch.zeros(R, C // 2, dtype=f16), torch.zeros(mr, dtype=u8),
+            torch.zeros(C, R // 2, dtype=f16), torch.zeros(mc, dtype=u8)]
+    cnt = torch.zeros(1, dtype=i64)
+
+    def bad(fn, *a, match):
+        with pytest.raises(ValueError, match=match):
+            fn(*a)
+
+    def ok_until_device(fn, *a):
+        with pytest.raises(ValueError, match="CUDA"):
+            fn(*a)
+
+    ok_until_device(sp.sp24_mask_step, w, idx, idx, cnt, *comp)
+    bad(sp.sp24_mask_search, w, idx[:8], match="idx")
+    bad(sp.sp24_mask_search, w, idx.to(torch.int8), match="idx")
+    bad(sp.sp24_mask_step, w, idx, idx[:4], cnt, *comp, match="idx_prev")
+    bad(sp.sp24_mask_step, w, idx, idx, cnt.to(torch.int32), *comp, match="flip_count")
+    bad(sp.sp24_mask_step, w, idx, idx, cnt, comp[0][:10], *comp[1:], match="row-compressed values")
+    bad(sp.sp24_mask_step, w, idx, idx, cnt, comp[0], comp[1][:100], *comp[2:], match="row-compressed metadata")
+    bad(sp.sp24_prune_compress, w, idx, comp[0], comp[1], comp[2].to(torch.bfloat16), comp[3],
+        match="column-compressed values")
+    x = torch.zeros(T, C, dtype=f16)
+    y = torch.zeros(T, R, dtype=f16)
+    ok_until_device(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, y, "gelu", y.clone())
+    bad(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, y[:-1], match="Y")
+    bad(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, y, "gelu", y[:, :R // 2].contiguous(), match="aux")
+    bad(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, y.float(), match="Y")
+    ok_until_device(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, torch.zeros(T, R // 2, dtype=f16), "geglu", y)
+    ok_until_device(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "dgelu", x.clone())
+    bad(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x[:1], match="dX")
+    bad(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "dgeglu", x.clone(), match="dX")
+    bad(sp.sp24_gemm_dgrad, y, comp[2][:10], comp[3], C, x, match="W\\^T values")
+    ok_until_device(sp.sp24_gemm_dense, x, w, y)
+    bad(sp.sp24_gemm_dense, x, w[:, :64].contiguous(), y, match="A:")
+    bad(sp.sp24_transpose, w, torch.zeros(C, R - 4, dtype=f16), match="out")
+    # weight gradient: MVUE(dY^T) [R x T] compressed along T, dW fp32 [R x C]
+    dy = torch.zeros(T, R, dtype=f16)
+    yv = torch.zeros(R, T // 2, dtype=f16)
+    ym = torch.zeros(sp.sp24_compressed_size(R, T)[1], dtype=u8)
+    dw = torch.zeros(R, C, dtype=f32)
+    ok_until_device(sp.sp24_mvue_sparsify, dy, 0, 0, yv, ym)
+    bad(sp.sp24_mvue_sparsify, dy, 0, 0, yv[:4], ym, match="values")
+    ok_until_device(sp.sp24_gemm_wgrad, x, yv, ym, R, dw)
+    bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw[:10], match="dW")
+    bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw.half(), match="dW")
+    bad(sp.sp24_gemm_wgrad_dense, x, torch.zeros(R, T, dtype=f16), dw.double(), match="dW")
+    g = torch.zeros(R, C, dtype=f32)
+    ok_until_device(sp.sp24_masked_decay, g, w, idx, 1e-4)
+    bad(sp.sp24_masked_decay, g.half(), w, idx, 1e-4, match="grad")
+    bad(sp.sp24_masked_decay, g[:8], w, idx, 1e-4, match="grad")
+    bad(sp.sp24_masked_decay, g, w, idx[:2], 1e-4, match="idx")
+    ok_until_device(sp.sp24_flip_rate, idx, idx, cnt)
+    bad(sp.sp24_flip_rate, idx[:3], idx, cnt, match="idx_prev")
+    bad(sp.sp24_flip_rate, idx, idx, torch.zeros(0, dtype=i64), match="count")
+
+
 def test_valid_call_without_a_device_reports_no_device():
     import torch
     if torch.cuda.is_available():

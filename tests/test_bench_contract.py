@@ -24,10 +24,11 @@ def test_reference_arm_prints_one_contract_line():
     assert REQUIRED <= set(d)
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["value"] > 0
-    assert d["config"]["workload"] == si.GPT2_355M.name
-    assert d["config"]["d_model"] == 1024 and d["config"]["d_ff"] == 4096 and d["config"]["tokens_per_gpu"] == 8192
+    # the default workload is the largest single-GPU configuration: the GPT-2 1.5B FFN
+    assert d["config"]["workload"] == si.GPT2_1P5B.name
+    assert d["config"]["d_model"] == 1600 and d["config"]["d_ff"] == 6400 and d["config"]["tokens_per_gpu"] == 32768
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "32 of 8192" in cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "32 of 32768" in cb["sample"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
@@ -45,3 +46,14 @@ def test_clock_sampler_summary_without_a_gpu():
 def test_headline_flops_are_the_four_ffn_gemms():
     wl = si.GPT2_355M
     assert wl.gemm_flops() == 4 * 2 * 8192 * 1024 * 4096
+
+
+def test_weight_sequence_is_cumulative_and_seeded():
+    wl = si.FFNWorkload("tiny", d=16, ff=32, tokens=16, dtype="f16", steps=3)
+    W1, W2 = wl.weights()
+    seq = bench.weight_sequence(wl, W1, W2)
+    assert [len(x) for x in seq] == [4, 4]
+    for li in range(2):
+        for t in range(3):
+            assert seq[li][t + 1].equal(si.perturb(seq[li][t], wl.perturb_seed(t, li)))
+    assert not seq[0][1].equal(seq[0][2])
