@@ -197,16 +197,6 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 
-def weight_sequence(wl: si.FFNWorkload, W1, W2):
-    """[[W1_0 .. W1_S], [W2_0 .. W2_S]] (host tensors) with W_(t+1) = round(W_t + N(0, 1e-4)),
-    the simulated training steps of the workload (S = max(1, wl.steps))."""
-    seq = [[W1], [W2]]
-    for t in range(max(1, wl.steps)):
-        for li in range(2):
-            seq[li].append(si.perturb(seq[li][-1], wl.perturb_seed(t, li)))
-    return seq
-
-
 class FFNStep:
     """Device buffers and the launch sequence of one step (kernel launches only)."""
 
@@ -228,7 +218,7 @@ class FFNStep:
         dev = "cuda"
         # The simulated training steps: W_(t+1) = round(W_t + N(0, 1e-4)), t = 0 .. S-1.
         self.S = max(1, wl.steps)
-        hostW = weight_sequence(wl, W1, W2)
+        hostW = wl.weight_sequence(W1, W2)
         self.host = {"W": hostW, "X": X, "dY": dY, "G1": G1, "G2": G2} if with_host else None
         self.W = [[w.to(dev) for w in hostW[li]] for li in range(2)]
         self.X, self.dY = X.to(dev), dY.to(dev)
@@ -303,20 +293,25 @@ class FFNStep:
         timed("gemm_dgrad2_dgelu",
               lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre), main)
         if wgrad:
-            # Weight gradients into the gradient buffers: dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X;
+            # Weight gradients into the gradient buffers, decayed in the same kernels:
+            # dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X, then + lambda W where pruned;
             # fresh draws every step and layer (offset 2 * step + layer).
             seed = wl.seeds["mvue"]
             (y2v, y2m), (y1v, y1m) = self.yh
             timed("mvue_dy", lambda: sp.sp24_mvue_sparsify(self.dY, seed, 2 * self.step_no + 1, y2v, y2m), main)
-            timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad(self.H, y2v, y2m, d, self.G[1]), main)
+            timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_decay(self.H, y2v, y2m, d, self.W[1][cur],
+                                                                    self.idx[1][cur], wl.lam, self.G[1]), main)
             timed("mvue_dh", lambda: sp.sp24_mvue_sparsify(self.dH, seed, 2 * self.step_no, y1v, y1m), main)
-            timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad(self.X, y1v, y1m, ff, self.G[0]), main)
+            timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad_decay(self.X, y1v, y1m, ff, self.W[0][cur],
+                                                                    self.idx[0][cur], wl.lam, self.G[0]), main)
         timed("gemm_dgrad1", lambda: sp.sp24_gemm_dgrad(self.dH, c1[2], c1[3], d, self.dX), main)
-        fork()
-        for li, stream in ((0, main), (1, side)):
-            timed("masked_decay", lambda li=li: sp.sp24_masked_decay(self.G[li], self.W[li][cur],
-                                                                      self.idx[li][cur], wl.lam), stream)
-        join()
+        if not wgrad:
+            # the gradients come from elsewhere: the masked decay as its own pass
+            fork()
+            for li, stream in ((0, main), (1, side)):
+                timed("masked_decay", lambda li=li: sp.sp24_masked_decay(self.G[li], self.W[li][cur],
+                                                                          self.idx[li][cur], wl.lam), stream)
+            join()
         self.step_no += 1
 
     def run_dense(self, events=None):
@@ -621,10 +616,11 @@ def run_wgrad_phase(args, step, wl, world, dev, flush, barrier, peaks):
     kernels = kernel_table(events, step.work(), peaks, FFNStep.WGRAD_KERNELS)
     flops = 6 * 2.0 * wl.tokens * wl.d * wl.ff
     return {"ms_per_step": round(ms, 4), "value": round(flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "launches_per_step": 12, "kernels": kernels,
-            "note": "the headline step plus both weight gradients: MVUE 2:4 sparsification of dY^T and dH^T "
+            "launches_per_step": 10, "kernels": kernels,
+            "note": "the headline step with both weight gradients: MVUE 2:4 sparsification of dY^T and dH^T "
                     "(Philox4x64-10 draws), dW2 = MVUE(dY^T) H and dW1 = MVUE(dH^T) X on the sparse tensor "
-                    "cores in fp32, then the masked decay of those gradients; FLOPs 6 x 2 T d ff"}
+                    "cores in fp32 with the masked decay applied in the same kernels' epilogues (no separate "
+                    "decay pass); FLOPs 6 x 2 T d ff"}
 
 
 def run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks):
@@ -825,7 +821,7 @@ def oracle_host(wl):
     W1, W2 = wl.weights()
     X, dY = wl.activations()
     G1, G2 = wl.grads()
-    seq = weight_sequence(wl, W1, W2)
+    seq = wl.weight_sequence(W1, W2)
     masks = [[oracle.mask_search(si.bits16(seq[li][0]), wl.dtype)] + [None] * max(1, wl.steps) for li in range(2)]
     return {"W": seq, "X": X, "dY": dY, "G1": G1, "G2": G2, "masks": masks}
 

@@ -243,6 +243,24 @@ SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const 
                             int64_t N, sp24_dtype dtype, float *dW, void *stream);
 
 /*
+ * Weight gradient and masked decay in one pass (abstract: the masked decay
+ * term on gradients; Software Dependencies row: the 2:4 MMs, MVUE and masked
+ * decay kernels).  dW[N x K] = Yhat * X as sp24_gemm_wgrad computes it, then,
+ * in the same kernel's epilogue, dW <- dW + lambda * W where the mask of W is 0
+ * (one fp32 fused multiply-add per pruned entry, as sp24_masked_decay does on
+ * the stored gradient, so the result has the same bits as sp24_gemm_wgrad
+ * followed by sp24_masked_decay).
+ *   X, vals, meta, dW  as for sp24_gemm_wgrad (dW overwritten)
+ *   W     device dtype [N x K] row-major, contiguous (the layer's weight)
+ *   idx   device uint8 [N/4][K/4], the mask of W (sp24_mask_search)
+ * T % 16 == 0, N % 16 == 0, K % 8 == 0; X, vals, meta, W and dW 16-byte
+ * aligned.  T == 0 gives the decay of a zero gradient.
+ */
+SP24_API sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
+                                  int64_t N, sp24_dtype dtype, const void *W, const uint8_t *idx, float lambda,
+                                  float *dW, void *stream);
+
+/*
  * Dense weight-gradient GEMM for the dense fine-tuning phase (abstract: dense
  * fine-tuning; Experiment Setup row: the last 1/6 of the steps):
  * dW[N x K] = dY^T[N x T] * X[T x K], fp32 accumulation and fp32 output in W's

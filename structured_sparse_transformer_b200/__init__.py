@@ -40,6 +40,7 @@ _SIGNATURES = {
     "sp24_transpose": [P, I64, I64, I32, P, P],
     "sp24_mvue_sparsify": [P, I64, I64, I64, I32, U64, U64, P, P, P],
     "sp24_gemm_wgrad": [P, I64, I64, P, P, I64, I32, P, P],
+    "sp24_gemm_wgrad_decay": [P, I64, I64, P, P, I64, I32, P, P, F32, P, P],
     "sp24_gemm_wgrad_dense": [P, I64, I64, P, I64, I32, P, P],
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
     "sp24_flip_rate": [P, P, I64, P, P],
@@ -121,24 +122,24 @@ def _need_device(*ts):
             raise ValueError("sp24 kernels take CUDA tensors only")
 
 
-def _expect(t, name: str, dtype, numel: int, exact: bool = True):
-    """Raises ValueError unless tensor `t` has `dtype` and holds `numel` elements (at least
-    `numel` when not `exact`): the kernels read and write exactly the sizes passed to the C
-    call, so a short or mistyped buffer would be accessed out of bounds."""
+def _expect(t, name: str, dtype, numel: int):
+    """Raises ValueError unless tensor `t` has `dtype` and holds at least `numel` elements:
+    the kernels read and write exactly the sizes passed to the C call, so a short or
+    mistyped buffer would be accessed out of bounds (a longer one is left alone past them)."""
     if t is None:
         return
     if t.dtype != dtype:
         raise ValueError(f"{name}: expected dtype {dtype}, got {t.dtype}")
     n = t.numel()
-    if (n != numel) if exact else (n < numel):
-        raise ValueError(f"{name}: expected {'' if exact else 'at least '}{numel} elements, got {n}")
+    if n < numel:
+        raise ValueError(f"{name}: expected at least {numel} elements, got {n}")
 
 
 def _expect_compressed(vals, meta, rows: int, cols: int, dtype, what: str):
     """vals [rows x cols/2] of `dtype` and the metadata bytes of an [rows x cols] operand."""
     import torch
     _expect(vals, f"{what} values", dtype, rows * (cols // 2))
-    _expect(meta, f"{what} metadata", torch.uint8, sp24_compressed_size(rows, cols)[1], exact=False)
+    _expect(meta, f"{what} metadata", torch.uint8, sp24_compressed_size(rows, cols)[1])
 
 
 def _shape2(t, name: str):
@@ -218,7 +219,7 @@ def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_r
     _dtype_code(W)
     _expect(idx, "idx", torch.uint8, (R // 4) * (C // 4))
     _expect(idx_prev, "idx_prev", torch.uint8, (R // 4) * (C // 4))
-    _expect(flip_count, "flip_count", torch.int64, 1, exact=False)
+    _expect(flip_count, "flip_count", torch.int64, 1)
     _expect_compressed(vals_row, meta_row, R, C, W.dtype, "row-compressed")
     _expect_compressed(vals_col, meta_col, C, R, W.dtype, "column-compressed")
     _need_device(idx, idx_prev, flip_count, vals_row, meta_row, vals_col, meta_col, W)
@@ -310,6 +311,22 @@ def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
                                 _stream(stream)))
 
 
+def sp24_gemm_wgrad_decay(X, vals, meta, N: int, W, idx, lam: float, dW, stream=None):
+    """dW[N, K] (fp32) <- Yhat[N, T] X[T, K], then dW + lam * W on the entries W's mask prunes."""
+    import torch
+    _need_rowmajor(X, vals, meta, W, idx, dW)
+    T, K = _shape2(X, "X")
+    _dtype_code(X)
+    _expect_compressed(vals, meta, N, T, X.dtype, "MVUE(dY^T)")
+    _expect(W, "W", X.dtype, N * K)
+    _expect(idx, "idx", torch.uint8, (N // 4) * (K // 4))
+    _expect(dW, "dW", torch.float32, N * K)
+    _need_device(X, vals, meta, W, idx, dW)
+    _check("sp24_gemm_wgrad_decay",
+           _lib.sp24_gemm_wgrad_decay(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(W), _ptr(idx),
+                                      float(lam), _ptr(dW), _stream(stream)))
+
+
 def sp24_gemm_wgrad_dense(X, dYt, dW, stream=None):
     """dW[N, K] (fp32) <- dYt[N, T] X[T, K] on the dense tensor-core path (dYt = dY transposed)."""
     import torch
@@ -344,7 +361,7 @@ def sp24_flip_rate(idx_prev, idx_cur, count, stream=None):
     _need_rowmajor(idx_prev, idx_cur, count)
     _expect(idx_cur, "idx_cur", torch.uint8, idx_cur.numel())
     _expect(idx_prev, "idx_prev", torch.uint8, idx_cur.numel())
-    _expect(count, "count", torch.int64, 1, exact=False)
+    _expect(count, "count", torch.int64, 1)
     _need_device(idx_prev, idx_cur, count)
     _check("sp24_flip_rate",
            _lib.sp24_flip_rate(_ptr(idx_prev), _ptr(idx_cur), idx_cur.numel(), _ptr(count), _stream(stream)))

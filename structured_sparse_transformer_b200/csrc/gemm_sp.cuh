@@ -56,6 +56,7 @@
 // error word, raises the CTA's abort flag, and the CTA drains and exits.
 #pragma once
 #include "sp24_common.cuh"
+#include "sp24_tables.cuh"
 
 namespace sp24 {
 
@@ -326,9 +327,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
                           const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
-                          uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out) {
+                          uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out,
+                          const uint16_t *__restrict__ dec_w, const uint8_t *__restrict__ dec_idx,
+                          float dec_lambda) {
   // T counts the B operand's rows of the output: tokens, or for the weight
   // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
+  // Weight gradient with dec_w set: the masked decay of dW in the epilogue, W and
+  // its pattern indices dec_idx [M/4][T/4] in the layout of dW (see below).
   using G = PairGeom<SPARSE, EPI>;
   constexpr bool WG = G::kWg;
   constexpr int kPairStages = G::kStages;
@@ -512,15 +517,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // round trip.  Register layout of tmem_ld_16x256b_x2: thread t holds row
     // t/4 (+8) at columns 2(t%4), +1 of each 8-column block, so each float2
     // store of a warp writes 8 rows x 32 contiguous bytes (whole sectors of dW).
+    // Masked decay (dec_w set): the two entries of a store that the mask of W
+    // prunes become fmaf(lambda, W, acc), the fp32 operation of the separate
+    // decay pass on the stored gradient, so both give the same bits.  The
+    // accumulator is not double-buffered here, so W's values and keep bits of
+    // all of a warp's stores are loaded before it waits for the tile, while the
+    // main loop still runs.
     const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     constexpr int kChunks = G::kBN / 16;
     constexpr int kPerWarp = (kChunks + kEpiGroups - 1) / kEpiGroups;
     constexpr int kBatch = 3;
+    const bool decay = dec_w != nullptr;
+    const int64_t idx_cols = ld_out >> 2;
     int j = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
       const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
       const int n0 = (tile / num_mt) * G::kBN;
+      // Decay operands of the warp's stores in this tile: W's two values (one
+      // 32-bit word) and their two keep bits; entries outside dW keep both.
+      uint32_t wv[kPerWarp][8], kb[kPerWarp];
+      if (decay) {
+#pragma unroll
+        for (int kc = 0; kc < kPerWarp; ++kc) {
+          const int ch = grp + kc * kEpiGroups;
+          kb[kc] = 0xFFFFu;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int h = e >> 2, i = (e >> 1) & 1, sub = e & 1;
+            const int row = m0 + 16 * h + 8 * sub + (lane >> 2);
+            const int col = n0 + 16 * ch + 8 * i + 2 * (lane & 3);
+            wv[kc][e] = 0u;
+            if (ch < kChunks && row < M && col < T) {
+              wv[kc][e] = __ldg(reinterpret_cast<const uint32_t *>(dec_w + (int64_t)row * ld_out + col));
+              const uint32_t pat = __ldg(dec_idx + (int64_t)(row >> 2) * idx_cols + (col >> 2));
+              const uint32_t two = ((uint32_t)g_tables.bits[pat] >> (4 * (row & 3) + (col & 3))) & 3u;
+              kb[kc] = (kb[kc] & ~(3u << (2 * e))) | (two << (2 * e));
+            }
+          }
+        }
+      }
       const bool got = mbar_wait_bounded(&acc_full[0], (uint32_t)j & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
@@ -554,10 +590,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               for (int sub = 0; sub < 2; ++sub) {
                 const int row = m0 + 16 * h + 8 * sub + (lane >> 2);
                 const int col = n0 + 16 * ch + 8 * i + 2 * (lane & 3);
-                if (row < M && col < T)
-                  *reinterpret_cast<float2 *>(out_f32 + (int64_t)row * ld_out + col) =
-                      make_float2(__uint_as_float(r[k][h][4 * i + 2 * sub]),
-                                  __uint_as_float(r[k][h][4 * i + 2 * sub + 1]));
+                float2 v = make_float2(__uint_as_float(r[k][h][4 * i + 2 * sub]),
+                                       __uint_as_float(r[k][h][4 * i + 2 * sub + 1]));
+                if (decay && k0 + k < kPerWarp) {
+                  const int e = 4 * h + 2 * i + sub;
+                  const uint32_t two = kb[k0 + k] >> (2 * e);
+                  if (!(two & 1u)) v.x = fmaf(dec_lambda, bits_to_f32<BF16>(wv[k0 + k][e] & 0xFFFFu), v.x);
+                  if (!(two & 2u)) v.y = fmaf(dec_lambda, bits_to_f32<BF16>(wv[k0 + k][e] >> 16), v.y);
+                }
+                if (row < M && col < T) *reinterpret_cast<float2 *>(out_f32 + (int64_t)row * ld_out + col) = v;
               }
         }
       }

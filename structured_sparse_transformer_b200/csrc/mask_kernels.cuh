@@ -28,11 +28,6 @@ namespace sp24 {
 
 using u64 = unsigned long long;
 
-// The pattern tables in global memory: threads index them with per-thread
-// pattern numbers, which the L1 cache serves without the serialisation that
-// divergent reads of __constant__ memory would take, and without a per-CTA copy.
-__device__ const PatternTables g_tables = make_pattern_tables();
-
 __device__ __forceinline__ u64 umax64(u64 a, u64 b) { return a > b ? a : b; }
 
 // Exact-key dynamic program.  v[4*i+j] = |w(i,j)| in fixed point << 12.
@@ -197,6 +192,77 @@ __device__ __noinline__ uint32_t search_block(const uint32_t (&w)[4][2], const u
 
 constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 
+__device__ const PackedTables g_packed = make_packed_tables();
+
+// Packed-key search of one block, exact when the block's nonzero magnitudes span
+// at most 10 binades (fp16) or 13 (bf16); otherwise returns kNeedsExact.
+//   * |w| becomes the integer v = |w| / U on a per-block unit U: the largest
+//     magnitude below 2^21 U (U = 2^-24 2^sh for fp16, 2^-133 2^sh for bf16),
+//     which is exact when every nonzero |w| is a multiple of U, i.e. when its
+//     exponent field is at least sh + 1 (checked on the raw bits with 16-bit
+//     lane max/min; zeros pass).  The conversion is one fp32 FMA,
+//     |w| 2^(-log2 U) + 2^23, whose low 23 bits hold v; shifted left by 8 the
+//     2^23 offset leaves the word and v << 8 remains.
+//   * A pattern's key is sum(v) << 8 plus the tie field of PackedTables, all
+//     below 2^32 (a sum of eight is below 2^24), so one unsigned max picks the
+//     largest exact sum and, among equal sums, the lowest pattern index.
+//   * The max over the 90 patterns is the same dynamic program over column-count
+//     states: per state, the best top and bottom combo, then the best total.
+template <bool BF16>
+__device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2], const uint8_t *__restrict__ decode) {
+  constexpr PackedTables PT = make_packed_tables();
+  constexpr int kMant = BF16 ? 7 : 10;               // explicit significand bits
+  uint32_t a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = w[k >> 1][k & 1] & 0x7FFF7FFFu;
+  uint32_t mx = __vmaxu2(__vmaxu2(__vmaxu2(a[0], a[1]), __vmaxu2(a[2], a[3])),
+                         __vmaxu2(__vmaxu2(a[4], a[5]), __vmaxu2(a[6], a[7])));
+  uint32_t m1[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m1[k] = __vsub2(a[k], 0x00010001u);   // zeros wrap to 0xFFFF
+  uint32_t mn = __vminu2(__vminu2(__vminu2(m1[0], m1[1]), __vminu2(m1[2], m1[3])),
+                         __vminu2(__vminu2(m1[4], m1[5]), __vminu2(m1[6], m1[7])));
+  mx = max(mx & 0xFFFFu, mx >> 16);
+  mn = min(mn & 0xFFFFu, mn >> 16);
+  const int emax = max((int)(mx >> kMant), 1);
+  const int sh = max(emax - (BF16 ? 14 : 11), 0);
+  const int E = (BF16 ? 133 : 24) - sh;              // U = 2^-E
+  const bool exact = (sh == 0 || mn + 1u >= ((uint32_t)(sh + 1) << kMant)) && E <= 127;
+  if (!exact) return kNeedsExact;
+  const float scale = __uint_as_float((uint32_t)(E + 127) << 23);
+  uint32_t P[4][6];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t h = (a[2 * i + (j >> 1)] >> ((j & 1) << 4)) & 0xFFFFu;
+      const float x = BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
+      v[j] = __float_as_uint(fmaf(x, scale, 8388608.0f)) << 8;
+    }
+#pragma unroll
+    for (int q = 0; q < 6; ++q) P[i][q] = v[pair_lo(q)] + v[pair_hi(q)];
+  }
+  uint32_t best = 0;
+#pragma unroll
+  for (int st = 0; st < kNumStates; ++st) {
+    uint32_t tb = 0, bb = 0;
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      if (i < PT.ntop[st]) {
+        const int c = PT.top[st][i];
+        tb = max(tb, P[0][c / 6] + P[1][c % 6] + (uint32_t)PT.tie_top[c]);
+      }
+      if (i < PT.nbot[st]) {
+        const int b = PT.bot[st][i];
+        bb = max(bb, P[2][b / 6] + P[3][b % 6] + (uint32_t)PT.tie_bot[b]);
+      }
+    }
+    best = max(best, tb + bb);
+  }
+  return decode[best & 0xFFu];
+}
+
 // Fast path of the search, on fp64 sums.  fp16: every |w| is an integer
 // multiple of 2^-24 below 2^17, so a sum of eight needs at most 44
 // significant bits and fp64 holds every partial sum exactly: the search is
@@ -276,9 +342,19 @@ __device__ __forceinline__ void load_unit(const uint16_t *__restrict__ W, int64_
   }
 }
 
-constexpr int kTile = 64;           // W tile: 64 rows x 64 columns per CTA
+constexpr int kTile = 64;           // quadrant of a chunk: 64 rows x 64 columns
 constexpr int kTileBlocks = kTile / 4;
-constexpr int kMaskThreads = 128;   // one unit (4 rows x 8 columns = two blocks) per thread
+constexpr int kQuadThreads = 128;   // one unit (4 rows x 8 columns = two blocks) per thread
+constexpr int kChunk = 2 * kTile;   // one tensor-core metadata chunk: 128 x 128
+#ifndef SP24_MASK_QUADS
+#define SP24_MASK_QUADS 2
+#endif
+// Quadrants per CTA: 4 (the whole chunk) or 2 (128 rows x 64 columns, the CTAs of
+// one chunk side by side).
+constexpr int kMaskQuads = SP24_MASK_QUADS;
+constexpr int kMaskThreads = kMaskQuads * kQuadThreads;
+constexpr int kMaskCtaCols = kMaskQuads == 4 ? kChunk : kTile;   // W columns per CTA
+static_assert(kMaskQuads == 2 || kMaskQuads == 4, "a CTA covers half a chunk or a whole one");
 
 // Nibble (4 * shift) of each of the four 16-bit codes in v, packed 4 bits apart.
 __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
@@ -287,41 +363,50 @@ __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
   return (lo & 0xFu) | ((lo >> 12) & 0xF0u) | ((hi & 0xFu) << 8) | ((hi >> 4) & 0xF000u);
 }
 
-// One CTA per 64x64 tile of W; thread t owns the unit at unit column t%8 and
-// block row t/8.  The tensor-core metadata comes in 2048-byte chunks of
-// 128x128 (see the GEMM); a tile writes its quadrant of the chunk, and with
-// COMPRESS the grid is rounded up to whole chunks so that rows and columns
-// past the matrix get the padding code.
+// Regions of 128x128 of W (one 2048-byte tensor-core metadata chunk of each
+// orientation) in quadrants of 64x64, 128 threads each; a CTA takes kMaskQuads
+// of them (the two quadrants of one column half, or all four).  Thread t of a
+// quadrant owns the unit at unit column t%8 and block row t/8.  Rows and
+// columns past the matrix get the padding code in the metadata.
 //   SEARCH:   compute the mask (else read it from idx)
 //   COMPRESS: write the compressed orientations whose pointers are non-null
 //             (values + tensor-core metadata)
 //   FLIP:     add the number of mask bits that differ from idx_prev to *flip_count
+// Search: every block takes the packed-key search; blocks it cannot certify
+// (magnitudes spread over more than 10 binades for fp16, 13 for bf16) are queued
+// in shared memory and, after a barrier, searched exactly by the first threads
+// of the CTA, so the slow path costs about one warp pass per chunk.
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
+__global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_tile_kernel(
     const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
     uint8_t *__restrict__ meta_col) {
-  __shared__ uint8_t s_idx[kTileBlocks][kTileBlocks];
-  __shared__ __align__(8) uint16_t s_rc[kTileBlocks][kTileBlocks];   // row codes, [block row][block col]
-  __shared__ __align__(8) uint16_t s_cc[kTileBlocks][kTileBlocks];   // column codes, [block col][block row]
-  __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kTile * 16 : 4];
-  __shared__ uint16_t s_queue[SEARCH ? kTileBlocks * kTileBlocks : 2];
+  __shared__ uint8_t s_idx[kMaskQuads][kTileBlocks][kTileBlocks];
+  __shared__ __align__(8) uint16_t s_rc[COMPRESS ? kMaskQuads : 1][kTileBlocks][kTileBlocks];   // row codes
+  __shared__ __align__(8) uint16_t s_cc[COMPRESS ? kMaskQuads : 1][kTileBlocks][kTileBlocks];   // [bc][br]
+  __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kMaskQuads : 1][COMPRESS ? kTile * 16 : 4];
+  __shared__ uint16_t s_queue[SEARCH ? kMaskQuads * kTileBlocks * kTileBlocks : 2];
   __shared__ int s_qn;
   __shared__ unsigned long long s_flip;
 
   const int tid = threadIdx.x;
+  const int qd = tid >> 7, lt = tid & (kQuadThreads - 1);
+  const int rh = kMaskQuads == 4 ? qd >> 1 : qd;
+  const int kh = kMaskQuads == 4 ? qd & 1 : (int)(blockIdx.x & 1);
+  const uint32_t chunk_x = kMaskQuads == 4 ? blockIdx.x : blockIdx.x >> 1;
+  const uint32_t chunks_x = kMaskQuads == 4 ? gridDim.x : gridDim.x >> 1;
   const uint16_t *bits_tab = g_tables.bits;
   const uint8_t *index_tab = g_tables.index;
   if (tid == 0) { s_flip = 0; s_qn = 0; }
   pdl_launch_dependents();
   pdl_wait();
 
-  const int64_t tile_r = (int64_t)blockIdx.y * kTile;
-  const int64_t tile_c = (int64_t)blockIdx.x * kTile;
+  const int64_t tile_r = (int64_t)blockIdx.y * kChunk + kTile * rh;
+  const int64_t tile_c = (int64_t)chunk_x * kChunk + kTile * kh;
   const int64_t bcols = C >> 2;
-  const int uc = tid & 7;
-  const int br = tid >> 3;
+  const int uc = lt & 7;
+  const int br = lt >> 3;
   const int64_t r0 = tile_r + 4 * br;
   const int64_t c0 = tile_c + 8 * uc;
   const bool row_ok = r0 < R;
@@ -344,8 +429,7 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
   }
   __syncthreads();
 
-  // Phase 1: search (SEARCH), or take the given mask (!SEARCH).  bf16 blocks
-  // the fast path cannot certify are queued for the exact integer search.
+  // Phase 1: search (SEARCH), or take the given mask (!SEARCH).
   uint32_t p[2];
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
@@ -355,36 +439,38 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
       uint32_t blk[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
-      p[b] = search_block_fast<BF16>(blk, index_tab);
-      if (BF16 && p[b] == kNeedsExact) {
+      p[b] = search_block_packed<BF16>(blk, g_packed.decode);
+      if (p[b] == kNeedsExact) {
         const int slot = atomicAdd(&s_qn, 1);
-        s_queue[slot] = (uint16_t)(br * kTileBlocks + 2 * uc + b);
+        s_queue[slot] = (uint16_t)((qd << 8) | (br << 4) | (2 * uc + b));
       }
     }
-    if (SEARCH && BF16) s_idx[br][2 * uc + b] = (uint8_t)p[b];
+    if (SEARCH) s_idx[qd][br][2 * uc + b] = (uint8_t)p[b];
   }
 
-  // Phase 1b (bf16): blocks the fast path could not certify take the exact integer search.
-  if (SEARCH && BF16) {
+  // Phase 1b: the exact search of the queued blocks, entry k by thread k.
+  if (SEARCH) {
     __syncthreads();
-    // Queue entry k goes to lane k/4 of warp k%4, so a few entries run on
-    // different schedulers instead of side by side in one warp.
     const int qn = s_qn;
-    for (int k = (tid >> 5) + 4 * (tid & 31); k < qn; k += kMaskThreads) {
-      const int id = s_queue[k];
-      const int qbr = id / kTileBlocks, qbc = id % kTileBlocks;
-      const uint16_t *src = W + (tile_r + 4 * qbr) * ldw + tile_c + 4 * qbc;
-      uint32_t blk[4][2];
+    if (qn > 0) {
+      for (int k = tid; k < qn; k += kMaskThreads) {
+        const int id = s_queue[k];
+        const int q = id >> 8, qbr = (id >> 4) & 15, qbc = id & 15;
+        const int qrh = kMaskQuads == 4 ? q >> 1 : q, qkh = kMaskQuads == 4 ? q & 1 : kh;
+        const uint16_t *src = W + ((int64_t)blockIdx.y * kChunk + kTile * qrh + 4 * qbr) * ldw +
+                              (int64_t)chunk_x * kChunk + kTile * qkh + 4 * qbc;
+        uint32_t blk[4][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src + i * ldw));
-        blk[i][0] = q.x; blk[i][1] = q.y;
+        for (int i = 0; i < 4; ++i) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src + i * ldw));
+          blk[i][0] = v.x; blk[i][1] = v.y;
+        }
+        s_idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, index_tab, bits_tab);
       }
-      s_idx[qbr][qbc] = (uint8_t)search_block<BF16>(blk, index_tab, bits_tab);
-    }
-    __syncthreads();
+      __syncthreads();
 #pragma unroll
-    for (int b = 0; b < 2; ++b) p[b] = s_idx[br][2 * uc + b];
+      for (int b = 0; b < 2; ++b) p[b] = s_idx[qd][br][2 * uc + b];
+    }
   }
 
   // Phase 2: outputs of this thread's two blocks.
@@ -401,8 +487,8 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
     for (int b = 0; b < 2; ++b) {
       rc[b] = g_tables.rowcode[p[b]];
       cc[b] = g_tables.colcode[p[b]];
-      s_rc[br][2 * uc + b] = (uint16_t)rc[b];
-      s_cc[2 * uc + b][br] = (uint16_t)cc[b];
+      s_rc[qd][br][2 * uc + b] = (uint16_t)rc[b];
+      s_cc[qd][2 * uc + b][br] = (uint16_t)cc[b];
     }
     if (ok0) {
       // Forward operand: kept values of each row, in column order.
@@ -429,7 +515,7 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
           const int word = 2 * b + (j >> 1);
           const uint32_t lo = (pick_row(w, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
           const uint32_t hi = (pick_row(w, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
-          s_vcol[vcol_word(8 * uc + 4 * b + j, br)] = lo | (hi << 16);
+          s_vcol[qd][vcol_word(8 * uc + 4 * b + j, br)] = lo | (hi << 16);
         }
       }
     }
@@ -443,14 +529,15 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
   if (FLIP && tid == 0 && s_flip) atomicAdd(flip_count, s_flip);
 
   if (COMPRESS) {
-    // Transposed values: W column c (a row of W^T) holds 32 kept values per tile.
+    // Transposed values: W column c (a row of W^T) holds 32 kept values per quadrant.
     const int64_t half_rows = R >> 1;
 #pragma unroll
-    for (int k = 0; k < (kTile * 4) / kMaskThreads; ++k) {
-      const int id = tid + kMaskThreads * k;
+    for (int k = 0; k < (kTile * 4) / kQuadThreads; ++k) {
+      const int id = lt + kQuadThreads * k;
       const int c_local = id >> 2, q = id & 3;
       if (vals_col && tile_c + c_local < C && tile_r + 16 * q + 16 <= R) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(&s_vcol[c_local * 16 + (((q ^ (c_local >> 3)) & 3) << 2)]);
+        const uint4 v =
+            *reinterpret_cast<const uint4 *>(&s_vcol[qd][c_local * 16 + (((q ^ (c_local >> 3)) & 3) << 2)]);
         const bool swap = (c_local >> 5) & 1;
         const uint4 o = swap ? make_uint4(v.z, v.w, v.x, v.y) : v;
         *reinterpret_cast<uint4 *>(vals_col + (tile_c + c_local) * half_rows + (tile_r >> 1) + 8 * q) = o;
@@ -460,26 +547,25 @@ __global__ void __launch_bounds__(kMaskThreads, 6) mask_tile_kernel(
     // word kk (one 32-column K step of the MMA) holds rows m and m+8,
     // m = (L%8) + 16*(L/16), groups 4*((L/8)%2) .. +3 of that K step; the
     // low 16 bits are row m, the high 16 bits row m+8, one nibble per group.
-    // This tile is quadrant (rh, kh) of its chunk: lanes 64*rh.., words 2*kh..
-    // for the rows of W, lanes 64*kh.., words 2*rh.. for its columns.  Thread
-    // t builds word t%2 of lane t/2 of the quadrant on each side.
-    const int rh = (int)(blockIdx.y & 1), kh = (int)(blockIdx.x & 1);
-    const int lq = tid >> 1, kx = tid & 1;
+    // Quadrant (rh, kh) fills lanes 64*rh.., words 2*kh.. of the chunk of the
+    // rows of W, and lanes 64*kh.., words 2*rh.. of the chunk of its columns.
+    // Thread t builds word t%2 of lane t/2 of the quadrant on each side.
+    const int lq = lt >> 1, kx = lt & 1;
     const int m_lo = (lq & 7) + ((lq >> 4) << 4);   // row of the quadrant (0..55)
     const int gq = kx * 8 + ((lq >> 3) & 1) * 4;     // first of four groups, in blocks of the quadrant
     const int shift = m_lo & 3;
     if (meta_row) {
-      const uint2 a = *reinterpret_cast<const uint2 *>(&s_rc[m_lo >> 2][gq]);
-      const uint2 c = *reinterpret_cast<const uint2 *>(&s_rc[(m_lo >> 2) + 2][gq]);
+      const uint2 a = *reinterpret_cast<const uint2 *>(&s_rc[qd][m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&s_rc[qd][(m_lo >> 2) + 2][gq]);
       const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
-      const size_t chunk = (size_t)(blockIdx.y >> 1) * (gridDim.x >> 1) + (blockIdx.x >> 1);
+      const size_t chunk = (size_t)blockIdx.y * chunks_x + chunk_x;
       *reinterpret_cast<uint32_t *>(meta_row + chunk * 2048 + (64 * rh + lq) * 16 + 4 * (2 * kh + kx)) = word;
     }
     if (meta_col) {
-      const uint2 a = *reinterpret_cast<const uint2 *>(&s_cc[m_lo >> 2][gq]);
-      const uint2 c = *reinterpret_cast<const uint2 *>(&s_cc[(m_lo >> 2) + 2][gq]);
+      const uint2 a = *reinterpret_cast<const uint2 *>(&s_cc[qd][m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&s_cc[qd][(m_lo >> 2) + 2][gq]);
       const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
-      const size_t chunk = (size_t)(blockIdx.x >> 1) * (gridDim.y >> 1) + (blockIdx.y >> 1);
+      const size_t chunk = (size_t)chunk_x * gridDim.y + blockIdx.y;
       *reinterpret_cast<uint32_t *>(meta_col + chunk * 2048 + (64 * kh + lq) * 16 + 4 * (2 * rh + kx)) = word;
     }
   }

@@ -134,9 +134,12 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 // SPARSE: A = kept values [M x Kd/2] + metadata chunks; dense: A = [M x Kd].
 // Weight gradient (kEpiWgrad): B = the layer input [Kd tokens x T columns]
 // read MN-major, out = fp32 [M x T]; tiles of 256 x 256.
+// Weight gradient with decay: dec_w/dec_idx/dec_lambda (the masked decay of dW in
+// the epilogue); null dec_w elsewhere.
 template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
-                               void *out, void *aux, cudaStream_t stream) {
+                               void *out, void *aux, cudaStream_t stream, const void *dec_w = nullptr,
+                               const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f) {
   using G = PairGeom<SPARSE, EPI>;
   const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
@@ -214,7 +217,7 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
-                    (int64_t)(G::kWg ? T : 0));
+                    (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda);
 }
 
 template <bool SPARSE>
@@ -264,9 +267,10 @@ sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
 sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint8_t *idx, const uint8_t *prev,
                           unsigned long long *flip, void *vr, void *mr, void *vc, void *mc, cudaStream_t s) {
-  // With COMPRESS the grid covers whole 128x128 metadata chunks (two tiles each way).
-  const int64_t g = COMPRESS ? 2 * kTile : kTile;
-  dim3 grid((unsigned)((C + g - 1) / g * (g / kTile)), (unsigned)((R + g - 1) / g * (g / kTile)));
+  // CTAs cover whole 128x128 regions (one metadata chunk of each orientation).
+  const int64_t chunks_x = (C + kChunk - 1) / kChunk, chunks_y = (R + kChunk - 1) / kChunk;
+  if (chunks_y > 65535 || chunks_x * (kChunk / kMaskCtaCols) > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  dim3 grid((unsigned)(chunks_x * (kChunk / kMaskCtaCols)), (unsigned)chunks_y);
   return launch_pdl(mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP>, grid, dim3(kMaskThreads), 0, s,
                     static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
                     static_cast<uint8_t *>(mr), static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc));
@@ -490,6 +494,29 @@ sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *val
   }
   return dtype == SP24_BF16 ? launch_gemm_pair_t<true, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s)
                             : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s);
+}
+
+sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
+                                  int64_t N, sp24_dtype dtype, const void *W, const uint8_t *idx, float lambda,
+                                  float *dW, void *stream) {
+  if (T < 0 || K < 0 || N < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (T % 16 || N % 16 || K % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!dW || !W || !idx || (T > 0 && (!X || !vals || !meta))) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dW) || !aligned16(W) || (T > 0 && (!aligned16(X) || !aligned16(vals) || !aligned16(meta))))
+    return SP24_ERR_MISALIGNED;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {   // an empty sum over tokens, then the decay of the zero gradient
+    if (cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
+    return sp24_masked_decay(dW, W, dtype, N, K, idx, lambda, stream);
+  }
+  return dtype == SP24_BF16
+             ? launch_gemm_pair_t<true, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s, W, idx, lambda)
+             : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s, W, idx, lambda);
 }
 
 sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N, sp24_dtype dtype,

@@ -100,4 +100,53 @@ __host__ __device__ constexpr PatternTables make_pattern_tables() {
   return t;
 }
 
+#ifdef __CUDACC__
+// The pattern tables in global memory: threads index them with per-thread
+// pattern numbers, which the L1 cache serves without the serialisation that
+// divergent reads of __constant__ memory would take, and without a per-CTA copy.
+__device__ const PatternTables g_tables = make_pattern_tables();
+#endif
+
+// Tables of the packed-key search (mask_kernels.cuh, search_block_packed).
+// A pattern's key is (exact sum of its |w|) << 8 plus an 8-bit tie field
+//   tie = (35 - top rank) * 6 + (5 - bottom class rank),
+// where a bottom combo's class rank is its position, in rank order, among the
+// bottom combos that need the same state (at most six).  Among patterns with equal
+// sums the larger tie field is the smaller (top rank, bottom rank), i.e. the lower
+// pattern index, and the field splits into a top part and a bottom part that ride
+// on the combo sums.  decode maps a tie field back to the pattern index.
+struct PackedTables {
+  uint8_t ntop[kNumStates];      // top combos producing each state
+  uint8_t top[kNumStates][6];    // their ranks, ascending
+  uint8_t nbot[kNumStates];      // bottom combos needing each state
+  uint8_t bot[kNumStates][6];    // their ranks, ascending
+  uint8_t tie_top[36];           // (35 - rank) * 6
+  uint8_t tie_bot[36];           // 5 - class rank
+  uint8_t decode[256];           // tie field -> pattern index (kPadIndex where unused)
+};
+
+__host__ __device__ constexpr PackedTables make_packed_tables() {
+  PackedTables t{};
+  const PatternTables pt = make_pattern_tables();
+  for (int s = 0; s < kNumStates; ++s) { t.ntop[s] = 0; t.nbot[s] = 0; }
+  for (int c = 0; c < 36; ++c) {
+    const int s = pt.top_state[c];
+    t.top[s][t.ntop[s]++] = (uint8_t)c;
+    t.tie_top[c] = (uint8_t)((35 - c) * 6);
+  }
+  for (int b = 0; b < 36; ++b) {
+    const int s = pt.bot_state[b];
+    t.tie_bot[b] = (uint8_t)(5 - t.nbot[s]);
+    t.bot[s][t.nbot[s]++] = (uint8_t)b;
+  }
+  for (int i = 0; i < 256; ++i) t.decode[i] = kPadIndex;
+  for (int s = 0; s < kNumStates; ++s)
+    for (int i = 0; i < t.ntop[s]; ++i)
+      for (int k = 0; k < t.nbot[s]; ++k) {
+        const int c = t.top[s][i], b = t.bot[s][k];
+        t.decode[t.tie_top[c] + t.tie_bot[b]] = pt.index[c * 36 + b];
+      }
+  return t;
+}
+
 }  // namespace sp24

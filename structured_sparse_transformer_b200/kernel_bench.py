@@ -9,7 +9,7 @@ W is [rows x cols] (N(0, 0.02), or the 8-level tie-heavy variant with
 T = --tokens rows of N(0, 1) activations: gemm_fwd computes [T x rows] from
 [T x cols], gemm_dgrad [T x cols] from [T x rows], gemm_wgrad the fp32
 [rows x cols] weight gradient from dY [T x rows] (MVUE-sparsified) and
-X [T x cols]; mvue sparsifies dY [T x rows] (bytes per dY element).  Each timed launch follows an
+X [T x cols] (gemm_wgrad_decay: with the masked decay of W's mask in its epilogue); mvue sparsifies dY [T x rows] (bytes per dY element).  Each timed launch follows an
 L2 flush (256 MiB write) and is timed alone with CUDA events on the current
 stream.  Prints one JSON line: average microseconds per launch and the
 algorithmic throughput (bytes for the memory-bound kernels, dense-equivalent
@@ -40,7 +40,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--kernel", required=True,
                     choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad", "gemm_dense_fwd", "gemm_dense_dgrad",
-                                                         "gemm_wgrad"])
+                                                         "gemm_wgrad", "gemm_wgrad_decay"])
     ap.add_argument("--rows", type=int, required=True)
     ap.add_argument("--cols", type=int, required=True)
     ap.add_argument("--tokens", type=int, default=8192)
@@ -87,7 +87,7 @@ def main(argv=None):
         aux = torch.empty(T, R, dtype=tdt, device=dev) if args.epi == "gelu" else None
         epi = "gelu" if args.epi == "gelu" else None
         fn = lambda: sp.sp24_gemm_fwd(x, bufs[0], bufs[1], R, y, epi, aux)
-    elif k in ("mvue", "gemm_wgrad"):
+    elif k in ("mvue", "gemm_wgrad", "gemm_wgrad_decay"):
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
         yv = torch.empty(R, T // 2, dtype=tdt, device=dev)
         ym = torch.empty(sp.sp24_compressed_size(R, T)[1], dtype=torch.uint8, device=dev)
@@ -97,7 +97,10 @@ def main(argv=None):
         else:
             x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
             dw = torch.empty(R, C, dtype=torch.float32, device=dev)
-            fn = lambda: sp.sp24_gemm_wgrad(x, yv, ym, R, dw)
+            if k == "gemm_wgrad":
+                fn = lambda: sp.sp24_gemm_wgrad(x, yv, ym, R, dw)
+            else:   # dW of W [rows x cols] with the masked decay in the epilogue
+                fn = lambda: sp.sp24_gemm_wgrad_decay(x, yv, ym, R, w, prev, 6e-5, dw)
     elif k == "transpose":
         wt = torch.empty(C, R, dtype=tdt, device=dev)
         fn = lambda: sp.sp24_transpose(w, wt)

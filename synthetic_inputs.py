@@ -96,6 +96,15 @@ class FFNWorkload:
         """Seed of the N(0, 1e-4) update of weight ``which`` (0: W1, 1: W2) at ``step``."""
         return self.seeds["perturb"] + 2 * step + which
 
+    def weight_sequence(self, W1, W2):
+        """[[W1_0 .. W1_S], [W2_0 .. W2_S]] with W_(t+1) = perturb(W_t): the weights of the
+        simulated training steps (S = max(1, steps)), seeds ``perturb_seed(t, layer)``."""
+        seq = [[W1], [W2]]
+        for t in range(max(1, self.steps)):
+            for li in range(2):
+                seq[li].append(perturb(seq[li][-1], self.perturb_seed(t, li)))
+        return seq
+
     def gemm_flops(self) -> int:
         """Dense-equivalent FLOPs of the four FFN GEMMs (fwd and dX for both layers)."""
         return 4 * 2 * self.tokens * self.d * self.ff

@@ -127,6 +127,14 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_gemm_wgrad", fake, 32, 64, odd, fake, 64, 0, fake, None) == \
         E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_gemm_wgrad_decay", fake, 32, 64, fake, fake, 64, 0, None, fake, ctypes.c_float(1e-4),
+                fake, None) == E["SP24_ERR_INVALID_ARG"]          # no weight
+    assert _raw("sp24_gemm_wgrad_decay", fake, 32, 64, fake, fake, 64, 0, fake, None, ctypes.c_float(1e-4),
+                fake, None) == E["SP24_ERR_INVALID_ARG"]          # no mask
+    assert _raw("sp24_gemm_wgrad_decay", fake, 32, 64, fake, fake, 64, 0, odd, fake, ctypes.c_float(1e-4),
+                fake, None) == E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_gemm_wgrad_decay", fake, 24, 64, fake, fake, 64, 0, fake, fake, ctypes.c_float(1e-4),
+                fake, None) == E["SP24_ERR_UNSUPPORTED_SHAPE"]
     assert _raw("sp24_gemm_wgrad_dense", fake, 24, 64, fake, 64, 0, fake, None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]
     assert _raw("sp24_gemm_wgrad_dense", fake, 32, 64, None, 64, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
@@ -212,6 +220,10 @@ def test_binding_rejects_wrong_dtype_and_short_buffers():
     bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw[:10], match="dW")
     bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw.half(), match="dW")
     bad(sp.sp24_gemm_wgrad_dense, x, torch.zeros(R, T, dtype=f16), dw.double(), match="dW")
+    wt = torch.zeros(R, C, dtype=f16)
+    ok_until_device(sp.sp24_gemm_wgrad_decay, x, yv, ym, R, wt, idx.reshape(-1)[:(R // 4) * (C // 4)].clone(), 1e-4, dw)
+    bad(sp.sp24_gemm_wgrad_decay, x, yv, ym, R, wt[:, :64].contiguous(), idx, 1e-4, dw, match="W:")
+    bad(sp.sp24_gemm_wgrad_decay, x, yv, ym, R, wt, idx[:1], 1e-4, dw, match="idx")
     g = torch.zeros(R, C, dtype=f32)
     ok_until_device(sp.sp24_masked_decay, g, w, idx, 1e-4)
     bad(sp.sp24_masked_decay, g.half(), w, idx, 1e-4, match="grad")

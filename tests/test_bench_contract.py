@@ -51,7 +51,7 @@ def test_headline_flops_are_the_four_ffn_gemms():
 def test_weight_sequence_is_cumulative_and_seeded():
     wl = si.FFNWorkload("tiny", d=16, ff=32, tokens=16, dtype="f16", steps=3)
     W1, W2 = wl.weights()
-    seq = bench.weight_sequence(wl, W1, W2)
+    seq = wl.weight_sequence(W1, W2)
     assert [len(x) for x in seq] == [4, 4]
     for li in range(2):
         for t in range(3):

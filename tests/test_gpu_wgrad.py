@@ -217,3 +217,46 @@ def test_ffn_weight_grads_1p5b_sampled_rows_and_columns():
         ref = oracle.weight_grad(oracle.to_f64(bits, dt), bf)
         got = dw[r0:r0 + 64][:, torch.from_numpy(cols).cuda()]
         _check_wgrad(got, ref, f"dW [{N}x{K}] rows {r0}.. sampled columns")
+
+
+@pytest.mark.parametrize("T,N,K,dtype", [(256, 128, 136, "f16"), (512, 272, 520, "bf16"), (1024, 4096, 1024, "f16"),
+                                         (2048, 1600, 6400, "f16"), (0, 64, 64, "f16")])
+def test_wgrad_decay_fused_equals_separate_passes(T, N, K, dtype):
+    """sp24_gemm_wgrad_decay = sp24_gemm_wgrad then sp24_masked_decay, bit for bit, and that
+    equals the oracle's masked decay (an fp32 fused multiply-add per pruned entry) of the
+    GPU's own undecayed gradient.  Ragged dW tiles (N, K not multiples of 256) included."""
+    tdt = si.DTYPES[dtype]
+    w = si.normal((N, K), 0.02, N + K, dtype)
+    x = si.normal((max(T, 16), K), 1.0, T + 3, dtype)[:T].contiguous()
+    dy = si.normal((max(T, 16), N), 1.0, T + 4, dtype)[:T].contiguous()
+    wd, xd = w.cuda(), x.cuda()
+    idx = torch.empty(N // 4, K // 4, dtype=torch.uint8, device="cuda")
+    sp.sp24_mask_search(wd, idx)
+    vals, meta = _alloc(N, max(T, 16), dtype)
+    if T:
+        sp.sp24_mvue_sparsify(dy.cuda(), 31, 7, vals, meta)
+    lam = 6e-5
+    plain = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    fused = torch.full((N, K), float("nan"), dtype=torch.float32, device="cuda")
+    if T:
+        sp.sp24_gemm_wgrad(xd, vals, meta, N, plain)
+        sp.sp24_gemm_wgrad_decay(xd, vals, meta, N, wd, idx, lam, fused)
+    else:
+        # an empty token range: the decay of a zero gradient
+        lib = sp.lib()
+        import ctypes
+        z = ctypes.c_void_p(0)
+        plain.zero_()
+        st = lib.sp24_gemm_wgrad_decay(z, 0, K, z, z, N, 0, ctypes.c_void_p(wd.data_ptr()),
+                                       ctypes.c_void_p(idx.data_ptr()), ctypes.c_float(lam),
+                                       ctypes.c_void_p(fused.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == 0
+    undecayed = plain.cpu().numpy().copy()
+    sp.sp24_masked_decay(plain, wd, idx, lam)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    got = fused.cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), plain.cpu().numpy().view(np.uint32))
+    ref = oracle.masked_decay(undecayed, si.bits16(w), dtype, idx.cpu().numpy(), lam)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    assert np.array_equal(idx.cpu().numpy(), oracle.mask_search(si.bits16(w), dtype))
