@@ -75,8 +75,15 @@ typedef enum sp24_epilogue {
    * 16g..16g+15 at 32g.., up rows at 32g+16..), so the accumulator columns of
    * one output feature sit 16 apart. */
   SP24_EPI_GEGLU = 3, /* out[T x N/2] = gelu(gate) * up; aux[T x N] <- acc (both halves) */
-  SP24_EPI_DGEGLU = 4 /* out[T x 2K] = (acc*up*gelu'(gate), acc*gelu(gate)) interleaved as
-                         aux; aux[T x 2K] holds the gated pre-activations */
+  SP24_EPI_DGEGLU = 4, /* out[T x 2K] = (acc*up*gelu'(gate), acc*gelu(gate)) interleaved as
+                          aux; aux[T x 2K] holds the gated pre-activations */
+  /* Derivative-saving GELU pair: the forward stores gelu'(pre-activation) as aux,
+   * so the input gradient multiplies by it and evaluates no GELU'.  The same
+   * product as SP24_EPI_GELU / SP24_EPI_DGELU, with the derivative rounded to the
+   * dtype instead of the pre-activation.  (Value 5 is the library's own
+   * weight-gradient epilogue and is not taken here.) */
+  SP24_EPI_GELU_DERIV = 6, /* out = gelu(acc); aux <- gelu'(acc) rounded to dtype */
+  SP24_EPI_MUL_AUX = 7     /* out = acc * aux; aux [T x K] holds gelu'(pre-activation) */
 } sp24_epilogue;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -148,9 +155,10 @@ SP24_API sp24_status sp24_mask_step(const void *W, sp24_dtype dtype, int64_t row
  *   vals_row, meta_row   device, W [N x K] compressed along K (sp24_prune_compress)
  *   Y         device [T x N] row-major, contiguous
  *   epi       SP24_EPI_NONE, or SP24_EPI_GELU: Y = gelu(acc) and aux[T x N] <- acc,
+ *             or SP24_EPI_GELU_DERIV: Y = gelu(acc) and aux[T x N] <- gelu'(acc),
  *             or SP24_EPI_GEGLU: Y is [T x N/2] = gelu(gate) * up for the stacked
  *             gate/up weight (N % 32 == 0) and aux[T x N] <- acc
- *   aux       device [T x N] for SP24_EPI_GELU / GEGLU, else ignored (may be NULL)
+ *   aux       device [T x N] for SP24_EPI_GELU / GEGLU / GELU_DERIV, else ignored (may be NULL)
  * fp32 accumulation; outputs rounded to dtype.  K % 16 == 0, N % 16 == 0,
  * T >= 0.  All pointers 16-byte aligned.
  */
@@ -165,6 +173,8 @@ SP24_API sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const vo
  *   vals_col, meta_col   device, W^T [K x N] compressed along N (sp24_prune_compress)
  *   dX        device [T x K]
  *   epi       SP24_EPI_NONE, or SP24_EPI_DGELU: dX = acc * gelu'(aux), aux [T x K],
+ *             or SP24_EPI_MUL_AUX: dX = acc * aux, aux [T x K] (the derivative that
+ *             SP24_EPI_GELU_DERIV stored),
  *             or SP24_EPI_DGEGLU (input gradient of the down projection of a
  *             gated FFN, acc = dH): dX is [T x 2K], the gradients of the gate
  *             and up pre-activations in the stacked layout of aux [T x 2K]
@@ -179,11 +189,12 @@ SP24_API sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const
  * procedure near the end of pre-training; Experiment Setup row: the last 1/6
  * of the total steps), on the same tcgen05 pipeline as the 2:4 GEMMs:
  *   out[T x M] = B[T x Kd] * A[M x Kd]^T
- * forward:        B = X  [T x K], A = W   [N x K]  (epi NONE or GELU)
- * input gradient: B = dY [T x N], A = W^T [K x N]  (epi NONE or DGELU;
+ * forward:        B = X  [T x K], A = W   [N x K]  (epi NONE, GELU or GELU_DERIV)
+ * input gradient: B = dY [T x N], A = W^T [K x N]  (epi NONE, DGELU or MUL_AUX;
  *                 W^T from sp24_transpose)
  *   B, A, out  device, row-major, contiguous; aux as in sp24_gemm_fwd (GELU:
- *              written with the pre-activation) or sp24_gemm_dgrad (DGELU: read)
+ *              written with the pre-activation, GELU_DERIV with gelu' of it) or
+ *              sp24_gemm_dgrad (DGELU, MUL_AUX: read)
  * fp32 accumulation; outputs rounded to dtype.  Kd % 16 == 0, M % 16 == 0,
  * T >= 0.  All pointers 16-byte aligned.
  */

@@ -61,7 +61,7 @@ STATUS = {0: "SP24_OK", 1: "SP24_ERR_INVALID_ARG", 2: "SP24_ERR_UNSUPPORTED_SHAP
           6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE"}
 SP24_F16, SP24_BF16 = 0, 1
 SP24_EPI_NONE, SP24_EPI_GELU, SP24_EPI_DGELU = 0, 1, 2
-EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4}
+EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4, "gelu_deriv": 6, "mul_aux": 7}
 
 
 class Sp24Error(RuntimeError):
@@ -230,8 +230,9 @@ def sp24_mask_step(W, idx, idx_prev=None, flip_count=None, vals_row=None, meta_r
 
 
 def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=None):
-    """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None, 'gelu' (aux <- pre-activation) or
-    'geglu' (W the stacked gate/up weight: Y[T, N/2] <- gelu(gate) * up, aux[T, N] <- pre-activations)."""
+    """Y[T, N] <- X[T, K] (W*m)^T, W given compressed along K; epi None, 'gelu' (aux <- pre-activation),
+    'gelu_deriv' (aux <- gelu' of the pre-activation) or 'geglu' (W the stacked gate/up weight:
+    Y[T, N/2] <- gelu(gate) * up, aux[T, N] <- pre-activations)."""
     _need_rowmajor(X, vals_row, meta_row, Y, aux)
     T, K = _shape2(X, "X")
     _dtype_code(X)
@@ -245,8 +246,9 @@ def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=N
 
 
 def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stream=None):
-    """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None, 'dgelu' (uses aux [T, K]) or
-    'dgeglu' (dX[T, 2K] <- gradients of the gated pre-activations in aux [T, 2K])."""
+    """dX[T, K] <- dY[T, N] (W*m), W^T given compressed along N; epi None, 'dgelu' (multiplies by gelu' of
+    the pre-activation in aux [T, K]), 'mul_aux' (multiplies by aux [T, K], the derivative 'gelu_deriv'
+    stored) or 'dgeglu' (dX[T, 2K] <- gradients of the gated pre-activations in aux [T, 2K])."""
     _need_rowmajor(dY, vals_col, meta_col, dX, aux)
     T, N = _shape2(dY, "dY")
     _dtype_code(dY)
@@ -261,7 +263,8 @@ def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stre
 
 
 def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
-    """out[T, M] <- B[T, Kd] A[M, Kd]^T on the dense tensor-core path; epi None, 'gelu' or 'dgelu'."""
+    """out[T, M] <- B[T, Kd] A[M, Kd]^T on the dense tensor-core path; epi None, 'gelu', 'dgelu',
+    'gelu_deriv' or 'mul_aux'."""
     _need_rowmajor(B, A, out, aux)
     T, Kd = _shape2(B, "B")
     M = _shape2(A, "A")[0]

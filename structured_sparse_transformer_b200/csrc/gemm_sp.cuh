@@ -84,7 +84,14 @@ constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at column
 // The weight gradient (wgrad) is its own variant: A = the MVUE-sparsified dY^T
 // [N x T], B = the layer input [T x K] read MN-major, out = dW [N x K] fp32 in
 // the natural orientation (see PairGeom and the wgrad epilogue below).
-enum : int { kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4, kEpiWgrad = 5 };
+// Derivative-saving pair: the forward writes gelu'(acc) as aux, so the input
+// gradient only multiplies by it (out = acc * aux); the same product as
+// GELU / GELU', with the derivative rounded to the dtype instead of the
+// pre-activation.
+enum : int {
+  kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4, kEpiWgrad = 5, kEpiGeluDeriv = 6,
+  kEpiMulAux = 7
+};
 constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in the stacked gated weight
 
 // Pipeline stage of the 2:4 GEMM (SPARSE) and of the dense GEMM of the dense
@@ -128,7 +135,9 @@ constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM addres
 // inputs.
 __host__ __device__ constexpr int epi_bufs(int epi) {
   return epi == kEpiWgrad ? 0
-                          : epi == kEpiNone ? 1 : (epi == kEpiGelu || epi == kEpiGeglu) ? 2 : (epi == kEpiDgelu ? 3 : 6);
+                          : epi == kEpiNone ? 1
+                          : (epi == kEpiGelu || epi == kEpiGeglu || epi == kEpiGeluDeriv) ? 2
+                          : ((epi == kEpiDgelu || epi == kEpiMulAux) ? 3 : 6);
 }
 // The wgrad variant keeps 8 KB unused after its barriers, so that its MN-major
 // B reads stay inside the allocation under any reading of the descriptor strides.
@@ -137,6 +146,10 @@ __host__ __device__ constexpr int pair_smem_bytes() {
   return PairGeom<SPARSE, EPI>::kStages * PairGeom<SPARSE, EPI>::kStageBytes + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
          kPairBarBytes + 1024 + (EPI == kEpiWgrad ? 8192 : 0);
 }
+static_assert(pair_smem_bytes<true, kEpiMulAux>() == pair_smem_bytes<true, kEpiDgelu>() &&
+                  pair_smem_bytes<false, kEpiMulAux>() == pair_smem_bytes<false, kEpiDgelu>() &&
+                  pair_smem_bytes<true, kEpiGeluDeriv>() == pair_smem_bytes<true, kEpiGelu>(),
+              "the derivative-saving pair stages like GELU / GELU'");
 static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<false, kEpiDgelu>() <= 232448 &&
                   pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448 &&
                   pair_smem_bytes<true, kEpiWgrad>() <= 232448,
@@ -368,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(drain, 1);
-    if (EPI == kEpiDgelu || EPI == kEpiDgeglu)
+    if (EPI == kEpiDgelu || EPI == kEpiDgeglu || EPI == kEpiMulAux)
       for (int i = 0; i < 2 * kEpiWarps; ++i) mbar_init(&aux_bars[i], 1);
     *s_abort = 0;
     fence_mbarrier_init();
@@ -619,7 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int grp = ew >> 2;
     const int q = warp & 3;
     constexpr int kMaxChunksPerWarp = (kPairChunks + kEpiGroups - 1) / kEpiGroups;
-    constexpr bool kPre = EPI == kEpiDgelu || EPI == kEpiDgeglu;       // TMA-loaded pre-activations
+    constexpr bool kPre = EPI == kEpiDgelu || EPI == kEpiDgeglu || EPI == kEpiMulAux;   // TMA-loaded aux tiles
     constexpr int kPreBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
     constexpr int kOutBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
     // Staging of warp ew: [out][aux] (GELU, gated), [out][pre 0][pre 1] (gradients).
@@ -748,7 +761,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         } else {
           uint32_t hx[2][4];
-          if (EPI == kEpiDgelu) {
+          if (EPI == kEpiDgelu || EPI == kEpiMulAux) {
             ldmatrix_x4_trans(pre_src + lane_off0, hx[0]);
             ldmatrix_x4_trans(pre_src + lane_off1, hx[1]);
           }
@@ -763,6 +776,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               if (EPI == kEpiGelu) {
                 y = gelu2(acc);
                 pa[h][i] = pack2<BF16>(acc.x, acc.y);
+              } else if (EPI == kEpiGeluDeriv) {
+                float2 gp;
+                gelu_and_grad2(acc, y, gp);
+                pa[h][i] = pack2<BF16>(gp.x, gp.y);
+              } else if (EPI == kEpiMulAux) {
+                float2 hv;
+                unpack2<BF16>(hx[h][i], hv.x, hv.y);
+                y = __fmul2_rn(acc, hv);
               } else if (EPI == kEpiDgelu) {
                 float2 hv;
                 unpack2<BF16>(hx[h][i], hv.x, hv.y);
@@ -773,7 +794,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);
           stmatrix_x4_trans(stg_u32 + lane_off1, po[1]);
-          if (EPI == kEpiGelu) {
+          if (EPI == kEpiGelu || EPI == kEpiGeluDeriv) {
             stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off0, pa[0]);
             stmatrix_x4_trans(stg_u32 + kEpiBufBytes + lane_off1, pa[1]);
           }
@@ -786,7 +807,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0 && m0 < M) {   // the TMA unit clips columns past the tensor and tokens >= T
           tma_store_2d(&tm_out, stg, out_col(m0), t0);
-          if (EPI == kEpiGelu || EPI == kEpiGeglu) tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
+          if (EPI == kEpiGelu || EPI == kEpiGeglu || EPI == kEpiGeluDeriv)
+            tma_store_2d(&tm_aux, stg + kEpiBufBytes, m0, t0);
           bulk_commit_group();
         }
         if (kPre && k + 2 < nk) pre_load(pre_col(m0), t0 + 2 * kEpiGroups * kEpiTokens);

@@ -193,6 +193,16 @@ __device__ __noinline__ uint32_t search_block(const uint32_t (&w)[4][2], const u
 constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 
 __device__ const PackedTables g_packed = make_packed_tables();
+__device__ const SelectTables g_select = make_select_tables();
+// 1, read at run time: multiply-adds by it keep integer additions on the FMA
+// pipe (the ALU pipe, half as wide, carries the maxima and the bit work).
+__device__ uint32_t g_one = 1u;
+
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 
 // Packed-key search of one block, exact when the block's nonzero magnitudes span
 // at most 10 binades (fp16) or 13 (bf16); otherwise returns kNeedsExact.
@@ -200,16 +210,19 @@ __device__ const PackedTables g_packed = make_packed_tables();
 //     magnitude below 2^21 U (U = 2^-24 2^sh for fp16, 2^-133 2^sh for bf16),
 //     which is exact when every nonzero |w| is a multiple of U, i.e. when its
 //     exponent field is at least sh + 1 (checked on the raw bits with 16-bit
-//     lane max/min; zeros pass).  The conversion is one fp32 FMA,
-//     |w| 2^(-log2 U) + 2^23, whose low 23 bits hold v; shifted left by 8 the
-//     2^23 offset leaves the word and v << 8 remains.
+//     lane max/min; zeros pass).
+//   * Pair sums on the FMA pipe: f = |w_a| / U + 2^23 and f + |w_b| / U are exact
+//     fp32 integers (below 2^24), whose low 23 bits hold v_a and v_a + v_b; one
+//     integer multiply-add turns the word into (v_a + v_b) << 8 plus the row's
+//     tie share (the 2^23 offset leaves the word).
 //   * A pattern's key is sum(v) << 8 plus the tie field of PackedTables, all
 //     below 2^32 (a sum of eight is below 2^24), so one unsigned max picks the
 //     largest exact sum and, among equal sums, the lowest pattern index.
 //   * The max over the 90 patterns is the same dynamic program over column-count
 //     states: per state, the best top and bottom combo, then the best total.
 template <bool BF16>
-__device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2], const uint8_t *__restrict__ decode) {
+__device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2], const uint8_t *__restrict__ decode,
+                                                        uint32_t one) {
   constexpr PackedTables PT = make_packed_tables();
   constexpr int kMant = BF16 ? 7 : 10;               // explicit significand bits
   uint32_t a[8];
@@ -230,18 +243,29 @@ __device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2
   const bool exact = (sh == 0 || mn + 1u >= ((uint32_t)(sh + 1) << kMant)) && E <= 127;
   if (!exact) return kNeedsExact;
   const float scale = __uint_as_float((uint32_t)(E + 127) << 23);
+  const uint32_t k256 = one << 8;
   uint32_t P[4][6];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    uint32_t v[4];
+    float x[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t h = (a[2 * i + (j >> 1)] >> ((j & 1) << 4)) & 0xFFFFu;
-      const float x = BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
-      v[j] = __float_as_uint(fmaf(x, scale, 8388608.0f)) << 8;
+    for (int hw = 0; hw < 2; ++hw) {
+      const uint32_t m2 = a[2 * i + hw];
+      if (BF16) {
+        x[2 * hw] = __uint_as_float(imad(m2, one << 16, 0u));
+        x[2 * hw + 1] = __uint_as_float(m2 & 0xFFFF0000u);
+      } else {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&m2));
+        x[2 * hw] = f.x;
+        x[2 * hw + 1] = f.y;
+      }
     }
+    const float f0 = fmaf(x[0], scale, 8388608.0f), f1 = fmaf(x[1], scale, 8388608.0f);
+    const float f2 = fmaf(x[2], scale, 8388608.0f);
+    const float ps[6] = {fmaf(x[1], scale, f0), fmaf(x[2], scale, f0), fmaf(x[3], scale, f0),
+                         fmaf(x[2], scale, f1), fmaf(x[3], scale, f1), fmaf(x[3], scale, f2)};
 #pragma unroll
-    for (int q = 0; q < 6; ++q) P[i][q] = v[pair_lo(q)] + v[pair_hi(q)];
+    for (int q = 0; q < 6; ++q) P[i][q] = imad(__float_as_uint(ps[q]), k256, pair_tie(i, q));
   }
   uint32_t best = 0;
 #pragma unroll
@@ -251,62 +275,16 @@ __device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2
     for (int i = 0; i < 6; ++i) {
       if (i < PT.ntop[st]) {
         const int c = PT.top[st][i];
-        tb = max(tb, P[0][c / 6] + P[1][c % 6] + (uint32_t)PT.tie_top[c]);
+        tb = max(tb, imad(P[0][c / 6], one, P[1][c % 6]));
       }
       if (i < PT.nbot[st]) {
         const int b = PT.bot[st][i];
-        bb = max(bb, P[2][b / 6] + P[3][b % 6] + (uint32_t)PT.tie_bot[b]);
+        bb = max(bb, P[2][b / 6] + P[3][b % 6]);
       }
     }
     best = max(best, tb + bb);
   }
   return decode[best & 0xFFu];
-}
-
-// Fast path of the search, on fp64 sums.  fp16: every |w| is an integer
-// multiple of 2^-24 below 2^17, so a sum of eight needs at most 44
-// significant bits and fp64 holds every partial sum exactly: the search is
-// exact for every block.  bf16: 8-bit significands and 3 carry bits fit the
-// 53-bit fp64 significand when the block's smallest nonzero magnitude is at
-// least its largest times 2^-42 (when that bound underflows fp32, every
-// magnitude is below 2^-84 and the sums still fit above the 2^-133
-// subnormal step); blocks that fail return kNeedsExact for the integer search.
-// Ranks: within a column-count state the first combo (lowest rank) reaching
-// the state's maximum wins (strict >); across states the smallest
-// (top rank, bottom rank) among the states reaching the global maximum wins.
-template <bool BF16>
-__device__ __forceinline__ uint32_t search_block_fast(const uint32_t (&w)[4][2], const uint8_t *index_tab) {
-  float v[16];
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t h = (w[c >> 2][(c >> 1) & 1] >> ((c & 1) << 4)) & 0x7FFFu;
-    v[c] = BF16 ? __uint_as_float(h << 16) : __half2float(__ushort_as_half((unsigned short)h));
-  }
-  if (BF16) {
-    float vmax = v[0], vmin = v[0] > 0.0f ? v[0] : __int_as_float(0x7F800000);
-#pragma unroll
-    for (int c = 1; c < 16; ++c) {
-      vmax = fmaxf(vmax, v[c]);
-      vmin = fminf(vmin, v[c] > 0.0f ? v[c] : __int_as_float(0x7F800000));
-    }
-    if (!(vmin >= vmax * 0x1p-42f)) return kNeedsExact;
-  }
-  double d[16];
-#pragma unroll
-  for (int c = 0; c < 16; ++c) d[c] = (double)v[c];
-  const uint32_t key = dp_state_key<double>(d);
-  return index_tab[(key >> 6) * 36 + (key & 63)];
-}
-
-__device__ __forceinline__ uint32_t half_of(const uint32_t (&row)[4], int blk, uint32_t k) {
-  const uint32_t wd = (k & 2) ? row[2 * blk + 1] : row[2 * blk];
-  return (wd >> ((k & 1) << 4)) & 0xFFFFu;
-}
-
-__device__ __forceinline__ uint32_t pick_row(const uint32_t (&w)[4][4], uint32_t i, int word) {
-  const uint32_t a = (i & 1) ? w[1][word] : w[0][word];
-  const uint32_t b = (i & 1) ? w[3][word] : w[2][word];
-  return (i & 2) ? b : a;
 }
 
 // Physical word of (W column c_local, block row br_local) in the transposed
@@ -342,19 +320,20 @@ __device__ __forceinline__ void load_unit(const uint16_t *__restrict__ W, int64_
   }
 }
 
-constexpr int kTile = 64;           // quadrant of a chunk: 64 rows x 64 columns
+constexpr int kTile = 64;           // quadrant of a metadata chunk: 64 rows x 64 columns
 constexpr int kTileBlocks = kTile / 4;
 constexpr int kQuadThreads = 128;   // one unit (4 rows x 8 columns = two blocks) per thread
 constexpr int kChunk = 2 * kTile;   // one tensor-core metadata chunk: 128 x 128
-#ifndef SP24_MASK_QUADS
-#define SP24_MASK_QUADS 2
+// A CTA tile is the two quadrants of one column half of a chunk: 128 rows x 64
+// columns of W, 256 threads (two CTA tiles side by side make a chunk).
+constexpr int kMaskThreads = 2 * kQuadThreads;
+constexpr int kMaskCtaCols = kTile;
+constexpr int kMaskTileBytes = kChunk * kTile * 2;   // 16 KB of W per CTA tile
+#ifndef SP24_MASK_CTAS_PER_SM
+#define SP24_MASK_CTAS_PER_SM 3
 #endif
-// Quadrants per CTA: 4 (the whole chunk) or 2 (128 rows x 64 columns, the CTAs of
-// one chunk side by side).
-constexpr int kMaskQuads = SP24_MASK_QUADS;
-constexpr int kMaskThreads = kMaskQuads * kQuadThreads;
-constexpr int kMaskCtaCols = kMaskQuads == 4 ? kChunk : kTile;   // W columns per CTA
-static_assert(kMaskQuads == 2 || kMaskQuads == 4, "a CTA covers half a chunk or a whole one");
+constexpr int kMaskCtasPerSm = SP24_MASK_CTAS_PER_SM;
+constexpr uint64_t kMaskDrainBudget = 1ull << 26;
 
 // Nibble (4 * shift) of each of the four 16-bit codes in v, packed 4 bits apart.
 __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
@@ -363,61 +342,110 @@ __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
   return (lo & 0xFu) | ((lo >> 12) & 0xF0u) | ((hi & 0xFu) << 8) | ((hi >> 4) & 0xF000u);
 }
 
-// Regions of 128x128 of W (one 2048-byte tensor-core metadata chunk of each
-// orientation) in quadrants of 64x64, 128 threads each; a CTA takes kMaskQuads
-// of them (the two quadrants of one column half, or all four).  Thread t of a
-// quadrant owns the unit at unit column t%8 and block row t/8.  Rows and
-// columns past the matrix get the padding code in the metadata.
+// Shared memory of one CTA tile.
+template <bool SEARCH, bool COMPRESS>
+struct MaskSmem {
+  uint8_t idx[2][kTileBlocks][kTileBlocks];
+  __align__(8) uint16_t rc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // row codes, [br][bc]
+  __align__(8) uint16_t cc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // column codes, [bc][br]
+  __align__(16) uint32_t vcol[COMPRESS ? 2 : 1][COMPRESS ? kTile * 16 : 4];
+  uint16_t queue[SEARCH ? 2 * kTileBlocks * kTileBlocks : 2];
+  int qn;
+};
+
+// Where a CTA tile's weights come from: straight from global memory (row pitch
+// ldw), or from a 128 x 64 tile that the tensor memory accelerator placed in
+// shared memory (zeros outside the matrix).  Coordinates are relative to the
+// CTA tile's first row and column.
+struct GlobalTileSrc {
+  const uint16_t *__restrict__ w;   // W at the CTA tile's origin
+  int64_t ldw;
+  bool vec16;                       // rows 16-byte aligned: one 128-bit load per unit row
+  __device__ __forceinline__ void unit(int r, int c, bool ok0, bool ok1, uint32_t (&v)[4][4]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[i][0] = v[i][1] = v[i][2] = v[i][3] = 0;
+      const uint16_t *src = w + (r + i) * ldw + c;
+      if (ok1 && vec16) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(src));
+        v[i][0] = q.x; v[i][1] = q.y; v[i][2] = q.z; v[i][3] = q.w;
+      } else if (ok1) {
+        const uint2 q0 = __ldg(reinterpret_cast<const uint2 *>(src));
+        const uint2 q1 = __ldg(reinterpret_cast<const uint2 *>(src + 4));
+        v[i][0] = q0.x; v[i][1] = q0.y; v[i][2] = q1.x; v[i][3] = q1.y;
+      } else if (ok0) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(src));
+        v[i][0] = q.x; v[i][1] = q.y;
+      }
+    }
+  }
+  __device__ __forceinline__ void block(int r, int c, uint32_t (&v)[4][2]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint2 q = __ldg(reinterpret_cast<const uint2 *>(w + (r + i) * ldw + c));
+      v[i][0] = q.x; v[i][1] = q.y;
+    }
+  }
+};
+
+struct SharedTileSrc {
+  const uint16_t *s;   // [128 rows][64 columns]
+  __device__ __forceinline__ void unit(int r, int c, bool, bool, uint32_t (&v)[4][4]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 q = *reinterpret_cast<const uint4 *>(s + (r + i) * kTile + c);
+      v[i][0] = q.x; v[i][1] = q.y; v[i][2] = q.z; v[i][3] = q.w;
+    }
+  }
+  __device__ __forceinline__ void block(int r, int c, uint32_t (&v)[4][2]) const {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint2 q = *reinterpret_cast<const uint2 *>(s + (r + i) * kTile + c);
+      v[i][0] = q.x; v[i][1] = q.y;
+    }
+  }
+};
+
+// One CTA tile: rows 128 cy .. +127, columns 128 cx + 64 kh .. +63 of W, the
+// quadrants rh = 0, 1 of column half kh of metadata chunk (cy, cx).  Thread t
+// of quadrant rh = t / 128 owns the unit at unit column t%8 and block row
+// (t%128)/8.  Rows and columns past the matrix get the padding code in the
+// metadata.
 //   SEARCH:   compute the mask (else read it from idx)
 //   COMPRESS: write the compressed orientations whose pointers are non-null
 //             (values + tensor-core metadata)
-//   FLIP:     add the number of mask bits that differ from idx_prev to *flip_count
+//   FLIP:     add the number of mask bits that differ from idx_prev to `flips`
 // Search: every block takes the packed-key search; blocks it cannot certify
 // (magnitudes spread over more than 10 binades for fp16, 13 for bf16) are queued
 // in shared memory and, after a barrier, searched exactly by the first threads
-// of the CTA, so the slow path costs about one warp pass per chunk.
-template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_tile_kernel(
-    const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
-    const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
-    uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
-    uint8_t *__restrict__ meta_col) {
-  __shared__ uint8_t s_idx[kMaskQuads][kTileBlocks][kTileBlocks];
-  __shared__ __align__(8) uint16_t s_rc[COMPRESS ? kMaskQuads : 1][kTileBlocks][kTileBlocks];   // row codes
-  __shared__ __align__(8) uint16_t s_cc[COMPRESS ? kMaskQuads : 1][kTileBlocks][kTileBlocks];   // [bc][br]
-  __shared__ __align__(16) uint32_t s_vcol[COMPRESS ? kMaskQuads : 1][COMPRESS ? kTile * 16 : 4];
-  __shared__ uint16_t s_queue[SEARCH ? kMaskQuads * kTileBlocks * kTileBlocks : 2];
-  __shared__ int s_qn;
-  __shared__ unsigned long long s_flip;
-
+// of the CTA, so the slow path costs about one warp pass per tile.  The body
+// has three CTA barriers; the caller separates consecutive tiles with a fourth.
+template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP, typename Src>
+__device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_t C, uint32_t cy, uint32_t cx,
+                                               int kh, uint32_t chunks_x, uint32_t chunks_y,
+                                               uint8_t *__restrict__ idx, const uint8_t *__restrict__ idx_prev,
+                                               unsigned &flips, uint16_t *__restrict__ vals_row,
+                                               uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
+                                               uint8_t *__restrict__ meta_col, MaskSmem<SEARCH, COMPRESS> &sm) {
   const int tid = threadIdx.x;
-  const int qd = tid >> 7, lt = tid & (kQuadThreads - 1);
-  const int rh = kMaskQuads == 4 ? qd >> 1 : qd;
-  const int kh = kMaskQuads == 4 ? qd & 1 : (int)(blockIdx.x & 1);
-  const uint32_t chunk_x = kMaskQuads == 4 ? blockIdx.x : blockIdx.x >> 1;
-  const uint32_t chunks_x = kMaskQuads == 4 ? gridDim.x : gridDim.x >> 1;
+  const int rh = tid >> 7, lt = tid & (kQuadThreads - 1);
   const uint16_t *bits_tab = g_tables.bits;
-  const uint8_t *index_tab = g_tables.index;
-  if (tid == 0) { s_flip = 0; s_qn = 0; }
-  pdl_launch_dependents();
-  pdl_wait();
-
-  const int64_t tile_r = (int64_t)blockIdx.y * kChunk + kTile * rh;
-  const int64_t tile_c = (int64_t)chunk_x * kChunk + kTile * kh;
+  const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
+  const int64_t tile_r0 = (int64_t)cy * kChunk, tile_c0 = (int64_t)cx * kChunk + kTile * kh;
+  const int64_t tile_r = tile_r0 + kTile * rh;
   const int64_t bcols = C >> 2;
   const int uc = lt & 7;
   const int br = lt >> 3;
-  const int64_t r0 = tile_r + 4 * br;
-  const int64_t c0 = tile_c + 8 * uc;
+  const int lr = kTile * rh + 4 * br, lc = 8 * uc;   // the unit, relative to the CTA tile
+  const int64_t r0 = tile_r0 + lr;
+  const int64_t c0 = tile_c0 + lc;
   const bool row_ok = r0 < R;
   const bool ok0 = row_ok && c0 + 4 <= C;
   const bool ok1 = row_ok && c0 + 8 <= C;
-  const bool vec16 = (ldw & 7) == 0;  // rows 16-byte aligned: one 128-bit load per row of a unit
   const int64_t bidx0 = (r0 >> 2) * bcols + (c0 >> 2);
 
-  // Every global load of the thread is issued before the first barrier.
   uint32_t w[4][4];
-  load_unit(W, ldw, r0, c0, R, C, vec16, w);
+  src.unit(lr, lc, ok0, ok1, w);
   uint32_t prev[2] = {0, 0}, given[2] = {kPadIndex, kPadIndex};
   if (FLIP) {
     if (ok0) prev[0] = idx_prev[bidx0];
@@ -427,7 +455,6 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
     if (ok0) given[0] = idx[bidx0];
     if (ok1) given[1] = idx[bidx0 + 1];
   }
-  __syncthreads();
 
   // Phase 1: search (SEARCH), or take the given mask (!SEARCH).
   uint32_t p[2];
@@ -439,42 +466,36 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
       uint32_t blk[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
-      p[b] = search_block_packed<BF16>(blk, g_packed.decode);
+      p[b] = search_block_packed<BF16>(blk, g_packed.decode, one);
       if (p[b] == kNeedsExact) {
-        const int slot = atomicAdd(&s_qn, 1);
-        s_queue[slot] = (uint16_t)((qd << 8) | (br << 4) | (2 * uc + b));
+        const int slot = atomicAdd(&sm.qn, 1);
+        sm.queue[slot] = (uint16_t)((rh << 8) | (br << 4) | (2 * uc + b));
       }
     }
-    if (SEARCH) s_idx[qd][br][2 * uc + b] = (uint8_t)p[b];
+    if (SEARCH) sm.idx[rh][br][2 * uc + b] = (uint8_t)p[b];
   }
 
   // Phase 1b: the exact search of the queued blocks, entry k by thread k.
   if (SEARCH) {
     __syncthreads();
-    const int qn = s_qn;
+    const int qn = sm.qn;
     if (qn > 0) {
       for (int k = tid; k < qn; k += kMaskThreads) {
-        const int id = s_queue[k];
+        const int id = sm.queue[k];
         const int q = id >> 8, qbr = (id >> 4) & 15, qbc = id & 15;
-        const int qrh = kMaskQuads == 4 ? q >> 1 : q, qkh = kMaskQuads == 4 ? q & 1 : kh;
-        const uint16_t *src = W + ((int64_t)blockIdx.y * kChunk + kTile * qrh + 4 * qbr) * ldw +
-                              (int64_t)chunk_x * kChunk + kTile * qkh + 4 * qbc;
         uint32_t blk[4][2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src + i * ldw));
-          blk[i][0] = v.x; blk[i][1] = v.y;
-        }
-        s_idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, index_tab, bits_tab);
+        src.block(kTile * q + 4 * qbr, 4 * qbc, blk);
+        sm.idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, g_tables.index, bits_tab);
       }
       __syncthreads();
 #pragma unroll
-      for (int b = 0; b < 2; ++b) p[b] = s_idx[qd][br][2 * uc + b];
+      for (int b = 0; b < 2; ++b) p[b] = sm.idx[rh][br][2 * uc + b];
     }
   }
 
-  // Phase 2: outputs of this thread's two blocks.
-  unsigned flips = 0;
+  // Phase 2: outputs of this thread's two blocks.  The unit is read again
+  // rather than kept live across the exact search's call.
+  if (SEARCH && COMPRESS) src.unit(lr, lc, ok0, ok1, w);
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     const bool ok = b ? ok1 : ok0;
@@ -487,19 +508,26 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
     for (int b = 0; b < 2; ++b) {
       rc[b] = g_tables.rowcode[p[b]];
       cc[b] = g_tables.colcode[p[b]];
-      s_rc[qd][br][2 * uc + b] = (uint16_t)rc[b];
-      s_cc[qd][2 * uc + b][br] = (uint16_t)cc[b];
+      sm.rc[rh][br][2 * uc + b] = (uint16_t)rc[b];
+      sm.cc[rh][2 * uc + b][br] = (uint16_t)cc[b];
     }
     if (ok0) {
-      // Forward operand: kept values of each row, in column order.
+      // Forward operand: kept values of each row, in column order (one byte
+      // permutation of the row's four values per row and block).
       if (vals_row) {
+        uint2 rsel[2];
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const uint64_t t = g_select.row[p[b]];
+          rsel[b] = make_uint2((uint32_t)t, (uint32_t)(t >> 32));
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           uint32_t packed[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
-            const uint32_t nib = (rc[b] >> (4 * i)) & 0xFu;
-            packed[b] = half_of(w[i], b, nib & 3u) | (half_of(w[i], b, nib >> 2) << 16);
+            const uint32_t sel = (i < 2 ? rsel[b].x : rsel[b].y) >> (16 * (i & 1));
+            packed[b] = __byte_perm(w[i][2 * b], w[i][2 * b + 1], sel);
           }
           uint16_t *dst = vals_row + (r0 + i) * (C >> 1) + (c0 >> 1);
           if (ok1) *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
@@ -507,26 +535,25 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
         }
       }
       // Input-gradient operand: kept values of each column, staged transposed.
+      // Column j's four values as two words (rows 0-1, rows 2-3), then one byte
+      // permutation picks its kept pair.
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
+        const uint64_t t = g_select.col[p[b]];
+        const uint2 csel = make_uint2((uint32_t)t, (uint32_t)(t >> 32));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint32_t nib = (cc[b] >> (4 * j)) & 0xFu;
-          const int word = 2 * b + (j >> 1);
-          const uint32_t lo = (pick_row(w, nib & 3u, word) >> ((j & 1) << 4)) & 0xFFFFu;
-          const uint32_t hi = (pick_row(w, nib >> 2, word) >> ((j & 1) << 4)) & 0xFFFFu;
-          s_vcol[qd][vcol_word(8 * uc + 4 * b + j, br)] = lo | (hi << 16);
+          const int wi = 2 * b + (j >> 1);
+          const uint32_t half = (j & 1) ? 0x7632u : 0x5410u;
+          const uint32_t c01 = __byte_perm(w[0][wi], w[1][wi], half);
+          const uint32_t c23 = __byte_perm(w[2][wi], w[3][wi], half);
+          const uint32_t sel = (j < 2 ? csel.x : csel.y) >> (16 * (j & 1));
+          sm.vcol[rh][vcol_word(8 * uc + 4 * b + j, br)] = __byte_perm(c01, c23, sel);
         }
       }
     }
   }
-
-  if (FLIP) {
-    const unsigned warp_sum = __reduce_add_sync(0xFFFFFFFFu, flips);
-    if ((tid & 31) == 0 && warp_sum) atomicAdd(&s_flip, (unsigned long long)warp_sum);
-  }
-  if (COMPRESS || FLIP) __syncthreads();
-  if (FLIP && tid == 0 && s_flip) atomicAdd(flip_count, s_flip);
+  if (COMPRESS) __syncthreads();
 
   if (COMPRESS) {
     // Transposed values: W column c (a row of W^T) holds 32 kept values per quadrant.
@@ -535,12 +562,12 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
     for (int k = 0; k < (kTile * 4) / kQuadThreads; ++k) {
       const int id = lt + kQuadThreads * k;
       const int c_local = id >> 2, q = id & 3;
-      if (vals_col && tile_c + c_local < C && tile_r + 16 * q + 16 <= R) {
+      if (vals_col && tile_c0 + c_local < C && tile_r + 16 * q + 16 <= R) {
         const uint4 v =
-            *reinterpret_cast<const uint4 *>(&s_vcol[qd][c_local * 16 + (((q ^ (c_local >> 3)) & 3) << 2)]);
+            *reinterpret_cast<const uint4 *>(&sm.vcol[rh][c_local * 16 + (((q ^ (c_local >> 3)) & 3) << 2)]);
         const bool swap = (c_local >> 5) & 1;
         const uint4 o = swap ? make_uint4(v.z, v.w, v.x, v.y) : v;
-        *reinterpret_cast<uint4 *>(vals_col + (tile_c + c_local) * half_rows + (tile_r >> 1) + 8 * q) = o;
+        *reinterpret_cast<uint4 *>(vals_col + (tile_c0 + c_local) * half_rows + (tile_r >> 1) + 8 * q) = o;
       }
     }
     // Metadata: one 2048-byte chunk per 128x128 region and orientation.  Lane L,
@@ -555,18 +582,135 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskQuads == 4 ? 2 : 3) mask_ti
     const int gq = kx * 8 + ((lq >> 3) & 1) * 4;     // first of four groups, in blocks of the quadrant
     const int shift = m_lo & 3;
     if (meta_row) {
-      const uint2 a = *reinterpret_cast<const uint2 *>(&s_rc[qd][m_lo >> 2][gq]);
-      const uint2 c = *reinterpret_cast<const uint2 *>(&s_rc[qd][(m_lo >> 2) + 2][gq]);
+      const uint2 a = *reinterpret_cast<const uint2 *>(&sm.rc[rh][m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&sm.rc[rh][(m_lo >> 2) + 2][gq]);
       const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
-      const size_t chunk = (size_t)blockIdx.y * chunks_x + chunk_x;
+      const size_t chunk = (size_t)cy * chunks_x + cx;
       *reinterpret_cast<uint32_t *>(meta_row + chunk * 2048 + (64 * rh + lq) * 16 + 4 * (2 * kh + kx)) = word;
     }
     if (meta_col) {
-      const uint2 a = *reinterpret_cast<const uint2 *>(&s_cc[qd][m_lo >> 2][gq]);
-      const uint2 c = *reinterpret_cast<const uint2 *>(&s_cc[qd][(m_lo >> 2) + 2][gq]);
+      const uint2 a = *reinterpret_cast<const uint2 *>(&sm.cc[rh][m_lo >> 2][gq]);
+      const uint2 c = *reinterpret_cast<const uint2 *>(&sm.cc[rh][(m_lo >> 2) + 2][gq]);
       const uint32_t word = gather_nibbles(a, shift) | (gather_nibbles(c, shift) << 16);
-      const size_t chunk = (size_t)chunk_x * gridDim.y + blockIdx.y;
+      const size_t chunk = (size_t)cx * chunks_y + cy;
       *reinterpret_cast<uint32_t *>(meta_col + chunk * 2048 + (64 * kh + lq) * 16 + 4 * (2 * rh + kx)) = word;
+    }
+  }
+}
+
+// Adds the CTA's flip count to *flip_count (one global atomic per CTA).
+__device__ __forceinline__ void mask_flip_flush(unsigned flips, unsigned long long *s_flip,
+                                                unsigned long long *__restrict__ flip_count) {
+  const unsigned warp_sum = __reduce_add_sync(0xFFFFFFFFu, flips);
+  if ((threadIdx.x & 31) == 0 && warp_sum) atomicAdd(s_flip, (unsigned long long)warp_sum);
+  __syncthreads();
+  if (threadIdx.x == 0 && *s_flip) atomicAdd(flip_count, *s_flip);
+}
+
+// One CTA per CTA tile, W read from global memory: the kernel for row pitches
+// that the tensor memory accelerator cannot take (ldw not a multiple of 8).
+template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
+__global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_tile_kernel(
+    const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
+    const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
+    uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
+    uint8_t *__restrict__ meta_col) {
+  __shared__ MaskSmem<SEARCH, COMPRESS> sm;
+  __shared__ unsigned long long s_flip;
+  if (threadIdx.x == 0) { s_flip = 0; sm.qn = 0; }
+  pdl_launch_dependents();
+  pdl_wait();
+  const uint32_t cy = blockIdx.y, cx = blockIdx.x >> 1, chunks_x = gridDim.x >> 1;
+  const int kh = (int)(blockIdx.x & 1);
+  const GlobalTileSrc src{W + (int64_t)cy * kChunk * ldw + (int64_t)cx * kChunk + kTile * kh, ldw, (ldw & 7) == 0};
+  __syncthreads();
+  unsigned flips = 0;
+  mask_tile_body<BF16, SEARCH, COMPRESS, FLIP>(src, R, C, cy, cx, kh, chunks_x, gridDim.y, idx, idx_prev, flips,
+                                               vals_row, meta_row, vals_col, meta_col, sm);
+  if (FLIP) mask_flip_flush(flips, &s_flip, flip_count);
+}
+
+// Persistent form: CTA b takes CTA tiles b, b + gridDim.x, ... (column halves
+// fastest, then chunks along a row of chunks, then down the rows), with two
+// 16 KB shared buffers of W: the tensor memory accelerator loads tile i + 2
+// into a buffer as soon as the CTA has finished reading tile i from it, so the
+// loads of the next two tiles overlap the work on this one.  Every wait is
+// bounded; on a timeout the CTA records the error, lets its copies land and exits.
+template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
+__global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_stream_kernel(
+    const __grid_constant__ CUtensorMap tm_w, int64_t R, int64_t C, uint8_t *__restrict__ idx,
+    const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
+    uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
+    uint8_t *__restrict__ meta_col, uint64_t wait_budget) {
+  __shared__ __align__(128) uint16_t s_w[2][kChunk * kTile];
+  __shared__ MaskSmem<SEARCH, COMPRESS> sm;
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ unsigned long long s_flip;
+  __shared__ volatile int s_abort;
+  const int tid = threadIdx.x;
+  const uint32_t chunks_x = (uint32_t)((C + kChunk - 1) / kChunk);
+  const uint32_t chunks_y = (uint32_t)((R + kChunk - 1) / kChunk);
+  const int64_t ntiles = 2ll * chunks_x * chunks_y;
+  auto tile_xy = [&](int64_t t, uint32_t &cy, uint32_t &cx, int &kh) {
+    kh = (int)(t & 1);
+    cx = (uint32_t)((t >> 1) % chunks_x);
+    cy = (uint32_t)((t >> 1) / chunks_x);
+  };
+  auto issue = [&](int64_t t, int buf) {
+    uint32_t cy, cx;
+    int kh;
+    tile_xy(t, cy, cx, kh);
+    mbar_arrive_expect_tx(&s_full[buf], kMaskTileBytes);
+    tma_load_2d(s_w[buf], &tm_w, &s_full[buf], (int)(cx * kChunk + kTile * kh), (int)(cy * kChunk));
+  };
+  if (tid == 0) {
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    fence_mbarrier_init();
+    prefetch_tensormap(&tm_w);
+    s_flip = 0;
+    s_abort = 0;
+    sm.qn = 0;
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
+  int64_t issued = 0, it = 0;   // copies issued (by thread 0) and tiles consumed
+  if (tid == 0) {
+    for (int k = 0; k < 2; ++k)
+      if ((int64_t)blockIdx.x + (int64_t)k * gridDim.x < ntiles) {
+        issue((int64_t)blockIdx.x + (int64_t)k * gridDim.x, k);
+        ++issued;
+      }
+  }
+  unsigned flips = 0;
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    const int buf = (int)(it & 1);
+    mbar_wait_bounded(&s_full[buf], (uint32_t)((it >> 1) & 1), wait_budget, &s_abort);
+    __syncthreads();
+    if (s_abort) break;
+    uint32_t cy, cx;
+    int kh;
+    tile_xy(t, cy, cx, kh);
+    const SharedTileSrc src{s_w[buf]};
+    mask_tile_body<BF16, SEARCH, COMPRESS, FLIP>(src, R, C, cy, cx, kh, chunks_x, chunks_y, idx, idx_prev, flips,
+                                                 vals_row, meta_row, vals_col, meta_col, sm);
+    __syncthreads();   // every read of this buffer and of the tile's shared state is done
+    if (tid == 0) {
+      sm.qn = 0;
+      const int64_t nt = t + 2ll * gridDim.x;
+      if (nt < ntiles) {
+        issue(nt, buf);
+        ++issued;
+      }
+    }
+  }
+  if (FLIP) mask_flip_flush(flips, &s_flip, flip_count);
+  // After an abort, let the copies still in flight land before the CTA exits.
+  if (tid == 0 && s_abort) {
+    for (int64_t k = it; k < issued; ++k) {
+      volatile int no_abort = 0;
+      mbar_wait_bounded(&s_full[k & 1], (uint32_t)((k >> 1) & 1), kMaskDrainBudget, &no_abort);
     }
   }
 }

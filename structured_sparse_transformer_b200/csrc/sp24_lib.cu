@@ -231,6 +231,12 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
                              : launch_gemm_pair_t<false, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
     case kEpiDgelu: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
                               : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiGeluDeriv:
+      return bf ? launch_gemm_pair_t<true, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                : launch_gemm_pair_t<false, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiMulAux:
+      return bf ? launch_gemm_pair_t<true, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
+                : launch_gemm_pair_t<false, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
     default: break;
   }
   if (SPARSE) {   // the gated epilogues serve the 2:4 GEMMs
@@ -245,13 +251,21 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
   return SP24_ERR_INVALID_ARG;
 }
 
+// The epilogues each product takes (bit e of the mask allows epilogue e).
+constexpr unsigned kFwdEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_GELU) | (1u << SP24_EPI_GEGLU) |
+                              (1u << SP24_EPI_GELU_DERIV);
+constexpr unsigned kDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) | (1u << SP24_EPI_DGEGLU) |
+                                (1u << SP24_EPI_MUL_AUX);
+constexpr unsigned kDenseEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_GELU) | (1u << SP24_EPI_DGELU) |
+                                (1u << SP24_EPI_GELU_DERIV) | (1u << SP24_EPI_MUL_AUX);
+
 sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
-                          sp24_dtype dt, const void *out, int epi, const void *aux, int allowed_epi) {
+                          sp24_dtype dt, const void *out, int epi, const void *aux, unsigned allowed_epis) {
   if (!B && T > 0) return SP24_ERR_INVALID_ARG;
   if (!vals || !meta || (!out && T > 0)) return SP24_ERR_INVALID_ARG;
   if (T < 0 || Kd <= 0 || M <= 0) return SP24_ERR_INVALID_ARG;
   if (!valid_dtype(dt)) return SP24_ERR_UNSUPPORTED_DTYPE;
-  if (epi != SP24_EPI_NONE && epi != allowed_epi && epi != allowed_epi + 2) return SP24_ERR_INVALID_ARG;
+  if (epi < 0 || epi > 31 || !((allowed_epis >> epi) & 1u)) return SP24_ERR_INVALID_ARG;
   if (epi == SP24_EPI_GEGLU && M % (2 * kGegluGroup)) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (epi != SP24_EPI_NONE && !aux) return SP24_ERR_INVALID_ARG;
   if (Kd % 16 || M % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
@@ -267,9 +281,21 @@ sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
 sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint8_t *idx, const uint8_t *prev,
                           unsigned long long *flip, void *vr, void *mr, void *vc, void *mc, cudaStream_t s) {
-  // CTAs cover whole 128x128 regions (one metadata chunk of each orientation).
+  // CTA tiles cover whole 128x128 regions (one metadata chunk of each orientation).
   const int64_t chunks_x = (C + kChunk - 1) / kChunk, chunks_y = (R + kChunk - 1) / kChunk;
   if (chunks_y > 65535 || chunks_x * (kChunk / kMaskCtaCols) > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ntiles = chunks_x * chunks_y * (kChunk / kMaskCtaCols);
+  CUtensorMap tm;
+  // Persistent form with tensor-memory-accelerator loads of W (row pitch a multiple of 16 bytes).
+  if (ldw % 8 == 0 && C <= INT32_MAX && R <= INT32_MAX &&
+      make_map_2d(&tm, W, (uint64_t)C, (uint64_t)R, (uint64_t)ldw * 2, kMaskCtaCols, kChunk,
+                  CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    const int64_t ctas = (int64_t)sm_count() * kMaskCtasPerSm;
+    const unsigned grid = (unsigned)(ntiles < ctas ? ntiles : ctas);
+    return launch_pdl(mask_stream_kernel<BF16, SEARCH, COMPRESS, FLIP>, dim3(grid), dim3(kMaskThreads), 0, s, tm, R,
+                      C, idx, prev, flip, static_cast<uint16_t *>(vr), static_cast<uint8_t *>(mr),
+                      static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc), (uint64_t)g_wait_budget.load());
+  }
   dim3 grid((unsigned)(chunks_x * (kChunk / kMaskCtaCols)), (unsigned)chunks_y);
   return launch_pdl(mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP>, grid, dim3(kMaskThreads), 0, s,
                     static_cast<const uint16_t *>(W), R, C, ldw, idx, prev, flip, static_cast<uint16_t *>(vr),
@@ -409,7 +435,7 @@ sp24_status sp24_prune_compress(const void *W, sp24_dtype dtype, int64_t rows, i
 
 sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const void *vals_row, const void *meta_row, int64_t N,
                           sp24_dtype dtype, void *Y, sp24_epilogue epi, void *aux, void *stream) {
-  sp24_status st = validate_gemm(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, SP24_EPI_GELU);
+  sp24_status st = validate_gemm(X, T, K, vals_row, meta_row, N, dtype, Y, epi, aux, kFwdEpis);
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;
@@ -419,7 +445,7 @@ sp24_status sp24_gemm_fwd(const void *X, int64_t T, int64_t K, const void *vals_
 sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *vals_col, const void *meta_col,
                             int64_t K, sp24_dtype dtype, void *dX, sp24_epilogue epi, const void *aux,
                             void *stream) {
-  sp24_status st = validate_gemm(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, aux, SP24_EPI_DGELU);
+  sp24_status st = validate_gemm(dY, T, N, vals_col, meta_col, K, dtype, dX, epi, aux, kDgradEpis);
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;
@@ -429,9 +455,7 @@ sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const void *va
 
 sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A, int64_t M, sp24_dtype dtype,
                             void *out, sp24_epilogue epi, void *aux, void *stream) {
-  if (epi != SP24_EPI_NONE && epi != SP24_EPI_GELU && epi != SP24_EPI_DGELU) return SP24_ERR_INVALID_ARG;
-  sp24_status st = validate_gemm(B, T, Kd, A, A, M, dtype, out, epi, aux, epi == SP24_EPI_NONE ? SP24_EPI_GELU : epi);
-  if (st == SP24_OK && epi != SP24_EPI_NONE && epi != SP24_EPI_GELU && epi != SP24_EPI_DGELU) st = SP24_ERR_INVALID_ARG;
+  sp24_status st = validate_gemm(B, T, Kd, A, A, M, dtype, out, epi, aux, kDenseEpis);
   if (st != SP24_OK) return st;
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;

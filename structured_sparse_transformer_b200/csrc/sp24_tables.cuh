@@ -109,21 +109,26 @@ __device__ const PatternTables g_tables = make_pattern_tables();
 
 // Tables of the packed-key search (mask_kernels.cuh, search_block_packed).
 // A pattern's key is (exact sum of its |w|) << 8 plus an 8-bit tie field
-//   tie = (35 - top rank) * 6 + (5 - bottom class rank),
-// where a bottom combo's class rank is its position, in rank order, among the
-// bottom combos that need the same state (at most six).  Among patterns with equal
-// sums the larger tie field is the smaller (top rank, bottom rank), i.e. the lower
-// pattern index, and the field splits into a top part and a bottom part that ride
-// on the combo sums.  decode maps a tie field back to the pattern index.
+//   tie = (35 - top rank) * 6 + (5 - q2),
+// q2 the pair rank of row 2.  Within one column-count state the bottom combos
+// that fit have distinct q2, in the order of their rank, so among patterns with
+// equal sums the larger tie field is the smaller (top rank, bottom rank), i.e.
+// the lower pattern index.  The field is linear in the row pair ranks,
+//   tie = 36 (5 - q0) + 6 (5 - q1) + (5 - q2),
+// so each row's share rides on that row's pair sums (pair_tie).  decode maps a
+// tie field back to the pattern index.
 struct PackedTables {
   uint8_t ntop[kNumStates];      // top combos producing each state
   uint8_t top[kNumStates][6];    // their ranks, ascending
   uint8_t nbot[kNumStates];      // bottom combos needing each state
   uint8_t bot[kNumStates][6];    // their ranks, ascending
-  uint8_t tie_top[36];           // (35 - rank) * 6
-  uint8_t tie_bot[36];           // 5 - class rank
   uint8_t decode[256];           // tie field -> pattern index (kPadIndex where unused)
 };
+
+// Row i's share of the tie field for pair rank q.
+__host__ __device__ constexpr uint32_t pair_tie(int i, int q) {
+  return i == 0 ? 36u * (5 - q) : (i == 1 ? 6u * (5 - q) : (i == 2 ? (uint32_t)(5 - q) : 0u));
+}
 
 __host__ __device__ constexpr PackedTables make_packed_tables() {
   PackedTables t{};
@@ -132,11 +137,9 @@ __host__ __device__ constexpr PackedTables make_packed_tables() {
   for (int c = 0; c < 36; ++c) {
     const int s = pt.top_state[c];
     t.top[s][t.ntop[s]++] = (uint8_t)c;
-    t.tie_top[c] = (uint8_t)((35 - c) * 6);
   }
   for (int b = 0; b < 36; ++b) {
     const int s = pt.bot_state[b];
-    t.tie_bot[b] = (uint8_t)(5 - t.nbot[s]);
     t.bot[s][t.nbot[s]++] = (uint8_t)b;
   }
   for (int i = 0; i < 256; ++i) t.decode[i] = kPadIndex;
@@ -144,8 +147,39 @@ __host__ __device__ constexpr PackedTables make_packed_tables() {
     for (int i = 0; i < t.ntop[s]; ++i)
       for (int k = 0; k < t.nbot[s]; ++k) {
         const int c = t.top[s][i], b = t.bot[s][k];
-        t.decode[t.tie_top[c] + t.tie_bot[b]] = pt.index[c * 36 + b];
+        const uint32_t tie = pair_tie(0, c / 6) + pair_tie(1, c % 6) + pair_tie(2, b / 6) + pair_tie(3, b % 6);
+        t.decode[tie] = pt.index[c * 36 + b];
       }
+  return t;
+}
+
+// Byte selectors of the compression (prmt): for pattern p and row i, the
+// selector that picks the row's two kept 16-bit values, in column order, from
+// the row's four values held as two words (columns 0-1, 2-3); for column j, the
+// selector that picks the column's two kept values, in row order, from the
+// column's four values held as two words (rows 0-1, 2-3).  Four 16-bit
+// selectors per pattern and orientation, row (column) i at bits 16 i.
+struct SelectTables {
+  uint64_t row[256];
+  uint64_t col[256];
+};
+
+__host__ __device__ constexpr uint64_t pair_selector(int lo, int hi) {
+  return (uint64_t)((2 * lo) | ((2 * lo + 1) << 4) | ((2 * hi) << 8) | ((2 * hi + 1) << 12));
+}
+
+__host__ __device__ constexpr SelectTables make_select_tables() {
+  SelectTables t{};
+  const PatternTables pt = make_pattern_tables();
+  for (int p = 0; p < 256; ++p) {
+    t.row[p] = 0;
+    t.col[p] = 0;
+    for (int i = 0; i < 4; ++i) {
+      const int rc = (pt.rowcode[p] >> (4 * i)) & 0xF, cc = (pt.colcode[p] >> (4 * i)) & 0xF;
+      t.row[p] |= pair_selector(rc & 3, rc >> 2) << (16 * i);
+      t.col[p] |= pair_selector(cc & 3, cc >> 2) << (16 * i);
+    }
+  }
   return t;
 }
 
