@@ -6,8 +6,9 @@ W_0 .. W_S of both layers follow W_(t+1) = round(W_t + N(0, 1e-4)) (S = 8 for
 the 1.5B shape), and step t runs
   mask step on W1 and W2 at W_(t+1) (transposable 2:4 search, flip count against
   the mask of W_t, compression of both orientations), forward GEMMs
-  (X -> gelu(X W1m^T) -> H W2m^T), input-gradient GEMMs (dY -> dH with the gelu'
-  epilogue -> dX), masked decay on both weights' gradients (lambda = 6e-5).
+  (X -> gelu(X W1m^T) -> H W2m^T, the first also storing gelu' of its
+  pre-activation), input-gradient GEMMs (dY -> dH = (dY W2m) * gelu' -> dX),
+  masked decay on both weights' gradients (lambda = 6e-5).
 Timed steps cycle through t = 0 .. S-1.  The metric is the dense-equivalent
 FLOPs of the four GEMMs divided by the step time (TFLOP/s); per-kernel times
 give the roofline.  The same JSON line carries the mask-search bandwidth sweep
@@ -231,7 +232,7 @@ class FFNStep:
         for li in range(2):   # the mask of W_0, against which step 0 counts its flips
             sp.sp24_mask_search(self.W[li][0], self.idx[li][0])
         self.H = torch.empty(T, ff, dtype=tdt, device=dev)
-        self.Hpre = torch.empty(T, ff, dtype=tdt, device=dev)
+        self.Gp = torch.empty(T, ff, dtype=tdt, device=dev)   # gelu' of the pre-activation
         self.dH = torch.empty(T, ff, dtype=tdt, device=dev)
         self.Y = torch.empty(T, d, dtype=tdt, device=dev)
         self.dX = torch.empty(T, d, dtype=tdt, device=dev)
@@ -287,11 +288,12 @@ class FFNStep:
             timed("mask_step", lambda li=li, c=c: sp.sp24_mask_step(
                 self.W[li][cur], self.idx[li][cur], self.idx[li][prev], self.flips[t, li:li + 1], *c), stream)
         c1, c2 = self.c
-        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu", self.Hpre), main)
+        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu_deriv", self.Gp),
+              main)
         join()
         timed("gemm_fwd2", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y), main)
         timed("gemm_dgrad2_dgelu",
-              lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "dgelu", self.Hpre), main)
+              lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "mul_aux", self.Gp), main)
         if wgrad:
             # Weight gradients into the gradient buffers, decayed in the same kernels:
             # dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X, then + lambda W where pruned;
@@ -339,9 +341,9 @@ class FFNStep:
         for li in range(2):
             timed("transpose", lambda li=li: sp.sp24_transpose(self.W[li][cur], self.Wt[li]))
         W1, W2 = self.W[0][cur], self.W[1][cur]
-        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu", self.Hpre))
+        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu_deriv", self.Gp))
         timed("gemm_fwd2", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
-        timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "dgelu", self.Hpre))
+        timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "mul_aux", self.Gp))
         timed("transpose_act", lambda: sp.sp24_transpose(self.dY, self.dYt))
         timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dYt, self.G[1]))
         timed("transpose_act", lambda: sp.sp24_transpose(self.dH, self.dHt))

@@ -60,7 +60,11 @@
 
 namespace sp24 {
 
-constexpr int kEpiWarps = 12;                          // epilogue warps: 3 per TMEM lane quadrant
+#ifndef SP24_EPI_WARPS
+#define SP24_EPI_WARPS 12
+#endif
+constexpr int kEpiWarps = SP24_EPI_WARPS;              // epilogue warps: kEpiWarps / 4 per TMEM lane quadrant
+static_assert(kEpiWarps == 8 || kEpiWarps == 12, "two or three epilogue warps per lane quadrant");
 constexpr int kEpiGroups = kEpiWarps / 4;              // warp groups taking alternate chunks
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemE = 2048;                           // metadata chunk (128 rows x 128 columns)

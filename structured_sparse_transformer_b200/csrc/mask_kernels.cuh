@@ -332,7 +332,10 @@ constexpr int kMaskTileBytes = kChunk * kTile * 2;   // 16 KB of W per CTA tile
 #ifndef SP24_MASK_CTAS_PER_SM
 #define SP24_MASK_CTAS_PER_SM 3
 #endif
-constexpr int kMaskCtasPerSm = SP24_MASK_CTAS_PER_SM;
+constexpr int kMaskCtasPerSm = SP24_MASK_CTAS_PER_SM;   // search and flip only
+// With compression a thread keeps more state live: two CTAs of 128 registers per thread.
+template <bool COMPRESS>
+constexpr int mask_ctas_per_sm() { return COMPRESS ? 2 : kMaskCtasPerSm; }
 constexpr uint64_t kMaskDrainBudget = 1ull << 26;
 
 // Nibble (4 * shift) of each of the four 16-bit codes in v, packed 4 bits apart.
@@ -342,9 +345,17 @@ __device__ __forceinline__ uint32_t gather_nibbles(uint2 v, int shift) {
   return (lo & 0xFu) | ((lo >> 12) & 0xF0u) | ((hi & 0xFu) << 8) | ((hi >> 4) & 0xF000u);
 }
 
-// Shared memory of one CTA tile.
+// Shared memory of one CTA tile, and the pattern tables the CTA reads per block
+// (copied from global memory once per CTA): pattern index p takes entry p & 127,
+// so the padding index 255 lands on entry 127, which holds its padding codes.
+constexpr int kTabEntries = 128;
 template <bool SEARCH, bool COMPRESS>
 struct MaskSmem {
+  uint2 rowsel[COMPRESS ? kTabEntries : 1];   // byte selectors of the kept pairs, rows
+  uint2 colsel[COMPRESS ? kTabEntries : 1];   // and columns
+  uint32_t codes[COMPRESS ? kTabEntries : 1]; // row codes | column codes << 16
+  uint16_t bits[kTabEntries];                 // kept-entry bit sets
+  uint8_t decode[SEARCH ? 256 : 4];           // tie field -> pattern index
   uint8_t idx[2][kTileBlocks][kTileBlocks];
   __align__(8) uint16_t rc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // row codes, [br][bc]
   __align__(8) uint16_t cc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // column codes, [bc][br]
@@ -352,6 +363,22 @@ struct MaskSmem {
   uint16_t queue[SEARCH ? 2 * kTileBlocks * kTileBlocks : 2];
   int qn;
 };
+
+template <bool SEARCH, bool COMPRESS>
+__device__ __forceinline__ void load_mask_tables(MaskSmem<SEARCH, COMPRESS> &sm) {
+  for (int e = threadIdx.x; e < kTabEntries; e += blockDim.x) {
+    const int pat = e == kTabEntries - 1 ? (int)kPadIndex : e;
+    if (COMPRESS) {
+      const uint64_t r = g_select.row[pat], c = g_select.col[pat];
+      sm.rowsel[e] = make_uint2((uint32_t)r, (uint32_t)(r >> 32));
+      sm.colsel[e] = make_uint2((uint32_t)c, (uint32_t)(c >> 32));
+      sm.codes[e] = (uint32_t)g_tables.rowcode[pat] | ((uint32_t)g_tables.colcode[pat] << 16);
+    }
+    sm.bits[e] = g_tables.bits[pat];
+  }
+  if (SEARCH)
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) sm.decode[e] = g_packed.decode[e];
+}
 
 // Where a CTA tile's weights come from: straight from global memory (row pitch
 // ldw), or from a 128 x 64 tile that the tensor memory accelerator placed in
@@ -426,11 +453,11 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
                                                uint8_t *__restrict__ idx, const uint8_t *__restrict__ idx_prev,
                                                unsigned &flips, uint16_t *__restrict__ vals_row,
                                                uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
-                                               uint8_t *__restrict__ meta_col, MaskSmem<SEARCH, COMPRESS> &sm) {
+                                               uint8_t *__restrict__ meta_col, MaskSmem<SEARCH, COMPRESS> &sm,
+                                               uint32_t one) {
   const int tid = threadIdx.x;
   const int rh = tid >> 7, lt = tid & (kQuadThreads - 1);
-  const uint16_t *bits_tab = g_tables.bits;
-  const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
+
   const int64_t tile_r0 = (int64_t)cy * kChunk, tile_c0 = (int64_t)cx * kChunk + kTile * kh;
   const int64_t tile_r = tile_r0 + kTile * rh;
   const int64_t bcols = C >> 2;
@@ -466,7 +493,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
       uint32_t blk[4][2];
 #pragma unroll
       for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
-      p[b] = search_block_packed<BF16>(blk, g_packed.decode, one);
+      p[b] = search_block_packed<BF16>(blk, sm.decode, one);
       if (p[b] == kNeedsExact) {
         const int slot = atomicAdd(&sm.qn, 1);
         sm.queue[slot] = (uint16_t)((rh << 8) | (br << 4) | (2 * uc + b));
@@ -485,7 +512,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
         const int q = id >> 8, qbr = (id >> 4) & 15, qbc = id & 15;
         uint32_t blk[4][2];
         src.block(kTile * q + 4 * qbr, 4 * qbc, blk);
-        sm.idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, g_tables.index, bits_tab);
+        sm.idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, g_tables.index, g_tables.bits);
       }
       __syncthreads();
 #pragma unroll
@@ -500,14 +527,15 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
   for (int b = 0; b < 2; ++b) {
     const bool ok = b ? ok1 : ok0;
     if (SEARCH && ok) idx[bidx0 + b] = (uint8_t)p[b];
-    if (FLIP && ok) flips += __popc((uint32_t)(bits_tab[prev[b]] ^ bits_tab[p[b]]));
+    if (FLIP && ok) flips += __popc((uint32_t)(sm.bits[prev[b] & 127] ^ sm.bits[p[b] & 127]));
   }
   if (COMPRESS) {
     uint32_t rc[2], cc[2];
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      rc[b] = g_tables.rowcode[p[b]];
-      cc[b] = g_tables.colcode[p[b]];
+      const uint32_t codes = sm.codes[p[b] & 127];
+      rc[b] = codes & 0xFFFFu;
+      cc[b] = codes >> 16;
       sm.rc[rh][br][2 * uc + b] = (uint16_t)rc[b];
       sm.cc[rh][2 * uc + b][br] = (uint16_t)cc[b];
     }
@@ -518,8 +546,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
         uint2 rsel[2];
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          const uint64_t t = g_select.row[p[b]];
-          rsel[b] = make_uint2((uint32_t)t, (uint32_t)(t >> 32));
+          rsel[b] = sm.rowsel[p[b] & 127];
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -539,8 +566,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
       // permutation picks its kept pair.
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
-        const uint64_t t = g_select.col[p[b]];
-        const uint2 csel = make_uint2((uint32_t)t, (uint32_t)(t >> 32));
+        const uint2 csel = sm.colsel[p[b] & 127];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int wi = 2 * b + (j >> 1);
@@ -610,7 +636,7 @@ __device__ __forceinline__ void mask_flip_flush(unsigned flips, unsigned long lo
 // One CTA per CTA tile, W read from global memory: the kernel for row pitches
 // that the tensor memory accelerator cannot take (ldw not a multiple of 8).
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_tile_kernel(
+__global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) mask_tile_kernel(
     const uint16_t *__restrict__ W, int64_t R, int64_t C, int64_t ldw, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
@@ -618,6 +644,8 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_tile_kernel
   __shared__ MaskSmem<SEARCH, COMPRESS> sm;
   __shared__ unsigned long long s_flip;
   if (threadIdx.x == 0) { s_flip = 0; sm.qn = 0; }
+  load_mask_tables(sm);
+  const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
   pdl_launch_dependents();
   pdl_wait();
   const uint32_t cy = blockIdx.y, cx = blockIdx.x >> 1, chunks_x = gridDim.x >> 1;
@@ -626,7 +654,7 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_tile_kernel
   __syncthreads();
   unsigned flips = 0;
   mask_tile_body<BF16, SEARCH, COMPRESS, FLIP>(src, R, C, cy, cx, kh, chunks_x, gridDim.y, idx, idx_prev, flips,
-                                               vals_row, meta_row, vals_col, meta_col, sm);
+                                               vals_row, meta_row, vals_col, meta_col, sm, one);
   if (FLIP) mask_flip_flush(flips, &s_flip, flip_count);
 }
 
@@ -637,7 +665,7 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_tile_kernel
 // loads of the next two tiles overlap the work on this one.  Every wait is
 // bounded; on a timeout the CTA records the error, lets its copies land and exits.
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
-__global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_stream_kernel(
+__global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) mask_stream_kernel(
     const __grid_constant__ CUtensorMap tm_w, int64_t R, int64_t C, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
@@ -672,6 +700,8 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_stream_kern
     s_abort = 0;
     sm.qn = 0;
   }
+  load_mask_tables(sm);
+  const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
   __syncthreads();
   pdl_launch_dependents();
   pdl_wait();
@@ -694,7 +724,7 @@ __global__ void __launch_bounds__(kMaskThreads, kMaskCtasPerSm) mask_stream_kern
     tile_xy(t, cy, cx, kh);
     const SharedTileSrc src{s_w[buf]};
     mask_tile_body<BF16, SEARCH, COMPRESS, FLIP>(src, R, C, cy, cx, kh, chunks_x, chunks_y, idx, idx_prev, flips,
-                                                 vals_row, meta_row, vals_col, meta_col, sm);
+                                                 vals_row, meta_row, vals_col, meta_col, sm, one);
     __syncthreads();   // every read of this buffer and of the tile's shared state is done
     if (tid == 0) {
       sm.qn = 0;

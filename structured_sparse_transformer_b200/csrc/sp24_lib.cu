@@ -290,7 +290,7 @@ sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint
   if (ldw % 8 == 0 && C <= INT32_MAX && R <= INT32_MAX &&
       make_map_2d(&tm, W, (uint64_t)C, (uint64_t)R, (uint64_t)ldw * 2, kMaskCtaCols, kChunk,
                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
-    const int64_t ctas = (int64_t)sm_count() * kMaskCtasPerSm;
+    const int64_t ctas = (int64_t)sm_count() * mask_ctas_per_sm<COMPRESS>();
     const unsigned grid = (unsigned)(ntiles < ctas ? ntiles : ctas);
     return launch_pdl(mask_stream_kernel<BF16, SEARCH, COMPRESS, FLIP>, dim3(grid), dim3(kMaskThreads), 0, s, tm, R,
                       C, idx, prev, flip, static_cast<uint16_t *>(vr), static_cast<uint8_t *>(mr),

@@ -8,7 +8,8 @@ masked decay on gradients; transposable masks for the input gradient).
 d = 1600, ff = 6400, 32768 tokens, fp16.  Eight steps W_(t+1) = round(W_t + N(0, 1e-4)) of
 both weights, each through the calls the benchmark times: the fused mask step (search, flip
 count against the previous step's mask, both compressions), the forward and input-gradient
-GEMMs of both layers with GELU between, and the masked decay of both gradients.  Per step:
+GEMMs of both layers with GELU between (the forward storing gelu' of its pre-activation, the
+input gradient multiplying by it), and the masked decay of both gradients.  Per step:
 masks, flip counts, compressed values and metadata, and decayed gradients bit for bit against
 the oracle; the four GEMMs at the stated tolerance on sampled token rows, each on the GPU's
 own inputs.
@@ -40,7 +41,7 @@ def test_gpt2_1p5b_eight_steps():
     idx_prev = [torch.empty(r // 4, c // 4, dtype=torch.uint8, device="cuda") for r, c in shapes]
     idx_cur = [torch.empty_like(i) for i in idx_prev]
     count = torch.zeros(2, dtype=torch.int64, device="cuda")
-    H, Hpre, dH = (torch.empty(T, ff, dtype=tdt, device="cuda") for _ in range(3))
+    H, Gp, dH = (torch.empty(T, ff, dtype=tdt, device="cuda") for _ in range(3))
     Y, dX = (torch.empty(T, d, dtype=tdt, device="cuda") for _ in range(2))
     o_prev = []
     for li in range(2):
@@ -56,9 +57,9 @@ def test_gpt2_1p5b_eight_steps():
             sp.sp24_mask_step(Wd[li], idx_cur[li], idx_prev[li], count[li:li + 1], *comp[li])
         vr1, mr1, vc1, mc1 = comp[0]
         vr2, mr2, vc2, mc2 = comp[1]
-        sp.sp24_gemm_fwd(Xd, vr1, mr1, ff, H, "gelu", Hpre)
+        sp.sp24_gemm_fwd(Xd, vr1, mr1, ff, H, "gelu_deriv", Gp)
         sp.sp24_gemm_fwd(H, vr2, mr2, d, Y)
-        sp.sp24_gemm_dgrad(dYd, vc2, mc2, ff, dH, "dgelu", Hpre)
+        sp.sp24_gemm_dgrad(dYd, vc2, mc2, ff, dH, "mul_aux", Gp)
         sp.sp24_gemm_dgrad(dH, vc1, mc1, d, dX)
         Gd = [G1.cuda(), G2.cuda()]
         for li in range(2):
@@ -87,13 +88,13 @@ def test_gpt2_1p5b_eight_steps():
         k1, k2 = oracle.dense_mask(o_cur[0]), oracle.dense_mask(o_cur[1])
         xs = oracle.to_f64(si.bits16(X)[rows], dt)
         pre = oracle.sparse_fwd(xs, w1f, k1)
-        hpre_gpu = f64_of(Hpre, dt)[rows]
-        assert_gemm_close(hpre_gpu, pre, dt, f"step {t} fwd1 pre-activation")
+        gp_gpu = f64_of(Gp, dt)[rows]
+        assert_gemm_close(gp_gpu, oracle.gelu_grad(pre), dt, f"step {t} fwd1 gelu'")
         assert_gemm_close(f64_of(H, dt)[rows], oracle.gelu(pre), dt, f"step {t} fwd1 gelu")
         assert_gemm_close(f64_of(Y, dt)[rows], oracle.sparse_fwd(f64_of(H, dt)[rows], w2f, k2), dt, f"step {t} fwd2")
         dys = oracle.to_f64(si.bits16(dY)[rows], dt)
-        assert_gemm_close(f64_of(dH, dt)[rows], oracle.sparse_dgrad(dys, w2f, k2) * oracle.gelu_grad(hpre_gpu), dt,
-                          f"step {t} dgrad2 dgelu")
+        assert_gemm_close(f64_of(dH, dt)[rows], oracle.sparse_dgrad(dys, w2f, k2) * gp_gpu, dt,
+                          f"step {t} dgrad2 times gelu'")
         assert_gemm_close(f64_of(dX, dt)[rows], oracle.sparse_dgrad(f64_of(dH, dt)[rows], w1f, k1), dt,
                           f"step {t} dgrad1")
         o_prev = o_cur
