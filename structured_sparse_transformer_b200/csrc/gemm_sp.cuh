@@ -115,7 +115,10 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // buffering: the weight-gradient tiles run one per pair at the FFN sizes).
 // The dense variant (dense fine-tuning) takes A = dY^T [N x T] dense, 64 tokens
 // per stage: A 16 KB + two 8 KB atoms, 6 stages; each 16-token K step issues
-// two dense MMAs of N = 128.
+// two dense MMAs of N = 128.  (Tiles of 128 dW columns with double-buffered
+// accumulators were measured 10-15% slower at the 1.5B shapes, although they
+// leave fewer column-waves idle: each stage then carries half the MMA work for
+// the same A tile and per-stage overhead.)
 template <bool SPARSE, int EPI>
 struct PairGeom {
   static constexpr bool kWg = EPI == kEpiWgrad;
@@ -148,7 +151,7 @@ __host__ __device__ constexpr int epi_bufs(int epi) {
 template <bool SPARSE, int EPI>
 __host__ __device__ constexpr int pair_smem_bytes() {
   return PairGeom<SPARSE, EPI>::kStages * PairGeom<SPARSE, EPI>::kStageBytes + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
-         kPairBarBytes + 1024 + (EPI == kEpiWgrad ? 8192 : 0);
+         kPairBarBytes + 1024 + (PairGeom<SPARSE, EPI>::kWg ? 8192 : 0);
 }
 static_assert(pair_smem_bytes<true, kEpiMulAux>() == pair_smem_bytes<true, kEpiDgelu>() &&
                   pair_smem_bytes<false, kEpiMulAux>() == pair_smem_bytes<false, kEpiDgelu>() &&
@@ -159,6 +162,7 @@ static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<fa
                   pair_smem_bytes<true, kEpiWgrad>() <= 232448,
               "shared memory per CTA");
 static_assert(pair_smem_bytes<false, kEpiWgrad>() <= 232448, "shared memory per CTA (dense wgrad)");
+
 // The producer loads A and two B atoms (and, sparse, the metadata chunk) per stage of a
 // weight-gradient pipeline: the stage, and the byte count armed on its barrier, hold all of them.
 static_assert(PairGeom<true, kEpiWgrad>::kStageBytes == kPairSmemA + 2 * (64 * 128 * 2) + kSmemE &&
@@ -430,13 +434,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (WG) {
           // MN-major atoms: x = dW column (b_row, b_row + 128), y = token.
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], b_row, kt * G::kBK);
-          tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 128, kt * G::kBK);
+          if (G::kBBoxes == 2)
+            tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 128, kt * G::kBK);
         } else {
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
           if (SPARSE) tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * G::kBK + 64, b_row);
         }
         if (SPARSE)
-          tma_load_2d_pair(st + kPairSmemA + 2 * G::kBBoxBytes, &tm_meta, &full[s], 0, chunk_row + kt);
+          tma_load_2d_pair(st + kPairSmemA + G::kBBoxes * G::kBBoxBytes, &tm_meta, &full[s], 0, chunk_row + kt);
       }
     }
     // The leader's `full` barriers count both CTAs' bytes: let every copy land.
@@ -462,7 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
     const uint64_t e_desc0 =
-        smem_desc(smem_u32(stage_base + kPairSmemA + 2 * G::kBBoxBytes), 128, 128, kSwizzleNone);
+        smem_desc(smem_u32(stage_base + kPairSmemA + G::kBBoxes * G::kBBoxBytes), 128, 128, kSwizzleNone);
     uint32_t g = 0;
     bool ok = true;
     int j = 0;
@@ -486,7 +491,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
             const uint64_t bk = bd + (uint64_t)(kk * (2048 >> 4));
             tc_mma_f16_pair(acc, ad + 2 * kk, bk, idesc, accum);
-            tc_mma_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
+            if (G::kBBoxes == 2)
+              tc_mma_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
           }
         } else if (WG) {
           const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;
@@ -500,7 +506,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
             const uint64_t bk = bd + (uint64_t)(kk * (4096 >> 4));
             tc_mma_sp_f16_pair(acc, ad + 2 * kk, bk, tm, id, accum);
-            tc_mma_sp_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), tm, id, accum);
+            if (G::kBBoxes == 2)
+              tc_mma_sp_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), tm, id, accum);
           }
         } else if (SPARSE) {
           const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
@@ -574,10 +581,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      const bool got = mbar_wait_bounded(&acc_full[0], (uint32_t)j & 1u, wait_budget, s_abort);
+      const int ab = j % G::kAccBufs;   // accumulator buffer of this tile
+      const bool got = mbar_wait_bounded(&acc_full[ab], (uint32_t)(j / G::kAccBufs) & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
-      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16);
+      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * G::kBN);
 #pragma unroll
       for (int k0 = 0; k0 < kPerWarp; k0 += kBatch) {
         uint32_t r[kBatch][2][8];
@@ -621,7 +629,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_leader(&acc_empty[0]);
+      if (lane == 0) mbar_arrive_leader(&acc_empty[ab]);
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------- epilogue (both CTAs)

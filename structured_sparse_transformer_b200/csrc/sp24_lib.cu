@@ -134,6 +134,42 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 // SPARSE: A = kept values [M x Kd/2] + metadata chunks; dense: A = [M x Kd].
 // Weight gradient (kEpiWgrad): B = the layer input [Kd tokens x T columns]
 // read MN-major, out = fp32 [M x T]; tiles of 256 x 256.
+// Per device, once: the shared-memory opt-in of an instantiation and the number
+// of its CTA pairs that fit at once (0: the set-up failed; -1: no device).
+template <bool BF16, int EPI, bool SPARSE>
+int gemm_pairs() {
+  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
+  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
+  static PerDevice pairs_cache;
+  const int dev = current_device();
+  if (dev < 0) return -1;
+  std::call_once(pairs_cache.once[dev], [&] {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess) {
+      cudaGetLastError();
+      pairs_cache.value[dev] = 0;
+      return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sm_count() / 2;
+    }
+    pairs_cache.value[dev] = n;
+  });
+  return pairs_cache.value[dev];
+}
+
 // Weight gradient with decay: dec_w/dec_idx/dec_lambda (the masked decay of dW in
 // the epilogue); null dec_w elsewhere.
 template <bool BF16, int EPI, bool SPARSE>
@@ -182,37 +218,8 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   if (!maps_ok) return SP24_ERR_CUDA;
   constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
   auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
-  // Per device, once: the shared-memory opt-in of this instantiation and the number
-  // of CTA pairs that fit at once (0 marks a failed set-up).
-  static PerDevice pairs_cache;
-  const int dev = current_device();
-  if (dev < 0) return SP24_ERR_NO_DEVICE;
-  std::call_once(pairs_cache.once[dev], [&] {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess) {
-      cudaGetLastError();
-      pairs_cache.value[dev] = 0;
-      return;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
-    cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = smem_bytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = sm_count() / 2;
-    }
-    pairs_cache.value[dev] = n;
-  });
-  const int max_pairs = pairs_cache.value[dev];
-  if (max_pairs <= 0) return SP24_ERR_CUDA;
+  const int max_pairs = gemm_pairs<BF16, EPI, SPARSE>();
+  if (max_pairs <= 0) return max_pairs == 0 ? SP24_ERR_CUDA : SP24_ERR_NO_DEVICE;
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
@@ -336,6 +343,14 @@ inline size_t meta_nibble_pos(int64_t r, int64_t g, int64_t cols, int *shift) {
   const int bit = 4 * (int)(gg % 4) + 16 * (int)((m / 8) % 2);
   *shift = bit % 8;
   return (size_t)(mt * kt_count + kt) * 2048 + (size_t)lane * 16 + (size_t)kk * 4 + (size_t)(bit / 8);
+}
+
+// Weight gradient: tiles of 256 rows x 256 columns of dW (see PairGeom).
+template <bool BF16, bool SPARSE>
+sp24_status launch_wgrad(const void *X, int64_t T, int64_t K, const void *A, const void *meta, int64_t N, float *dW,
+                         cudaStream_t s, const void *dec_w = nullptr, const uint8_t *dec_idx = nullptr,
+                         float dec_lambda = 0.0f) {
+  return launch_gemm_pair_t<BF16, kEpiWgrad, SPARSE>(X, K, T, A, meta, N, dW, nullptr, s, dec_w, dec_idx, dec_lambda);
 }
 
 }  // namespace
@@ -516,8 +531,8 @@ sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *val
   if (T == 0) {   // an empty sum over tokens
     return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
   }
-  return dtype == SP24_BF16 ? launch_gemm_pair_t<true, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s)
-                            : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s);
+  return dtype == SP24_BF16 ? launch_wgrad<true, true>(X, T, K, vals, meta, N, dW, s)
+                            : launch_wgrad<false, true>(X, T, K, vals, meta, N, dW, s);
 }
 
 sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
@@ -538,9 +553,8 @@ sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const voi
     if (cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) != cudaSuccess) return SP24_ERR_CUDA;
     return sp24_masked_decay(dW, W, dtype, N, K, idx, lambda, stream);
   }
-  return dtype == SP24_BF16
-             ? launch_gemm_pair_t<true, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s, W, idx, lambda)
-             : launch_gemm_pair_t<false, kEpiWgrad, true>(X, K, T, vals, meta, N, dW, nullptr, s, W, idx, lambda);
+  return dtype == SP24_BF16 ? launch_wgrad<true, true>(X, T, K, vals, meta, N, dW, s, W, idx, lambda)
+                            : launch_wgrad<false, true>(X, T, K, vals, meta, N, dW, s, W, idx, lambda);
 }
 
 sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N, sp24_dtype dtype,
@@ -558,8 +572,8 @@ sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const voi
   if (T == 0) {   // an empty sum over tokens
     return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
   }
-  return dtype == SP24_BF16 ? launch_gemm_pair_t<true, kEpiWgrad, false>(X, K, T, dYt, nullptr, N, dW, nullptr, s)
-                            : launch_gemm_pair_t<false, kEpiWgrad, false>(X, K, T, dYt, nullptr, N, dW, nullptr, s);
+  return dtype == SP24_BF16 ? launch_wgrad<true, false>(X, T, K, dYt, nullptr, N, dW, s)
+                            : launch_wgrad<false, false>(X, T, K, dYt, nullptr, N, dW, s);
 }
 
 sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,
