@@ -26,16 +26,20 @@
  *     column pairs (each row's pair ranked (0,1)<(0,2)<(0,3)<(1,2)<(1,3)<(2,3),
  *     row 0 most significant).  sp24_pattern_table() returns the patterns.
  *   - Device pointers (marked "device") are caller-owned device memory; host
- *     pointers (marked "host") are caller-owned host memory.  The library never
- *     allocates, frees or keeps a pointer after a call returns.
+ *     pointers (marked "host") are caller-owned host memory.  The library
+ *     keeps no caller pointer after a call returns.  It allocates only the
+ *     weight-gradient workspace (see sp24_gemm_wgrad): one per (device,
+ *     stream), made by the first call on that stream that needs it and kept
+ *     for the life of the process.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls that launch work are asynchronous and stream-ordered.
  *   - Argument checks (shapes, dtypes, alignment, null pointers) run on the
  *     host before anything is launched; a failed check launches nothing.
  *   - Weights must be finite; results for NaN/Inf weights are unspecified
  *     (never out-of-bounds accesses).
- *   - A kernel that gives up waiting (bounded spin on an mbarrier) records it
- *     in a per-device error word and exits; sp24_device_status() reports it.
+ *   - A kernel that gives up waiting (bounded spin on an mbarrier or on a
+ *     counter in global memory) records it in a per-device error word and
+ *     exits; sp24_device_status() reports it.
  */
 #ifndef SP24_H
 #define SP24_H
@@ -249,6 +253,16 @@ SP24_API sp24_status sp24_mvue_sparsify(const void *dY, int64_t T, int64_t N, in
  *   vals, meta  device, from sp24_mvue_sparsify with the same T and N
  *   dW    device fp32 [N x K] contiguous, overwritten (zeros when T == 0)
  * T % 16 == 0, N % 16 == 0, K % 8 == 0; all pointers 16-byte aligned.
+ * Tiles of 256 x 256 of dW run in waves over the device's CTA pairs (P, 74 on
+ * a 148-SM B200).  When the tile count is not a multiple of P, the r tiles of
+ * the last wave are split along T into s = min(P / r, 8, ceil(T / 128)) parts
+ * on all P pairs; the pair with each tile's first tokens adds the other parts'
+ * fp32 partial sums (in part order, so results are reproducible run to run)
+ * and stores the tile.  The partial sums go through a workspace of 147,456
+ * bytes per CTA plus 48 bytes of counters (2 P CTAs: about 21 MB on B200),
+ * allocated with cudaMalloc by the first such call on each (device, stream)
+ * and reused by later ones; a failed allocation returns SP24_ERR_CUDA.
+ * Launches on one stream run in order, so they share that workspace safely.
  */
 SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
                             int64_t N, sp24_dtype dtype, float *dW, void *stream);
@@ -265,7 +279,8 @@ SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const 
  *   W     device dtype [N x K] row-major, contiguous (the layer's weight)
  *   idx   device uint8 [N/4][K/4], the mask of W (sp24_mask_search)
  * T % 16 == 0, N % 16 == 0, K % 8 == 0; X, vals, meta, W and dW 16-byte
- * aligned.  T == 0 gives the decay of a zero gradient.
+ * aligned.  T == 0 gives the decay of a zero gradient.  Tiles, split tail and
+ * workspace as for sp24_gemm_wgrad.
  */
 SP24_API sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
                                   int64_t N, sp24_dtype dtype, const void *W, const uint8_t *idx, float lambda,
@@ -281,6 +296,8 @@ SP24_API sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, 
  *   dYt   device [N x T] row-major, contiguous (dY transposed)
  *   dW    device fp32 [N x K] contiguous, overwritten (zeros when T == 0)
  * T % 16 == 0, N % 16 == 0, K % 8 == 0; all pointers 16-byte aligned.
+ * Tiles, split tail and workspace as for sp24_gemm_wgrad (64 tokens per K step:
+ * s <= ceil(T / 64)).
  */
 SP24_API sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N,
                                   sp24_dtype dtype, float *dW, void *stream);
@@ -321,7 +338,10 @@ SP24_API sp24_status sp24_meta_from_canonical(const uint16_t *canon, int64_t row
 /*
  * Synchronizes `stream`, then reads and clears the current device's error
  * word.  Returns SP24_ERR_TIMEOUT if a kernel gave up waiting since the last
- * query, SP24_ERR_CUDA if synchronization failed, else SP24_OK.
+ * query, SP24_ERR_CUDA if synchronization failed, else SP24_OK.  After a
+ * timeout it also waits for the whole device and zeroes the counters of every
+ * weight-gradient workspace of the device, which a launch that gave up may have
+ * left raised; results of the calls before the query are then unspecified.
  */
 SP24_API sp24_status sp24_device_status(void *stream);
 

@@ -180,6 +180,54 @@ static_assert(PairGeom<true, kEpiNone>::kStageBytes % 1024 == 0 && PairGeom<fals
 static_assert(kPairMetaCol + 4 * PairGeom<true, kEpiNone>::kStages <= kTmemCols, "tensor memory budget");
 static_assert(2 * PairGeom<false, kEpiNone>::kStages + 16 + 2 * kEpiWarps <= kPairBarBytes / 8, "barrier space");
 
+// Work schedule of a CTA pair: a sequence of segments (tile, K steps kb..ke-1).
+// Data-parallel (every GEMM): pair p takes tiles p, p + P, p + 2P, ... over all
+// num_kt K steps, so the P pairs of a wave walk K in step and share each K
+// window of both operands in L2.  Split tail (the weight gradient, when
+// `split` > 1): the full waves stay data-parallel, and the r = tiles mod P
+// tiles of the last wave are cut along K into `split` (<= P / r) parts of
+// num_kt / split steps; part j of tail tile i goes to pair i * split + j.  The
+// pair holding part 0 (K steps from 0) adds the other parts' partial
+// accumulators, written by pairs i * split + 1 .. i * split + split - 1 while it
+// runs its own part, and stores the tile.
+struct PairSchedule {
+  int tile, pair, npairs, num_tiles, num_kt, split, full_tiles;
+  bool tail_taken;
+  __device__ PairSchedule(int sp, int p, int np, int tiles, int kt)
+      : tile(p), pair(p), npairs(np), num_tiles(tiles), num_kt(kt), split(sp),
+        full_tiles(sp > 1 ? (tiles / np) * np : tiles), tail_taken(false) {}
+  __device__ bool next(int &t, int &kb, int &ke) {
+    if (tile < full_tiles) {
+      t = tile;
+      kb = 0;
+      ke = num_kt;
+      tile += npairs;
+      return true;
+    }
+    if (split > 1 && !tail_taken) {
+      tail_taken = true;
+      if (pair < (num_tiles - full_tiles) * split) {
+        const int part = pair % split;
+        t = full_tiles + pair / split;
+        kb = part * num_kt / split;
+        ke = (part + 1) * num_kt / split;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+// Partial accumulator of one CTA of a split tail tile (128 rows x 256 columns of dW, fp32):
+// per epilogue warp, its 16-column chunks as [chunk][row half][8-column block]
+// [lane] float4s, the registers of tmem_ld_16x256b_x2 as loaded, so the CTA
+// that adds it reads back exactly what the same warp and lane of its own
+// accumulator hold.  Ready counters: one per epilogue warp, raised by 1 per
+// lane with release semantics once the lane's stores are issued.
+constexpr int kWgChunksPerWarp = (256 / 16 + kEpiGroups - 1) / kEpiGroups;
+constexpr int kMaxSplit = 8;   // parts of a split tail tile (part 0 adds the others one after another)
+constexpr int64_t kSkPartFloatsPerCta = (int64_t)kEpiWarps * kWgChunksPerWarp * 4 * 32 * 4;
+
 // GELU (exact erf form) and its derivative for the epilogues:
 //   gelu(x) = x Phi(x),  gelu'(x) = Phi(x) + x phi(x),
 //   Phi(x) = 1 - erfc(x/sqrt2)/2 (x >= 0),  erfc(|x|/sqrt2)/2 (x < 0),
@@ -350,11 +398,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           const __grid_constant__ CUtensorMap tm_aux, int M, int T, int num_kt,
                           uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out,
                           const uint16_t *__restrict__ dec_w, const uint8_t *__restrict__ dec_idx,
-                          float dec_lambda) {
+                          float dec_lambda, float *__restrict__ sk_part, unsigned *__restrict__ sk_flags,
+                          int sk_split) {
   // T counts the B operand's rows of the output: tokens, or for the weight
   // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
   // Weight gradient with dec_w set: the masked decay of dW in the epilogue, W and
   // its pattern indices dec_idx [M/4][T/4] in the layout of dW (see below).
+  // Weight gradient with sk_part set: the split-tail schedule with sk_split
+  // parts per tail tile, partial accumulators in sk_part (kSkPartFloatsPerCta
+  // per CTA) and ready counters in sk_flags (kEpiWarps per CTA, zero at launch
+  // and left zero).
   using G = PairGeom<SPARSE, EPI>;
   constexpr bool WG = G::kWg;
   constexpr int kPairStages = G::kStages;
@@ -381,6 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int num_mt = (M + 2 * kPairRows - 1) / (2 * kPairRows);
   const int num_row_tiles = (M + kPairRows - 1) / kPairRows;
   const int num_tiles = num_mt * ((T + G::kBN - 1) / G::kBN);
+  const int split = (WG && sk_part != nullptr) ? sk_split : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -415,14 +469,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------ producer (both CTAs)
     uint32_t g = 0;
     bool ok = true;
-    for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+    PairSchedule sched(split, pair, npairs, num_tiles, num_kt);
+    int tile, kb, ke;
+    while (ok && sched.next(tile, kb, ke)) {
       const int mt = tile % num_mt;
       const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
       const int b_row = (tile / num_mt) * G::kBN + (int)rank * (WG ? 64 : kPairBNh);
       // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
       // it the last real metadata chunk so every code the MMA sees is valid.
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
-      for (int kt = 0; kt < num_kt; ++kt, ++g) {
+      for (int kt = kb; kt < ke; ++kt, ++g) {
         const int s = (int)(g % kPairStages);
         if (!mbar_wait_bounded(&empty[s], ((g / kPairStages) & 1u) ^ 1u, wait_budget, s_abort)) {
           ok = false;
@@ -471,13 +527,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint32_t g = 0;
     bool ok = true;
     int j = 0;
-    for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++j) {
+    PairSchedule sched(split, pair, npairs, num_tiles, num_kt);
+    int tile, kb, ke;
+    for (; ok && sched.next(tile, kb, ke); ++j) {
       const int b = j % G::kAccBufs;
       const uint32_t use = (uint32_t)(j / G::kAccBufs);
       if (!(ok = mbar_wait_bounded(&acc_empty[b], (use & 1u) ^ 1u, wait_budget, s_abort))) break;
       tc_fence_after();
       const uint32_t acc = tmem_base + (uint32_t)(b * G::kBN);
-      for (int kt = 0; kt < num_kt; ++kt, ++g) {
+      for (int kt = kb; kt < ke; ++kt, ++g) {
         const int s = (int)(g % kPairStages);
         if (!(ok = mbar_wait_bounded(&full[s], (g / kPairStages) & 1u, wait_budget, s_abort))) break;
         tc_fence_after();
@@ -488,7 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           // swizzled rows and B 16 tokens (2048 bytes); atom 1 of B sits 8 KB after atom 0.
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
+            const uint32_t accum = (kt != kb || kk != 0) ? 1u : 0u;
             const uint64_t bk = bd + (uint64_t)(kk * (2048 >> 4));
             tc_mma_f16_pair(acc, ad + 2 * kk, bk, idesc, accum);
             if (G::kBBoxes == 2)
@@ -503,7 +561,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t tm = t_meta + 2 * (kk >> 1);
             const uint32_t id = idesc | (uint32_t)(kk & 1);
-            const uint32_t accum = (kt != 0 || kk != 0) ? 1u : 0u;
+            const uint32_t accum = (kt != kb || kk != 0) ? 1u : 0u;
             const uint64_t bk = bd + (uint64_t)(kk * (4096 >> 4));
             tc_mma_sp_f16_pair(acc, ad + 2 * kk, bk, tm, id, accum);
             if (G::kBBoxes == 2)
@@ -514,13 +572,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_cp_128x128b_pair(t_meta, e_desc0 + so);
           // The metadata operand address must be 2-column aligned; the low column
           // bit travels in the descriptor's sparsity-selector field instead.
-          tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != 0 ? 1u : 0u);
+          tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != kb ? 1u : 0u);
           tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
           tc_mma_sp_f16_pair(acc, ad + 4, bd + (kPairSmemBBox >> 4), t_meta + 2, idesc, 1u);
           tc_mma_sp_f16_pair(acc, ad + 6, bd + (kPairSmemBBox >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
         } else {
           // Four K = 16 steps through the 128-byte swizzled rows of A and B (32 bytes each).
-          tc_mma_f16_pair(acc, ad, bd, idesc, kt != 0 ? 1u : 0u);
+          tc_mma_f16_pair(acc, ad, bd, idesc, kt != kb ? 1u : 0u);
           tc_mma_f16_pair(acc, ad + 2, bd + 2, idesc, 1u);
           tc_mma_f16_pair(acc, ad + 4, bd + 4, idesc, 1u);
           tc_mma_f16_pair(acc, ad + 6, bd + 6, idesc, 1u);
@@ -551,11 +609,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     constexpr int kChunks = G::kBN / 16;
     constexpr int kPerWarp = (kChunks + kEpiGroups - 1) / kEpiGroups;
-    constexpr int kBatch = 3;
-    const bool decay = dec_w != nullptr;
+    constexpr int kBatch = 2;
+    static_assert(!WG || kPerWarp == kWgChunksPerWarp, "split-tail partial layout");
     const int64_t idx_cols = ld_out >> 2;
+    const int ew = warp - 2;
+    // Split tail: this CTA's partial slot and counter; the CTA of the same rank in
+    // pair p + d uses slot and counter blockIdx.x + 2d.
+    float4 *part_own = split > 1 ? reinterpret_cast<float4 *>(sk_part + (int64_t)blockIdx.x * kSkPartFloatsPerCta) +
+                                       (int64_t)ew * kPerWarp * 4 * 32 + lane
+                                 : nullptr;
+    unsigned *flag_own = split > 1 ? sk_flags + (int64_t)blockIdx.x * kEpiWarps + ew : nullptr;
     int j = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++j) {
+    PairSchedule sched(split, pair, npairs, num_tiles, num_kt);
+    int tile, kbeg, kend;
+    for (; sched.next(tile, kbeg, kend); ++j) {
+      const bool to_part = kbeg > 0;                   // a later part of a split tile: another pair stores it
+      const bool merge = kbeg == 0 && kend < num_kt;   // part 0: pairs p + 1 .. p + split - 1 hold the rest
+      const bool decay = dec_w != nullptr && !to_part;
       const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
       const int n0 = (tile / num_mt) * G::kBN;
       // Decay operands of the warp's stores in this tile: W's two values (one
@@ -585,6 +655,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool got = mbar_wait_bounded(&acc_full[ab], (uint32_t)(j / G::kAccBufs) & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) break;
       tc_fence_after();
+      if (merge) {
+        // The other parts of this tile: all 32 lanes of the same warp of each
+        // have released their stores (the parts run side by side in the last
+        // wave).  Each lane then acquires every counter itself.
+        bool ready = true;
+        if (lane == 0)
+          for (int d = 1; d < split && ready; ++d)
+            ready = flag_wait_bounded(flag_own + 2 * d * kEpiWarps, 32u, wait_budget, s_abort);
+        if (!__shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0)) break;
+        for (int d = 1; d < split; ++d) (void)flag_load_acquire(flag_own + 2 * d * kEpiWarps);
+      }
       const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(ab * G::kBN);
 #pragma unroll
       for (int k0 = 0; k0 < kPerWarp; k0 += kBatch) {
@@ -603,10 +684,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           reg_fence(r[k][0]);
           reg_fence(r[k][1]);
         }
+        // Part 0 of a split tile: its own sum, then parts 1, 2, ... in order (fp32
+        // additions into the loaded accumulator), a chunk's four loads at a time.
+        if (merge) {
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            if (grp + (k0 + k) * kEpiGroups >= kChunks) break;
+            for (int d = 1; d < split; ++d) {
+              const float4 *src = part_own + 2 * d * kSkPartFloatsPerCta / 4 + (k0 + k) * 4 * 32;
+              float4 pv[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) pv[e] = __ldcg(src + e * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint32_t *a = &r[k][e >> 1][4 * (e & 1)];
+                a[0] = __float_as_uint(__fadd_rn(__uint_as_float(a[0]), pv[e].x));
+                a[1] = __float_as_uint(__fadd_rn(__uint_as_float(a[1]), pv[e].y));
+                a[2] = __float_as_uint(__fadd_rn(__uint_as_float(a[2]), pv[e].z));
+                a[3] = __float_as_uint(__fadd_rn(__uint_as_float(a[3]), pv[e].w));
+              }
+            }
+          }
+        }
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
           const int ch = grp + (k0 + k) * kEpiGroups;
           if (ch >= kChunks) break;
+          if (to_part) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int i = 0; i < 2; ++i)
+                part_own[((k0 + k) * 4 + 2 * h + i) * 32] =
+                    make_float4(__uint_as_float(r[k][h][4 * i]), __uint_as_float(r[k][h][4 * i + 1]),
+                                __uint_as_float(r[k][h][4 * i + 2]), __uint_as_float(r[k][h][4 * i + 3]));
+            continue;
+          }
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -626,6 +739,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 if (row < M && col < T) *reinterpret_cast<float2 *>(out_f32 + (int64_t)row * ld_out + col) = v;
               }
         }
+      }
+      if (to_part) flag_add_release(flag_own, 1u);   // this lane's partial stores are issued
+      if (merge) {
+        __syncwarp();   // every lane has read the partials: the counters return to zero for the next launch
+        if (lane == 0)
+          for (int d = 1; d < split; ++d) flag_store_relaxed(flag_own + 2 * d * kEpiWarps, 0u);
       }
       tc_fence_before();
       __syncwarp();

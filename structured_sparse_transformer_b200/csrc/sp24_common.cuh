@@ -90,6 +90,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// ------------------------------------------------ flags between CTAs (global)
+// Release increment of a counter in global memory (device scope): the
+// thread's earlier stores are visible to any thread whose acquire load sees it.
+__device__ __forceinline__ void flag_add_release(unsigned *flag, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned flag_load_acquire(const unsigned *flag) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void flag_store_relaxed(unsigned *flag, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+// Wait until *flag >= target, at most `budget` clock cycles; on timeout raise
+// the CTA's abort flag and the device error word, like mbar_wait_bounded.
+__device__ __forceinline__ bool flag_wait_bounded(const unsigned *flag, unsigned target, uint64_t budget,
+                                                  volatile int *abort_flag) {
+  if (flag_load_acquire(flag) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (*abort_flag) return false;
+    if ((uint64_t)(clock64() - t0) > budget) {
+      *abort_flag = 1;
+      record_device_error(kDevErrTimeout);
+      return false;
+    }
+    __nanosleep(256);
+    if (flag_load_acquire(flag) >= target) return true;
+  }
+}
+
 // ------------------------------------------ programmatic dependent launch
 // Every kernel here is launched with programmatic stream serialisation: the
 // next kernel in the stream may be scheduled (and run its prologue) while

@@ -9,7 +9,9 @@
 #include <string.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "sp24.h"
 #include "gemm_sp.cuh"
@@ -170,6 +172,63 @@ int gemm_pairs() {
   return pairs_cache.value[dev];
 }
 
+// Split-tail workspace of the weight gradient, one per (device, stream), so that
+// launches on different streams never share one (launches on one stream run
+// one after another): the partial accumulators and ready counters of every
+// CTA of a full-width launch.  Allocated on first use and kept for the life of
+// the process.  The counters start at zero and every launch that completes
+// leaves them at zero; after a kernel gives up waiting, sp24_device_status
+// clears them.
+struct SkWorkspace {
+  float *part = nullptr;
+  unsigned *flags = nullptr;
+  int ctas = 0;
+};
+std::mutex g_sk_mutex;
+std::map<std::pair<int, cudaStream_t>, SkWorkspace> g_sk_workspaces;
+
+sp24_status sk_workspace(cudaStream_t stream, int ctas, SkWorkspace *out) {
+  const int dev = current_device();
+  if (dev < 0) return SP24_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_sk_mutex);
+  SkWorkspace &w = g_sk_workspaces[std::make_pair(dev, stream)];
+  if (w.ctas < ctas) {
+    // cudaFree waits for the device, so no earlier launch still uses the old buffers.
+    if (w.part) cudaFree(w.part);
+    if (w.flags) cudaFree(w.flags);
+    w = SkWorkspace{};
+    float *part = nullptr;
+    unsigned *flags = nullptr;
+    if (cudaMalloc(&part, (size_t)ctas * kSkPartFloatsPerCta * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&flags, (size_t)ctas * kEpiWarps * sizeof(unsigned)) != cudaSuccess ||
+        cudaMemsetAsync(flags, 0, (size_t)ctas * kEpiWarps * sizeof(unsigned), stream) != cudaSuccess) {
+      cudaGetLastError();
+      if (part) cudaFree(part);
+      if (flags) cudaFree(flags);
+      return SP24_ERR_CUDA;
+    }
+    w.part = part;
+    w.flags = flags;
+    w.ctas = ctas;
+  }
+  *out = w;
+  return SP24_OK;
+}
+
+// Zero the ready counters of every split-tail workspace of the current device
+// (after a kernel gave up waiting, one may have been left raised).
+sp24_status sk_clear_flags() {
+  const int dev = current_device();
+  if (dev < 0) return SP24_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_sk_mutex);
+  if (cudaDeviceSynchronize() != cudaSuccess) return SP24_ERR_CUDA;
+  for (auto &kv : g_sk_workspaces)
+    if (kv.first.first == dev && cudaMemset(kv.second.flags, 0, (size_t)kv.second.ctas * kEpiWarps * sizeof(unsigned)) !=
+                                     cudaSuccess)
+      return SP24_ERR_CUDA;
+  return SP24_OK;
+}
+
 // Weight gradient with decay: dec_w/dec_idx/dec_lambda (the masked decay of dW in
 // the epilogue); null dec_w elsewhere.
 template <bool BF16, int EPI, bool SPARSE>
@@ -222,9 +281,25 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   if (max_pairs <= 0) return max_pairs == 0 ? SP24_ERR_CUDA : SP24_ERR_NO_DEVICE;
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
-  return launch_pdl(kernel, dim3(2 * pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
+  // Weight gradient: when the last wave would leave pairs idle, split its r
+  // tiles along K into min(P / r, 8, num_kt) parts on all P pairs.
+  SkWorkspace ws;
+  int split = 1, grid_pairs = pairs;
+  const int64_t tail = tiles % max_pairs;
+  if (G::kWg && tail != 0) {
+    int64_t s = max_pairs / tail < num_kt ? max_pairs / tail : num_kt;
+    if (s > kMaxSplit) s = kMaxSplit;
+    if (s > 1) {
+      const sp24_status st = sk_workspace(stream, 2 * max_pairs, &ws);
+      if (st != SP24_OK) return st;
+      split = (int)s;
+      grid_pairs = max_pairs;
+    }
+  }
+  return launch_pdl(kernel, dim3(2 * grid_pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
-                    (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda);
+                    (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda, ws.part,
+                    ws.flags, split);
 }
 
 template <bool SPARSE>
@@ -648,6 +723,7 @@ sp24_status sp24_device_status(void *stream) {
   unsigned int word = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess) return SP24_ERR_CUDA;
   if (word && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return SP24_ERR_CUDA;
+  if (word && sk_clear_flags() != SP24_OK) return SP24_ERR_CUDA;
   return (word & kDevErrTimeout) ? SP24_ERR_TIMEOUT : SP24_OK;
 }
 

@@ -84,6 +84,38 @@ def test_mvue_leading_dimension_and_wide_bf16_groups():
     assert np.array_equal(got, bits)
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_mvue_raw_bit_groups_over_wide_exponent_spans(dtype):
+    """Groups of raw bits whose nonzero exponent fields span 0 to 24 binades, with
+    subnormals, zeros, the largest finite values (whose estimates S/2 overflow to
+    infinity on both sides) and random signs."""
+    T, N = 512, 192
+    mant, emax_field = (10, 30) if dtype == "f16" else (7, 254)
+    rng = np.random.default_rng(23 if dtype == "f16" else 24)
+    G = T // 4 * N
+    span = rng.integers(0, 25, G)
+    top = rng.integers(np.minimum(span, emax_field - 1), emax_field + 1)   # largest exponent field
+    e = top[:, None] - rng.integers(0, span[:, None] + 1, (G, 4))
+    e[:, 0] = np.where(rng.random(G) < 0.5, top, e[:, 0])
+    e = np.clip(e, 0, emax_field)
+    m = rng.integers(0, 1 << mant, (G, 4))
+    m[rng.random((G, 4)) < 0.05] = (1 << mant) - 1                        # with e = top: the largest finite
+    bits = (e << mant) | m
+    bits[rng.random((G, 4)) < 0.1] = 0
+    bits |= rng.integers(0, 2, (G, 4)) << 15
+    bits = bits.astype(np.uint16).reshape(T // 4, N, 4).transpose(0, 2, 1).reshape(T, N)
+    dy = torch.from_numpy(bits.view(np.int16)).view(si.DTYPES[dtype])
+    vals, meta = _alloc(N, T, dtype)
+    sp.sp24_mvue_sparsify(dy.cuda(), 5, 9, vals, meta)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    obits, keep, _ = oracle.mvue_sparsify_t(np.ascontiguousarray(bits), dtype, 5, 9)
+    ovals, ometa = oracle.compress_rows(obits, keep)
+    assert np.array_equal(si.bits16(vals.cpu()), ovals)
+    got, canon = _yhat_of(vals, meta, N, T, dtype)
+    assert np.array_equal(canon, ometa)
+
+
 def test_mvue_draws_depend_on_seed_and_offset_only():
     T, N = 256, 64
     dy = si.normal((T, N), 1.0, 9, "f16").cuda()
@@ -119,6 +151,53 @@ def test_wgrad_small(T, N, K, dtype):
     yhat, _ = _yhat_of(vals, meta, N, T, dtype)
     ref = oracle.weight_grad(oracle.to_f64(yhat, dtype), oracle.to_f64(si.bits16(x), dtype))
     _check_wgrad(dw, ref, f"wgrad {T}x{N}x{K}")
+
+
+@pytest.mark.parametrize("T,N,K,dtype", [(1024, 2560, 2048, "f16"), (896, 2608, 1800, "bf16")])
+def test_wgrad_stream_k_full_matrix(T, N, K, dtype):
+    """dW with more tiles than CTA pairs and not a multiple of them (80 and 88 tiles of
+    256 x 256 on 74 pairs): the stream-K schedule, where two pairs share a tile's K
+    steps and one adds the other's partial.  Every entry against the fp64 product
+    of the GPU's own Yhat, and the same bits from a second call."""
+    dy = si.normal((T, N), 1.0, T + 5, dtype)
+    x = si.normal((T, K), 1.0, T + 6, dtype)
+    vals, meta = _alloc(N, T, dtype)
+    sp.sp24_mvue_sparsify(dy.cuda(), 13, 2, vals, meta)
+    xd = x.cuda()
+    dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    again = torch.full((N, K), float("nan"), dtype=torch.float32, device="cuda")
+    sp.sp24_gemm_wgrad(xd, vals, meta, N, dw)
+    sp.sp24_gemm_wgrad(xd, vals, meta, N, again)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    assert torch.equal(dw.view(torch.int32), again.view(torch.int32))
+    yhat, _ = _yhat_of(vals, meta, N, T, dtype)
+    ref = oracle.weight_grad(oracle.to_f64(yhat, dtype), oracle.to_f64(si.bits16(x), dtype))
+    _check_wgrad(dw, ref, f"wgrad {T}x{N}x{K}")
+
+
+def test_wgrad_stream_k_timeout_reports_status_and_next_call_is_exact():
+    """A zero wait budget makes the stream-K launch give up (no bounded wait can
+    succeed late); the status reports it and clears any ready counter left raised,
+    so the next launch with the normal budget gives the same bits as before."""
+    T, N, K, dtype = 1024, 2560, 2048, "f16"
+    dy = si.normal((T, N), 1.0, 41, dtype)
+    x = si.normal((T, K), 1.0, 42, dtype).cuda()
+    vals, meta = _alloc(N, T, dtype)
+    sp.sp24_mvue_sparsify(dy.cuda(), 3, 4, vals, meta)
+    good = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    sp.sp24_gemm_wgrad(x, vals, meta, N, good)
+    assert sp.sp24_device_status() == 0
+    dw = torch.zeros(N, K, dtype=torch.float32, device="cuda")
+    sp.sp24_set_wait_budget(0)
+    try:
+        sp.sp24_gemm_wgrad(x, vals, meta, N, dw)
+        assert sp.sp24_device_status() == 6          # SP24_ERR_TIMEOUT
+    finally:
+        sp.sp24_set_wait_budget(1 << 32)
+    sp.sp24_gemm_wgrad(x, vals, meta, N, dw)
+    assert sp.sp24_device_status() == 0
+    assert torch.equal(dw.view(torch.int32), good.view(torch.int32))
 
 
 def test_wgrad_zero_tokens_gives_zeros():
