@@ -65,7 +65,9 @@ typedef enum sp24_status {
   SP24_ERR_MISALIGNED = 4,        /* a pointer or row pitch is not 16-byte aligned */
   SP24_ERR_CUDA = 5,              /* a CUDA runtime/driver call or launch failed */
   SP24_ERR_TIMEOUT = 6,           /* a kernel gave up waiting (see sp24_device_status) */
-  SP24_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+  SP24_ERR_NO_DEVICE = 7,         /* no sm_100 device is current */
+  SP24_ERR_SCRATCH_TOO_SMALL = 8  /* the call needs more than a fixed scratch holds
+                                     (sp24_gemm_wgrad_noalloc) */
 } sp24_status;
 
 typedef enum sp24_dtype { SP24_F16 = 0, SP24_BF16 = 1 } sp24_dtype;
@@ -266,6 +268,30 @@ SP24_API sp24_status sp24_mvue_sparsify(const void *dY, int64_t T, int64_t N, in
  */
 SP24_API sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
                             int64_t N, sp24_dtype dtype, float *dW, void *stream);
+
+/*
+ * sp24_gemm_wgrad without any device allocation.  The pages have no
+ * counterpart: this is a library entry point for callers that must not
+ * allocate device memory inside the call, for example a process whose device
+ * memory is all taken by its own allocator (a cudaMalloc there would fail), or a
+ * loop that must not pay for cudaMalloc's implicit synchronization on a
+ * stream's first call.  Same arguments, checks, kernel, split rule and result
+ * bits as sp24_gemm_wgrad; the split tail's partial sums go through one fixed
+ * scratch array in the library's static device memory instead of the
+ * per-stream workspace.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine; it zeroes the scratch's ready counters with cudaMemsetAsync on
+ * `stream` before each launch.
+ *   Limit: the scratch holds the partial sums of 128 CTAs (18,874,368 bytes)
+ *   and their counters (6,144 bytes).  A call whose split tail would use more,
+ *   i.e. 2 * r * s > 128 for r tail tiles split s ways (see sp24_gemm_wgrad),
+ *   launches nothing and returns SP24_ERR_SCRATCH_TOO_SMALL; calls without a
+ *   split tail use none of it.
+ *   Concurrency: every call on a device uses the same scratch, whatever its
+ *   stream or host thread, so calls that overlap in time race on it and give
+ *   wrong results; order them (one stream, or events between streams).
+ */
+SP24_API sp24_status sp24_gemm_wgrad_noalloc(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
+                                    int64_t N, sp24_dtype dtype, float *dW, void *stream);
 
 /*
  * Weight gradient and masked decay in one pass (abstract: the masked decay

@@ -40,6 +40,7 @@ _SIGNATURES = {
     "sp24_transpose": [P, I64, I64, I32, P, P],
     "sp24_mvue_sparsify": [P, I64, I64, I64, I32, U64, U64, P, P, P],
     "sp24_gemm_wgrad": [P, I64, I64, P, P, I64, I32, P, P],
+    "sp24_gemm_wgrad_noalloc": [P, I64, I64, P, P, I64, I32, P, P],
     "sp24_gemm_wgrad_decay": [P, I64, I64, P, P, I64, I32, P, P, F32, P, P],
     "sp24_gemm_wgrad_dense": [P, I64, I64, P, I64, I32, P, P],
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
@@ -58,7 +59,7 @@ _lib.sp24_status_string.restype = ctypes.c_char_p
 
 STATUS = {0: "SP24_OK", 1: "SP24_ERR_INVALID_ARG", 2: "SP24_ERR_UNSUPPORTED_SHAPE",
           3: "SP24_ERR_UNSUPPORTED_DTYPE", 4: "SP24_ERR_MISALIGNED", 5: "SP24_ERR_CUDA",
-          6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE"}
+          6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE", 8: "SP24_ERR_SCRATCH_TOO_SMALL"}
 SP24_F16, SP24_BF16 = 0, 1
 SP24_EPI_NONE, SP24_EPI_GELU, SP24_EPI_DGELU = 0, 1, 2
 EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4, "gelu_deriv": 6, "mul_aux": 7}
@@ -312,6 +313,22 @@ def sp24_gemm_wgrad(X, vals, meta, N: int, dW, stream=None):
     _check("sp24_gemm_wgrad",
            _lib.sp24_gemm_wgrad(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(dW),
                                 _stream(stream)))
+
+
+def sp24_gemm_wgrad_noalloc(X, vals, meta, N: int, dW, stream=None):
+    """sp24_gemm_wgrad through the library's fixed static scratch: no device allocation in the
+    call; calls overlapping in time race on the scratch; SP24_ERR_SCRATCH_TOO_SMALL when the
+    split tail would need more than it holds."""
+    import torch
+    _need_rowmajor(X, vals, meta, dW)
+    T, K = _shape2(X, "X")
+    _dtype_code(X)
+    _expect_compressed(vals, meta, N, T, X.dtype, "MVUE(dY^T)")
+    _expect(dW, "dW", torch.float32, N * K)
+    _need_device(X, vals, meta, dW)
+    _check("sp24_gemm_wgrad_noalloc",
+           _lib.sp24_gemm_wgrad_noalloc(_ptr(X), T, K, _ptr(vals), _ptr(meta), N, _dtype_code(X), _ptr(dW),
+                                        _stream(stream)))
 
 
 def sp24_gemm_wgrad_decay(X, vals, meta, N: int, W, idx, lam: float, dW, stream=None):

@@ -229,12 +229,45 @@ sp24_status sk_clear_flags() {
   return SP24_OK;
 }
 
+// Fixed scratch of sp24_gemm_wgrad_noalloc, in the module's static device
+// memory (zero at load): the split-tail partial sums of kNoAllocCtas CTAs, then
+// their ready counters.
+constexpr int kNoAllocCtas = 128;
+constexpr size_t kNoAllocPartBytes = (size_t)kNoAllocCtas * kSkPartFloatsPerCta * sizeof(float);
+constexpr size_t kNoAllocBytes = kNoAllocPartBytes + (size_t)kNoAllocCtas * kEpiWarps * sizeof(unsigned);
+static_assert(kNoAllocPartBytes % 256 == 0, "counters start 256-byte aligned");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Its address on the current device, looked up once per device (with that
+// device current) and checked.
+sp24_status noalloc_scratch(SkWorkspace *out) {
+  static std::once_flag once[kMaxDevices];
+  static void *addr[kMaxDevices];
+  static cudaError_t err[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return SP24_ERR_NO_DEVICE;
+  std::call_once(once[dev], [dev] {
+    void *p = nullptr;
+    err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err[dev] != cudaSuccess) cudaGetLastError();
+    addr[dev] = p;
+  });
+  if (err[dev] != cudaSuccess || addr[dev] == nullptr) return SP24_ERR_CUDA;
+  out->part = static_cast<float *>(addr[dev]);
+  out->flags = reinterpret_cast<unsigned *>(static_cast<unsigned char *>(addr[dev]) + kNoAllocPartBytes);
+  out->ctas = kNoAllocCtas;
+  return SP24_OK;
+}
+
 // Weight gradient with decay: dec_w/dec_idx/dec_lambda (the masked decay of dW in
-// the epilogue); null dec_w elsewhere.
+// the epilogue); null dec_w elsewhere.  `fixed`: a caller-given split-tail
+// scratch (its counters are zeroed here before the launch) instead of the
+// per-stream workspace; null for every entry point but sp24_gemm_wgrad_noalloc.
 template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream, const void *dec_w = nullptr,
-                               const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f) {
+                               const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f,
+                               const SkWorkspace *fixed = nullptr) {
   using G = PairGeom<SPARSE, EPI>;
   const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
@@ -290,8 +323,18 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
     int64_t s = max_pairs / tail < num_kt ? max_pairs / tail : num_kt;
     if (s > kMaxSplit) s = kMaxSplit;
     if (s > 1) {
-      const sp24_status st = sk_workspace(stream, 2 * max_pairs, &ws);
-      if (st != SP24_OK) return st;
+      if (fixed) {   // CTAs 0 .. 2 tail s - 1 use their partial slots and counters
+        const int64_t used = 2 * tail * s;
+        if (used > fixed->ctas) return SP24_ERR_SCRATCH_TOO_SMALL;
+        ws = *fixed;
+        if (cudaMemsetAsync(ws.flags, 0, (size_t)used * kEpiWarps * sizeof(unsigned), stream) != cudaSuccess) {
+          cudaGetLastError();
+          return SP24_ERR_CUDA;
+        }
+      } else {
+        const sp24_status st = sk_workspace(stream, 2 * max_pairs, &ws);
+        if (st != SP24_OK) return st;
+      }
       split = (int)s;
       grid_pairs = max_pairs;
     }
@@ -424,8 +467,9 @@ inline size_t meta_nibble_pos(int64_t r, int64_t g, int64_t cols, int *shift) {
 template <bool BF16, bool SPARSE>
 sp24_status launch_wgrad(const void *X, int64_t T, int64_t K, const void *A, const void *meta, int64_t N, float *dW,
                          cudaStream_t s, const void *dec_w = nullptr, const uint8_t *dec_idx = nullptr,
-                         float dec_lambda = 0.0f) {
-  return launch_gemm_pair_t<BF16, kEpiWgrad, SPARSE>(X, K, T, A, meta, N, dW, nullptr, s, dec_w, dec_idx, dec_lambda);
+                         float dec_lambda = 0.0f, const SkWorkspace *fixed = nullptr) {
+  return launch_gemm_pair_t<BF16, kEpiWgrad, SPARSE>(X, K, T, A, meta, N, dW, nullptr, s, dec_w, dec_idx, dec_lambda,
+                                                     fixed);
 }
 
 }  // namespace
@@ -442,6 +486,7 @@ const char *sp24_status_string(sp24_status st) {
     case SP24_ERR_CUDA: return "SP24_ERR_CUDA";
     case SP24_ERR_TIMEOUT: return "SP24_ERR_TIMEOUT";
     case SP24_ERR_NO_DEVICE: return "SP24_ERR_NO_DEVICE";
+    case SP24_ERR_SCRATCH_TOO_SMALL: return "SP24_ERR_SCRATCH_TOO_SMALL";
   }
   return "SP24_UNKNOWN_STATUS";
 }
@@ -608,6 +653,28 @@ sp24_status sp24_gemm_wgrad(const void *X, int64_t T, int64_t K, const void *val
   }
   return dtype == SP24_BF16 ? launch_wgrad<true, true>(X, T, K, vals, meta, N, dW, s)
                             : launch_wgrad<false, true>(X, T, K, vals, meta, N, dW, s);
+}
+
+sp24_status sp24_gemm_wgrad_noalloc(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
+                                    int64_t N, sp24_dtype dtype, float *dW, void *stream) {
+  if (T < 0 || K < 0 || N < 0) return SP24_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
+  if (T % 16 || N % 16 || K % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (T > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!dW || (T > 0 && (!X || !vals || !meta))) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (T > 0 && (!aligned16(X) || !aligned16(vals) || !aligned16(meta)))) return SP24_ERR_MISALIGNED;
+  sp24_status st = check_device();
+  if (st != SP24_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {   // an empty sum over tokens
+    return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  }
+  SkWorkspace fixed;
+  st = noalloc_scratch(&fixed);
+  if (st != SP24_OK) return st;
+  return dtype == SP24_BF16 ? launch_wgrad<true, true>(X, T, K, vals, meta, N, dW, s, nullptr, nullptr, 0.0f, &fixed)
+                            : launch_wgrad<false, true>(X, T, K, vals, meta, N, dW, s, nullptr, nullptr, 0.0f, &fixed);
 }
 
 sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const void *vals, const void *meta,
