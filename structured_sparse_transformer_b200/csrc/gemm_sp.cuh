@@ -842,8 +842,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           ++pre_used;
           pre_src = stg_u32 + kOutBytes + kPreBytes * (seq & 1);
         }
-        if (lane == 0) bulk_wait_group_read<0>();   // the previous chunk's stores have read the staging tiles
-        __syncwarp();
+        // The staging tiles are rewritten only once the previous chunk's TMA
+        // stores have read them: the gated epilogues wait here, the others after
+        // their arithmetic (which then overlaps those reads).
+        auto staging_free = [&]() {
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+        };
+        if (EPI == kEpiGeglu || EPI == kEpiDgeglu) staging_free();
         // Register i of half h: tokens 8(i/2) + 2(lane%4) + {0, 1} of feature
         // 16h + 8(i%2) + lane/4 (TMEM registers 4(i/2) + 2(i%2) + {0, 1}).
         if (EPI == kEpiGeglu) {
@@ -923,6 +929,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               po[h][i] = pack2<BF16>(y.x, y.y);
             }
           }
+          staging_free();
           stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);
           stmatrix_x4_trans(stg_u32 + lane_off1, po[1]);
           if (EPI == kEpiGelu || EPI == kEpiGeluDeriv) {
