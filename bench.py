@@ -319,14 +319,12 @@ class FFNStep:
     def run_dense(self, events=None):
         """One step of the dense fine-tuning phase (the last 1/6 of the steps):
         W^T of both weights (they change every step), the six FFN products on
-        the dense tensor-core path (the weight gradients take dY^T and dH^T from
-        the transpose kernel); no mask, compression or decay."""
+        the dense tensor-core path (the weight gradients read dY and dH as
+        stored); no mask, compression or decay."""
         sp, torch = self.sp, self.torch
         cur = self.step_no % self.S + 1
         if not hasattr(self, "Wt"):
             self.Wt = [torch.empty(w[0].shape[1], w[0].shape[0], dtype=w[0].dtype, device="cuda") for w in self.W]
-            self.dYt = torch.empty(self.dY.shape[1], self.dY.shape[0], dtype=self.dY.dtype, device="cuda")
-            self.dHt = torch.empty(self.dH.shape[1], self.dH.shape[0], dtype=self.dH.dtype, device="cuda")
 
         def timed(name, fn):
             if events is None:
@@ -344,10 +342,8 @@ class FFNStep:
         timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu_deriv", self.Gp))
         timed("gemm_fwd2", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
         timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "mul_aux", self.Gp))
-        timed("transpose_act", lambda: sp.sp24_transpose(self.dY, self.dYt))
-        timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dYt, self.G[1]))
-        timed("transpose_act", lambda: sp.sp24_transpose(self.dH, self.dHt))
-        timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dHt, self.G[0]))
+        timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dY, self.G[1]))
+        timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dH, self.G[0]))
         timed("gemm_dgrad1", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
         self.step_no += 1
 
@@ -643,16 +639,15 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks):
     n_el = wl.d * wl.ff
     work = {k: ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff) for k in FFNStep.GEMMS + ("gemm_wgrad2", "gemm_wgrad1")}
     work["transpose"] = ("GB/s", 4 * n_el)
-    work["transpose_act"] = ("GB/s", 4 * wl.tokens * (wl.d + wl.ff) / 2)
     dense_peaks = dict(peaks)
     dense_peaks["bf16_tflops"] = peaks["bf16_tflops"] / 2.0   # kernel_table doubles it for the 2:4 peak
     kernels = kernel_table(events, work, dense_peaks, list(work))
     return {"ms_per_step": round(ms, 4),
             "value": round(6 * 2.0 * wl.tokens * wl.d * wl.ff * world / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "kernels": kernels,
-            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights, dY^T and dH^T, and "
-                    "the six FFN products (forward, input gradient, weight gradient) on the dense tcgen05 "
-                    "path, same workload; FLOPs 6 x 2 T d ff; GEMM peak = the dense bf16 burst"}
+            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights and the six FFN "
+                    "products (forward, input gradient, weight gradient reading dY and dH as stored) on the "
+                    "dense tcgen05 path, same workload; FLOPs 6 x 2 T d ff; GEMM peak = the dense bf16 burst"}
 
 
 class GegluStep:

@@ -316,16 +316,17 @@ SP24_API sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, 
  * Dense weight-gradient GEMM for the dense fine-tuning phase (abstract: dense
  * fine-tuning; Experiment Setup row: the last 1/6 of the steps):
  * dW[N x K] = dY^T[N x T] * X[T x K], fp32 accumulation and fp32 output in W's
- * layout, on the same tcgen05 pipeline (X read as stored, dY^T from
- * sp24_transpose of dY).
+ * layout, on the same tcgen05 pipeline.  Both operands are read as stored (the
+ * tensor memory accelerator loads them in 64-column atoms, MN-major): no
+ * transpose of dY.
  *   X     device [T x K] row-major, contiguous
- *   dYt   device [N x T] row-major, contiguous (dY transposed)
+ *   dY    device [T x N] row-major, contiguous (the output gradient)
  *   dW    device fp32 [N x K] contiguous, overwritten (zeros when T == 0)
  * T % 16 == 0, N % 16 == 0, K % 8 == 0; all pointers 16-byte aligned.
  * Tiles, split tail and workspace as for sp24_gemm_wgrad (64 tokens per K step:
  * s <= ceil(T / 64)).
  */
-SP24_API sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N,
+SP24_API sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dY, int64_t N,
                                   sp24_dtype dtype, float *dW, void *stream);
 
 /*

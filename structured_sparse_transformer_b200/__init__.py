@@ -347,18 +347,20 @@ def sp24_gemm_wgrad_decay(X, vals, meta, N: int, W, idx, lam: float, dW, stream=
                                       float(lam), _ptr(dW), _stream(stream)))
 
 
-def sp24_gemm_wgrad_dense(X, dYt, dW, stream=None):
-    """dW[N, K] (fp32) <- dYt[N, T] X[T, K] on the dense tensor-core path (dYt = dY transposed)."""
+def sp24_gemm_wgrad_dense(X, dY, dW, stream=None):
+    """dW[N, K] (fp32) <- dY[T, N]^T X[T, K] on the dense tensor-core path (dY as stored)."""
     import torch
-    _need_rowmajor(X, dYt, dW)
+    _need_rowmajor(X, dY, dW)
     T, K = _shape2(X, "X")
-    N = _shape2(dYt, "dYt")[0]
+    T2, N = _shape2(dY, "dY")
+    if T2 != T:
+        raise ValueError(f"dY has {T2} rows, X has {T}")
     _dtype_code(X)
-    _expect(dYt, "dYt", X.dtype, N * T)
+    _expect(dY, "dY", X.dtype, N * T)
     _expect(dW, "dW", torch.float32, N * K)
-    _need_device(X, dYt, dW)
+    _need_device(X, dY, dW)
     _check("sp24_gemm_wgrad_dense",
-           _lib.sp24_gemm_wgrad_dense(_ptr(X), T, K, _ptr(dYt), N, _dtype_code(X), _ptr(dW), _stream(stream)))
+           _lib.sp24_gemm_wgrad_dense(_ptr(X), T, K, _ptr(dY), N, _dtype_code(X), _ptr(dW), _stream(stream)))
 
 
 def sp24_masked_decay(grad, W, idx, lam: float, stream=None):

@@ -113,8 +113,9 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // 64-column halves make the 128), into accumulator columns 0 and 128: an MMA
 // never spans two atoms along N.  One 256-column accumulator (no double
 // buffering: the weight-gradient tiles run one per pair at the FFN sizes).
-// The dense variant (dense fine-tuning) takes A = dY^T [N x T] dense, 64 tokens
-// per stage: A 16 KB + two 8 KB atoms, 6 stages; each 16-token K step issues
+// The dense variant (dense fine-tuning) takes A = dY [T x N] as stored, read
+// MN-major like B (two 8 KB atoms of 64 rows of dW x 64 tokens), 64 tokens per
+// stage: A 16 KB + two 8 KB atoms of B, 6 stages; each 16-token K step issues
 // two dense MMAs of N = 128.  (Tiles of 128 dW columns with double-buffered
 // accumulators were measured 10-15% slower at the 1.5B shapes, although they
 // leave fewer column-waves idle: each stage then carries half the MMA work for
@@ -486,7 +487,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         uint8_t *st = stage_base + s * kPairStageBytes;
         if (is_leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
-        tma_load_2d_pair(st, &tm_a, &full[s], kt * G::kAcols, a_row);
+        if (WG && !SPARSE) {
+          // Dense weight gradient: A = dY as stored, MN-major, in two 64-row atoms
+          // (x = dW row, y = token), 8 KB apart.
+          tma_load_2d_pair(st, &tm_a, &full[s], a_row, kt * G::kBK);
+          tma_load_2d_pair(st + kPairSmemA / 2, &tm_a, &full[s], a_row + 64, kt * G::kBK);
+        } else {
+          tma_load_2d_pair(st, &tm_a, &full[s], kt * G::kAcols, a_row);
+        }
         if (WG) {
           // MN-major atoms: x = dW column (b_row, b_row + 128), y = token.
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], b_row, kt * G::kBK);
@@ -515,12 +523,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // Its B descriptor steps 8-token groups 1024 bytes apart (the stride field);
     // an MMA reads a single 64-column atom per CTA, so the field for the stride
     // between atoms along N is never used and is given the same 1024.
+    // Dense wgrad: A MN-major too (bit 15); its descriptor's leading field is the
+    // 8 KB between its two 64-row atoms, its stride field the 1024 bytes between
+    // 8-token groups.
     constexpr uint32_t idesc = WG ? ((SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, 128)
-                                             : make_idesc_dense(BF16, 2 * kPairRows, 128)) |
+                                             : (make_idesc_dense(BF16, 2 * kPairRows, 128) | (1u << 15))) |
                                     (1u << 16))
                                : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN)
                                         : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
-    const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), 16, 1024, kSwizzle128B);
+    const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), (WG && !SPARSE) ? kPairSmemA / 2 : 16, 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
     const uint64_t e_desc0 =
         smem_desc(smem_u32(stage_base + kPairSmemA + G::kBBoxes * G::kBBoxBytes), 128, 128, kSwizzleNone);
@@ -542,15 +553,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const uint64_t so = (uint64_t)((s * kPairStageBytes) >> 4);
         const uint64_t ad = a_desc0 + so, bd = b_desc0 + so;
         if (WG && !SPARSE) {
-          // Dense weight gradient: K step kk of 16 tokens moves A 32 bytes along its
-          // swizzled rows and B 16 tokens (2048 bytes); atom 1 of B sits 8 KB after atom 0.
+          // Dense weight gradient: K step kk of 16 tokens moves A and B 16 tokens
+          // (2048 bytes) each; atom 1 of B sits 8 KB after atom 0.
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kt != kb || kk != 0) ? 1u : 0u;
+            const uint64_t ak = ad + (uint64_t)(kk * (2048 >> 4));
             const uint64_t bk = bd + (uint64_t)(kk * (2048 >> 4));
-            tc_mma_f16_pair(acc, ad + 2 * kk, bk, idesc, accum);
+            tc_mma_f16_pair(acc, ak, bk, idesc, accum);
             if (G::kBBoxes == 2)
-              tc_mma_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
+              tc_mma_f16_pair(acc + 128, ak, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
           }
         } else if (WG) {
           const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;

@@ -277,9 +277,13 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
                                          CU_TENSOR_MAP_SWIZZLE_128B)
                            : make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh,
                                          CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!make_map_2d(&ta, vals, a_cols, (uint64_t)M, a_cols * 2, G::kAcols, kPairRows, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !b_ok)
-    return SP24_ERR_CUDA;
+  // Dense weight gradient: A = dY [Kd tokens x M] read MN-major in 64 x kBK boxes.
+  const bool a_ok = (G::kWg && !SPARSE)
+                        ? make_map_2d(&ta, vals, (uint64_t)M, (uint64_t)Kd, (uint64_t)M * 2, 64, (uint32_t)G::kBK,
+                                      CU_TENSOR_MAP_SWIZZLE_128B)
+                        : make_map_2d(&ta, vals, a_cols, (uint64_t)M, a_cols * 2, G::kAcols, kPairRows,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!a_ok || !b_ok) return SP24_ERR_CUDA;
   if (SPARSE) {
     if (!make_map_2d(&tm, meta, kSmemE / 8, (uint64_t)(row_tiles * num_kt), kSmemE, kSmemE / 8, 1,
                      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT64))
@@ -699,23 +703,23 @@ sp24_status sp24_gemm_wgrad_decay(const void *X, int64_t T, int64_t K, const voi
                             : launch_wgrad<false, true>(X, T, K, vals, meta, N, dW, s, W, idx, lambda);
 }
 
-sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dYt, int64_t N, sp24_dtype dtype,
+sp24_status sp24_gemm_wgrad_dense(const void *X, int64_t T, int64_t K, const void *dY, int64_t N, sp24_dtype dtype,
                                   float *dW, void *stream) {
   if (T < 0 || K < 0 || N < 0) return SP24_ERR_INVALID_ARG;
   if (!valid_dtype(dtype)) return SP24_ERR_UNSUPPORTED_DTYPE;
   if (T % 16 || N % 16 || K % 8) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (T > INT32_MAX || K > INT32_MAX || N > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (N == 0 || K == 0) return SP24_OK;
-  if (!dW || (T > 0 && (!X || !dYt))) return SP24_ERR_INVALID_ARG;
-  if (!aligned16(dW) || (T > 0 && (!aligned16(X) || !aligned16(dYt)))) return SP24_ERR_MISALIGNED;
+  if (!dW || (T > 0 && (!X || !dY))) return SP24_ERR_INVALID_ARG;
+  if (!aligned16(dW) || (T > 0 && (!aligned16(X) || !aligned16(dY)))) return SP24_ERR_MISALIGNED;
   sp24_status st = check_device();
   if (st != SP24_OK) return st;
   cudaStream_t s = as_stream(stream);
   if (T == 0) {   // an empty sum over tokens
     return cudaMemsetAsync(dW, 0, (size_t)N * (size_t)K * sizeof(float), s) == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
   }
-  return dtype == SP24_BF16 ? launch_wgrad<true, false>(X, T, K, dYt, nullptr, N, dW, s)
-                            : launch_wgrad<false, false>(X, T, K, dYt, nullptr, N, dW, s);
+  return dtype == SP24_BF16 ? launch_wgrad<true, false>(X, T, K, dY, nullptr, N, dW, s)
+                            : launch_wgrad<false, false>(X, T, K, dY, nullptr, N, dW, s);
 }
 
 sp24_status sp24_masked_decay(float *grad, const void *W, sp24_dtype dtype, int64_t rows, int64_t cols,

@@ -219,7 +219,8 @@ def test_binding_rejects_wrong_dtype_and_short_buffers():
     ok_until_device(sp.sp24_gemm_wgrad, x, yv, ym, R, dw)
     bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw[:10], match="dW")
     bad(sp.sp24_gemm_wgrad, x, yv, ym, R, dw.half(), match="dW")
-    bad(sp.sp24_gemm_wgrad_dense, x, torch.zeros(R, T, dtype=f16), dw.double(), match="dW")
+    bad(sp.sp24_gemm_wgrad_dense, x, torch.zeros(T, R, dtype=f16), dw.double(), match="dW")
+    bad(sp.sp24_gemm_wgrad_dense, x, torch.zeros(R, T, dtype=f16), dw, match="rows")
     wt = torch.zeros(R, C, dtype=f16)
     ok_until_device(sp.sp24_gemm_wgrad_decay, x, yv, ym, R, wt, idx.reshape(-1)[:(R // 4) * (C // 4)].clone(), 1e-4, dw)
     bad(sp.sp24_gemm_wgrad_decay, x, yv, ym, R, wt[:, :64].contiguous(), idx, 1e-4, dw, match="W:")

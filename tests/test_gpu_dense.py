@@ -104,12 +104,11 @@ def _check_wgrad(dw, ref, what=""):
 @pytest.mark.parametrize("T,N,K,dtype", [(128, 256, 256, "f16"), (256, 272, 200, "f16"), (144, 160, 520, "bf16"),
                                          (16, 16, 8, "f16"), (2048, 512, 1024, "f16")])
 def test_dense_weight_grad(T, N, K, dtype):
-    """dW = dY^T X with dY^T from the transpose kernel (ragged M, N and K tiles)."""
+    """dW = dY^T X with both operands read as stored (ragged M, N and K tiles)."""
     dy = si.normal((T, N), 1.0, T + 5, dtype)
     x = si.normal((T, K), 1.0, T + 6, dtype)
-    dyt = _transpose(dy.cuda())
     dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
-    sp.sp24_gemm_wgrad_dense(x.cuda(), dyt, dw)
+    sp.sp24_gemm_wgrad_dense(x.cuda(), dy.cuda(), dw)
     torch.cuda.synchronize()
     assert sp.sp24_device_status() == 0
     ref = oracle.dense_weight_grad(oracle.to_f64(si.bits16(dy), dtype), oracle.to_f64(si.bits16(x), dtype))
@@ -123,9 +122,8 @@ def test_dense_weight_grads_full_size_sampled_rows(wl):
     rng = np.random.default_rng(2)
     for g, b in ((dY, H), (dH, X)):
         N, K = g.shape[1], b.shape[1]
-        gt = _transpose(g.cuda())
         dw = torch.empty(N, K, dtype=torch.float32, device="cuda")
-        sp.sp24_gemm_wgrad_dense(b.cuda(), gt, dw)
+        sp.sp24_gemm_wgrad_dense(b.cuda(), g.cuda(), dw)
         torch.cuda.synchronize()
         assert sp.sp24_device_status() == 0
         rows = np.sort(rng.choice(N, 64, replace=False))
