@@ -400,11 +400,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out,
                           const uint16_t *__restrict__ dec_w, const uint8_t *__restrict__ dec_idx,
                           float dec_lambda, float *__restrict__ sk_part, unsigned *__restrict__ sk_flags,
-                          int sk_split) {
+                          int sk_split, int cols_fastest) {
   // T counts the B operand's rows of the output: tokens, or for the weight
   // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
   // Weight gradient with dec_w set: the masked decay of dW in the epilogue, W and
   // its pattern indices dec_idx [M/4][T/4] in the layout of dW (see below).
+  // Weight gradient with cols_fastest set: tiles are numbered along dW's
+  // columns first, so a wave of pairs shares the row tiles' A operand (chosen
+  // when A is the larger operand, which each wave would otherwise read again).
   // Weight gradient with sk_part set: the split-tail schedule with sk_split
   // parts per tail tile, partial accumulators in sk_part (kSkPartFloatsPerCta
   // per CTA) and ready counters in sk_flags (kEpiWarps per CTA, zero at launch
@@ -434,7 +437,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_mt = (M + 2 * kPairRows - 1) / (2 * kPairRows);
   const int num_row_tiles = (M + kPairRows - 1) / kPairRows;
-  const int num_tiles = num_mt * ((T + G::kBN - 1) / G::kBN);
+  const int num_nt = (T + G::kBN - 1) / G::kBN;
+  const int num_tiles = num_mt * num_nt;
+  const bool by_cols = WG && cols_fastest != 0;
+  auto tile_mt = [&](int t) { return by_cols ? t / num_nt : t % num_mt; };
+  auto tile_nt = [&](int t) { return by_cols ? t % num_nt : t / num_mt; };
   const int split = (WG && sk_part != nullptr) ? sk_split : 1;
 
   if (threadIdx.x == 0) {
@@ -473,9 +480,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     PairSchedule sched(split, pair, npairs, num_tiles, num_kt);
     int tile, kb, ke;
     while (ok && sched.next(tile, kb, ke)) {
-      const int mt = tile % num_mt;
+      const int mt = tile_mt(tile);
       const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
-      const int b_row = (tile / num_mt) * G::kBN + (int)rank * (WG ? 64 : kPairBNh);
+      const int b_row = tile_nt(tile) * G::kBN + (int)rank * (WG ? 64 : kPairBNh);
       // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
       // it the last real metadata chunk so every code the MMA sees is valid.
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
@@ -638,8 +645,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool to_part = kbeg > 0;                   // a later part of a split tile: another pair stores it
       const bool merge = kbeg == 0 && kend < num_kt;   // part 0: pairs p + 1 .. p + split - 1 hold the rest
       const bool decay = dec_w != nullptr && !to_part;
-      const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
-      const int n0 = (tile / num_mt) * G::kBN;
+      const int m0 = tile_mt(tile) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
+      const int n0 = tile_nt(tile) * G::kBN;
       // Decay operands of the warp's stores in this tile: W's two values (one
       // 32-bit word) and their two keep bits; entries outside dW keep both.
       uint32_t wv[kPerWarp][8], kb[kPerWarp];

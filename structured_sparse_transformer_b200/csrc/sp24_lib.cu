@@ -318,6 +318,11 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   if (max_pairs <= 0) return max_pairs == 0 ? SP24_ERR_CUDA : SP24_ERR_NO_DEVICE;
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  // Weight gradient: number the tiles along dW's columns first when the A
+  // operand is the larger one (each wave of pairs then reads it once).
+  const double a_bytes = (double)M * (double)Kd * (SPARSE ? 1.0 + 1.0 / 8 : 2.0);
+  const double b_bytes = (double)Kd * (double)T * 2.0;
+  const int cols_fastest = (G::kWg && a_bytes > b_bytes) ? 1 : 0;
   // Weight gradient: when the last wave would leave pairs idle, split its r
   // tiles along K into min(P / r, 8, num_kt) parts on all P pairs.
   SkWorkspace ws;
@@ -346,7 +351,7 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   return launch_pdl(kernel, dim3(2 * grid_pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
                     (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda, ws.part,
-                    ws.flags, split);
+                    ws.flags, split, cols_fastest);
 }
 
 template <bool SPARSE>
