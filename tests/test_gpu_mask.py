@@ -104,6 +104,65 @@ def test_mask_search_sweep_sampled_rows(shape, seed, kind):
         assert np.array_equal(got[br:br + 1], exp), br
 
 
+def _device_weights(R, C, seed, kind, update_seed=None):
+    """fp16 [R, C] drawn on the device in row slabs: N(0, 0.02) (or its 8-level tie-heavy
+    rounding), optionally followed by one N(0, 1e-4) update."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    w = torch.empty(R, C, dtype=torch.float16, device="cuda")
+    for r0 in range(0, R, 1024):
+        x = torch.randn(min(1024, R - r0), C, device="cuda", generator=g) * 0.02
+        if kind == "tie":
+            x = torch.clamp(torch.round(x / 2.0**-6), -4, 3) * 2.0**-6
+        w[r0:r0 + x.shape[0]] = x.half()
+    if update_seed is not None:
+        g.manual_seed(update_seed)
+        for r0 in range(0, R, 1024):
+            sl = w[r0:r0 + 1024]
+            sl.copy_((sl.float() + torch.randn(sl.shape, device="cuda", generator=g) * 1e-4).half())
+    return w
+
+
+@pytest.mark.parametrize("kind,seed", [("normal", 31), ("tie", 32)])
+def test_mask_step_at_the_sweep_size(kind, seed):
+    """The fused mask step on a 2 GiB fp16 weight (16384 x 65536, the sweep's largest size):
+    the mask and the flip count equal the separate search and flip kernels in full, and 12
+    sampled 16-row strips of the mask and of both compressed orientations equal the oracle."""
+    R, C = 16384, 65536
+    w0 = _device_weights(R, C, seed, kind)
+    prev = torch.empty(R // 4, C // 4, dtype=torch.uint8, device="cuda")
+    sp.sp24_mask_search(w0, prev)
+    del w0
+    w1 = _device_weights(R, C, seed, kind, update_seed=seed + 100)
+    idx = torch.empty_like(prev)
+    count = torch.zeros(1, dtype=torch.int64, device="cuda")
+    bufs = sp.alloc_compressed(R, C, torch.float16)
+    sp.sp24_mask_step(w1, idx, prev, count, *bufs)
+    sep = torch.empty_like(prev)
+    sp.sp24_mask_search(w1, sep)
+    cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sp.sp24_flip_rate(prev, sep, cnt)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    assert torch.equal(idx, sep)
+    assert int(count.item()) == int(cnt.item()) > 0
+    mr = sp.sp24_meta_to_canonical(bufs[1].cpu().numpy().tobytes(), R, C)
+    mc = sp.sp24_meta_to_canonical(bufs[3].cpu().numpy().tobytes(), C, R)
+    vr, vc = bufs[0], bufs[2]
+    idx_h = idx.cpu().numpy()
+    rng = np.random.default_rng(seed)
+    for s16 in np.sort(rng.choice(R // 16, 12, replace=False)):
+        r0 = 16 * int(s16)
+        bits = si.bits16(w1[r0:r0 + 16].cpu())
+        i_o = oracle.mask_search(bits, "f16")
+        assert np.array_equal(idx_h[r0 // 4:r0 // 4 + 4], i_o), r0
+        (vr_o, mr_o), (vc_o, mc_o) = oracle.compress_both(bits, i_o)
+        assert np.array_equal(bits_of(vr[r0:r0 + 16]), vr_o), r0
+        assert np.array_equal(mr[r0:r0 + 16], mr_o), r0
+        assert np.array_equal(bits_of(vc[:, r0 // 2:r0 // 2 + 8].contiguous()), vc_o), r0
+        assert np.array_equal(mc[:, r0 // 16:r0 // 16 + 1], mc_o), r0
+
+
 # -------------------------------------------------------------- compression
 
 def _compress_gpu(w_cpu, idx_np):
