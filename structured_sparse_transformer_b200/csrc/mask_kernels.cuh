@@ -454,7 +454,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
                                                unsigned &flips, uint16_t *__restrict__ vals_row,
                                                uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
                                                uint8_t *__restrict__ meta_col, MaskSmem<SEARCH, COMPRESS> &sm,
-                                               uint32_t one) {
+                                               uint32_t one, const uint8_t *s_prev = nullptr) {
   const int tid = threadIdx.x;
   const int rh = tid >> 7, lt = tid & (kQuadThreads - 1);
 
@@ -475,8 +475,14 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
   src.unit(lr, lc, ok0, ok1, w);
   uint32_t prev[2] = {0, 0}, given[2] = {kPadIndex, kPadIndex};
   if (FLIP) {
-    if (ok0) prev[0] = idx_prev[bidx0];
-    if (ok1) prev[1] = idx_prev[bidx0 + 1];
+    if (s_prev) {   // the previous mask's tile, staged with W: [32 block rows][16 block columns]
+      const int pr = (kTile / 4) * rh + br;
+      if (ok0) prev[0] = s_prev[pr * (kTile / 4) + 2 * uc];
+      if (ok1) prev[1] = s_prev[pr * (kTile / 4) + 2 * uc + 1];
+    } else {
+      if (ok0) prev[0] = idx_prev[bidx0];
+      if (ok1) prev[1] = idx_prev[bidx0 + 1];
+    }
   }
   if (!SEARCH) {
     if (ok0) given[0] = idx[bidx0];
@@ -669,8 +675,11 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
     const __grid_constant__ CUtensorMap tm_w, int64_t R, int64_t C, uint8_t *__restrict__ idx,
     const uint8_t *__restrict__ idx_prev, unsigned long long *__restrict__ flip_count,
     uint16_t *__restrict__ vals_row, uint8_t *__restrict__ meta_row, uint16_t *__restrict__ vals_col,
-    uint8_t *__restrict__ meta_col, uint64_t wait_budget) {
+    uint8_t *__restrict__ meta_col, uint64_t wait_budget, const __grid_constant__ CUtensorMap tm_prev,
+    int prev_tma) {
   __shared__ __align__(128) uint16_t s_w[2][kChunk * kTile];
+  // FLIP with prev_tma: the previous mask's bytes of each tile arrive with it.
+  __shared__ __align__(128) uint8_t s_prev[2][(kChunk / 4) * (kTile / 4)];
   __shared__ MaskSmem<SEARCH, COMPRESS> sm;
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ unsigned long long s_flip;
@@ -688,14 +697,18 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
     uint32_t cy, cx;
     int kh;
     tile_xy(t, cy, cx, kh);
-    mbar_arrive_expect_tx(&s_full[buf], kMaskTileBytes);
+    const bool with_prev = FLIP && prev_tma;
+    mbar_arrive_expect_tx(&s_full[buf], kMaskTileBytes + (with_prev ? (uint32_t)sizeof(s_prev[0]) : 0u));
     tma_load_2d(s_w[buf], &tm_w, &s_full[buf], (int)(cx * kChunk + kTile * kh), (int)(cy * kChunk));
+    if (with_prev)
+      tma_load_2d(s_prev[buf], &tm_prev, &s_full[buf], (int)((cx * kChunk + kTile * kh) / 4), (int)(cy * (kChunk / 4)));
   };
   if (tid == 0) {
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
     fence_mbarrier_init();
     prefetch_tensormap(&tm_w);
+    if (FLIP && prev_tma) prefetch_tensormap(&tm_prev);
     s_flip = 0;
     s_abort = 0;
     sm.qn = 0;
@@ -724,7 +737,8 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
     tile_xy(t, cy, cx, kh);
     const SharedTileSrc src{s_w[buf]};
     mask_tile_body<BF16, SEARCH, COMPRESS, FLIP>(src, R, C, cy, cx, kh, chunks_x, chunks_y, idx, idx_prev, flips,
-                                                 vals_row, meta_row, vals_col, meta_col, sm, one);
+                                                 vals_row, meta_row, vals_col, meta_col, sm, one,
+                                                 (FLIP && prev_tma) ? s_prev[buf] : nullptr);
     __syncthreads();   // every read of this buffer and of the tile's shared state is done
     if (tid == 0) {
       sm.qn = 0;

@@ -426,9 +426,18 @@ sp24_status launch_mask_t(const void *W, int64_t R, int64_t C, int64_t ldw, uint
                   CU_TENSOR_MAP_SWIZZLE_NONE)) {
     const int64_t ctas = (int64_t)sm_count() * mask_ctas_per_sm<COMPRESS>();
     const unsigned grid = (unsigned)(ntiles < ctas ? ntiles : ctas);
+    // The previous mask travels with each W tile by TMA ([R/4][C/4] bytes, a 16 x 32
+    // box per tile) when its row pitch is a multiple of 16 bytes; else plain loads.
+    CUtensorMap tp = tm;
+    const int prev_tma = (FLIP && prev && (C / 4) % 16 == 0 && aligned16(prev) &&
+                          make_map_2d(&tp, prev, (uint64_t)(C / 4), (uint64_t)(R / 4), (uint64_t)(C / 4), kMaskCtaCols / 4,
+                                      kChunk / 4, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+                             ? 1
+                             : 0;
     return launch_pdl(mask_stream_kernel<BF16, SEARCH, COMPRESS, FLIP>, dim3(grid), dim3(kMaskThreads), 0, s, tm, R,
                       C, idx, prev, flip, static_cast<uint16_t *>(vr), static_cast<uint8_t *>(mr),
-                      static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc), (uint64_t)g_wait_budget.load());
+                      static_cast<uint16_t *>(vc), static_cast<uint8_t *>(mc), (uint64_t)g_wait_budget.load(), tp,
+                      prev_tma);
   }
   dim3 grid((unsigned)(chunks_x * (kChunk / kMaskCtaCols)), (unsigned)chunks_y);
   return launch_pdl(mask_tile_kernel<BF16, SEARCH, COMPRESS, FLIP>, grid, dim3(kMaskThreads), 0, s,
