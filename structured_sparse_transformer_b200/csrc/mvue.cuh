@@ -165,20 +165,12 @@ __device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, i
   int i2 = capped ? m : count_le(e1, e2, e3, __dadd_rn(q1, step));
   const bool empty = capped && !(tot > 0.0);        // at most one nonzero entry
   if (empty) i1 = m == 0 ? 1 : 0;
-  // Only a rounded cumulative sum puts both points in one entry: the second
-  // goes to the next nonzero entry after it, else the last nonzero one before.
-  // (Warp-uniform branch: all 32 lanes of the warp call this function.)
-  const bool collide = !capped && i2 == i1;
-  if (__any_sync(0xFFFFFFFFu, collide) && collide) {
-    int nxt = -1, prv = -1;
-#pragma unroll
-    for (int j = 3; j >= 0; --j)
-      if (j > i1 && q[j] != 0u) nxt = j;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (j < i1 && q[j] != 0u) prv = j;
-    i2 = nxt >= 0 ? nxt : prv;
-  }
+  // In the first case the two points always select two different nonzero
+  // entries, although the cumulative sums are rounded: round-to-nearest-even is
+  // monotone, so the second point (half the total past the first) passes the
+  // first point's entry; the one way to stay would need the total to round up
+  // by half an ulp of the last entry's complement, and ties-to-even then makes
+  // that entry reach half the total, i.e. the group capped.
   const uint32_t sgn4 = ((lo >> 15) & 1u) | ((lo >> 30) & 2u) | ((hi >> 13) & 4u) | ((hi >> 28) & 8u);
   const uint32_t mag = empty ? 0u : mvue_bits<BF16>(step);
   const uint32_t b1 = empty ? 0u : (mag | sign_of(sgn4, i1));
