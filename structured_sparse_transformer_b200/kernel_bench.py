@@ -46,7 +46,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=8192)
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16")
     ap.add_argument("--dist", choices=["normal", "tie"], default="normal")
-    ap.add_argument("--epi", choices=["none", "gelu", "dgelu", "gelu_deriv", "mul_aux"], default="none")
+    ap.add_argument("--epi", choices=["none", "gelu", "dgelu", "gelu_deriv", "mul_aux", "geglu", "dgeglu"],
+                    default="none")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--seed", type=int, default=0)
@@ -83,8 +84,9 @@ def main(argv=None):
         sp.sp24_mask_search(w, idx)
     elif k == "gemm_fwd":
         x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
-        y = torch.empty(T, R, dtype=tdt, device=dev)
-        epi = args.epi if args.epi in ("gelu", "gelu_deriv") else None
+        epi = args.epi if args.epi in ("gelu", "gelu_deriv", "geglu") else None
+        # geglu: W is the stacked gate/up weight [rows = 2 ff, cols]; out [T, ff], aux [T, 2 ff]
+        y = torch.empty(T, R // 2 if epi == "geglu" else R, dtype=tdt, device=dev)
         aux = torch.empty(T, R, dtype=tdt, device=dev) if epi else None
         fn = lambda: sp.sp24_gemm_fwd(x, bufs[0], bufs[1], R, y, epi, aux)
     elif k in ("mvue", "gemm_wgrad", "gemm_wgrad_decay"):
@@ -120,9 +122,11 @@ def main(argv=None):
         fn = lambda: sp.sp24_gemm_dense(dy, wt, dx, epi, aux)
     else:
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
-        dx = torch.empty(T, C, dtype=tdt, device=dev)
-        epi = args.epi if args.epi in ("dgelu", "mul_aux") else None
-        aux = torch.randn(T, C, device=dev, generator=gen).to(tdt) if epi else None
+        epi = args.epi if args.epi in ("dgelu", "mul_aux", "dgeglu") else None
+        # dgeglu: W is the down projection [rows = d, cols = ff]; aux and dX are [T, 2 ff]
+        width = 2 * C if epi == "dgeglu" else C
+        dx = torch.empty(T, width, dtype=tdt, device=dev)
+        aux = torch.randn(T, width, device=dev, generator=gen).to(tdt) if epi else None
         fn = lambda: sp.sp24_gemm_dgrad(dy, bufs[2], bufs[3], C, dx, epi, aux)
 
     for _ in range(args.warmup):
