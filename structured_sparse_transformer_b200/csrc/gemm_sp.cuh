@@ -19,12 +19,14 @@
 // with SPARSE = false runs the dense fine-tuning products.
 //
 // CTA pairs (clusters of 2, tcgen05 cta_group::2).  A pair computes a tile of
-// 256 output features x 224 tokens: each CTA holds 128 rows of the compressed
-// operand and 112 token rows of the activations in its own shared memory, and
-// the pair's even (leader) CTA issues MMAs of M = 256, N = 224, K = 32 that
-// read both.  Per CTA and 128-wide K step this moves 46 KB (A 16 KB, B 28 KB,
-// metadata 2 KB) for 7.3 MFLOP dense-equivalent; a single-CTA 128 x 128 tile
-// moves 50 KB for 4.2 MFLOP and is bound by the latency of its L2 -> SM stream.
+// 256 output features x N tokens (N = 240, or 224 where the epilogue's staging
+// leaves no room; see PairGeom): each CTA holds 128 rows of the compressed
+// operand and N/2 token rows of the activations in its own shared memory, and
+// the pair's even (leader) CTA issues MMAs of M = 256, N, K = 32 that read
+// both.  At N = 240, per CTA and 128-wide K step this moves 48 KB (A 16 KB,
+// B 30 KB, metadata 2 KB) for 7.9 MFLOP dense-equivalent; a single-CTA
+// 128 x 128 tile moves 50 KB for 4.2 MFLOP and is bound by the latency of its
+// L2 -> SM stream.
 // Persistent: each pair walks tiles pair, pair + npairs, ... (feature tiles
 // fastest, so the pairs running at once share token tiles through L2).
 //
@@ -35,11 +37,11 @@
 // cross-warp barrier: TMEM -> registers (two adjacent tokens of one feature
 // per thread) -> packed 16-bit pairs -> stmatrix.trans into its own staging
 // tile [16 tokens x 32 features] -> one TMA store per chunk and output.
-// Shared memory: a 4-stage ring of {A 128x64 kept values, B 112x128 as two
+// Shared memory: a 4-stage ring of {A 128x64 kept values, B (N/2)x128 as two
 // boxes (both 128B-swizzled), the 2 KB metadata chunk}, then 1 KB staging
 // tiles per epilogue warp (out; + aux for GELU; two pre-activation tiles for
 // dGELU).
-// Tensor memory per CTA: two 224-column fp32 accumulators (tile i+1 runs its
+// Tensor memory per CTA: two N-column fp32 accumulators (tile i+1 runs its
 // MMAs while tile i drains) and 4 metadata columns per stage.
 // Protocol:
 //   - both producers TMA-load their halves, counting bytes on the leader's
@@ -73,12 +75,9 @@ constexpr int kTmemCols = 512;
 constexpr uint64_t kDrainBudget = 1ull << 26;
 
 constexpr int kPairRows = 128;                         // compressed-operand rows per CTA
-constexpr int kPairBN = 224;                           // tokens per pair tile
-constexpr int kPairBNh = kPairBN / 2;                  // token rows per CTA
 constexpr int kPairSmemA = kPairRows * 64 * 2;        // 16 KB: 128 rows x 64 values (128B swizzle)
-constexpr int kPairSmemBBox = kPairBNh * 64 * 2;       // 14 KB: 112 token rows x 64 K
-constexpr int kPairChunks = kPairBN / kEpiTokens;      // 14
-constexpr int kPairMetaCol = 2 * kPairBN;              // accumulators at columns 0 and 224
+constexpr int kPairBNWide = 240;                       // tokens per pair tile where shared memory allows
+constexpr int kPairBNNarrow = 224;                     // else
 
 // Epilogues: none; GELU (aux <- pre-activation); GELU' (aux = pre-activation,
 // read); gated GELU on a gate/up-interleaved output (out = gelu(gate) * up at
@@ -120,20 +119,6 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // accumulators were measured 10-15% slower at the 1.5B shapes, although they
 // leave fewer column-waves idle: each stage then carries half the MMA work for
 // the same A tile and per-stage overhead.)
-template <bool SPARSE, int EPI>
-struct PairGeom {
-  static constexpr bool kWg = EPI == kEpiWgrad;
-  static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
-  static constexpr int kAcols = 64;                      // A values per row and stage
-  static constexpr int kBN = kWg ? 256 : kPairBN;        // B columns (tokens, or dW columns) per pair tile
-  static constexpr int kBBoxes = (SPARSE || kWg) ? 2 : 1;  // wgrad: two 64-column atoms
-  static constexpr int kBBoxBytes = kWg ? 64 * kBK * 2 : kPairSmemBBox;
-  static constexpr int kMeta = SPARSE ? kSmemE : 0;
-  static constexpr int kStageBytes = kPairSmemA + kBBoxes * kBBoxBytes + kMeta;
-  static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
-  static constexpr int kAccBufs = kWg ? 1 : 2;
-  static constexpr int kMetaCol = kAccBufs * kBN;        // metadata columns after the accumulators
-};
 constexpr int kEpiBufBytes = kEpiTokens * 32 * 2;      // staging tile: 16 tokens x 32 features, 64B-swizzled
 constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM address, abort flag
 
@@ -147,17 +132,45 @@ __host__ __device__ constexpr int epi_bufs(int epi) {
                           : (epi == kEpiGelu || epi == kEpiGeglu || epi == kEpiGeluDeriv) ? 2
                           : ((epi == kEpiDgelu || epi == kEpiMulAux) ? 3 : 6);
 }
+
+// Tokens per pair tile (kBN): 240 where the shared memory still holds the same
+// number of stages, else 224.  TMEM holds two accumulators of kBN columns and 4
+// metadata columns per stage (2 x 240 + 16 = 496 of 512).  240 = 15 chunks of
+// 16 tokens, five per epilogue warp group; 240 tokens per pair are 120 B rows
+// per CTA, a 15 KB box (a whole number of 1 KB swizzle atoms).
+template <bool SPARSE, int EPI>
+struct PairGeom {
+  static constexpr bool kWg = EPI == kEpiWgrad;
+  static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
+  static constexpr int kAcols = 64;                      // A values per row and stage
+  static constexpr int kBBoxes = (SPARSE || kWg) ? 2 : 1;  // wgrad: two 64-column atoms
+  static constexpr int kMeta = SPARSE ? kSmemE : 0;
+  static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
+  static constexpr int kAccBufs = kWg ? 1 : 2;
+  static constexpr int box_bytes(int bn) { return kWg ? 64 * kBK * 2 : (bn / 2) * 64 * 2; }
+  static constexpr int smem_for(int bn) {
+    return kStages * (kPairSmemA + kBBoxes * box_bytes(bn) + kMeta) + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
+           kPairBarBytes + 1024 + (kWg ? 8192 : 0);
+  }
+  static constexpr int kBN = kWg ? 256 : (smem_for(kPairBNWide) <= 232448 ? kPairBNWide : kPairBNNarrow);
+  static constexpr int kBBoxBytes = box_bytes(kBN);      // one B box (or wgrad atom)
+  static constexpr int kStageBytes = kPairSmemA + kBBoxes * kBBoxBytes + kMeta;
+  static constexpr int kChunks = kBN / kEpiTokens;       // 16-token epilogue chunks per tile
+  static constexpr int kMetaCol = kAccBufs * kBN;        // metadata columns after the accumulators
+};
 // The wgrad variant keeps 8 KB unused after its barriers, so that its MN-major
 // B reads stay inside the allocation under any reading of the descriptor strides.
 template <bool SPARSE, int EPI>
 __host__ __device__ constexpr int pair_smem_bytes() {
-  return PairGeom<SPARSE, EPI>::kStages * PairGeom<SPARSE, EPI>::kStageBytes + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
-         kPairBarBytes + 1024 + (PairGeom<SPARSE, EPI>::kWg ? 8192 : 0);
+  return PairGeom<SPARSE, EPI>::smem_for(PairGeom<SPARSE, EPI>::kBN);
 }
 static_assert(pair_smem_bytes<true, kEpiMulAux>() == pair_smem_bytes<true, kEpiDgelu>() &&
                   pair_smem_bytes<false, kEpiMulAux>() == pair_smem_bytes<false, kEpiDgelu>() &&
                   pair_smem_bytes<true, kEpiGeluDeriv>() == pair_smem_bytes<true, kEpiGelu>(),
               "the derivative-saving pair stages like GELU / GELU'");
+static_assert(PairGeom<true, kEpiNone>::kBN == 240 && PairGeom<true, kEpiGeluDeriv>::kBN == 240 &&
+                  PairGeom<true, kEpiMulAux>::kBN == 224 && PairGeom<false, kEpiMulAux>::kBN == 240,
+              "tile widths of the headline variants");
 static_assert(pair_smem_bytes<true, kEpiDgelu>() <= 232448 && pair_smem_bytes<false, kEpiDgelu>() <= 232448 &&
                   pair_smem_bytes<true, kEpiDgeglu>() <= 232448 && pair_smem_bytes<false, kEpiDgeglu>() <= 232448 &&
                   pair_smem_bytes<true, kEpiWgrad>() <= 232448,
@@ -176,9 +189,12 @@ static_assert(PairGeom<true, kEpiWgrad>::kStageBytes % 1024 == 0 && PairGeom<tru
 static_assert(PairGeom<true, kEpiWgrad>::kMetaCol + 4 * PairGeom<true, kEpiWgrad>::kStages <= kTmemCols,
               "tensor memory budget (wgrad)");
 static_assert(PairGeom<true, kEpiNone>::kStageBytes % 1024 == 0 && PairGeom<false, kEpiNone>::kStageBytes % 1024 == 0 &&
-                  kPairSmemA % 1024 == 0 && kPairSmemBBox % 1024 == 0,
+                  PairGeom<true, kEpiMulAux>::kStageBytes % 1024 == 0 && kPairSmemA % 1024 == 0 &&
+                  PairGeom<true, kEpiNone>::kBBoxBytes % 1024 == 0 && PairGeom<true, kEpiMulAux>::kBBoxBytes % 1024 == 0,
               "128B-swizzled tiles need 1 KB aligned starts");
-static_assert(kPairMetaCol + 4 * PairGeom<true, kEpiNone>::kStages <= kTmemCols, "tensor memory budget");
+static_assert(PairGeom<true, kEpiNone>::kMetaCol + 4 * PairGeom<true, kEpiNone>::kStages <= kTmemCols &&
+                  PairGeom<true, kEpiDgeglu>::kMetaCol + 4 * PairGeom<true, kEpiDgeglu>::kStages <= kTmemCols,
+              "tensor memory budget");
 static_assert(2 * PairGeom<false, kEpiNone>::kStages + 16 + 2 * kEpiWarps <= kPairBarBytes / 8, "barrier space");
 
 // Work schedule of a CTA pair: a sequence of segments (tile, K steps kb..ke-1).
@@ -482,7 +498,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     while (ok && sched.next(tile, kb, ke)) {
       const int mt = tile_mt(tile);
       const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
-      const int b_row = tile_nt(tile) * G::kBN + (int)rank * (WG ? 64 : kPairBNh);
+      const int b_row = tile_nt(tile) * G::kBN + (int)rank * (WG ? 64 : G::kBN / 2);
       // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
       // it the last real metadata chunk so every code the MMA sees is valid.
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
@@ -509,7 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 128, kt * G::kBK);
         } else {
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
-          if (SPARSE) tma_load_2d_pair(st + kPairSmemA + kPairSmemBBox, &tm_b, &full[s], kt * G::kBK + 64, b_row);
+          if (SPARSE) tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], kt * G::kBK + 64, b_row);
         }
         if (SPARSE)
           tma_load_2d_pair(st + kPairSmemA + G::kBBoxes * G::kBBoxBytes, &tm_meta, &full[s], 0, chunk_row + kt);
@@ -536,8 +552,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     constexpr uint32_t idesc = WG ? ((SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, 128)
                                              : (make_idesc_dense(BF16, 2 * kPairRows, 128) | (1u << 15))) |
                                     (1u << 16))
-                               : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, kPairBN)
-                                        : make_idesc_dense(BF16, 2 * kPairRows, kPairBN);
+                               : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, G::kBN)
+                                        : make_idesc_dense(BF16, 2 * kPairRows, G::kBN);
     const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), (WG && !SPARSE) ? kPairSmemA / 2 : 16, 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
     const uint64_t e_desc0 =
@@ -587,14 +603,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               tc_mma_sp_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), tm, id, accum);
           }
         } else if (SPARSE) {
-          const uint32_t t_meta = tmem_base + kPairMetaCol + 4 * s;
+          const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;
           tc_cp_128x128b_pair(t_meta, e_desc0 + so);
           // The metadata operand address must be 2-column aligned; the low column
           // bit travels in the descriptor's sparsity-selector field instead.
           tc_mma_sp_f16_pair(acc, ad, bd, t_meta, idesc, kt != kb ? 1u : 0u);
           tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
-          tc_mma_sp_f16_pair(acc, ad + 4, bd + (kPairSmemBBox >> 4), t_meta + 2, idesc, 1u);
-          tc_mma_sp_f16_pair(acc, ad + 6, bd + (kPairSmemBBox >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
+          tc_mma_sp_f16_pair(acc, ad + 4, bd + (G::kBBoxBytes >> 4), t_meta + 2, idesc, 1u);
+          tc_mma_sp_f16_pair(acc, ad + 6, bd + (G::kBBoxBytes >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
         } else {
           // Four K = 16 steps through the 128-byte swizzled rows of A and B (32 bytes each).
           tc_mma_f16_pair(acc, ad, bd, idesc, kt != kb ? 1u : 0u);
@@ -781,7 +797,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int ew = warp - 2;
     const int grp = ew >> 2;
     const int q = warp & 3;
-    constexpr int kMaxChunksPerWarp = (kPairChunks + kEpiGroups - 1) / kEpiGroups;
+    constexpr int kMaxChunksPerWarp = (G::kChunks + kEpiGroups - 1) / kEpiGroups;
     constexpr bool kPre = EPI == kEpiDgelu || EPI == kEpiDgeglu || EPI == kEpiMulAux;   // TMA-loaded aux tiles
     constexpr int kPreBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
     constexpr int kOutBytes = EPI == kEpiDgeglu ? 2 * kEpiBufBytes : kEpiBufBytes;
@@ -818,8 +834,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = pair; tile < num_tiles && alive; tile += npairs, ++j) {
       const int b = j & 1;
       const int m0 = (tile % num_mt) * 2 * kPairRows + (int)rank * kPairRows + 32 * q;
-      const int n0 = (tile / num_mt) * kPairBN;
-      const int nchunks = min(kPairChunks, (T - n0 + kEpiTokens - 1) / kEpiTokens);
+      const int n0 = (tile / num_mt) * G::kBN;
+      const int nchunks = min(G::kChunks, (T - n0 + kEpiTokens - 1) / kEpiTokens);
       const int nk = grp < nchunks ? (nchunks - 1 - grp) / kEpiGroups + 1 : 0;   // this warp's chunks
       if (kPre)
         for (int k = 0; k < 2 && k < nk; ++k) pre_load(pre_col(m0), n0 + (grp + k * kEpiGroups) * kEpiTokens);
@@ -830,7 +846,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       uint32_t r[kMaxChunksPerWarp][2][8];
-      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * kPairBN);
+      const uint32_t t_base = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * G::kBN);
 #pragma unroll
       for (int k = 0; k < kMaxChunksPerWarp; ++k) {
         if (k < nk) {

@@ -132,7 +132,7 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 
 // ---------------------------------------------------------------- GEMM launch
 
-// CTA-pair kernel: clusters of two CTAs, 256 x 224 tiles (see gemm_sp.cuh).
+// CTA-pair kernel: clusters of two CTAs, tiles of 256 rows x 240 or 224 tokens (see gemm_sp.cuh).
 // SPARSE: A = kept values [M x Kd/2] + metadata chunks; dense: A = [M x Kd].
 // Weight gradient (kEpiWgrad): B = the layer input [Kd tokens x T columns]
 // read MN-major, out = fp32 [M x T]; tiles of 256 x 256.
@@ -275,7 +275,7 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
   CUtensorMap ta, tb, tm;
   const bool b_ok = G::kWg ? make_map_2d(&tb, B, (uint64_t)T, (uint64_t)Kd, (uint64_t)T * 2, 64, (uint32_t)G::kBK,
                                          CU_TENSOR_MAP_SWIZZLE_128B)
-                           : make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, kPairBNh,
+                           : make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, (uint32_t)(G::kBN / 2),
                                          CU_TENSOR_MAP_SWIZZLE_128B);
   // Dense weight gradient: A = dY [Kd tokens x M] read MN-major in 64 x kBK boxes.
   const bool a_ok = (G::kWg && !SPARSE)
