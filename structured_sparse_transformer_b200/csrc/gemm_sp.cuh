@@ -133,12 +133,13 @@ __host__ __device__ constexpr int epi_bufs(int epi) {
                           : ((epi == kEpiDgelu || epi == kEpiMulAux) ? 3 : 6);
 }
 
-// Tokens per pair tile (kBN): 240 where the shared memory still holds the same
-// number of stages, else 224.  TMEM holds two accumulators of kBN columns and 4
+// Tokens per pair tile (kBN): with WIDE, 240 where the shared memory still
+// holds the same number of stages, else 224 (the host picks WIDE per call: the
+// wider tile is cheaper per token but can leave a wave less full).  TMEM holds two accumulators of kBN columns and 4
 // metadata columns per stage (2 x 240 + 16 = 496 of 512).  240 = 15 chunks of
 // 16 tokens, five per epilogue warp group; 240 tokens per pair are 120 B rows
 // per CTA, a 15 KB box (a whole number of 1 KB swizzle atoms).
-template <bool SPARSE, int EPI>
+template <bool SPARSE, int EPI, bool WIDE = true>
 struct PairGeom {
   static constexpr bool kWg = EPI == kEpiWgrad;
   static constexpr int kBK = SPARSE ? 128 : 64;          // logical K per stage
@@ -152,7 +153,7 @@ struct PairGeom {
     return kStages * (kPairSmemA + kBBoxes * box_bytes(bn) + kMeta) + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
            kPairBarBytes + 1024 + (kWg ? 8192 : 0);
   }
-  static constexpr int kBN = kWg ? 256 : (smem_for(kPairBNWide) <= 232448 ? kPairBNWide : kPairBNNarrow);
+  static constexpr int kBN = kWg ? 256 : ((WIDE && smem_for(kPairBNWide) <= 232448) ? kPairBNWide : kPairBNNarrow);
   static constexpr int kBBoxBytes = box_bytes(kBN);      // one B box (or wgrad atom)
   static constexpr int kStageBytes = kPairSmemA + kBBoxes * kBBoxBytes + kMeta;
   static constexpr int kChunks = kBN / kEpiTokens;       // 16-token epilogue chunks per tile
@@ -160,9 +161,9 @@ struct PairGeom {
 };
 // The wgrad variant keeps 8 KB unused after its barriers, so that its MN-major
 // B reads stay inside the allocation under any reading of the descriptor strides.
-template <bool SPARSE, int EPI>
+template <bool SPARSE, int EPI, bool WIDE = true>
 __host__ __device__ constexpr int pair_smem_bytes() {
-  return PairGeom<SPARSE, EPI>::smem_for(PairGeom<SPARSE, EPI>::kBN);
+  return PairGeom<SPARSE, EPI, WIDE>::smem_for(PairGeom<SPARSE, EPI, WIDE>::kBN);
 }
 static_assert(pair_smem_bytes<true, kEpiMulAux>() == pair_smem_bytes<true, kEpiDgelu>() &&
                   pair_smem_bytes<false, kEpiMulAux>() == pair_smem_bytes<false, kEpiDgelu>() &&
@@ -408,7 +409,7 @@ __device__ __forceinline__ void unpack2(uint32_t v, float &lo, float &hi) {
   }
 }
 
-template <bool BF16, int EPI, bool SPARSE>
+template <bool BF16, int EPI, bool SPARSE, bool WIDE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     sp24_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                           const __grid_constant__ CUtensorMap tm_meta, const __grid_constant__ CUtensorMap tm_out,
@@ -428,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // parts per tail tile, partial accumulators in sk_part (kSkPartFloatsPerCta
   // per CTA) and ready counters in sk_flags (kEpiWarps per CTA, zero at launch
   // and left zero).
-  using G = PairGeom<SPARSE, EPI>;
+  using G = PairGeom<SPARSE, EPI, WIDE>;
   constexpr bool WG = G::kWg;
   constexpr int kPairStages = G::kStages;
   constexpr int kPairStageBytes = G::kStageBytes;

@@ -138,10 +138,10 @@ bool make_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t ou
 // read MN-major, out = fp32 [M x T]; tiles of 256 x 256.
 // Per device, once: the shared-memory opt-in of an instantiation and the number
 // of its CTA pairs that fit at once (0: the set-up failed; -1: no device).
-template <bool BF16, int EPI, bool SPARSE>
+template <bool BF16, int EPI, bool SPARSE, bool WIDE = false>
 int gemm_pairs() {
-  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
-  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
+  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI, WIDE>();
+  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE, WIDE>;
   static PerDevice pairs_cache;
   const int dev = current_device();
   if (dev < 0) return -1;
@@ -263,12 +263,11 @@ sp24_status noalloc_scratch(SkWorkspace *out) {
 // the epilogue); null dec_w elsewhere.  `fixed`: a caller-given split-tail
 // scratch (its counters are zeroed here before the launch) instead of the
 // per-stream workspace; null for every entry point but sp24_gemm_wgrad_noalloc.
-template <bool BF16, int EPI, bool SPARSE>
-sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
-                               void *out, void *aux, cudaStream_t stream, const void *dec_w = nullptr,
-                               const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f,
-                               const SkWorkspace *fixed = nullptr) {
-  using G = PairGeom<SPARSE, EPI>;
+template <bool BF16, int EPI, bool SPARSE, bool WIDE>
+sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                               void *out, void *aux, cudaStream_t stream, const void *dec_w, const uint8_t *dec_idx,
+                               float dec_lambda, const SkWorkspace *fixed) {
+  using G = PairGeom<SPARSE, EPI, WIDE>;
   const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
   const uint64_t a_cols = SPARSE ? (uint64_t)(Kd / 2) : (uint64_t)Kd;
@@ -312,9 +311,9 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
                           CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (!maps_ok) return SP24_ERR_CUDA;
-  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI>();
-  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE>;
-  const int max_pairs = gemm_pairs<BF16, EPI, SPARSE>();
+  constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI, WIDE>();
+  auto kernel = sp24_gemm_pair_kernel<BF16, EPI, SPARSE, WIDE>;
+  const int max_pairs = gemm_pairs<BF16, EPI, SPARSE, WIDE>();
   if (max_pairs <= 0) return max_pairs == 0 ? SP24_ERR_CUDA : SP24_ERR_NO_DEVICE;
   const int64_t tiles = ((M + 2 * kPairRows - 1) / (2 * kPairRows)) * ((T + G::kBN - 1) / G::kBN);
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
@@ -352,6 +351,34 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
                     (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda, ws.part,
                     ws.flags, split, cols_fastest);
+}
+
+// Tile width per call, for the variants that have both: the busiest pair's token
+// columns, ceil(tiles / pairs) x width, with the 240-token tile counted 5% cheaper
+// per token (measured on the 1.5B FFN launches, where its waves are as full);
+// where waves quantise differently (e.g. 148 tiles of 224 tokens on 74 pairs
+// against 140 of 240) the narrower tile is kept.
+template <bool BF16, int EPI, bool SPARSE>
+sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
+                               void *out, void *aux, cudaStream_t stream, const void *dec_w = nullptr,
+                               const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f,
+                               const SkWorkspace *fixed = nullptr) {
+  constexpr int kWideBN = PairGeom<SPARSE, EPI, true>::kBN, kNarrowBN = PairGeom<SPARSE, EPI, false>::kBN;
+  if constexpr (kWideBN != kNarrowBN) {
+    const int P = gemm_pairs<BF16, EPI, SPARSE, false>();
+    if (P > 0) {
+      const int64_t mt = (M + 2 * kPairRows - 1) / (2 * kPairRows);
+      auto busiest = [&](int bn) {
+        const int64_t tiles = mt * ((T + bn - 1) / bn);
+        return (double)((tiles + P - 1) / P) * (double)bn;
+      };
+      if (busiest(kWideBN) * 0.95 < busiest(kNarrowBN))
+        return launch_gemm_pair_w<BF16, EPI, SPARSE, true>(B, T, Kd, vals, meta, M, out, aux, stream, dec_w, dec_idx,
+                                                           dec_lambda, fixed);
+    }
+  }
+  return launch_gemm_pair_w<BF16, EPI, SPARSE, false>(B, T, Kd, vals, meta, M, out, aux, stream, dec_w, dec_idx,
+                                                      dec_lambda, fixed);
 }
 
 template <bool SPARSE>
