@@ -318,13 +318,11 @@ class FFNStep:
 
     def run_dense(self, events=None):
         """One step of the dense fine-tuning phase (the last 1/6 of the steps):
-        W^T of both weights (they change every step), the six FFN products on
-        the dense tensor-core path (the weight gradients read dY and dH as
-        stored); no mask, compression or decay."""
+        the six FFN products on the dense tensor-core path, every operand read
+        as stored (the input gradients load W MN-major, the weight gradients dY
+        and dH); no mask, compression or decay."""
         sp, torch = self.sp, self.torch
         cur = self.step_no % self.S + 1
-        if not hasattr(self, "Wt"):
-            self.Wt = [torch.empty(w[0].shape[1], w[0].shape[0], dtype=w[0].dtype, device="cuda") for w in self.W]
 
         def timed(name, fn):
             if events is None:
@@ -336,15 +334,13 @@ class FFNStep:
             e.record()
             events.setdefault(name, []).append((s, e))
 
-        for li in range(2):
-            timed("transpose", lambda li=li: sp.sp24_transpose(self.W[li][cur], self.Wt[li]))
         W1, W2 = self.W[0][cur], self.W[1][cur]
         timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_dense(self.X, W1, self.H, "gelu_deriv", self.Gp))
         timed("gemm_fwd2", lambda: sp.sp24_gemm_dense(self.H, W2, self.Y))
-        timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dense(self.dY, self.Wt[1], self.dH, "mul_aux", self.Gp))
+        timed("gemm_dgrad2_dgelu", lambda: sp.sp24_gemm_dgrad_dense(self.dY, W2, self.dH, "mul_aux", self.Gp))
         timed("gemm_wgrad2", lambda: sp.sp24_gemm_wgrad_dense(self.H, self.dY, self.G[1]))
         timed("gemm_wgrad1", lambda: sp.sp24_gemm_wgrad_dense(self.X, self.dH, self.G[0]))
-        timed("gemm_dgrad1", lambda: sp.sp24_gemm_dense(self.dH, self.Wt[0], self.dX))
+        timed("gemm_dgrad1", lambda: sp.sp24_gemm_dgrad_dense(self.dH, W1, self.dX))
         self.step_no += 1
 
     # algorithmic bytes / flops per launch of each kernel
@@ -636,18 +632,16 @@ def run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks):
     st = sp.sp24_device_status()
     if st != 0:
         raise RuntimeError(f"device status after the dense phase: {sp.sp24_status_string(st)}")
-    n_el = wl.d * wl.ff
     work = {k: ("TFLOP/s", 2.0 * wl.tokens * wl.d * wl.ff) for k in FFNStep.GEMMS + ("gemm_wgrad2", "gemm_wgrad1")}
-    work["transpose"] = ("GB/s", 4 * n_el)
     dense_peaks = dict(peaks)
     dense_peaks["bf16_tflops"] = peaks["bf16_tflops"] / 2.0   # kernel_table doubles it for the 2:4 peak
     kernels = kernel_table(events, work, dense_peaks, list(work))
     return {"ms_per_step": round(ms, 4),
             "value": round(6 * 2.0 * wl.tokens * wl.d * wl.ff * world / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "kernels": kernels,
-            "note": "dense fine-tuning phase (last 1/6 of the steps): W^T of both weights and the six FFN "
-                    "products (forward, input gradient, weight gradient reading dY and dH as stored) on the "
-                    "dense tcgen05 path, same workload; FLOPs 6 x 2 T d ff; GEMM peak = the dense bf16 burst"}
+            "note": "dense fine-tuning phase (last 1/6 of the steps): the six FFN products (forward, input "
+                    "gradient reading W as stored, weight gradient reading dY and dH as stored) on the dense "
+                    "tcgen05 path, same workload; FLOPs 6 x 2 T d ff; GEMM peak = the dense bf16 burst"}
 
 
 class GegluStep:

@@ -15,7 +15,8 @@
  *     weight-gradient product (sp24_gemm_wgrad), and the GEGLU kernel (the gated
  *     epilogues of sp24_gemm_fwd / sp24_gemm_dgrad);
  *   - abstract and Experiment Setup row: dense fine-tuning for the last 1/6 of
- *     the steps (sp24_gemm_dense, sp24_gemm_wgrad_dense, sp24_transpose).
+ *     the steps (sp24_gemm_dense, sp24_gemm_dgrad_dense, sp24_gemm_wgrad_dense,
+ *     sp24_transpose).
  *
  * Conventions shared by every call
  *   - Matrices are row-major.  W is [rows x cols] with leading dimension ldw
@@ -206,6 +207,24 @@ SP24_API sp24_status sp24_gemm_dgrad(const void *dY, int64_t T, int64_t N, const
  */
 SP24_API sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A, int64_t M,
                             sp24_dtype dtype, void *out, sp24_epilogue epi, void *aux, void *stream);
+
+/*
+ * Dense input gradient for the dense fine-tuning phase (abstract: dense
+ * fine-tuning; Experiment Setup row: the last 1/6 of the steps), with the
+ * weight read as stored:
+ *   dX[T x K] = dY[T x N] * W[N x K]
+ * The same product as sp24_gemm_dense(dY, W^T) without forming W^T: the tensor
+ * memory accelerator loads W in 64-column atoms, MN-major for the tensor cores.
+ *   dY   device [T x N] row-major, contiguous (the output gradient)
+ *   W    device [N x K] row-major, contiguous (the layer's weight)
+ *   dX   device [T x K] row-major, contiguous, overwritten
+ *   epi  NONE, DGELU or MUL_AUX; aux as in sp24_gemm_dgrad ([T x K], read)
+ * fp32 accumulation; outputs rounded to dtype.  N % 16 == 0, K % 16 == 0,
+ * T >= 0 (T == 0: nothing is written).  All pointers 16-byte aligned.
+ */
+SP24_API sp24_status sp24_gemm_dgrad_dense(const void *dY, int64_t T, int64_t N, const void *W, int64_t K,
+                                  sp24_dtype dtype, void *dX, sp24_epilogue epi, const void *aux,
+                                  void *stream);
 
 /*
  * out[cols x rows] = in[rows x cols]^T for 16-bit elements (bit copy): the

@@ -37,6 +37,7 @@ _SIGNATURES = {
     "sp24_gemm_fwd": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
     "sp24_gemm_dgrad": [P, I64, I64, P, P, I64, I32, P, I32, P, P],
     "sp24_gemm_dense": [P, I64, I64, P, I64, I32, P, I32, P, P],
+    "sp24_gemm_dgrad_dense": [P, I64, I64, P, I64, I32, P, I32, P, P],
     "sp24_transpose": [P, I64, I64, I32, P, P],
     "sp24_mvue_sparsify": [P, I64, I64, I64, I32, U64, U64, P, P, P],
     "sp24_gemm_wgrad": [P, I64, I64, P, P, I64, I32, P, P],
@@ -277,6 +278,24 @@ def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
     _check("sp24_gemm_dense",
            _lib.sp24_gemm_dense(_ptr(B), T, Kd, _ptr(A), M, _dtype_code(B), _ptr(out), EPILOGUES[epi], _ptr(aux),
                                 _stream(stream)))
+
+
+def sp24_gemm_dgrad_dense(dY, W, dX, epi=None, aux=None, stream=None):
+    """dX[T, K] <- dY[T, N] W[N, K] on the dense tensor-core path with W read as stored;
+    epi None, 'dgelu' or 'mul_aux'."""
+    _need_rowmajor(dY, W, dX, aux)
+    T, N = _shape2(dY, "dY")
+    N2, K = _shape2(W, "W")
+    if N2 != N:
+        raise ValueError(f"W has {N2} rows, dY has {N} columns")
+    _dtype_code(dY)
+    _expect(W, "W", dY.dtype, N * K)
+    _expect(dX, "dX", dY.dtype, T * K)
+    _expect(aux, "aux", dY.dtype, T * K)
+    _need_device(dY, W, dX, aux)
+    _check("sp24_gemm_dgrad_dense",
+           _lib.sp24_gemm_dgrad_dense(_ptr(dY), T, N, _ptr(W), K, _dtype_code(dY), _ptr(dX), EPILOGUES[epi],
+                                      _ptr(aux), _stream(stream)))
 
 
 def sp24_transpose(x, out, stream=None):

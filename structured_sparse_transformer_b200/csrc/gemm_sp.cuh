@@ -148,8 +148,8 @@ struct PairGeom {
   static constexpr int kMeta = SPARSE ? kSmemE : 0;
   static constexpr int kStages = SPARSE ? (EPI == kEpiDgeglu ? 3 : 4) : (EPI == kEpiDgeglu ? 4 : 6);
   static constexpr int kAccBufs = kWg ? 1 : 2;
-  static constexpr int box_bytes(int bn) { return kWg ? 64 * kBK * 2 : (bn / 2) * 64 * 2; }
-  static constexpr int smem_for(int bn) {
+  __host__ __device__ static constexpr int box_bytes(int bn) { return kWg ? 64 * kBK * 2 : (bn / 2) * 64 * 2; }
+  __host__ __device__ static constexpr int smem_for(int bn) {
     return kStages * (kPairSmemA + kBBoxes * box_bytes(bn) + kMeta) + kEpiWarps * epi_bufs(EPI) * kEpiBufBytes +
            kPairBarBytes + 1024 + (kWg ? 8192 : 0);
   }
@@ -417,7 +417,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out,
                           const uint16_t *__restrict__ dec_w, const uint8_t *__restrict__ dec_idx,
                           float dec_lambda, float *__restrict__ sk_part, unsigned *__restrict__ sk_flags,
-                          int sk_split, int cols_fastest) {
+                          int sk_split, int cols_fastest, int a_mn) {
   // T counts the B operand's rows of the output: tokens, or for the weight
   // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
   // Weight gradient with dec_w set: the masked decay of dW in the epilogue, W and
@@ -429,6 +429,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // parts per tail tile, partial accumulators in sk_part (kSkPartFloatsPerCta
   // per CTA) and ready counters in sk_flags (kEpiWarps per CTA, zero at launch
   // and left zero).
+  // Dense with a_mn set: A is read as stored [K x M] (M contiguous), MN-major
+  // like the dense weight gradient's A: the input gradient takes W itself.
   using G = PairGeom<SPARSE, EPI, WIDE>;
   constexpr bool WG = G::kWg;
   constexpr int kPairStages = G::kStages;
@@ -511,9 +513,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         uint8_t *st = stage_base + s * kPairStageBytes;
         if (is_leader) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
-        if (WG && !SPARSE) {
-          // Dense weight gradient: A = dY as stored, MN-major, in two 64-row atoms
-          // (x = dW row, y = token), 8 KB apart.
+        if (!SPARSE && (WG || a_mn)) {
+          // Dense A read as stored, MN-major, in two 64-row atoms 8 KB apart
+          // (x = output row, y = K): dY for the weight gradient, W for the input
+          // gradient.
           tma_load_2d_pair(st, &tm_a, &full[s], a_row, kt * G::kBK);
           tma_load_2d_pair(st + kPairSmemA / 2, &tm_a, &full[s], a_row + 64, kt * G::kBK);
         } else {
@@ -555,7 +558,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                     (1u << 16))
                                : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, G::kBN)
                                         : make_idesc_dense(BF16, 2 * kPairRows, G::kBN);
-    const uint64_t a_desc0 = smem_desc(smem_u32(stage_base), (WG && !SPARSE) ? kPairSmemA / 2 : 16, 1024, kSwizzle128B);
+    // Dense input gradient with a_mn: the same MN-major A as the dense wgrad (bit 15).
+    const uint32_t idesc_amn = idesc | (1u << 15);
+    const uint64_t a_desc0 =
+        smem_desc(smem_u32(stage_base), (!SPARSE && (WG || a_mn)) ? kPairSmemA / 2 : 16, 1024, kSwizzle128B);
     const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
     const uint64_t e_desc0 =
         smem_desc(smem_u32(stage_base + kPairSmemA + G::kBBoxes * G::kBBoxBytes), 128, 128, kSwizzleNone);
@@ -612,6 +618,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_mma_sp_f16_pair(acc, ad + 2, bd + 4, t_meta, idesc | 1u, 1u);
           tc_mma_sp_f16_pair(acc, ad + 4, bd + (G::kBBoxBytes >> 4), t_meta + 2, idesc, 1u);
           tc_mma_sp_f16_pair(acc, ad + 6, bd + (G::kBBoxBytes >> 4) + 4, t_meta + 2, idesc | 1u, 1u);
+        } else if (a_mn) {
+          // A MN-major: a K = 16 step moves A 16 rows of 128 bytes (2048 bytes) and
+          // B 32 bytes along its swizzled rows.
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_f16_pair(acc, ad + (uint64_t)(kk * (2048 >> 4)), bd + 2 * kk, idesc_amn,
+                            (kt != kb || kk != 0) ? 1u : 0u);
         } else {
           // Four K = 16 steps through the 128-byte swizzled rows of A and B (32 bytes each).
           tc_mma_f16_pair(acc, ad, bd, idesc, kt != kb ? 1u : 0u);

@@ -266,7 +266,7 @@ sp24_status noalloc_scratch(SkWorkspace *out) {
 template <bool BF16, int EPI, bool SPARSE, bool WIDE>
 sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream, const void *dec_w, const uint8_t *dec_idx,
-                               float dec_lambda, const SkWorkspace *fixed) {
+                               float dec_lambda, const SkWorkspace *fixed, bool a_mn) {
   using G = PairGeom<SPARSE, EPI, WIDE>;
   const int num_kt = (int)((Kd + G::kBK - 1) / G::kBK);
   const int64_t row_tiles = (M + kPairRows - 1) / kPairRows;
@@ -276,8 +276,10 @@ sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void 
                                          CU_TENSOR_MAP_SWIZZLE_128B)
                            : make_map_2d(&tb, B, (uint64_t)Kd, (uint64_t)T, (uint64_t)Kd * 2, 64, (uint32_t)(G::kBN / 2),
                                          CU_TENSOR_MAP_SWIZZLE_128B);
-  // Dense weight gradient: A = dY [Kd tokens x M] read MN-major in 64 x kBK boxes.
-  const bool a_ok = (G::kWg && !SPARSE)
+  // Dense weight gradient (A = dY [Kd tokens x M]) and dense input gradient with
+  // a_mn (A = W [Kd x M]): A read MN-major in 64 x kBK boxes.
+  a_mn = a_mn && !SPARSE && !G::kWg;
+  const bool a_ok = (G::kWg && !SPARSE) || a_mn
                         ? make_map_2d(&ta, vals, (uint64_t)M, (uint64_t)Kd, (uint64_t)M * 2, 64, (uint32_t)G::kBK,
                                       CU_TENSOR_MAP_SWIZZLE_128B)
                         : make_map_2d(&ta, vals, a_cols, (uint64_t)M, a_cols * 2, G::kAcols, kPairRows,
@@ -350,7 +352,7 @@ sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void 
   return launch_pdl(kernel, dim3(2 * grid_pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
                     (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda, ws.part,
-                    ws.flags, split, cols_fastest);
+                    ws.flags, split, cols_fastest, a_mn ? 1 : 0);
 }
 
 // Tile width per call, for the variants that have both: the busiest pair's token
@@ -362,7 +364,7 @@ template <bool BF16, int EPI, bool SPARSE>
 sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                                void *out, void *aux, cudaStream_t stream, const void *dec_w = nullptr,
                                const uint8_t *dec_idx = nullptr, float dec_lambda = 0.0f,
-                               const SkWorkspace *fixed = nullptr) {
+                               const SkWorkspace *fixed = nullptr, bool a_mn = false) {
   constexpr int kWideBN = PairGeom<SPARSE, EPI, true>::kBN, kNarrowBN = PairGeom<SPARSE, EPI, false>::kBN;
   if constexpr (kWideBN != kNarrowBN) {
     const int P = gemm_pairs<BF16, EPI, SPARSE, false>();
@@ -374,38 +376,38 @@ sp24_status launch_gemm_pair_t(const void *B, int64_t T, int64_t Kd, const void 
       };
       if (busiest(kWideBN) * 0.95 < busiest(kNarrowBN))
         return launch_gemm_pair_w<BF16, EPI, SPARSE, true>(B, T, Kd, vals, meta, M, out, aux, stream, dec_w, dec_idx,
-                                                           dec_lambda, fixed);
+                                                           dec_lambda, fixed, a_mn);
     }
   }
   return launch_gemm_pair_w<BF16, EPI, SPARSE, false>(B, T, Kd, vals, meta, M, out, aux, stream, dec_w, dec_idx,
-                                                      dec_lambda, fixed);
+                                                      dec_lambda, fixed, a_mn);
 }
 
 template <bool SPARSE>
 sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
-                        sp24_dtype dt, void *out, int epi, void *aux, cudaStream_t s) {
+                        sp24_dtype dt, void *out, int epi, void *aux, cudaStream_t s, bool a_mn = false) {
   const bool bf = dt == SP24_BF16;
   switch (epi) {
-    case kEpiNone: return bf ? launch_gemm_pair_t<true, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_pair_t<false, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
-    case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                             : launch_gemm_pair_t<false, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
-    case kEpiDgelu: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                              : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+    case kEpiNone: return bf ? launch_gemm_pair_t<true, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                             : launch_gemm_pair_t<false, kEpiNone, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
+    case kEpiGelu: return bf ? launch_gemm_pair_t<true, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                             : launch_gemm_pair_t<false, kEpiGelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
+    case kEpiDgelu: return bf ? launch_gemm_pair_t<true, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                              : launch_gemm_pair_t<false, kEpiDgelu, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
     case kEpiGeluDeriv:
-      return bf ? launch_gemm_pair_t<true, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                : launch_gemm_pair_t<false, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+      return bf ? launch_gemm_pair_t<true, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                : launch_gemm_pair_t<false, kEpiGeluDeriv, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
     case kEpiMulAux:
-      return bf ? launch_gemm_pair_t<true, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s)
-                : launch_gemm_pair_t<false, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s);
+      return bf ? launch_gemm_pair_t<true, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                : launch_gemm_pair_t<false, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
     default: break;
   }
   if (SPARSE) {   // the gated epilogues serve the 2:4 GEMMs
     switch (epi) {
-      case kEpiGeglu: return bf ? launch_gemm_pair_t<true, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s)
-                                : launch_gemm_pair_t<false, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s);
-      case kEpiDgeglu: return bf ? launch_gemm_pair_t<true, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s)
-                                 : launch_gemm_pair_t<false, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s);
+      case kEpiGeglu: return bf ? launch_gemm_pair_t<true, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                                : launch_gemm_pair_t<false, kEpiGeglu, true>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
+      case kEpiDgeglu: return bf ? launch_gemm_pair_t<true, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                                 : launch_gemm_pair_t<false, kEpiDgeglu, true>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
       default: break;
     }
   }
@@ -419,6 +421,7 @@ constexpr unsigned kDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) |
                                 (1u << SP24_EPI_MUL_AUX);
 constexpr unsigned kDenseEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_GELU) | (1u << SP24_EPI_DGELU) |
                                 (1u << SP24_EPI_GELU_DERIV) | (1u << SP24_EPI_MUL_AUX);
+constexpr unsigned kDenseDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) | (1u << SP24_EPI_MUL_AUX);
 
 sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                           sp24_dtype dt, const void *out, int epi, const void *aux, unsigned allowed_epis) {
@@ -640,6 +643,16 @@ sp24_status sp24_gemm_dense(const void *B, int64_t T, int64_t Kd, const void *A,
   if ((st = check_device()) != SP24_OK) return st;
   if (T == 0) return SP24_OK;
   return launch_gemm<false>(B, T, Kd, A, nullptr, M, dtype, out, epi, aux, as_stream(stream));
+}
+
+sp24_status sp24_gemm_dgrad_dense(const void *dY, int64_t T, int64_t N, const void *W, int64_t K, sp24_dtype dtype,
+                                  void *dX, sp24_epilogue epi, const void *aux, void *stream) {
+  sp24_status st = validate_gemm(dY, T, N, W, W, K, dtype, dX, epi, aux, kDenseDgradEpis);
+  if (st != SP24_OK) return st;
+  if ((st = check_device()) != SP24_OK) return st;
+  if (T == 0) return SP24_OK;
+  return launch_gemm<false>(dY, T, N, W, nullptr, K, dtype, dX, epi, const_cast<void *>(aux), as_stream(stream),
+                            /*a_mn=*/true);
 }
 
 sp24_status sp24_transpose(const void *in, int64_t rows, int64_t cols, sp24_dtype dtype, void *out, void *stream) {

@@ -45,6 +45,8 @@ def main(argv=None):
     ap.add_argument("--cols", type=int, required=True)
     ap.add_argument("--tokens", type=int, default=8192)
     ap.add_argument("--dtype", choices=["f16", "bf16"], default="f16")
+    ap.add_argument("--via-transpose", action="store_true",
+                    help="gemm_dense_dgrad: multiply by W^T formed with sp24_transpose")
     ap.add_argument("--dist", choices=["normal", "tie"], default="normal")
     ap.add_argument("--epi", choices=["none", "gelu", "dgelu", "gelu_deriv", "mul_aux", "geglu", "dgeglu"],
                     default="none")
@@ -113,13 +115,17 @@ def main(argv=None):
         epi = "gelu" if args.epi == "gelu" else None
         fn = lambda: sp.sp24_gemm_dense(x, w, y, epi, aux)
     elif k == "gemm_dense_dgrad":
+        # dX = dY W with W read as stored (--via-transpose: sp24_gemm_dense on W^T)
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
-        wt = torch.empty(C, R, dtype=tdt, device=dev)
-        sp.sp24_transpose(w, wt)
         dx = torch.empty(T, C, dtype=tdt, device=dev)
-        aux = torch.randn(T, C, device=dev, generator=gen).to(tdt) if args.epi == "dgelu" else None
-        epi = "dgelu" if args.epi == "dgelu" else None
-        fn = lambda: sp.sp24_gemm_dense(dy, wt, dx, epi, aux)
+        epi = args.epi if args.epi in ("dgelu", "mul_aux") else None
+        aux = torch.randn(T, C, device=dev, generator=gen).to(tdt) if epi else None
+        if args.via_transpose:
+            wt = torch.empty(C, R, dtype=tdt, device=dev)
+            sp.sp24_transpose(w, wt)
+            fn = lambda: sp.sp24_gemm_dense(dy, wt, dx, epi, aux)
+        else:
+            fn = lambda: sp.sp24_gemm_dgrad_dense(dy, w, dx, epi, aux)
     else:
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
         epi = args.epi if args.epi in ("dgelu", "mul_aux", "dgeglu") else None

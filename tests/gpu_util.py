@@ -38,3 +38,20 @@ def assert_gemm_close(got: np.ndarray, ref_f64: np.ndarray, dtype: str, what: st
     assert fro <= FRO_TOL, f"{what}: relative Frobenius error {fro:.3e} > {FRO_TOL}"
     assert elem <= ELEM_TOL, f"{what}: max element relative error {elem:.3e} > {ELEM_TOL}"
     return fro, elem
+
+
+def assert_gemm_within_accumulation_bound(got: np.ndarray, ref_f64: np.ndarray, abs_prod: np.ndarray, n: int,
+                                          dtype: str, what: str = ""):
+    """Long contractions over whole matrices: the relative Frobenius bound above, and on every
+    element |got - ref| <= n 2^-24 sum_k |a_k b_k| + 2 ulp(ref) of the output dtype (the
+    textbook bound of an fp32 sum of n products, plus the output rounding).  abs_prod is
+    |A| |B|, the sum of the products' magnitudes.  Near-cancelling elements, whose relative
+    error the fixed floor above would judge, get their absolute error budget instead; a wrong
+    or missing term in every element still moves the Frobenius error far past 1e-3."""
+    ref_q = oracle.round_to(ref_f64, dtype)
+    fro, _ = gemm_errors(got, ref_q)
+    assert fro <= FRO_TOL, f"{what}: relative Frobenius error {fro:.3e} > {FRO_TOL}"
+    ulp = 2.0 ** (-10 if dtype == "f16" else -7)
+    bound = n * 2.0 ** -24 * abs_prod + 2 * ulp * np.abs(ref_q) + 2.0 ** -24
+    worst = float(np.max(np.abs(got - ref_q) / bound))
+    assert worst <= 1.0, f"{what}: an element exceeds the accumulation bound ({worst:.3f} of it)"

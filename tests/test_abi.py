@@ -100,6 +100,16 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_INVALID_ARG"]                       # no such epilogue
     assert _raw("sp24_gemm_dense", fake, 8, 32, odd, 16, 0, fake, 0, None, None) == \
         E["SP24_ERR_MISALIGNED"]
+    assert _raw("sp24_gemm_dgrad_dense", fake, 8, 24, fake, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # N (the contraction) % 16
+    assert _raw("sp24_gemm_dgrad_dense", fake, 8, 32, fake, 24, 0, fake, 0, None, None) == \
+        E["SP24_ERR_UNSUPPORTED_SHAPE"]                # K (the output width) % 16
+    assert _raw("sp24_gemm_dgrad_dense", fake, 8, 32, fake, 16, 0, fake, 1, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # GELU is not an input-gradient epilogue
+    assert _raw("sp24_gemm_dgrad_dense", fake, 8, 32, fake, 16, 0, fake, 7, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # MUL_AUX without aux
+    assert _raw("sp24_gemm_dgrad_dense", fake, 8, 32, odd, 16, 0, fake, 0, None, None) == \
+        E["SP24_ERR_MISALIGNED"]
     assert _raw("sp24_transpose", fake, 8, 8, 5, fake, None) == E["SP24_ERR_UNSUPPORTED_DTYPE"]
     assert _raw("sp24_transpose", None, 8, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
     assert _raw("sp24_transpose", fake, -2, 8, 0, fake, None) == E["SP24_ERR_INVALID_ARG"]
@@ -209,6 +219,10 @@ def test_binding_rejects_wrong_dtype_and_short_buffers():
     ok_until_device(sp.sp24_gemm_dense, x, w, y)
     bad(sp.sp24_gemm_dense, x, w[:, :64].contiguous(), y, match="A:")
     bad(sp.sp24_transpose, w, torch.zeros(C, R - 4, dtype=f16), match="out")
+    ok_until_device(sp.sp24_gemm_dgrad_dense, y, w, x, "mul_aux", x.clone())
+    bad(sp.sp24_gemm_dgrad_dense, y, w[:32].contiguous(), x, match="W has 32 rows")
+    bad(sp.sp24_gemm_dgrad_dense, y, w, x[:, :64].contiguous(), match="dX")
+    bad(sp.sp24_gemm_dgrad_dense, y, w, x, "mul_aux", x[:1].clone(), match="aux")
     # weight gradient: MVUE(dY^T) [R x T] compressed along T, dW fp32 [R x C]
     dy = torch.zeros(T, R, dtype=f16)
     yv = torch.zeros(R, T // 2, dtype=f16)

@@ -4,7 +4,8 @@
 fine-tuning procedure near the end of pre-training) and Experiment Setup row
 (dense fine-tuning takes the last 1/6 of the total steps): the FFN products
 run dense, on the same tcgen05 pipeline as the 2:4 GEMMs.  The input gradient
-takes W^T from the transpose kernel.  Tolerances as in gpu_util.
+reads W as stored (sp24_gemm_dgrad_dense, W loaded MN-major) or takes W^T from
+the transpose kernel (sp24_gemm_dense).  Tolerances as in gpu_util.
 """
 import numpy as np
 import pytest
@@ -13,7 +14,7 @@ import torch
 import oracle
 import synthetic_inputs as si
 import structured_sparse_transformer_b200 as sp
-from gpu_util import assert_gemm_close, f64_of
+from gpu_util import assert_gemm_close, assert_gemm_within_accumulation_bound, f64_of
 
 pytestmark = pytest.mark.gpu
 
@@ -69,8 +70,8 @@ def test_dense_ffn_chain_with_gelu_sampled_rows(wl):
     dX = torch.empty(T, d, dtype=tdt, device="cuda")
     sp.sp24_gemm_dense(X.cuda(), W1d, H, "gelu", Hpre)
     sp.sp24_gemm_dense(H, W2d, Y)
-    sp.sp24_gemm_dense(dY.cuda(), _transpose(W2d), dH, "dgelu", Hpre)
-    sp.sp24_gemm_dense(dH, _transpose(W1d), dX)
+    sp.sp24_gemm_dgrad_dense(dY.cuda(), W2d, dH, "dgelu", Hpre)
+    sp.sp24_gemm_dgrad_dense(dH, W1d, dX)
     torch.cuda.synchronize()
     rows = np.arange(3, T, 32)
     w1f, w2f = oracle.to_f64(si.bits16(W1), dt), oracle.to_f64(si.bits16(W2), dt)
@@ -81,6 +82,48 @@ def test_dense_ffn_chain_with_gelu_sampled_rows(wl):
     dh_ref = oracle.dense_dgrad(oracle.to_f64(si.bits16(dY)[rows], dt), w2f) * oracle.gelu_grad(f64_of(Hpre, dt)[rows])
     assert_gemm_close(f64_of(dH, dt)[rows], dh_ref, dt, "dgrad2 dgelu")
     assert_gemm_close(f64_of(dX, dt)[rows], oracle.dense_dgrad(f64_of(dH, dt)[rows], w1f), dt, "dgrad1")
+
+
+@pytest.mark.parametrize("T,N,K,dtype", [(128, 128, 128, "f16"), (200, 256, 384, "f16"), (77, 144, 400, "bf16"),
+                                         (1, 16, 16, "f16"), (300, 1600, 208, "f16"), (513, 208, 1600, "bf16"),
+                                         (1000, 6400, 1600, "f16"), (640, 1600, 6400, "f16")])
+def test_dense_dgrad_reads_w_as_stored(T, N, K, dtype):
+    """dX = dY W with W [N x K] loaded MN-major (ragged T, K tiles of 64-column atoms, K steps
+    past N): every element against the fp64 product within the fp32 accumulation bound, and
+    the same bits as the product with W^T from the transpose (the same MMAs in the same K
+    order; only the shared-memory layout of A differs)."""
+    w = si.normal((N, K), 0.02, N + K + 1, dtype)
+    dy = si.normal((T, N), 1.0, T + 2, dtype)
+    wd, dyd = w.cuda(), dy.cuda()
+    dx = torch.full((T, K), float("nan"), dtype=w.dtype, device="cuda")
+    sp.sp24_gemm_dgrad_dense(dyd, wd, dx)
+    dx_t = torch.empty_like(dx)
+    sp.sp24_gemm_dense(dyd, _transpose(wd), dx_t)
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    assert torch.equal(dx.view(torch.int16), dx_t.view(torch.int16))
+    dyf, wf = oracle.to_f64(si.bits16(dy), dtype), oracle.to_f64(si.bits16(w), dtype)
+    ref = oracle.dense_dgrad(dyf, wf)
+    assert_gemm_within_accumulation_bound(f64_of(dx, dtype), ref, np.abs(dyf) @ np.abs(wf), N, dtype,
+                                          f"dgrad, W as stored {T}x{N}x{K}")
+
+
+@pytest.mark.parametrize("epi", ["dgelu", "mul_aux"])
+def test_dense_dgrad_epilogues_read_w_as_stored(epi):
+    """The input-gradient epilogues on the MN-major weight: dGELU of a stored pre-activation,
+    and the product with a stored derivative."""
+    T, N, K, dtype = 456, 512, 1040, "f16"
+    w = si.normal((N, K), 0.02, 9, dtype)
+    dy = si.normal((T, N), 1.0, 10, dtype)
+    aux = si.normal((T, K), 1.0, 11, dtype)
+    dx = torch.empty(T, K, dtype=w.dtype, device="cuda")
+    sp.sp24_gemm_dgrad_dense(dy.cuda(), w.cuda(), dx, epi, aux.cuda())
+    torch.cuda.synchronize()
+    assert sp.sp24_device_status() == 0
+    acc = oracle.dense_dgrad(oracle.to_f64(si.bits16(dy), dtype), oracle.to_f64(si.bits16(w), dtype))
+    a = oracle.to_f64(si.bits16(aux), dtype)
+    ref = acc * (oracle.gelu_grad(a) if epi == "dgelu" else a)
+    assert_gemm_close(f64_of(dx, dtype), ref, dtype, f"dgrad {epi}, W as stored")
 
 
 def test_dense_zero_tokens_is_a_no_op():
