@@ -194,8 +194,8 @@ constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 
 __device__ const PackedTables g_packed = make_packed_tables();
 __device__ const SelectTables g_select = make_select_tables();
-// 1, read at run time: multiply-adds by it keep integer additions on the FMA
-// pipe (the ALU pipe, half as wide, carries the maxima and the bit work).
+// 1, read at run time: multiply-adds by it keep the pair sums' integer steps
+// on the FMA pipe (the ALU pipe, half as wide, carries the maxima and the bit work).
 __device__ uint32_t g_one = 1u;
 
 __device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
@@ -219,7 +219,8 @@ __device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
 //     below 2^32 (a sum of eight is below 2^24), so one unsigned max picks the
 //     largest exact sum and, among equal sums, the lowest pattern index.
 //   * The max over the 90 patterns is the same dynamic program over column-count
-//     states: per state, the best top and bottom combo, then the best total.
+//     states: per state, the best top and bottom combo, then the best total, each
+//     step one add-then-max.
 template <bool BF16>
 __device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2], const uint8_t *__restrict__ decode,
                                                         uint32_t one) {
@@ -275,14 +276,14 @@ __device__ __forceinline__ uint32_t search_block_packed(const uint32_t (&w)[4][2
     for (int i = 0; i < 6; ++i) {
       if (i < PT.ntop[st]) {
         const int c = PT.top[st][i];
-        tb = max(tb, imad(P[0][c / 6], one, P[1][c % 6]));
+        tb = __viaddmax_u32(P[0][c / 6], P[1][c % 6], tb);
       }
       if (i < PT.nbot[st]) {
         const int b = PT.bot[st][i];
-        bb = max(bb, P[2][b / 6] + P[3][b % 6]);
+        bb = __viaddmax_u32(P[2][b / 6], P[3][b % 6], bb);
       }
     }
-    best = max(best, tb + bb);
+    best = __viaddmax_u32(tb, bb, best);
   }
   return decode[best & 0xFFu];
 }
