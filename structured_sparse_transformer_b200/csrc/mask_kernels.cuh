@@ -361,8 +361,8 @@ struct MaskSmem {
   __align__(8) uint16_t rc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // row codes, [br][bc]
   __align__(8) uint16_t cc[COMPRESS ? 2 : 1][kTileBlocks][kTileBlocks];   // column codes, [bc][br]
   __align__(16) uint32_t vcol[COMPRESS ? 2 : 1][COMPRESS ? kTile * 16 : 4];
-  uint16_t queue[SEARCH ? 2 * kTileBlocks * kTileBlocks : 2];
-  int qn;
+  // Blocks of each warp that need the exact search (two per lane at most).
+  uint16_t wq[SEARCH ? kMaskThreads / 32 : 1][SEARCH ? 64 : 2];
 };
 
 template <bool SEARCH, bool COMPRESS>
@@ -492,6 +492,7 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
 
   // Phase 1: search (SEARCH), or take the given mask (!SEARCH).
   uint32_t p[2];
+  bool need[2] = {false, false};
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     const bool ok = b ? ok1 : ok0;
@@ -501,29 +502,35 @@ __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_
 #pragma unroll
       for (int i = 0; i < 4; ++i) { blk[i][0] = w[i][2 * b]; blk[i][1] = w[i][2 * b + 1]; }
       p[b] = search_block_packed<BF16>(blk, sm.decode, one);
-      if (p[b] == kNeedsExact) {
-        const int slot = atomicAdd(&sm.qn, 1);
-        sm.queue[slot] = (uint16_t)((rh << 8) | (br << 4) | (2 * uc + b));
-      }
+      need[b] = p[b] == kNeedsExact;
     }
-    if (SEARCH) sm.idx[rh][br][2 * uc + b] = (uint8_t)p[b];
   }
 
-  // Phase 1b: the exact search of the queued blocks, entry k by thread k.
+  // Phase 1b: the blocks that need the exact search, searched by the lanes of
+  // their own warp (entry k of the warp's queue by lane k mod 32), with no
+  // barrier across the CTA.  The queue lists them by lane, block 0 before 1.
   if (SEARCH) {
-    __syncthreads();
-    const int qn = sm.qn;
-    if (qn > 0) {
-      for (int k = tid; k < qn; k += kMaskThreads) {
-        const int id = sm.queue[k];
+    const unsigned n0 = __ballot_sync(0xFFFFFFFFu, need[0]), n1 = __ballot_sync(0xFFFFFFFFu, need[1]);
+    if (n0 | n1) {
+      const int lane = tid & 31, wid = tid >> 5;
+      const unsigned below = (1u << lane) - 1u;
+      int pos = __popc(n0 & below) + __popc(n1 & below);
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+        if (need[b]) sm.wq[wid][pos++] = (uint16_t)((rh << 8) | (br << 4) | (2 * uc + b));
+      const int wn = __popc(n0) + __popc(n1);
+      __syncwarp();
+      for (int k = lane; k < wn; k += 32) {
+        const int id = sm.wq[wid][k];
         const int q = id >> 8, qbr = (id >> 4) & 15, qbc = id & 15;
         uint32_t blk[4][2];
         src.block(kTile * q + 4 * qbr, 4 * qbc, blk);
         sm.idx[q][qbr][qbc] = (uint8_t)search_block<BF16>(blk, g_tables.index, g_tables.bits);
       }
-      __syncthreads();
+      __syncwarp();
 #pragma unroll
-      for (int b = 0; b < 2; ++b) p[b] = sm.idx[rh][br][2 * uc + b];
+      for (int b = 0; b < 2; ++b)
+        if (need[b]) p[b] = sm.idx[rh][br][2 * uc + b];
     }
   }
 
@@ -650,7 +657,7 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
     uint8_t *__restrict__ meta_col) {
   __shared__ MaskSmem<SEARCH, COMPRESS> sm;
   __shared__ unsigned long long s_flip;
-  if (threadIdx.x == 0) { s_flip = 0; sm.qn = 0; }
+  if (threadIdx.x == 0) s_flip = 0;
   load_mask_tables(sm);
   const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
   pdl_launch_dependents();
@@ -671,6 +678,12 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
 // into a buffer as soon as the CTA has finished reading tile i from it, so the
 // loads of the next two tiles overlap the work on this one.  Every wait is
 // bounded; on a timeout the CTA records the error, lets its copies land and exits.
+// One CTA barrier per tile (two with compression): each thread waits for its
+// tile's copy itself, and the decision to stop is taken after the end-of-tile
+// barrier on a flag of that tile's parity, so a thread already waiting on the
+// next tile cannot change the flag the others are about to read.  A tile whose
+// wait ran out is computed on whatever the buffer holds; its outputs are void
+// (the device status reports the timeout), and every index stays in bounds.
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP>
 __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) mask_stream_kernel(
     const __grid_constant__ CUtensorMap tm_w, int64_t R, int64_t C, uint8_t *__restrict__ idx,
@@ -684,7 +697,7 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
   __shared__ MaskSmem<SEARCH, COMPRESS> sm;
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ unsigned long long s_flip;
-  __shared__ volatile int s_abort;
+  __shared__ volatile int s_abort[2];   // per tile parity
   const int tid = threadIdx.x;
   const uint32_t chunks_x = (uint32_t)((C + kChunk - 1) / kChunk);
   const uint32_t chunks_y = (uint32_t)((R + kChunk - 1) / kChunk);
@@ -711,8 +724,8 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
     prefetch_tensormap(&tm_w);
     if (FLIP && prev_tma) prefetch_tensormap(&tm_prev);
     s_flip = 0;
-    s_abort = 0;
-    sm.qn = 0;
+    s_abort[0] = 0;
+    s_abort[1] = 0;
   }
   load_mask_tables(sm);
   const uint32_t one = *reinterpret_cast<volatile const uint32_t *>(&g_one);
@@ -728,11 +741,10 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
       }
   }
   unsigned flips = 0;
+  bool aborted = false;
   for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
     const int buf = (int)(it & 1);
-    mbar_wait_bounded(&s_full[buf], (uint32_t)((it >> 1) & 1), wait_budget, &s_abort);
-    __syncthreads();
-    if (s_abort) break;
+    mbar_wait_bounded(&s_full[buf], (uint32_t)((it >> 1) & 1), wait_budget, &s_abort[buf]);
     uint32_t cy, cx;
     int kh;
     tile_xy(t, cy, cx, kh);
@@ -741,8 +753,11 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
                                                  vals_row, meta_row, vals_col, meta_col, sm, one,
                                                  (FLIP && prev_tma) ? s_prev[buf] : nullptr);
     __syncthreads();   // every read of this buffer and of the tile's shared state is done
+    if (s_abort[buf]) {
+      aborted = true;
+      break;
+    }
     if (tid == 0) {
-      sm.qn = 0;
       const int64_t nt = t + 2ll * gridDim.x;
       if (nt < ntiles) {
         issue(nt, buf);
@@ -752,7 +767,7 @@ __global__ void __launch_bounds__(kMaskThreads, mask_ctas_per_sm<COMPRESS>()) ma
   }
   if (FLIP) mask_flip_flush(flips, &s_flip, flip_count);
   // After an abort, let the copies still in flight land before the CTA exits.
-  if (tid == 0 && s_abort) {
+  if (tid == 0 && aborted) {
     for (int64_t k = it; k < issued; ++k) {
       volatile int no_abort = 0;
       mbar_wait_bounded(&s_full[k & 1], (uint32_t)((k >> 1) & 1), kMaskDrainBudget, &no_abort);
