@@ -107,15 +107,14 @@ constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in 
 // 256 columns.  B comes from the row-major layer input [T x K] (K contiguous),
 // i.e. MN-major for the MMA: per stage each CTA loads two 128B-swizzled atoms
 // of 64 columns x 128 tokens (16 KB each; atom a of CTA r holds columns
-// 128a + 64r .. +63 of the tile), so a stage is 50 KB and 4 stages fit.  Each
-// 32-token K step issues two MMAs of N = 128 (one per atom; the pair's two
-// 64-column halves make the 128), into accumulator columns 0 and 128: an MMA
-// never spans two atoms along N.  One 256-column accumulator (no double
+// 128r + 64a .. +63 of the tile), so a stage is 50 KB and 4 stages fit.  Each
+// 32-token K step issues one MMA of N = 256 (each CTA's 128 columns, its two
+// atoms one descriptor stride apart).  One 256-column accumulator (no double
 // buffering: the weight-gradient tiles run one per pair at the FFN sizes).
 // The dense variant (dense fine-tuning) takes A = dY [T x N] as stored, read
 // MN-major like B (two 8 KB atoms of 64 rows of dW x 64 tokens), 64 tokens per
 // stage: A 16 KB + two 8 KB atoms of B, 6 stages; each 16-token K step issues
-// two dense MMAs of N = 128.  (Tiles of 128 dW columns with double-buffered
+// one dense MMA of N = 256.  (Tiles of 128 dW columns with double-buffered
 // accumulators were measured 10-15% slower at the 1.5B shapes, although they
 // leave fewer column-waves idle: each stage then carries half the MMA work for
 // the same A tile and per-stage overhead.)
@@ -501,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     while (ok && sched.next(tile, kb, ke)) {
       const int mt = tile_mt(tile);
       const int a_row = mt * 2 * kPairRows + (int)rank * kPairRows;
-      const int b_row = tile_nt(tile) * G::kBN + (int)rank * (WG ? 64 : G::kBN / 2);
+      const int b_row = tile_nt(tile) * G::kBN + (int)rank * (WG ? 128 : G::kBN / 2);
       // A pair tile past the last 128-row tile reads zero rows (TMA fill); give
       // it the last real metadata chunk so every code the MMA sees is valid.
       const int chunk_row = min(2 * mt + (int)rank, num_row_tiles - 1) * num_kt;
@@ -523,10 +522,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_pair(st, &tm_a, &full[s], kt * G::kAcols, a_row);
         }
         if (WG) {
-          // MN-major atoms: x = dW column (b_row, b_row + 128), y = token.
+          // MN-major atoms: x = dW column (b_row, b_row + 64), y = token.
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], b_row, kt * G::kBK);
           if (G::kBBoxes == 2)
-            tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 128, kt * G::kBK);
+            tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], b_row + 64, kt * G::kBK);
         } else {
           tma_load_2d_pair(st + kPairSmemA, &tm_b, &full[s], kt * G::kBK, b_row);
           if (SPARSE) tma_load_2d_pair(st + kPairSmemA + G::kBBoxBytes, &tm_b, &full[s], kt * G::kBK + 64, b_row);
@@ -546,15 +545,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ----------------------------------------------------- MMA issuer (leader)
     // Descriptors of stage 0; stage s and K step kk only move the 14-bit start
     // address field (all of shared memory is below 2^18 bytes, so it never carries).
-    // wgrad: N = 128 per MMA and B MN-major (instruction descriptor bit 16).
-    // Its B descriptor steps 8-token groups 1024 bytes apart (the stride field);
-    // an MMA reads a single 64-column atom per CTA, so the field for the stride
-    // between atoms along N is never used and is given the same 1024.
+    // wgrad: one MMA of N = 256 per K step, B MN-major (instruction descriptor
+    // bit 16): each CTA holds 128 of the tile's columns as two 64-column atoms,
+    // and the B descriptor's leading field is the atom stride (kBBoxBytes), its
+    // stride field the 1024 bytes between 8-token groups.
     // Dense wgrad: A MN-major too (bit 15); its descriptor's leading field is the
     // 8 KB between its two 64-row atoms, its stride field the 1024 bytes between
     // 8-token groups.
-    constexpr uint32_t idesc = WG ? ((SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, 128)
-                                             : (make_idesc_dense(BF16, 2 * kPairRows, 128) | (1u << 15))) |
+    constexpr uint32_t idesc = WG ? ((SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, 256)
+                                             : (make_idesc_dense(BF16, 2 * kPairRows, 256) | (1u << 15))) |
                                     (1u << 16))
                                : SPARSE ? make_idesc_sparse(BF16, 2 * kPairRows, G::kBN)
                                         : make_idesc_dense(BF16, 2 * kPairRows, G::kBN);
@@ -562,7 +561,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t idesc_amn = idesc | (1u << 15);
     const uint64_t a_desc0 =
         smem_desc(smem_u32(stage_base), (!SPARSE && (WG || a_mn)) ? kPairSmemA / 2 : 16, 1024, kSwizzle128B);
-    const uint64_t b_desc0 = smem_desc(smem_u32(stage_base + kPairSmemA), WG ? 1024 : 16, 1024, kSwizzle128B);
+    const uint64_t b_desc0 =
+        smem_desc(smem_u32(stage_base + kPairSmemA), WG ? G::kBBoxBytes : 16, 1024, kSwizzle128B);
     const uint64_t e_desc0 =
         smem_desc(smem_u32(stage_base + kPairSmemA + G::kBBoxes * G::kBBoxBytes), 128, 128, kSwizzleNone);
     uint32_t g = 0;
@@ -588,11 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t accum = (kt != kb || kk != 0) ? 1u : 0u;
-            const uint64_t ak = ad + (uint64_t)(kk * (2048 >> 4));
-            const uint64_t bk = bd + (uint64_t)(kk * (2048 >> 4));
-            tc_mma_f16_pair(acc, ak, bk, idesc, accum);
-            if (G::kBBoxes == 2)
-              tc_mma_f16_pair(acc + 128, ak, bk + (uint64_t)(G::kBBoxBytes >> 4), idesc, accum);
+            tc_mma_f16_pair(acc, ad + (uint64_t)(kk * (2048 >> 4)), bd + (uint64_t)(kk * (2048 >> 4)), idesc, accum);
           }
         } else if (WG) {
           const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;
@@ -604,10 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const uint32_t tm = t_meta + 2 * (kk >> 1);
             const uint32_t id = idesc | (uint32_t)(kk & 1);
             const uint32_t accum = (kt != kb || kk != 0) ? 1u : 0u;
-            const uint64_t bk = bd + (uint64_t)(kk * (4096 >> 4));
-            tc_mma_sp_f16_pair(acc, ad + 2 * kk, bk, tm, id, accum);
-            if (G::kBBoxes == 2)
-              tc_mma_sp_f16_pair(acc + 128, ad + 2 * kk, bk + (uint64_t)(G::kBBoxBytes >> 4), tm, id, accum);
+            tc_mma_sp_f16_pair(acc, ad + 2 * kk, bd + (uint64_t)(kk * (4096 >> 4)), tm, id, accum);
           }
         } else if (SPARSE) {
           const uint32_t t_meta = tmem_base + G::kMetaCol + 4 * s;

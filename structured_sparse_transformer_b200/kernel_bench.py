@@ -9,7 +9,9 @@ W is [rows x cols] (N(0, 0.02), or the 8-level tie-heavy variant with
 T = --tokens rows of N(0, 1) activations: gemm_fwd computes [T x rows] from
 [T x cols], gemm_dgrad [T x cols] from [T x rows], gemm_wgrad the fp32
 [rows x cols] weight gradient from dY [T x rows] (MVUE-sparsified) and
-X [T x cols] (gemm_wgrad_decay: with the masked decay of W's mask in its epilogue); mvue sparsifies dY [T x rows] (bytes per dY element).  Each timed launch follows an
+X [T x cols] (gemm_wgrad_decay: with the masked decay of W's mask in its epilogue;
+gemm_wgrad_dense: dY dense, read as stored); mvue sparsifies dY [T x rows] (bytes per dY
+element).  Each timed launch follows an
 L2 flush (256 MiB write) and is timed alone with CUDA events on the current
 stream.  Prints one JSON line: average microseconds per launch and the
 algorithmic throughput (bytes for the memory-bound kernels, dense-equivalent
@@ -40,7 +42,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--kernel", required=True,
                     choices=sorted(BYTES_PER_ELEMENT) + ["gemm_fwd", "gemm_dgrad", "gemm_dense_fwd", "gemm_dense_dgrad",
-                                                         "gemm_wgrad", "gemm_wgrad_decay"])
+                                                         "gemm_wgrad", "gemm_wgrad_decay", "gemm_wgrad_dense"])
     ap.add_argument("--rows", type=int, required=True)
     ap.add_argument("--cols", type=int, required=True)
     ap.add_argument("--tokens", type=int, default=8192)
@@ -105,6 +107,12 @@ def main(argv=None):
                 fn = lambda: sp.sp24_gemm_wgrad(x, yv, ym, R, dw)
             else:   # dW of W [rows x cols] with the masked decay in the epilogue
                 fn = lambda: sp.sp24_gemm_wgrad_decay(x, yv, ym, R, w, prev, 6e-5, dw)
+    elif k == "gemm_wgrad_dense":
+        # dW [rows x cols] fp32 = dY^T X, dY [T x rows] and X [T x cols] read as stored
+        dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
+        x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
+        dw = torch.empty(R, C, dtype=torch.float32, device=dev)
+        fn = lambda: sp.sp24_gemm_wgrad_dense(x, dy, dw)
     elif k == "transpose":
         wt = torch.empty(C, R, dtype=tdt, device=dev)
         fn = lambda: sp.sp24_transpose(w, wt)
