@@ -194,15 +194,6 @@ constexpr uint32_t kNeedsExact = 0xFFu;  // fast path could not certify its sums
 
 __device__ const PackedTables g_packed = make_packed_tables();
 __device__ const SelectTables g_select = make_select_tables();
-// 1, read at run time: multiply-adds by it keep the pair sums' integer steps
-// on the FMA pipe (the ALU pipe, half as wide, carries the maxima and the bit work).
-__device__ uint32_t g_one = 1u;
-
-__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
 
 // Packed-key search of one block, exact when the block's nonzero magnitudes span
 // at most 10 binades (fp16) or 13 (bf16); otherwise returns kNeedsExact.

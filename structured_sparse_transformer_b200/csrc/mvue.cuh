@@ -116,13 +116,20 @@ __device__ __forceinline__ double mag_f64(uint32_t m) {
   return (double)__half2float(__ushort_as_half((unsigned short)m));
 }
 
-// Entry i (0..3) of a group held as lo = v0 | v1 << 16, hi = v2 | v3 << 16.
-__device__ __forceinline__ uint32_t pick_raw(uint32_t lo, uint32_t hi, int i) {
-  return ((i < 2 ? lo : hi) >> (16 * (i & 1))) & 0xFFFFu;
-}
+// Integer constants formed from the run-time 1 (multiply-adds by them stay on
+// the FMA pipe; the ALU pipe is this kernel's busy one).
+struct MvueConsts {
+  uint32_t k4, k16, k22, k10, k64k;   // 4, 16, 0x22, 0x10, 65536
+  __device__ __forceinline__ explicit MvueConsts(uint32_t one)
+      : k4(one << 2), k16(one << 4), k22(one * 0x22u), k10(one << 4), k64k(one << 16) {}
+};
 
-// Sign bit (as bit 15) of entry i, from the group's 4-bit sign mask.
-__device__ __forceinline__ uint32_t sign_of(uint32_t sgn4, int i) { return ((sgn4 >> i) & 1u) << 15; }
+// Entry i (0..3) of a group held as lo = v0 | v1 << 16, hi = v2 | v3 << 16, in
+// the low 16 bits of one byte permutation (selector 0x22 i + 0x10 picks bytes
+// 2i and 2i + 1 of the pair; the upper 16 bits are left unspecified).
+__device__ __forceinline__ uint32_t entry_bits(uint32_t lo, uint32_t hi, int i, const MvueConsts &K) {
+  return __byte_perm(lo, hi, imad((uint32_t)i, K.k22, K.k10));
+}
 
 // One group of four (16-bit storage bits in lo/hi), without branches on the
 // group's case: the cumulative sums run over w = |v| with the largest entry
@@ -131,26 +138,22 @@ __device__ __forceinline__ uint32_t sign_of(uint32_t sgn4, int i) { return ((sgn
 // estimates have the magnitude `step` (S/2, or R) except the entry kept as is,
 // so one rounding RNE_dtype(RNE_fp32(step)) serves both and the signs come from
 // the stored bits.  The largest |v| is found on the magnitude bits (for finite
-// values their order is that of the magnitudes; equal magnitudes, equal bits).
-// Returns the kept positions pa < pb and their output bits.
+// values their order is that of the magnitudes; equal magnitudes, equal bits):
+// keys (bits << 2) | (3 - i) make one unsigned max pick the largest, lowest
+// index first.  Returns the metadata code pa | pb << 2 of the kept positions
+// pa < pb and their output bits packed as bits(pa) | bits(pb) << 16.
 template <bool BF16>
-__device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, int &pa, int &pb, uint32_t &ba,
-                                           uint32_t &bb) {
+__device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, const MvueConsts &K,
+                                           uint32_t &code, uint32_t &packed) {
   const uint32_t lm = lo & 0x7FFF7FFFu, hm = hi & 0x7FFF7FFFu;
   double a[4];
   mag2_f64<BF16>(lm, a[0], a[1]);
   mag2_f64<BF16>(hm, a[2], a[3]);
   const double s = __dadd_rn(__dadd_rn(__dadd_rn(a[0], a[1]), a[2]), a[3]);
-  const uint32_t q[4] = {lm & 0xFFFFu, lm >> 16, hm & 0xFFFFu, hm >> 16};
-  int m = 0;
-  uint32_t qm = q[0];
-#pragma unroll
-  for (int i = 1; i < 4; ++i)
-    if (q[i] > qm) {
-      qm = q[i];
-      m = i;
-    }
-  const double am = mag_f64<BF16>(qm);
+  const uint32_t km = max(max(imad(lm & 0xFFFFu, K.k4, 3u), imad(lm >> 16, K.k4, 2u)),
+                          max(imad(hm & 0xFFFFu, K.k4, 1u), imad(hm >> 16, K.k4, 0u)));
+  const int m = 3 - (int)(km & 3u);
+  const double am = mag_f64<BF16>(km >> 2);
   const bool capped = __dadd_rn(am, am) >= s;
   double w[4];
 #pragma unroll
@@ -162,7 +165,7 @@ __device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, i
   const double step = capped ? tot : __dmul_rn(tot, 0.5);
   const double q1 = __dmul_rn(u, step);
   int i1 = count_le(e1, e2, e3, q1);
-  int i2 = capped ? m : count_le(e1, e2, e3, __dadd_rn(q1, step));
+  const int i2 = capped ? m : count_le(e1, e2, e3, __dadd_rn(q1, step));
   const bool empty = capped && !(tot > 0.0);        // at most one nonzero entry
   if (empty) i1 = m == 0 ? 1 : 0;
   // In the first case the two points always select two different nonzero
@@ -171,15 +174,14 @@ __device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, i
   // first point's entry; the one way to stay would need the total to round up
   // by half an ulp of the last entry's complement, and ties-to-even then makes
   // that entry reach half the total, i.e. the group capped.
-  const uint32_t sgn4 = ((lo >> 15) & 1u) | ((lo >> 30) & 2u) | ((hi >> 13) & 4u) | ((hi >> 28) & 8u);
   const uint32_t mag = empty ? 0u : mvue_bits<BF16>(step);
-  const uint32_t b1 = empty ? 0u : (mag | sign_of(sgn4, i1));
-  const uint32_t b2 = capped ? pick_raw(lo, hi, m) : (mag | sign_of(sgn4, i2));
-  if (i1 < i2) {
-    pa = i1; pb = i2; ba = b1; bb = b2;
-  } else {
-    pa = i2; pb = i1; ba = b2; bb = b1;
-  }
+  // Entry i1 takes the estimate's magnitude and its own sign (nothing when empty);
+  // entry i2 keeps its stored bits when it is the capped entry m (i2 == m then).
+  const uint32_t b1 = (entry_bits(lo, hi, i1, K) & (empty ? 0u : 0x8000u)) | mag;
+  const uint32_t b2 = (entry_bits(lo, hi, i2, K) & (capped ? 0xFFFFu : 0x8000u)) | (capped ? 0u : mag);
+  const bool fwd = i1 < i2;
+  code = fwd ? imad((uint32_t)i2, K.k4, (uint32_t)i1) : imad((uint32_t)i1, K.k4, (uint32_t)i2);
+  packed = fwd ? imad(b2, K.k64k, b1) : imad(b1, K.k64k, b2);
 }
 
 template <bool BF16>
@@ -215,24 +217,23 @@ __global__ void __launch_bounds__(kMvueThreads) mvue_sparsify_kernel(
   const int64_t n = n0 + p;
   uint64_t rnd[4] = {(uint64_t)(tseg >> 5), (uint64_t)n, 0ull, 0ull};
   philox4x64_10(rnd, keys);
-  uint32_t nib = 0x44444444u;                               // padding: positions 0, 1
+  const MvueConsts K(load_one());
+  uint32_t nib = 0;                                         // built from group 7 down (Horner, base 16)
   uint32_t packed[8];
   const uint32_t sel = (p & 1) ? 0x7632u : 0x5410u;         // this column's halves of the staged words
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 7; j >= 0; --j) {
     packed[j] = 0u;
+    uint32_t code = 4u;                                     // padding: positions 0, 1
     if (j < ngroups) {
       const uint32_t *col = &s_tile[32 * w + 4 * j][p >> 1];
       const uint32_t lo = __byte_perm(col[0], col[kMvueCols / 2], sel);
       const uint32_t hi = __byte_perm(col[kMvueCols], col[3 * kMvueCols / 2], sel);
       const uint32_t u32 = (uint32_t)(rnd[j >> 1] >> (32 * (j & 1)));
       const double u = (double)(u32 >> 8) * 0x1p-24;
-      int pa, pb;
-      uint32_t ba, bb;
-      mvue_group<BF16>(lo, hi, u, pa, pb, ba, bb);
-      nib = (nib & ~(0xFu << (4 * j))) | ((uint32_t)(pa | (pb << 2)) << (4 * j));
-      packed[j] = ba | (bb << 16);
+      mvue_group<BF16>(lo, hi, u, K, code, packed[j]);
     }
+    nib = imad(nib, K.k16, code);
   }
   if (n < N && ngroups > 0) {
     uint16_t *dst = vals + n * (T >> 1) + (tseg >> 1);

@@ -395,4 +395,19 @@ __host__ __device__ constexpr uint32_t make_idesc_sparse(bool bf16, int m, int n
          | ((uint32_t)(m >> 4) << 24);  // M / 16
 }
 
+// ------------------------------------------------ integer work on the FMA pipe
+// 1, read at run time.  Integer multiply-adds by it, or by constants formed from
+// it, stay integer multiply-adds, which issue to the FMA pipe: kernels whose ALU
+// pipe (half as wide as the issue rate) is the busy one move additions, shifts
+// and field packing there.
+__device__ uint32_t g_one = 1u;
+
+__device__ __forceinline__ uint32_t imad(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t load_one() { return *reinterpret_cast<volatile const uint32_t *>(&g_one); }
+
 }  // namespace sp24
