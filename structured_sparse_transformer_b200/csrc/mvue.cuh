@@ -152,12 +152,14 @@ __device__ __forceinline__ void mvue_group(uint32_t lo, uint32_t hi, double u, c
   const double s = __dadd_rn(__dadd_rn(__dadd_rn(a[0], a[1]), a[2]), a[3]);
   const uint32_t km = max(max(imad(lm & 0xFFFFu, K.k4, 3u), imad(lm >> 16, K.k4, 2u)),
                           max(imad(hm & 0xFFFFu, K.k4, 1u), imad(hm >> 16, K.k4, 0u)));
-  const int m = 3 - (int)(km & 3u);
+  const int m = (int)((km & 3u) ^ 3u);
   const double am = mag_f64<BF16>(km >> 2);
   const bool capped = __dadd_rn(am, am) >= s;
+  // A 16-bit magnitude widened to fp64 has a zero low word, so zeroing the
+  // entry kept outright only selects the high word.
   double w[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = (capped && i == m) ? 0.0 : a[i];
+  for (int i = 0; i < 4; ++i) w[i] = __hiloint2double((capped && i == m) ? 0 : __double2hiint(a[i]), 0);
   const double e1 = w[0];
   const double e2 = __dadd_rn(e1, w[1]);
   const double e3 = __dadd_rn(e2, w[2]);
