@@ -121,7 +121,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int, period_s: float = 0.2):
         import threading
         self.gpu, self.period = gpu_index, period_s
-        self.samples = []
+        self.samples = []   # (monotonic time, SM MHz, max SM MHz, active reasons)
+        self.marks = []     # (phase name, monotonic time at its start)
         self.error = None
         self.source = None
         self._nvml = self._open_nvml()
@@ -171,7 +172,7 @@ class ClockSampler:
         self.source = "nvml" if self._nvml else "nvidia-smi"
         while not self._stop.is_set():
             try:
-                self.samples.append(query())
+                self.samples.append((time.monotonic(), *query()))
             except Exception as e:  # a field unsupported: stop sampling, keep what was read
                 self.error = str(e)[:200]
                 return
@@ -185,15 +186,27 @@ class ClockSampler:
         self._stop.set()
         self._thread.join(timeout=15)
 
+    def mark(self, phase: str):
+        """Start of a named phase of the run (the previous one ends here)."""
+        self.marks.append((phase, time.monotonic()))
+
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"]}
-        sm = [x[0] for x in self.samples]
-        reasons = sorted(set().union(*[x[2] for x in self.samples]))
+        sm = [x[1] for x in self.samples]
+        reasons = sorted(set().union(*[x[3] for x in self.samples]))
         period = "~5 ms" if self.source == "nvml" else "~200 ms"
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+        phases = {}
+        for i, (name, t0) in enumerate(self.marks):
+            t1 = self.marks[i + 1][1] if i + 1 < len(self.marks) else float("inf")
+            v = [x[1] for x in self.samples if t0 <= x[0] < t1]
+            if v:
+                phases[name] = {"sm_mhz_median": statistics.median(v), "sm_mhz_min": min(v), "samples": len(v)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[2] for x in self.samples),
                 "sm_min_mhz": min(sm), "samples": len(sm), "reasons": reasons, "source": self.source,
-                "window": f"warm-up through the end-to-end loop, one query per {period}"}
+                "window": f"warm-up of the headline step through the mask-search sweep, one query per {period} "
+                          "(fewer while the host is busy)",
+                "phases": phases}
 
 
 # ------------------------------------------------------------------ our arm
@@ -418,6 +431,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     clk = ClockSampler(torch.cuda.current_device()).__enter__()
     try:
+        clk.mark("headline warm-up and timed steps")
         for _ in range(args.warmup):
             step.run()
         torch.cuda.synchronize()
@@ -431,20 +445,28 @@ def run_ours(args, wl, rank, world, local_rank):
         # every launch (an event between two launches serialises them).
         events = {}
         barrier()
+        clk.mark("headline event pass")
         for _ in range(args.steps):
             flush.fill_(1.0)
             step.run(events)
         barrier()
         peaks, peak_kind = load_peaks()
         kernels = kernel_table(events, step.work(), peaks, FFNStep.KERNELS)
+        clk.mark("weight-gradient step")
         wgrad = run_wgrad_phase(args, step, wl, world, dev, flush, barrier, peaks)
+        clk.mark("dense step")
         dense = run_dense_phase(args, step, wl, world, dev, flush, barrier, peaks)
+        clk.mark("gated step")
         geglu = run_geglu_phase(args, step, wl, world, dev, flush, barrier)
+        clk.mark("end to end")
         e2e = run_e2e(args, step, wl, world, dev, barrier)
         del step
         torch.cuda.empty_cache()
+        clk.mark("gpt2-355m")
         secondary = run_secondary(args, si.GPT2_355M, rank, world, dev, flush, barrier, peaks)
+        clk.mark("mask-search sweep")
         sweep = None if args.no_sweep else run_sweep(args, dev, flush, barrier, peaks)
+        clk.mark("end")
     finally:
         clk.__exit__()
     total_ms = max_over_ranks(step_ms, world, dev)

@@ -43,6 +43,19 @@ def test_clock_sampler_summary_without_a_gpu():
         assert s["sm_mhz"] is None and s["reasons"]
 
 
+def test_clock_sampler_splits_samples_by_phase():
+    """Samples are attributed to the phase whose mark precedes them; the last phase runs on."""
+    c = bench.ClockSampler(0, period_s=0.01)
+    c.source = "nvml"
+    c.marks = [("a", 0.0), ("b", 10.0)]
+    c.samples = [(1.0, 1900.0, 1965.0, set()), (2.0, 1800.0, 1965.0, {"sw_power_cap"}),
+                 (11.0, 1500.0, 1965.0, set()), (-1.0, 1000.0, 1965.0, set())]
+    s = c.summary()
+    assert s["phases"]["a"] == {"sm_mhz_median": 1850.0, "sm_mhz_min": 1800.0, "samples": 2}
+    assert s["phases"]["b"] == {"sm_mhz_median": 1500.0, "sm_mhz_min": 1500.0, "samples": 1}
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 4 and s["sm_min_mhz"] == 1000.0
+
+
 def test_headline_flops_are_the_four_ffn_gemms():
     wl = si.GPT2_355M
     assert wl.gemm_flops() == 4 * 2 * 8192 * 1024 * 4096
