@@ -19,8 +19,9 @@
 // with SPARSE = false runs the dense fine-tuning products.
 //
 // CTA pairs (clusters of 2, tcgen05 cta_group::2).  A pair computes a tile of
-// 256 output features x N tokens (N = 240, or 224 where the epilogue's staging
-// leaves no room; see PairGeom): each CTA holds 128 rows of the compressed
+// 256 output features x N tokens (N = 240 or 224; 224 only where the epilogue's
+// staging leaves no room for 240, or, for variants built both ways, where the
+// host finds the waves fuller at 224; see PairGeom): each CTA holds 128 rows of the compressed
 // operand and N/2 token rows of the activations in its own shared memory, and
 // the pair's even (leader) CTA issues MMAs of M = 256, N, K = 32 that read
 // both.  At N = 240, per CTA and 128-wide K step this moves 48 KB (A 16 KB,

@@ -436,9 +436,10 @@ struct SharedTileSrc {
 //   FLIP:     add the number of mask bits that differ from idx_prev to `flips`
 // Search: every block takes the packed-key search; blocks it cannot certify
 // (magnitudes spread over more than 10 binades for fp16, 13 for bf16) are queued
-// in shared memory and, after a barrier, searched exactly by the first threads
-// of the CTA, so the slow path costs about one warp pass per tile.  The body
-// has three CTA barriers; the caller separates consecutive tiles with a fourth.
+// per warp and searched exactly by the lanes of their own warp, with no barrier
+// across the CTA.  The body has one CTA barrier with COMPRESS (the compressed
+// operands are staged across the CTA's threads) and none without; the caller
+// separates consecutive tiles with one more.
 template <bool BF16, bool SEARCH, bool COMPRESS, bool FLIP, typename Src>
 __device__ __forceinline__ void mask_tile_body(const Src &src, int64_t R, int64_t C, uint32_t cy, uint32_t cx,
                                                int kh, uint32_t chunks_x, uint32_t chunks_y,
