@@ -131,6 +131,9 @@ def test_dense_zero_tokens_is_a_no_op():
     x = torch.empty(0, 128, dtype=torch.float16, device="cuda")
     y = torch.empty(0, 128, dtype=torch.float16, device="cuda")
     sp.sp24_gemm_dense(x, w, y)
+    sp.sp24_gemm_dgrad_dense(x, w, y)
+    sp.sp24_gemm_dgrad_dense(x, w, y, "mul_aux", y)
+    torch.cuda.synchronize()
     assert sp.sp24_device_status() == 0
 
 
