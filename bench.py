@@ -245,7 +245,10 @@ class FFNStep:
         for li in range(2):   # the mask of W_0, against which step 0 counts its flips
             sp.sp24_mask_search(self.W[li][0], self.idx[li][0])
         self.H = torch.empty(T, ff, dtype=tdt, device=dev)
-        self.Gp = torch.empty(T, ff, dtype=tdt, device=dev)   # gelu' of the pre-activation
+        # gelu' of the pre-activation, sized for either layout: the 2:4 step keeps it in the
+        # layout choose_aux_layout() measured faster, the dense step row-major
+        self.Gp = torch.empty(sp.aux_elements(T, ff, "gelu_deriv_packed"), dtype=tdt, device=dev)
+        self.aux_pair = ("gelu_deriv_packed", "mul_aux_packed")
         self.dH = torch.empty(T, ff, dtype=tdt, device=dev)
         self.Y = torch.empty(T, d, dtype=tdt, device=dev)
         self.dX = torch.empty(T, d, dtype=tdt, device=dev)
@@ -301,12 +304,13 @@ class FFNStep:
             timed("mask_step", lambda li=li, c=c: sp.sp24_mask_step(
                 self.W[li][cur], self.idx[li][cur], self.idx[li][prev], self.flips[t, li:li + 1], *c), stream)
         c1, c2 = self.c
-        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, "gelu_deriv", self.Gp),
+        timed("gemm_fwd1_gelu", lambda: sp.sp24_gemm_fwd(self.X, c1[0], c1[1], ff, self.H, self.aux_pair[0],
+                                                         self.Gp),
               main)
         join()
         timed("gemm_fwd2", lambda: sp.sp24_gemm_fwd(self.H, c2[0], c2[1], d, self.Y), main)
         timed("gemm_dgrad2_dgelu",
-              lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, "mul_aux", self.Gp), main)
+              lambda: sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], ff, self.dH, self.aux_pair[1], self.Gp), main)
         if wgrad:
             # Weight gradients into the gradient buffers, decayed in the same kernels:
             # dW2 = MVUE(dY^T) H, dW1 = MVUE(dH^T) X, then + lambda W where pruned;
@@ -328,6 +332,31 @@ class FFNStep:
                                                                           self.idx[li][cur], wl.lam), stream)
             join()
         self.step_no += 1
+
+    def choose_aux_layout(self, reps: int = 3):
+        """Times the derivative-saving pair (forward 1 storing GELU', input gradient 2 multiplying
+        by it) with the derivative row-major and packed, on the step's own operands, and keeps
+        the faster for the 2:4 step.  The packed layout lets the input gradient take wider
+        tiles at some shapes and costs a little at others.  Needs one step run first (the
+        compressed weights)."""
+        sp, torch, wl = self.sp, self.torch, self.wl
+        c1, c2 = self.c
+        best = None
+        for pair in (("gelu_deriv", "mul_aux"), ("gelu_deriv_packed", "mul_aux_packed")):
+            times = []
+            for _ in range(reps):
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                sp.sp24_gemm_fwd(self.X, c1[0], c1[1], wl.ff, self.H, pair[0], self.Gp)
+                sp.sp24_gemm_dgrad(self.dY, c2[2], c2[3], wl.ff, self.dH, pair[1], self.Gp)
+                e.record()
+                torch.cuda.synchronize()
+                times.append(s.elapsed_time(e))
+            t = min(times)
+            if best is None or t < best[0]:
+                best = (t, pair)
+        self.aux_pair = best[1]
+        return {"aux_layout": "packed" if "packed" in best[1][0] else "row-major"}
 
     def run_dense(self, events=None):
         """One step of the dense fine-tuning phase (the last 1/6 of the steps):
@@ -434,6 +463,7 @@ def run_ours(args, wl, rank, world, local_rank):
         clk.mark("headline warm-up and timed steps")
         for _ in range(args.warmup):
             step.run()
+        aux_choice = step.choose_aux_layout()
         torch.cuda.synchronize()
         status("after warm-up")
         # Timed region: the step's launches back to back (each kernel may start
@@ -499,6 +529,8 @@ def run_ours(args, wl, rank, world, local_rank):
                    "perturbation": "W_(t+1) = round(W_t + N(0, 1e-4)) per weight; timed steps cycle t = 0..S-1",
                    "parallelism": f"dp{world} replicas, no collective",
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)",
+                   "gelu_derivative": aux_choice["aux_layout"] + " (the faster of the two layouts, timed on "
+                                      "the step's own operands after warm-up)",
                    "kernel_times": "second pass of the same steps with events around each launch, all on "
                                    "one stream (the timed steps run the second layer's mask step and "
                                    "decay concurrently on a side stream)"},
@@ -534,6 +566,7 @@ def run_secondary(args, wl, rank, world, dev, flush, barrier, peaks):
     step = FFNStep(wl, rank, with_host=False)
     for _ in range(args.warmup):
         step.run()
+    aux_choice = step.choose_aux_layout()
     ms = max_over_ranks(timed_steps(step.run, args.steps, flush, barrier), world, dev) / args.steps
     events = {}
     for _ in range(args.steps):
@@ -546,7 +579,7 @@ def run_secondary(args, wl, rank, world, dev, flush, barrier, peaks):
     kernels = kernel_table(events, step.work(), peaks, FFNStep.KERNELS)
     del step
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff, "tokens_per_gpu": wl.tokens,
+    return {"workload": wl.name, "d_model": wl.d, "d_ff": wl.ff, "tokens_per_gpu": wl.tokens, **aux_choice,
             "ms_per_step": round(ms, 4), "value": round(wl.gemm_flops() * world / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "kernels": kernels}
 

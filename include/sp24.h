@@ -90,8 +90,31 @@ typedef enum sp24_epilogue {
    * dtype instead of the pre-activation.  (Value 5 is the library's own
    * weight-gradient epilogue and is not taken here.) */
   SP24_EPI_GELU_DERIV = 6, /* out = gelu(acc); aux <- gelu'(acc) rounded to dtype */
-  SP24_EPI_MUL_AUX = 7     /* out = acc * aux; aux [T x K] holds gelu'(pre-activation) */
+  SP24_EPI_MUL_AUX = 7,    /* out = acc * aux; aux [T x K] holds gelu'(pre-activation) */
+  /* The same pair with aux in the packed chunk layout below instead of
+   * row-major: the kernels write and read it straight from the registers that
+   * hold the accumulator, with no staging in shared memory. */
+  SP24_EPI_GELU_DERIV_PACKED = 8, /* out = gelu(acc); aux (packed) <- gelu'(acc) */
+  SP24_EPI_MUL_AUX_PACKED = 9     /* out = acc * aux; aux (packed) holds gelu'(pre-activation) */
 } sp24_epilogue;
+
+/*
+ * Packed chunk layout of a 16-bit [T x M] matrix (the aux of the _PACKED
+ * epilogues, M the output width of the product that writes or reads it):
+ * blocks of 16 tokens x 32 features, 1024 bytes each; block (t/16, m/32)
+ * starts at element ((t/16) * ceil(M/32) + m/32) * 512.  In a block, element
+ * (t, m) with t' = t % 16, m' = m % 32, h = m' / 16, f = m' % 16 sits at
+ *   256 h + 8 (4 (f % 8) + (t' % 8) / 2) + 2 (2 (t' / 8) + f / 8) + t' % 2.
+ * Blocks past T or M are part of the buffer (ceil(T/16) x ceil(M/32) blocks);
+ * their padding entries are unspecified.  The buffer must be 16-byte aligned.
+ */
+SP24_API sp24_status sp24_aux_packed_size(int64_t T, int64_t M, size_t *bytes);
+
+/* Host index maps of the packed layout (host memory, 16-bit elements):
+ * sp24_aux_pack writes every block of packed (padding entries 0) from
+ * rowmajor [T x M]; sp24_aux_unpack writes rowmajor from packed. */
+SP24_API sp24_status sp24_aux_pack(const void *rowmajor, int64_t T, int64_t M, void *packed);
+SP24_API sp24_status sp24_aux_unpack(const void *packed, int64_t T, int64_t M, void *rowmajor);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 SP24_API const char *sp24_status_string(sp24_status status);

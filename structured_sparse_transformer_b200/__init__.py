@@ -47,6 +47,9 @@ _SIGNATURES = {
     "sp24_masked_decay": [P, P, I32, I64, I64, P, F32, P],
     "sp24_flip_rate": [P, P, I64, P, P],
     "sp24_meta_to_canonical": [P, I64, I64, P],
+    "sp24_aux_packed_size": [I64, I64, P],
+    "sp24_aux_pack": [P, I64, I64, P],
+    "sp24_aux_unpack": [P, I64, I64, P],
     "sp24_meta_from_canonical": [P, I64, I64, P],
     "sp24_device_status": [P],
     "sp24_set_wait_budget": [U64],
@@ -63,7 +66,9 @@ STATUS = {0: "SP24_OK", 1: "SP24_ERR_INVALID_ARG", 2: "SP24_ERR_UNSUPPORTED_SHAP
           6: "SP24_ERR_TIMEOUT", 7: "SP24_ERR_NO_DEVICE", 8: "SP24_ERR_SCRATCH_TOO_SMALL"}
 SP24_F16, SP24_BF16 = 0, 1
 SP24_EPI_NONE, SP24_EPI_GELU, SP24_EPI_DGELU = 0, 1, 2
-EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4, "gelu_deriv": 6, "mul_aux": 7}
+EPILOGUES = {None: 0, "none": 0, "gelu": 1, "dgelu": 2, "geglu": 3, "dgeglu": 4, "gelu_deriv": 6, "mul_aux": 7,
+             "gelu_deriv_packed": 8, "mul_aux_packed": 9}
+PACKED_EPILOGUES = ("gelu_deriv_packed", "mul_aux_packed")
 
 
 class Sp24Error(RuntimeError):
@@ -166,6 +171,38 @@ def sp24_compressed_size(rows: int, cols: int, dtype: int = SP24_F16):
     return v.value, m.value
 
 
+def sp24_aux_packed_size(T: int, M: int) -> int:
+    """Bytes of a 16-bit [T, M] matrix in the packed chunk layout (the _packed epilogues' aux)."""
+    out = ctypes.c_size_t(0)
+    _check("sp24_aux_packed_size", _lib.sp24_aux_packed_size(T, M, ctypes.byref(out)))
+    return out.value
+
+
+def aux_elements(T: int, M: int, epi) -> int:
+    """16-bit elements of the aux buffer of a [T, M] product with epilogue epi."""
+    return sp24_aux_packed_size(T, M) // 2 if epi in PACKED_EPILOGUES else T * M
+
+
+def sp24_aux_pack(rowmajor, T: int, M: int):
+    """Row-major uint16 [T, M] (numpy, host) -> the packed chunk layout (numpy uint16, padding 0)."""
+    import numpy as np
+    src = np.ascontiguousarray(rowmajor, dtype=np.uint16).reshape(T, M)
+    out = np.zeros(sp24_aux_packed_size(T, M) // 2, dtype=np.uint16)
+    _check("sp24_aux_pack", _lib.sp24_aux_pack(src.ctypes.data, T, M, out.ctypes.data))
+    return out
+
+
+def sp24_aux_unpack(packed, T: int, M: int):
+    """The packed chunk layout (numpy uint16, host) -> row-major uint16 [T, M] (numpy)."""
+    import numpy as np
+    src = np.ascontiguousarray(packed, dtype=np.uint16).reshape(-1)
+    if src.size * 2 < sp24_aux_packed_size(T, M):
+        raise ValueError(f"packed aux has {src.size} elements, needs {sp24_aux_packed_size(T, M) // 2}")
+    out = np.zeros((T, M), dtype=np.uint16)
+    _check("sp24_aux_unpack", _lib.sp24_aux_unpack(src.ctypes.data, T, M, out.ctypes.data))
+    return out
+
+
 def sp24_meta_to_canonical(meta_bytes: bytes, rows: int, cols: int):
     """Device-layout metadata (host bytes) -> canonical uint16 words [rows][cols/16] (numpy)."""
     import numpy as np
@@ -240,7 +277,7 @@ def sp24_gemm_fwd(X, vals_row, meta_row, N: int, Y, epi=None, aux=None, stream=N
     _dtype_code(X)
     _expect_compressed(vals_row, meta_row, N, K, X.dtype, "W")
     _expect(Y, "Y", X.dtype, T * (N // 2 if epi == "geglu" else N))
-    _expect(aux, "aux", X.dtype, T * N)
+    _expect(aux, "aux", X.dtype, aux_elements(T, N, epi))
     _need_device(X, vals_row, meta_row, Y, aux)
     _check("sp24_gemm_fwd",
            _lib.sp24_gemm_fwd(_ptr(X), T, K, _ptr(vals_row), _ptr(meta_row), N, _dtype_code(X), _ptr(Y),
@@ -257,7 +294,7 @@ def sp24_gemm_dgrad(dY, vals_col, meta_col, K: int, dX, epi=None, aux=None, stre
     _expect_compressed(vals_col, meta_col, K, N, dY.dtype, "W^T")
     width = 2 * K if epi == "dgeglu" else K
     _expect(dX, "dX", dY.dtype, T * width)
-    _expect(aux, "aux", dY.dtype, T * width)
+    _expect(aux, "aux", dY.dtype, aux_elements(T, width, epi))
     _need_device(dY, vals_col, meta_col, dX, aux)
     _check("sp24_gemm_dgrad",
            _lib.sp24_gemm_dgrad(_ptr(dY), T, N, _ptr(vals_col), _ptr(meta_col), K, _dtype_code(dY), _ptr(dX),
@@ -273,7 +310,7 @@ def sp24_gemm_dense(B, A, out, epi=None, aux=None, stream=None):
     _dtype_code(B)
     _expect(A, "A", B.dtype, M * Kd)
     _expect(out, "out", B.dtype, T * M)
-    _expect(aux, "aux", B.dtype, T * M)
+    _expect(aux, "aux", B.dtype, aux_elements(T, M, epi))
     _need_device(B, A, out, aux)
     _check("sp24_gemm_dense",
            _lib.sp24_gemm_dense(_ptr(B), T, Kd, _ptr(A), M, _dtype_code(B), _ptr(out), EPILOGUES[epi], _ptr(aux),
@@ -291,7 +328,7 @@ def sp24_gemm_dgrad_dense(dY, W, dX, epi=None, aux=None, stream=None):
     _dtype_code(dY)
     _expect(W, "W", dY.dtype, N * K)
     _expect(dX, "dX", dY.dtype, T * K)
-    _expect(aux, "aux", dY.dtype, T * K)
+    _expect(aux, "aux", dY.dtype, aux_elements(T, K, epi))
     _need_device(dY, W, dX, aux)
     _check("sp24_gemm_dgrad_dense",
            _lib.sp24_gemm_dgrad_dense(_ptr(dY), T, N, _ptr(W), K, _dtype_code(dY), _ptr(dX), EPILOGUES[epi],

@@ -94,8 +94,19 @@ constexpr int kPairBNNarrow = 224;                     // else
 // pre-activation.
 enum : int {
   kEpiNone = 0, kEpiGelu = 1, kEpiDgelu = 2, kEpiGeglu = 3, kEpiDgeglu = 4, kEpiWgrad = 5, kEpiGeluDeriv = 6,
-  kEpiMulAux = 7
+  kEpiMulAux = 7,
+  // The derivative-saving pair with the derivative in the packed chunk layout
+  // (below): written and read straight from registers, no staging tile.
+  kEpiGeluDerivPacked = 8,
+  kEpiMulAuxPacked = 9
 };
+// Packed chunk layout of a 16-bit [T x M] matrix: blocks of 16 tokens x 32
+// features (1 KB), block (t / 16, m / 32) at element offset
+// ((t / 16) * ceil(M / 32) + m / 32) * 512.  Inside a block, half h (features
+// 16h .. 16h + 15) is 512 bytes; lane l's 16 bytes at 16 l hold the four 32-bit
+// registers i = 0..3 of the epilogue fragment: tokens 8 (i / 2) + 2 (l % 4) + {0, 1}
+// (low, high half) of feature 16 h + 8 (i % 2) + l / 4.  A warp's fragment of one
+// chunk is then two 512-byte runs, stored and loaded with 16-byte accesses.
 constexpr int kGegluGroup = 16;   // rows of W_gate, then of W_up, alternate in the stacked gated weight
 
 // Pipeline stage of the 2:4 GEMM (SPARSE) and of the dense GEMM of the dense
@@ -128,7 +139,7 @@ constexpr int kPairBarBytes = 512;                     // mbarriers, TMEM addres
 // inputs.
 __host__ __device__ constexpr int epi_bufs(int epi) {
   return epi == kEpiWgrad ? 0
-                          : epi == kEpiNone ? 1
+                          : (epi == kEpiNone || epi == kEpiGeluDerivPacked || epi == kEpiMulAuxPacked) ? 1
                           : (epi == kEpiGelu || epi == kEpiGeglu || epi == kEpiGeluDeriv) ? 2
                           : ((epi == kEpiDgelu || epi == kEpiMulAux) ? 3 : 6);
 }
@@ -417,7 +428,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                           uint64_t wait_budget, float *__restrict__ out_f32, int64_t ld_out,
                           const uint16_t *__restrict__ dec_w, const uint8_t *__restrict__ dec_idx,
                           float dec_lambda, float *__restrict__ sk_part, unsigned *__restrict__ sk_flags,
-                          int sk_split, int cols_fastest, int a_mn) {
+                          int sk_split, int cols_fastest, int a_mn, uint16_t *__restrict__ aux_packed,
+                          int aux_nbf) {
   // T counts the B operand's rows of the output: tokens, or for the weight
   // gradient the columns of dW (out_f32 [M x T], leading dimension ld_out).
   // Weight gradient with dec_w set: the masked decay of dW in the epilogue, W and
@@ -429,6 +441,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // parts per tail tile, partial accumulators in sk_part (kSkPartFloatsPerCta
   // per CTA) and ready counters in sk_flags (kEpiWarps per CTA, zero at launch
   // and left zero).
+  // Packed-derivative epilogues: aux_packed in the packed chunk layout with
+  // aux_nbf = ceil(M / 32) feature blocks per token block.
   // Dense with a_mn set: A is read as stored [K x M] (M contiguous), MN-major
   // like the dense weight gradient's A: the input gradient takes W itself.
   using G = PairGeom<SPARSE, EPI, WIDE>;
@@ -837,6 +851,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tma_load_2d(stg + kOutBytes + kPreBytes * (seq & 1), &tm_aux, bar, x, y);
       }
     };
+    // This lane's 16 bytes of half 0 of the packed block holding chunk (t0, m0);
+    // half 1 is 256 elements further.
+    auto packed_at = [&](int t0, int m0) {
+      return aux_packed + ((((size_t)(t0 >> 4) * (size_t)aux_nbf + (size_t)(m0 >> 5)) << 9) + 8 * (size_t)lane);
+    };
+    uint4 pk_cur[2], pk_nxt[2];   // MulAuxPacked: this chunk's and the next chunk's derivative
+    auto packed_load = [&](int t0, int m0, uint4 (&v)[2]) {
+      if (m0 < M) {
+        const uint16_t *src = packed_at(t0, m0);
+        v[0] = __ldg(reinterpret_cast<const uint4 *>(src));
+        v[1] = __ldg(reinterpret_cast<const uint4 *>(src + 256));
+      } else {
+        v[0] = v[1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
     bool alive = true;
     int j = 0;
     for (int tile = pair; tile < num_tiles && alive; tile += npairs, ++j) {
@@ -847,6 +876,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const int nk = grp < nchunks ? (nchunks - 1 - grp) / kEpiGroups + 1 : 0;   // this warp's chunks
       if (kPre)
         for (int k = 0; k < 2 && k < nk; ++k) pre_load(pre_col(m0), n0 + (grp + k * kEpiGroups) * kEpiTokens);
+      if (EPI == kEpiMulAuxPacked && nk > 0) packed_load(n0 + grp * kEpiTokens, m0, pk_nxt);
       const bool got = mbar_wait_bounded(&acc_full[b], (uint32_t)(j >> 1) & 1u, wait_budget, s_abort);
       if (!__all_sync(0xFFFFFFFFu, got)) {
         alive = false;
@@ -893,6 +923,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
         };
         if (EPI == kEpiGeglu || EPI == kEpiDgeglu) staging_free();
+        if (EPI == kEpiMulAuxPacked) {
+          pk_cur[0] = pk_nxt[0];
+          pk_cur[1] = pk_nxt[1];
+          if (k + 1 < nk) packed_load(t0 + kEpiGroups * kEpiTokens, m0, pk_nxt);   // one chunk ahead
+        }
         // Register i of half h: tokens 8(i/2) + 2(lane%4) + {0, 1} of feature
         // 16h + 8(i%2) + lane/4 (TMEM registers 4(i/2) + 2(i%2) + {0, 1}).
         if (EPI == kEpiGeglu) {
@@ -945,6 +980,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             ldmatrix_x4_trans(pre_src + lane_off0, hx[0]);
             ldmatrix_x4_trans(pre_src + lane_off1, hx[1]);
           }
+          if (EPI == kEpiMulAuxPacked) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              hx[h][0] = pk_cur[h].x;
+              hx[h][1] = pk_cur[h].y;
+              hx[h][2] = pk_cur[h].z;
+              hx[h][3] = pk_cur[h].w;
+            }
+          }
           uint32_t po[2][4], pa[2][4];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -956,11 +1000,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               if (EPI == kEpiGelu) {
                 y = gelu2(acc);
                 pa[h][i] = pack2<BF16>(acc.x, acc.y);
-              } else if (EPI == kEpiGeluDeriv) {
+              } else if (EPI == kEpiGeluDeriv || EPI == kEpiGeluDerivPacked) {
                 float2 gp;
                 gelu_and_grad2(acc, y, gp);
                 pa[h][i] = pack2<BF16>(gp.x, gp.y);
-              } else if (EPI == kEpiMulAux) {
+              } else if (EPI == kEpiMulAux || EPI == kEpiMulAuxPacked) {
                 float2 hv;
                 unpack2<BF16>(hx[h][i], hv.x, hv.y);
                 y = __fmul2_rn(acc, hv);
@@ -971,6 +1015,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               }
               po[h][i] = pack2<BF16>(y.x, y.y);
             }
+          }
+          if (EPI == kEpiGeluDerivPacked && m0 < M) {   // the derivative, straight from registers
+            uint16_t *dst = packed_at(t0, m0);
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(pa[0][0], pa[0][1], pa[0][2], pa[0][3]);
+            *reinterpret_cast<uint4 *>(dst + 256) = make_uint4(pa[1][0], pa[1][1], pa[1][2], pa[1][3]);
           }
           staging_free();
           stmatrix_x4_trans(stg_u32 + lane_off0, po[0]);

@@ -309,8 +309,8 @@ sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void 
               make_map_2d(&tx, aux, (uint64_t)M * 2, (uint64_t)T, (uint64_t)M * 4, 64, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_128B);
   } else {
     maps_ok = make_map_2d(&to, out, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B) &&
-              make_map_2d(&tx, EPI == kEpiNone ? out : aux, (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens,
-                          CU_TENSOR_MAP_SWIZZLE_64B);
+              make_map_2d(&tx, (EPI == kEpiNone || EPI == kEpiGeluDerivPacked || EPI == kEpiMulAuxPacked) ? out : aux,
+                          (uint64_t)M, (uint64_t)T, (uint64_t)M * 2, 32, kEpiTokens, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   if (!maps_ok) return SP24_ERR_CUDA;
   constexpr int smem_bytes = pair_smem_bytes<SPARSE, EPI, WIDE>();
@@ -352,7 +352,9 @@ sp24_status launch_gemm_pair_w(const void *B, int64_t T, int64_t Kd, const void 
   return launch_pdl(kernel, dim3(2 * grid_pairs), dim3(kGemmThreads), smem_bytes, stream, ta, tb, tm, to, tx, (int)M,
                     (int)T, num_kt, (uint64_t)g_wait_budget.load(), G::kWg ? static_cast<float *>(out) : nullptr,
                     (int64_t)(G::kWg ? T : 0), static_cast<const uint16_t *>(dec_w), dec_idx, dec_lambda, ws.part,
-                    ws.flags, split, cols_fastest, a_mn ? 1 : 0);
+                    ws.flags, split, cols_fastest, a_mn ? 1 : 0,
+                    (EPI == kEpiGeluDerivPacked || EPI == kEpiMulAuxPacked) ? static_cast<uint16_t *>(aux) : nullptr,
+                    (int)((M + 31) / 32));
 }
 
 // Tile width per call, for the variants that have both: the busiest pair's token
@@ -400,6 +402,12 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
     case kEpiMulAux:
       return bf ? launch_gemm_pair_t<true, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
                 : launch_gemm_pair_t<false, kEpiMulAux, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
+    case kEpiGeluDerivPacked:
+      return bf ? launch_gemm_pair_t<true, kEpiGeluDerivPacked, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                : launch_gemm_pair_t<false, kEpiGeluDerivPacked, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
+    case kEpiMulAuxPacked:
+      return bf ? launch_gemm_pair_t<true, kEpiMulAuxPacked, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn)
+                : launch_gemm_pair_t<false, kEpiMulAuxPacked, SPARSE>(B, T, Kd, vals, meta, M, out, aux, s, nullptr, nullptr, 0.0f, nullptr, a_mn);
     default: break;
   }
   if (SPARSE) {   // the gated epilogues serve the 2:4 GEMMs
@@ -416,12 +424,18 @@ sp24_status launch_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, 
 
 // The epilogues each product takes (bit e of the mask allows epilogue e).
 constexpr unsigned kFwdEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_GELU) | (1u << SP24_EPI_GEGLU) |
-                              (1u << SP24_EPI_GELU_DERIV);
+                              (1u << SP24_EPI_GELU_DERIV) | (1u << SP24_EPI_GELU_DERIV_PACKED);
 constexpr unsigned kDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) | (1u << SP24_EPI_DGEGLU) |
-                                (1u << SP24_EPI_MUL_AUX);
+                                (1u << SP24_EPI_MUL_AUX) | (1u << SP24_EPI_MUL_AUX_PACKED);
 constexpr unsigned kDenseEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_GELU) | (1u << SP24_EPI_DGELU) |
-                                (1u << SP24_EPI_GELU_DERIV) | (1u << SP24_EPI_MUL_AUX);
-constexpr unsigned kDenseDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) | (1u << SP24_EPI_MUL_AUX);
+                                (1u << SP24_EPI_GELU_DERIV) | (1u << SP24_EPI_MUL_AUX) |
+                                (1u << SP24_EPI_GELU_DERIV_PACKED) | (1u << SP24_EPI_MUL_AUX_PACKED);
+constexpr unsigned kDenseDgradEpis = (1u << SP24_EPI_NONE) | (1u << SP24_EPI_DGELU) | (1u << SP24_EPI_MUL_AUX) |
+                                     (1u << SP24_EPI_MUL_AUX_PACKED);
+static_assert((int)SP24_EPI_GELU_DERIV_PACKED == (int)kEpiGeluDerivPacked &&
+                  (int)SP24_EPI_MUL_AUX_PACKED == (int)kEpiMulAuxPacked &&
+                  (int)SP24_EPI_GELU_DERIV == (int)kEpiGeluDeriv && (int)SP24_EPI_MUL_AUX == (int)kEpiMulAux,
+              "public and kernel epilogue numbers");
 
 sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals, const void *meta, int64_t M,
                           sp24_dtype dt, const void *out, int epi, const void *aux, unsigned allowed_epis) {
@@ -431,7 +445,7 @@ sp24_status validate_gemm(const void *B, int64_t T, int64_t Kd, const void *vals
   if (!valid_dtype(dt)) return SP24_ERR_UNSUPPORTED_DTYPE;
   if (epi < 0 || epi > 31 || !((allowed_epis >> epi) & 1u)) return SP24_ERR_INVALID_ARG;
   if (epi == SP24_EPI_GEGLU && M % (2 * kGegluGroup)) return SP24_ERR_UNSUPPORTED_SHAPE;
-  if (epi != SP24_EPI_NONE && !aux) return SP24_ERR_INVALID_ARG;
+  if (epi != SP24_EPI_NONE && !aux && T > 0) return SP24_ERR_INVALID_ARG;   // T == 0 touches nothing
   if (Kd % 16 || M % 16) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (T > INT32_MAX || M > INT32_MAX || Kd > INT32_MAX) return SP24_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(B) || !aligned16(vals) || !aligned16(meta) || !aligned16(out) ||
@@ -520,6 +534,17 @@ sp24_status launch_wgrad(const void *X, int64_t T, int64_t K, const void *A, con
                                                      fixed);
 }
 
+}  // namespace
+
+namespace {
+// (packed chunk layout of the derivative-saving epilogues; see gemm_sp.cuh)
+// Element offset, in the packed chunk layout of a [T x M] matrix, of (t, m).
+size_t aux_packed_offset(int64_t t, int64_t m, int64_t M) {
+  const int64_t tin = t & 15, fin = m & 31, h = fin >> 4, ff = fin & 15;
+  const int64_t lane = 4 * (ff & 7) + ((tin & 7) >> 1), reg = 2 * (tin >> 3) + (ff >> 3);
+  const int64_t block = (t >> 4) * ((M + 31) / 32) + (m >> 5);
+  return (size_t)(block * 512 + h * 256 + lane * 8 + reg * 2 + (tin & 1));
+}
 }  // namespace
 
 extern "C" {
@@ -804,6 +829,33 @@ sp24_status sp24_flip_rate(const uint8_t *idx_prev, const uint8_t *idx_cur, int6
   const int64_t want = (nblocks / 16 + 255) / 256 + 1;
   const int grid = (int)(want < (int64_t)sm_count() * 8 ? want : (int64_t)sm_count() * 8);
   return launch_pdl(flip_count_kernel, dim3(grid), dim3(256), 0, s, idx_prev, idx_cur, nblocks, d_count);
+}
+
+sp24_status sp24_aux_packed_size(int64_t T, int64_t M, size_t *bytes) {
+  if (T < 0 || M < 0 || !bytes) return SP24_ERR_INVALID_ARG;
+  *bytes = (size_t)((T + 15) / 16) * (size_t)((M + 31) / 32) * 1024u;
+  return SP24_OK;
+}
+
+sp24_status sp24_aux_pack(const void *rowmajor, int64_t T, int64_t M, void *packed) {
+  if (T < 0 || M < 0 || (T > 0 && M > 0 && (!rowmajor || !packed))) return SP24_ERR_INVALID_ARG;
+  const uint16_t *src = static_cast<const uint16_t *>(rowmajor);
+  uint16_t *dst = static_cast<uint16_t *>(packed);
+  size_t bytes = 0;
+  sp24_aux_packed_size(T, M, &bytes);
+  if (bytes) memset(dst, 0, bytes);
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t m = 0; m < M; ++m) dst[aux_packed_offset(t, m, M)] = src[t * M + m];
+  return SP24_OK;
+}
+
+sp24_status sp24_aux_unpack(const void *packed, int64_t T, int64_t M, void *rowmajor) {
+  if (T < 0 || M < 0 || (T > 0 && M > 0 && (!rowmajor || !packed))) return SP24_ERR_INVALID_ARG;
+  const uint16_t *src = static_cast<const uint16_t *>(packed);
+  uint16_t *dst = static_cast<uint16_t *>(rowmajor);
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t m = 0; m < M; ++m) dst[t * M + m] = src[aux_packed_offset(t, m, M)];
+  return SP24_OK;
 }
 
 sp24_status sp24_meta_to_canonical(const void *meta_dev_layout_host, int64_t rows, int64_t cols, uint16_t *canon) {

@@ -50,7 +50,8 @@ def main(argv=None):
     ap.add_argument("--via-transpose", action="store_true",
                     help="gemm_dense_dgrad: multiply by W^T formed with sp24_transpose")
     ap.add_argument("--dist", choices=["normal", "tie"], default="normal")
-    ap.add_argument("--epi", choices=["none", "gelu", "dgelu", "gelu_deriv", "mul_aux", "geglu", "dgeglu"],
+    ap.add_argument("--epi", choices=["none", "gelu", "dgelu", "gelu_deriv", "mul_aux", "geglu", "dgeglu",
+                                      "gelu_deriv_packed", "mul_aux_packed"],
                     default="none")
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
@@ -88,10 +89,10 @@ def main(argv=None):
         sp.sp24_mask_search(w, idx)
     elif k == "gemm_fwd":
         x = torch.randn(T, C, device=dev, generator=gen).to(tdt)
-        epi = args.epi if args.epi in ("gelu", "gelu_deriv", "geglu") else None
+        epi = args.epi if args.epi in ("gelu", "gelu_deriv", "geglu", "gelu_deriv_packed") else None
         # geglu: W is the stacked gate/up weight [rows = 2 ff, cols]; out [T, ff], aux [T, 2 ff]
         y = torch.empty(T, R // 2 if epi == "geglu" else R, dtype=tdt, device=dev)
-        aux = torch.empty(T, R, dtype=tdt, device=dev) if epi else None
+        aux = torch.empty(sp.aux_elements(T, R, epi), dtype=tdt, device=dev) if epi else None
         fn = lambda: sp.sp24_gemm_fwd(x, bufs[0], bufs[1], R, y, epi, aux)
     elif k in ("mvue", "gemm_wgrad", "gemm_wgrad_decay"):
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
@@ -136,11 +137,11 @@ def main(argv=None):
             fn = lambda: sp.sp24_gemm_dgrad_dense(dy, w, dx, epi, aux)
     else:
         dy = torch.randn(T, R, device=dev, generator=gen).to(tdt)
-        epi = args.epi if args.epi in ("dgelu", "mul_aux", "dgeglu") else None
+        epi = args.epi if args.epi in ("dgelu", "mul_aux", "dgeglu", "mul_aux_packed") else None
         # dgeglu: W is the down projection [rows = d, cols = ff]; aux and dX are [T, 2 ff]
         width = 2 * C if epi == "dgeglu" else C
         dx = torch.empty(T, width, dtype=tdt, device=dev)
-        aux = torch.randn(T, width, device=dev, generator=gen).to(tdt) if epi else None
+        aux = torch.randn(sp.aux_elements(T, width, epi), device=dev, generator=gen).to(tdt) if epi else None
         fn = lambda: sp.sp24_gemm_dgrad(dy, bufs[2], bufs[3], C, dx, epi, aux)
 
     for _ in range(args.warmup):

@@ -79,6 +79,12 @@ def test_host_validation_rejects_bad_arguments_without_a_device():
         E["SP24_ERR_INVALID_ARG"]                       # DGELU is not a forward epilogue
     assert _raw("sp24_gemm_dgrad", fake, 8, 32, fake, fake, 16, 0, fake, 1, fake, None) == \
         E["SP24_ERR_INVALID_ARG"]                       # GELU is not an input-gradient epilogue
+    assert _raw("sp24_gemm_dgrad", fake, 8, 32, fake, fake, 16, 0, fake, 8, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # the packed GELU' writer is a forward epilogue
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 16, 0, fake, 9, fake, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # the packed multiply is an input-gradient epilogue
+    assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 16, 0, fake, 8, None, None) == \
+        E["SP24_ERR_INVALID_ARG"]                       # packed GELU' without aux
     assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 48, 0, fake, 3, fake, None) == \
         E["SP24_ERR_UNSUPPORTED_SHAPE"]                # GEGLU needs whole gate/up row groups
     assert _raw("sp24_gemm_fwd", fake, 8, 32, fake, fake, 64, 0, fake, 4, fake, None) == \
@@ -213,6 +219,9 @@ def test_binding_rejects_wrong_dtype_and_short_buffers():
     bad(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, y.float(), match="Y")
     ok_until_device(sp.sp24_gemm_fwd, x, comp[0], comp[1], R, torch.zeros(T, R // 2, dtype=f16), "geglu", y)
     ok_until_device(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "dgelu", x.clone())
+    pk = torch.zeros(sp.sp24_aux_packed_size(T, C) // 2, dtype=f16)
+    ok_until_device(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "mul_aux_packed", pk)
+    bad(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "mul_aux_packed", pk[:-8].clone(), match="aux")
     bad(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x[:1], match="dX")
     bad(sp.sp24_gemm_dgrad, y, comp[2], comp[3], C, x, "dgeglu", x.clone(), match="dX")
     bad(sp.sp24_gemm_dgrad, y, comp[2][:10], comp[3], C, x, match="W\\^T values")
