@@ -333,13 +333,18 @@ class FFNStep:
             join()
         self.step_no += 1
 
-    def choose_aux_layout(self, reps: int = 3):
+    def choose_aux_layout(self, reps: int = 3, force: str = "auto"):
         """Times the derivative-saving pair (forward 1 storing GELU', input gradient 2 multiplying
         by it) with the derivative row-major and packed, on the step's own operands, and keeps
         the faster for the 2:4 step.  The packed layout lets the input gradient take wider
         tiles at some shapes and costs a little at others.  Needs one step run first (the
-        compressed weights)."""
+        compressed weights).  `force` ("packed" or "row-major") skips the timing, for runs under
+        a profiler, whose serialised launches make the events meaningless."""
         sp, torch, wl = self.sp, self.torch, self.wl
+        if force != "auto":
+            self.aux_pair = (("gelu_deriv_packed", "mul_aux_packed") if force == "packed"
+                             else ("gelu_deriv", "mul_aux"))
+            return {"aux_layout": force}
         c1, c2 = self.c
         best = None
         for pair in (("gelu_deriv", "mul_aux"), ("gelu_deriv_packed", "mul_aux_packed")):
@@ -463,7 +468,7 @@ def run_ours(args, wl, rank, world, local_rank):
         clk.mark("headline warm-up and timed steps")
         for _ in range(args.warmup):
             step.run()
-        aux_choice = step.choose_aux_layout()
+        aux_choice = step.choose_aux_layout(force=args.aux_layout)
         torch.cuda.synchronize()
         status("after warm-up")
         # Timed region: the step's launches back to back (each kernel may start
@@ -529,8 +534,9 @@ def run_ours(args, wl, rank, world, local_rank):
                    "perturbation": "W_(t+1) = round(W_t + N(0, 1e-4)) per weight; timed steps cycle t = 0..S-1",
                    "parallelism": f"dp{world} replicas, no collective",
                    "l2": "flushed before every timed step (256 MiB write, outside the step events)",
-                   "gelu_derivative": aux_choice["aux_layout"] + " (the faster of the two layouts, timed on "
-                                      "the step's own operands after warm-up)",
+                   "gelu_derivative": aux_choice["aux_layout"] + (" (the faster of the two layouts, timed on "
+                                                                  "the step's own operands after warm-up)"
+                                                                  if args.aux_layout == "auto" else " (as asked)"),
                    "kernel_times": "second pass of the same steps with events around each launch, all on "
                                    "one stream (the timed steps run the second layer's mask step and "
                                    "decay concurrently on a side stream)"},
@@ -566,7 +572,7 @@ def run_secondary(args, wl, rank, world, dev, flush, barrier, peaks):
     step = FFNStep(wl, rank, with_host=False)
     for _ in range(args.warmup):
         step.run()
-    aux_choice = step.choose_aux_layout()
+    aux_choice = step.choose_aux_layout(force=args.aux_layout)
     ms = max_over_ranks(timed_steps(step.run, args.steps, flush, barrier), world, dev) / args.steps
     events = {}
     for _ in range(args.steps):
@@ -953,6 +959,8 @@ def main(argv=None):
     ap.add_argument("--sweep-iters", type=int, default=5)
     ap.add_argument("--cpu-tokens", type=int, default=256, help="token rows of the oracle's GEMM sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--aux-layout", choices=["auto", "packed", "row-major"], default="auto",
+                    help="layout of the stored GELU' in the 2:4 step (auto: the faster, timed after warm-up)")
     ap.add_argument("--gemm-traffic", type=float, default=None, help="ncu DRAM bytes per GEMM launch")
     ap.add_argument("--mask-traffic", type=float, default=None, help="ncu DRAM bytes per mask-step launch")
     args = ap.parse_args(argv)
