@@ -26,7 +26,7 @@ def _bits(t):
 
 @pytest.mark.parametrize("dense", [False, True])
 @pytest.mark.parametrize("T,d,ff,dtype", [(1000, 1600, 6400, "f16"), (300, 400, 208, "bf16"), (77, 64, 48, "f16"),
-                                          (4096, 1024, 4096, "bf16")])
+                                          (4096, 1024, 4096, "bf16"), (1, 32, 16, "f16")])
 def test_packed_pair_equals_the_row_major_pair(T, d, ff, dtype, dense):
     tdt = si.DTYPES[dtype]
     W1 = si.normal((ff, d), 0.02, T + ff, dtype).cuda()     # layer 1: X [T, d] -> H [T, ff]
